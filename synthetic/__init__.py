@@ -1,0 +1,148 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests/benchmark and by the oracle's tests.
+
+This module draws random numbers and lays them out; it holds none of the decoder's arithmetic.
+Weights are random-init (no trained checkpoint exists here); ids are uniform; logits for the
+standalone sampler workload are Gaussian with sparse spikes.
+
+Weight layout (row-major, PyTorch ``Linear`` convention: [out_features, in_features]):
+  emb        [V, d]            bf16   embedding table
+  head       [V, d]            bf16   untied vocabulary projection
+  final_norm [d]               fp32   RMSNorm gain
+  per layer:
+    attn_norm [d]              fp32
+    w_qkv     [(Hq+2Hkv)*dh, d] bf16  Q rows, then K rows, then V rows
+    w_o       [d, Hq*dh]        bf16
+    ffn_norm  [d]              fp32
+    w_router  [E, d]            bf16
+    w_gate_up [E, 2F, d]        bf16  per expert: F gate rows, then F up rows
+    w_down    [E, d, F]         bf16
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class ModelConfig:
+    d_model: int
+    n_q: int
+    n_kv: int
+    d_head: int
+    n_exp: int
+    top_k: int
+    d_ff: int
+    n_layers: int
+    vocab: int
+    rms_eps: float = 1e-6
+    rope_theta: float = 10000.0
+
+    @property
+    def qkv_rows(self) -> int:
+        return (self.n_q + 2 * self.n_kv) * self.d_head
+
+
+# Tiny oracle model: 2 layers, d 256, 4 Q / 2 KV heads of dim 64, 8 experts top-2, FFN 512, V 4096.
+TINY = ModelConfig(d_model=256, n_q=4, n_kv=2, d_head=64, n_exp=8, top_k=2, d_ff=512, n_layers=2, vocab=4096)
+# Full-width decoder layer of the Gemma-4-26B-A4B shape: d 2816, 16 Q / 8 KV heads of dim 128,
+# 128 experts top-8 with FFN 704, vocabulary 262144.
+FULL = ModelConfig(d_model=2816, n_q=16, n_kv=8, d_head=128, n_exp=128, top_k=8, d_ff=704, n_layers=30,
+                   vocab=262144)
+ONE_LAYER = dataclasses.replace(FULL, n_layers=1)
+
+CANVAS = 256
+MAX_STEPS = 48
+T_START, T_END = 0.8, 0.4
+ENTROPY_BOUND = 0.1
+STOP_MEAN_ENTROPY = 0.005
+
+
+def default_rerand_entropy(vocab: int) -> float:
+    """Threshold above which a non-committing position is re-randomised (a stated default: half of
+    the maximum entropy ln V)."""
+    return 0.5 * math.log(vocab)
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _normal_bf16(shape, std, gen, device) -> torch.Tensor:
+    t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    t.mul_(std)
+    return t.to(torch.bfloat16)
+
+
+def make_layer_weights(cfg: ModelConfig, gen: torch.Generator, device="cpu", w_std=0.02,
+                       router_std=None) -> dict:
+    d, E, F = cfg.d_model, cfg.n_exp, cfg.d_ff
+    if router_std is None:
+        router_std = w_std
+    return {
+        "attn_norm": torch.ones(d, dtype=torch.float32, device=device),
+        "w_qkv": _normal_bf16((cfg.qkv_rows, d), w_std, gen, device),
+        "w_o": _normal_bf16((d, cfg.n_q * cfg.d_head), w_std, gen, device),
+        "ffn_norm": torch.ones(d, dtype=torch.float32, device=device),
+        "w_router": _normal_bf16((E, d), router_std, gen, device),
+        "w_gate_up": _normal_bf16((E, 2 * F, d), w_std, gen, device),
+        "w_down": _normal_bf16((E, d, F), w_std, gen, device),
+    }
+
+
+def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, router_std=None,
+                       head_scale=1.0) -> dict:
+    """Random-init weights N(0, w_std^2) rounded to bf16 (round-to-nearest-even), norm gains 1.
+    ``head_scale`` multiplies the LM head's std (a larger head gives confident rows that commit)."""
+    gen = _gen(seed, device)
+    w = {
+        "emb": _normal_bf16((cfg.vocab, cfg.d_model), w_std, gen, device),
+        "layers": [make_layer_weights(cfg, gen, device, w_std, router_std) for _ in range(cfg.n_layers)],
+        "final_norm": torch.ones(cfg.d_model, dtype=torch.float32, device=device),
+    }
+    w["head"] = _normal_bf16((cfg.vocab, cfg.d_model), w_std * head_scale, gen, device)
+    return w
+
+
+def make_ids(n: int, vocab: int, seed: int, device="cpu") -> torch.Tensor:
+    return torch.randint(0, vocab, (n,), generator=_gen(seed, device), device=device, dtype=torch.int32)
+
+
+def make_hidden(n: int, d: int, seed: int, device="cpu") -> torch.Tensor:
+    """N(0,1) hidden states, rounded to bf16-representable values, held as fp32."""
+    t = torch.randn((n, d), generator=_gen(seed, device), device=device, dtype=torch.float32)
+    return t.to(torch.bfloat16).to(torch.float32)
+
+
+def make_prefix_kv(n_layers: int, P: int, n_kv: int, dh: int, seed: int, device="cpu"):
+    """Synthetic committed-prefix cache: K (taken as already rotated) and V ~ N(0,1) in bf16,
+    one [P, n_kv, dh] pair per layer."""
+    gen = _gen(seed, device)
+    ks, vs = [], []
+    for _ in range(n_layers):
+        ks.append(torch.randn((P, n_kv, dh), generator=gen, device=device).to(torch.bfloat16))
+        vs.append(torch.randn((P, n_kv, dh), generator=gen, device=device).to(torch.bfloat16))
+    return ks, vs
+
+
+def make_sampler_logits(rows: int, vocab: int, seed: int, std=3.0, spike=12.0, spike_every=10,
+                        device="cpu"):
+    """fp32 logits ~ N(0, std^2); rows r with r % spike_every == 0 get +spike at one uniformly
+    chosen column.  Returns (logits, spike_columns)."""
+    gen = _gen(seed, device)
+    logits = torch.randn((rows, vocab), generator=gen, device=device, dtype=torch.float32).mul_(std)
+    spike_rows = torch.arange(0, rows, spike_every, device=device)
+    cols = torch.randint(0, vocab, (spike_rows.numel(),), generator=gen, device=device)
+    if spike:
+        logits[spike_rows, cols] += spike
+    return logits, cols
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """The raw bf16 bit patterns of a CPU bf16 tensor, as a uint16 numpy array (no copy)."""
+    assert t.dtype == torch.bfloat16
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
