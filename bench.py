@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark: canvas denoise steps/s of the block-diffusion decoder on B200.
+
+Workload (default, "full_b1"): the full synthetic 30-layer stack at batch 1 -- d_model 2816, 16 Q /
+8 KV heads of dim 128, 128 experts top-8 with expert FFN 704, vocabulary 262144, bf16 random-init
+weights generated on the device; a 2048-token prompt prefilled into the KV cache; canvases of 256
+positions denoised with 12 fixed steps per block.  One benchmark step = one dg_canvas_step: the
+whole hot path (embedding, 30 x [RMSNorm, QKV+RoPE, canvas attention, O+residual, RMSNorm, router,
+top-k, bucketing, expert GEMMs, combine], final norm, vocabulary logits, sampler, stop test).
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent batch-1 replica (its own
+seed): there is no exchange in the path, so no collective is used except the barrier and the
+max-over-ranks reduction of the timing.  --impl reference times the CPU oracle on a bounded sample
+of the same workload (rank 0 only).
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CANVAS = 256
+PROMPT = 2048
+BLOCKS = 4
+FIXED_STEPS = 12
+METRIC = "canvas denoise steps/s"
+WORKLOAD = ("full_b1: 30-layer Gemma-4-26B-A4B-shaped MoE (d 2816, 16/8 heads x 128, 128 experts top-8, "
+            "FFN 704, vocab 262144), bf16 random-init (residual-scaled; every step routes the canvas to all "
+            "128 experts of every layer), batch 1, 2048-token prompt, 256-token canvas, 12 fixed steps per block")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=24)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# the CUDA path
+# ------------------------------------------------------------------------------------------------
+def setup_full(rank, device):
+    import torch
+
+    import synthetic
+    from block_discrete_diffusion_b200 import dg
+
+    cfg = synthetic.FULL
+    w = synthetic.make_model_weights(cfg, seed=2 + 1000 * rank, device=device, **synthetic.full_stack_init(cfg))
+    model = dg.dg_model_create(cfg, w)
+    max_ctx = PROMPT + BLOCKS * CANVAS
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=2 + 1000 * rank, device=device)
+    dg.dg_prefill(seqs, prompt, [PROMPT])
+    prm = dg.sampler_params(cfg.vocab, seed=2 + 1000 * rank, fixed_steps=FIXED_STEPS)
+    st = {
+        "ids": torch.empty(CANVAS, dtype=torch.int32, device=device),
+        "commit": torch.empty(CANVAS, dtype=torch.uint8, device=device),
+        "H": torch.empty(CANVAS, device=device),
+        "stop": torch.empty(1, dtype=torch.int32, device=device),
+    }
+    torch.cuda.synchronize()
+    return cfg, w, model, seqs, prm, st
+
+
+def run_steps(dg, seqs, prm, st, k, state):
+    """k canvas steps; a new canvas every FIXED_STEPS steps (the block's step budget)."""
+    for _ in range(k):
+        if state["step"] % FIXED_STEPS == 0:
+            dg.dg_canvas_init(seqs, prm, st["ids"], st["commit"])
+        dg.dg_canvas_step(seqs, prm, st["ids"], st["commit"], st["H"], st["stop"])
+        state["step"] += 1
+
+
+def expert_up_bytes(cfg):
+    """Algorithmic bytes of one grouped gate|up launch at batch 1: every expert's [2F x d] bf16
+    weights (all 128 experts are routed to with probability 1 - 128*(120/128)^256 > 0.99999), the
+    gathered activations read once, the SwiGLU rows written once."""
+    A = CANVAS * cfg.top_k
+    return cfg.n_exp * 2 * cfg.d_ff * cfg.d_model * 2 + A * cfg.d_model * 2 + A * cfg.d_ff * 2
+
+
+def main_dg(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    from block_discrete_diffusion_b200 import build, dg
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    cfg, w, model, seqs, prm, st = setup_full(rank, device)
+    state = {"step": 0}
+    run_steps(dg, seqs, prm, st, args.warmup, state)
+    torch.cuda.synchronize()
+    code = dg.dg_device_error(seqs)
+    assert code == 0, f"device error {code} during warm-up"
+
+    # ---- timed region: K canvas steps, inputs (48 GB of weights) far larger than L2 ----
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dg.dg_stats_reset(seqs, timing=False)
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        run_steps(dg, seqs, prm, st, args.steps, state)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    t = e0.elapsed_time(e1) / 1e3
+    launches = sum(v[0] for v in dg.dg_stats_read(seqs).values())
+    if world > 1:
+        tt = torch.tensor([t], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    value = world * args.steps / t
+    ms_per_step = 1e3 * t / args.steps
+
+    # ---- per-kernel device time (CUDA events around each launch, same stream), separate pass ----
+    dg.dg_stats_reset(seqs, timing=True)
+    run_steps(dg, seqs, prm, st, args.steps, state)
+    stats = dg.dg_stats_read(seqs)
+    dg.dg_stats_reset(seqs, timing=False)
+    kernel_ms = {k: round(v[1] / args.steps, 4) for k, v in stats.items() if v[0]}
+    dominant = max(stats, key=lambda k: stats[k][1])
+    hbm, tflops, peak_kind = peaks()
+    up_launch_s = stats["expert_up"][1] / 1e3 / max(stats["expert_up"][0], 1)
+    up_bytes = expert_up_bytes(cfg)
+    roofline = {"kernel": "expert_up (grouped gate|up GEMM + SwiGLU)", "bound": "hbm",
+                "achieved": round(up_bytes / up_launch_s / 1e9, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(up_bytes / up_launch_s / 1e9 / hbm, 4), "traffic": None,
+                "algorithmic_bytes_per_launch": up_bytes, "launch_ms": round(up_launch_s * 1e3, 4),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind,
+                "dominant_by_time": dominant}
+
+    # ---- end to end through the C ABI with host buffers: H2D ids/commit, step, D2H results ----
+    h_ids = torch.empty(CANVAS, dtype=torch.int32).pin_memory()
+    h_commit = torch.empty(CANVAS, dtype=torch.uint8).pin_memory()
+    h_H = torch.empty(CANVAS).pin_memory()
+    h_stop = torch.empty(1, dtype=torch.int32).pin_memory()
+    dg.dg_canvas_init(seqs, prm, st["ids"], st["commit"])
+    h_ids.copy_(st["ids"])
+    h_commit.copy_(st["commit"])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    k_e2e = min(args.steps, FIXED_STEPS)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    dg.dg_canvas_init(seqs, prm, st["ids"], st["commit"])
+    for _ in range(k_e2e):
+        st["ids"].copy_(h_ids, non_blocking=True)
+        st["commit"].copy_(h_commit, non_blocking=True)
+        dg.dg_canvas_step(seqs, prm, st["ids"], st["commit"], st["H"], st["stop"])
+        h_ids.copy_(st["ids"], non_blocking=True)
+        h_commit.copy_(st["commit"], non_blocking=True)
+        h_H.copy_(st["H"], non_blocking=True)
+        h_stop.copy_(st["stop"], non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    te = f0.elapsed_time(f1) / 1e3
+    if world > 1:
+        tt = torch.tensor([te], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        te = float(tt.item())
+    state["step"] = 0
+    e2e = {"value": round(world * k_e2e / te, 3), "unit": "steps/s", "h2d_bytes_per_step": CANVAS * 4 + CANVAS,
+           "d2h_bytes_per_step": CANVAS * 4 + CANVAS + CANVAS * 4 + 4}
+
+    # ---- committed tokens/s: dg_decode of 4 blocks x 12 fixed steps with a commit pass per block ----
+    seqs2 = dg.dg_seqs_create(model, 1, PROMPT + BLOCKS * CANVAS)
+    import synthetic
+    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=2 + 1000 * rank, device=device)
+    dg.dg_prefill(seqs2, prompt, [PROMPT])
+    out = torch.empty(1, BLOCKS * CANVAS, dtype=torch.int32, device=device)
+    torch.cuda.synchronize()
+    g0 = time.perf_counter()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    n_out, steps_per_block = dg.dg_decode(seqs2, prm, BLOCKS, out)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    td = d0.elapsed_time(d1) / 1e3
+    committed_tok_s = sum(n_out) / td
+    code = dg.dg_device_error(seqs)
+    assert code == 0, f"device error {code}"
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(cfg, w, sample_rows_layer=256, head_rows=32, samp_rows=256)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 3), "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CANVAS,
+                           "parallelism": f"replicas x{world} (independent sequences, no exchange)",
+                           "l2": "inputs larger than L2: 48.2 GB of weights streamed per step"},
+                "committed_tok_s": round(committed_tok_s, 1),
+                "decode": {"blocks": BLOCKS, "steps_per_block": steps_per_block, "tokens": sum(n_out),
+                           "seconds": round(td, 4), "includes": "canvas init, 12 steps and a commit pass per block"},
+                "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "kernel_ms_per_step": kernel_ms,
+                "clocks": clk.summary(), "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------------------
+def _host_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v else os.cpu_count()
+
+
+def _cpu_layer_model(cfg, layer_w):
+    import dataclasses
+
+    import oracle
+    c1 = dataclasses.replace(cfg, n_layers=1)
+    cpu_layer = {k: v.detach().cpu() for k, v in layer_w.items()}
+    return oracle.Model(c1, {"layers": [cpu_layer]})
+
+
+def cpu_baseline_sample(cfg, w, sample_rows_layer, head_rows, samp_rows, rounds=1):
+    """Time the oracle on a bounded sample of one canvas step and extrapolate to the whole step:
+    one decoder layer on `sample_rows_layer` canvas rows (x 30 layers x 256/rows), the vocabulary
+    head on `head_rows` rows and the sampler on `samp_rows` rows (each x 256/rows).  Inputs are
+    synthetic (hidden states N(0,1), a 2048-token prefix N(0,1), logits N(0, 3^2))."""
+    import numpy as np
+
+    import oracle
+    import synthetic
+    M1 = _cpu_layer_model(cfg, w["layers"][0])
+    head = w["head"].detach().cpu()
+    final_norm = w["final_norm"].detach().cpu()
+    Mh = oracle.Model(cfg, {"layers": [], "head": head, "final_norm": final_norm}, layers=[])
+    ks, vs = synthetic.make_prefix_kv(1, PROMPT, cfg.n_kv, cfg.d_head, seed=5)
+    kc, vc = ks[0].double().numpy(), vs[0].double().numpy()
+    x = synthetic.make_hidden(CANVAS, cfg.d_model, seed=6).double().numpy()
+    logits, _ = synthetic.make_sampler_logits(samp_rows, cfg.vocab, seed=7)
+    lg = logits.numpy()
+    t_layer = t_head = t_samp = 0.0
+    for _ in range(rounds):
+        n = sample_rows_layer
+        t0 = time.perf_counter()
+        oracle.layer_forward(M1, 0, x[:n], np.arange(PROMPT, PROMPT + n), PROMPT, kc, vc)
+        t_layer += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.head(Mh, x[:head_rows])
+        t_head += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.sample_rows(lg, None, np.arange(samp_rows), 0.8, 7, 0)
+        t_samp += time.perf_counter() - t0
+    t_layer, t_head, t_samp = t_layer / rounds, t_head / rounds, t_samp / rounds
+    step_s = (cfg.n_layers * t_layer * CANVAS / sample_rows_layer + t_head * CANVAS / head_rows
+              + t_samp * CANVAS / samp_rows)
+    return {"value": round(1.0 / step_s, 6), "unit": "steps/s", "cores": _host_threads(), "kind": "oracle",
+            "sample": (f"1 of {cfg.n_layers} layers on {sample_rows_layer} of 256 canvas rows "
+                       f"({t_layer:.2f} s), LM head on {head_rows} rows ({t_head:.2f} s), sampler on {samp_rows} rows "
+                       f"({t_samp:.2f} s); extrapolated to one full step ({step_s:.1f} s)"),
+            "seconds_measured": round(t_layer + t_head + t_samp, 2)}
+
+
+def main_reference(args):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return
+    import torch
+
+    import synthetic
+    cfg = synthetic.FULL
+    # weights of one layer and of the head, generated on the host (the oracle never sees the GPU)
+    gen = torch.Generator().manual_seed(2)
+    init = synthetic.full_stack_init(cfg)
+    layer = synthetic.make_layer_weights(cfg, gen, "cpu", router_std=init["router_std"], out_std=init["out_std"])
+    head = (torch.randn((cfg.vocab, cfg.d_model), generator=gen) * 0.02).to(torch.bfloat16)
+    w = {"layers": [layer], "head": head, "final_norm": torch.ones(cfg.d_model)}
+    for _ in range(args.warmup):
+        cpu_baseline_sample(cfg, w, 64, 4, 32)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline_sample(cfg, w, 64, 4, 32))
+    wall = time.perf_counter() - t0
+    step_s = statistics.mean(1.0 / v["value"] for v in vals)
+    value = 1.0 / step_s
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "steps/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": CANVAS, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "steps/s", "cores": _host_threads(), "kind": "oracle",
+                             "sample": "per step: " + vals[-1]["sample"]},
+            "e2e": {"value": round(value, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_seconds": round(wall, 1)}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_dg(a)

@@ -1,0 +1,818 @@
+// dg_api.cu -- the C ABI (include/dg.h): handles, workspace layout, TMA descriptors and the launch
+// sequences of prefill, canvas step, block commit and the decode loop.  Host code only; every step
+// of the method runs in the kernels of gemm.cu, attention.cu, misc.cu and sampler.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "dg.h"
+#include "dg_kernels.h"
+
+#define DG_API extern "C" __attribute__((visibility("default")))
+
+using namespace dg;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+dg_status fail(dg_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define CK(call)                                                                                     \
+  do {                                                                                               \
+    cudaError_t e_ = (call);                                                                         \
+    if (e_ != cudaSuccess) return fail(DG_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                                       __FILE__, __LINE__);                                          \
+  } while (0)
+
+constexpr int kCanvas = 256;
+constexpr int kSplitTargetCtas = 296;   // two waves of CTAs over the 148 SMs
+constexpr int kMaxSplits = 16;
+
+// ---------------------------------------------------------------------------------------------
+// TMA descriptor creation through the driver entry point (no libcuda link dependency)
+// ---------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 [rows][cols] (cols contiguous), box box_rows x 64, 128-byte swizzle.
+dg_status map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (cols * 2) % 16)
+    return fail(DG_ERR_INVALID_ARG, "TMA operand not 16-byte aligned (ptr %p, row bytes %llu)", ptr,
+                (unsigned long long)(cols * 2));
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (2d, %llux%llu box %u) failed: %d",
+                                     (unsigned long long)rows, (unsigned long long)cols, box_rows, (int)r);
+  return DG_OK;
+}
+
+// 3-D bf16 [d2][d1][d0] (d0 contiguous), box {64, box1, 1}, 128-byte swizzle.
+dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (3d) failed: %d", (int)r);
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// workspace layout
+// ---------------------------------------------------------------------------------------------
+struct WsLayout {
+  int R, A, split_cap, chunks;
+  size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
+      y, logits, samp, rope, cids, ccommit, cH, cstop, total;
+};
+
+int attn_split_cap(const dg_model_config& c, int n_seq) {
+  const int G = c.n_q / c.n_kv;
+  const int qtiles = (G * kCanvas + 127) / 128;
+  const int base = qtiles * n_seq * c.n_kv;
+  return std::max(1, std::min(kMaxSplits, (kSplitTargetCtas + base - 1) / base));
+}
+
+WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
+  WsLayout L{};
+  L.R = n_seq * kCanvas;
+  L.A = L.R * c.top_k;
+  L.split_cap = attn_split_cap(c, n_seq);
+  L.chunks = sampler_chunks(c.vocab);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 1023) & ~size_t(1023);
+    return o;
+  };
+  const size_t d = c.d_model, R = L.R, A = L.A, dh = c.d_head, nq = c.n_q;
+  L.err = take(64);
+  L.seqP = take(sizeof(int) * n_seq);
+  L.x = take(4 * R * d);
+  L.xn = take(2 * R * d);
+  L.q = take(2 * (size_t)n_seq * nq * kCanvas * dh);
+  L.opart = take(4 * (size_t)L.split_cap * n_seq * nq * kCanvas * dh);
+  L.ml = take(8 * (size_t)L.split_cap * n_seq * nq * kCanvas);
+  L.attn = take(2 * R * nq * dh);
+  L.rlog = take(4 * R * c.n_exp);
+  L.sel = take(4 * A);
+  L.gate = take(4 * A);
+  L.counts = take(4 * (size_t)c.n_exp);
+  L.offsets = take(4 * (size_t)(c.n_exp + 1));
+  L.perm_gate = take(4 * A);
+  L.perm_tok = take(4 * A);
+  L.slot = take(4 * A);
+  L.xp = take(2 * A * d);
+  L.hb = take(2 * A * (size_t)c.d_ff);
+  L.y = take(4 * A * d);
+  L.logits = take(4 * R * (size_t)c.vocab);
+  L.samp = take(4 * 8 * R * (size_t)L.chunks);
+  L.rope = take(8 * (size_t)max_ctx * (dh / 2));
+  L.cids = take(4 * R);
+  L.ccommit = take(R);
+  L.cH = take(4 * R);
+  L.cstop = take(4 * (size_t)n_seq);
+  L.total = off + 1024;   // slack for base alignment
+  return L;
+}
+
+bool shape_ok(const dg_model_config* c, const char** why) {
+  if (!c) return (*why = "null config", false);
+  if (c->d_head != 64 && c->d_head != 128) return (*why = "d_head must be 64 or 128", false);
+  if (c->d_model <= 0 || c->d_model % 128) return (*why = "d_model must be a positive multiple of 128", false);
+  if (c->d_ff <= 0 || c->d_ff % 64) return (*why = "d_ff must be a positive multiple of 64", false);
+  if (c->n_q <= 0 || c->n_kv <= 0 || c->n_q % c->n_kv) return (*why = "n_q must be a multiple of n_kv", false);
+  if ((c->n_q * c->d_head) % 128 || (c->n_kv * c->d_head) % 128)
+    return (*why = "n_q*d_head and n_kv*d_head must be multiples of 128", false);
+  if (c->n_exp <= 0 || c->n_exp > 256) return (*why = "n_exp must be in [1, 256]", false);
+  if (c->top_k <= 0 || c->top_k > 32 || c->top_k > c->n_exp) return (*why = "top_k must be in [1, min(32, n_exp)]", false);
+  if (c->n_layers <= 0) return (*why = "n_layers must be positive", false);
+  if (c->vocab <= 0 || c->vocab % 1024) return (*why = "vocab must be a positive multiple of 1024", false);
+  return true;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// handles
+// ---------------------------------------------------------------------------------------------
+struct LayerMaps {
+  CUtensorMap wqkv, wo, wrouter, wgu, wdown;
+};
+
+struct dg_model {
+  dg_model_config cfg;
+  const __nv_bfloat16 *emb, *head;
+  const float* final_norm;
+  std::vector<dg_layer_weights> layers;
+  std::vector<LayerMaps> maps;
+  CUtensorMap head_map;
+};
+
+struct dg_seqs {
+  dg_model* m;
+  int n_seq, max_ctx;
+  cudaStream_t st;
+  __nv_bfloat16 *kc, *vt;
+  WsLayout L;
+  uint8_t* ws;
+  // typed workspace views
+  int *err, *seqP;
+  float *x, *opart, *ml, *rlog, *gate, *perm_gate, *y, *logits, *samp;
+  __nv_bfloat16 *xn, *q, *attn, *xp, *hb;
+  int32_t *sel, *counts, *offsets, *perm_tok, *slot, *cids, *cstop;
+  uint8_t* ccommit;
+  float* cH;
+  float2* rope;
+  CUtensorMap xn_map, attn_map, xp_map, hb_map, q_map, k_map, v_map;
+  std::vector<int> P;   // host mirror of the committed lengths
+  int step;
+  bool block_open;
+  int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
+  // statistics: launches per kernel class; optional event timing
+  long long launches[DG_K_COUNT];
+  double ms[DG_K_COUNT];
+  bool timing;
+  std::vector<cudaEvent_t> events;            // pairs (start, end)
+  std::vector<std::pair<int, int>> pending;   // (class, pair index) not yet folded into ms
+  int next_pair;
+  ~dg_seqs() {
+    for (cudaEvent_t e : events) cudaEventDestroy(e);
+  }
+};
+
+namespace {
+
+constexpr int kEventPairs = 4096;
+
+cudaError_t stats_fold(dg_seqs* s) {
+  if (s->pending.empty()) return cudaSuccess;
+  cudaError_t e = cudaStreamSynchronize(s->st);
+  if (e != cudaSuccess) return e;
+  for (auto& pr : s->pending) {
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, s->events[2 * pr.second], s->events[2 * pr.second + 1]);
+    if (e != cudaSuccess) return e;
+    s->ms[pr.first] += t;
+  }
+  s->pending.clear();
+  s->next_pair = 0;
+  return cudaSuccess;
+}
+
+int stats_begin(dg_seqs* s) {
+  if (!s->timing) return -1;
+  if (s->next_pair >= kEventPairs && stats_fold(s) != cudaSuccess) return -1;
+  const int i = s->next_pair++;
+  cudaEventRecord(s->events[2 * i], s->st);
+  return i;
+}
+
+void stats_end(dg_seqs* s, int cls, int n_kernels, int pair) {
+  s->launches[cls] += n_kernels;
+  if (pair >= 0) {
+    cudaEventRecord(s->events[2 * pair + 1], s->st);
+    s->pending.emplace_back(cls, pair);
+  }
+}
+
+}  // namespace
+
+// launch `call` (n_kernels kernels of class cls) on the handle's stream, counted and optionally timed
+#define LAUNCH(s, cls, n_kernels, call)     \
+  do {                                      \
+    const int pair_ = stats_begin(s);       \
+    CK(call);                               \
+    stats_end(s, cls, n_kernels, pair_);    \
+  } while (0)
+
+DG_API const char* dg_last_error(void) { return g_err; }
+
+DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w, dg_model** out) {
+  const char* why = "";
+  if (!out) return fail(DG_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  if (!shape_ok(cfg, &why)) return fail(DG_ERR_INVALID_ARG, "model config: %s", why);
+  if (!w || !w->layers || !aligned16(w->emb) || !aligned16(w->head) || !aligned16(w->final_norm))
+    return fail(DG_ERR_INVALID_ARG, "weights: null or unaligned emb/head/final_norm/layers");
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const dg_layer_weights& L = w->layers[l];
+    if (!aligned16(L.attn_norm) || !aligned16(L.w_qkv) || !aligned16(L.w_o) || !aligned16(L.ffn_norm) ||
+        !aligned16(L.w_router) || !aligned16(L.w_gate_up) || !aligned16(L.w_down))
+      return fail(DG_ERR_INVALID_ARG, "layer %d: null or unaligned weight pointer", l);
+  }
+  dg_model* m = new (std::nothrow) dg_model();
+  if (!m) return fail(DG_ERR_INVALID_ARG, "host allocation failed");
+  m->cfg = *cfg;
+  m->emb = static_cast<const __nv_bfloat16*>(w->emb);
+  m->head = static_cast<const __nv_bfloat16*>(w->head);
+  m->final_norm = static_cast<const float*>(w->final_norm);
+  m->layers.assign(w->layers, w->layers + cfg->n_layers);
+  m->maps.resize(cfg->n_layers);
+  const dg_model_config& c = *cfg;
+  const uint64_t d = c.d_model, qkv = (uint64_t)(c.n_q + 2 * c.n_kv) * c.d_head;
+  dg_status st = DG_OK;
+  for (int l = 0; l < c.n_layers && st == DG_OK; ++l) {
+    const dg_layer_weights& L = m->layers[l];
+    LayerMaps& M = m->maps[l];
+    if ((st = map_2d(&M.wqkv, L.w_qkv, qkv, d, 128)) != DG_OK) break;
+    if ((st = map_2d(&M.wo, L.w_o, d, (uint64_t)c.n_q * c.d_head, 64)) != DG_OK) break;
+    if ((st = map_2d(&M.wrouter, L.w_router, c.n_exp, d, 128)) != DG_OK) break;
+    if ((st = map_2d(&M.wgu, L.w_gate_up, (uint64_t)c.n_exp * 2 * c.d_ff, d, 64)) != DG_OK) break;
+    if ((st = map_2d(&M.wdown, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
+  }
+  if (st == DG_OK) st = map_2d(&m->head_map, w->head, c.vocab, d, 256);
+  if (st != DG_OK) {
+    delete m;
+    return st;
+  }
+  *out = m;
+  return DG_OK;
+}
+
+DG_API void dg_model_destroy(dg_model* m) { delete m; }
+
+DG_API size_t dg_kv_bytes(const dg_model_config* cfg, int n_seq, int max_ctx) {
+  const char* why;
+  if (!shape_ok(cfg, &why) || n_seq <= 0 || max_ctx <= 0 || max_ctx % kCanvas) return 0;
+  return 2ull * cfg->n_layers * n_seq * cfg->n_kv * (size_t)max_ctx * cfg->d_head * 2ull;
+}
+
+DG_API size_t dg_workspace_bytes(const dg_model_config* cfg, int n_seq, int max_ctx) {
+  const char* why;
+  if (!shape_ok(cfg, &why) || n_seq <= 0 || max_ctx <= 0 || max_ctx % kCanvas) return 0;
+  return ws_layout(*cfg, n_seq, max_ctx).total;
+}
+
+DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, size_t kv_bytes, void* ws,
+                                size_t ws_bytes, void* stream, dg_seqs** out) {
+  if (!out) return fail(DG_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  if (!m) return fail(DG_ERR_INVALID_ARG, "model is null");
+  if (n_seq <= 0 || max_ctx <= 0 || max_ctx % kCanvas)
+    return fail(DG_ERR_INVALID_ARG, "n_seq must be > 0 and max_ctx a positive multiple of 256");
+  const dg_model_config& c = m->cfg;
+  const size_t need_kv = dg_kv_bytes(&c, n_seq, max_ctx);
+  const size_t need_ws = dg_workspace_bytes(&c, n_seq, max_ctx);
+  if (!kv || !ws) return fail(DG_ERR_INVALID_ARG, "kv and ws must be device buffers");
+  if (kv_bytes < need_kv) return fail(DG_ERR_CAPACITY, "kv buffer %zu bytes < %zu needed", kv_bytes, need_kv);
+  if (ws_bytes < need_ws) return fail(DG_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need_ws);
+  if (!aligned16(kv)) return fail(DG_ERR_INVALID_ARG, "kv buffer must be 16-byte aligned");
+
+  dg_seqs* s = new (std::nothrow) dg_seqs();
+  if (!s) return fail(DG_ERR_INVALID_ARG, "host allocation failed");
+  s->m = m;
+  s->n_seq = n_seq;
+  s->max_ctx = max_ctx;
+  s->st = static_cast<cudaStream_t>(stream);
+  s->L = ws_layout(c, n_seq, max_ctx);
+  s->ws = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 1023) & ~uintptr_t(1023));
+  const size_t half_kv = need_kv / 2;
+  s->kc = static_cast<__nv_bfloat16*>(kv);
+  s->vt = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(kv) + half_kv);
+  uint8_t* b = s->ws;
+  const WsLayout& L = s->L;
+  s->err = reinterpret_cast<int*>(b + L.err);
+  s->seqP = reinterpret_cast<int*>(b + L.seqP);
+  s->x = reinterpret_cast<float*>(b + L.x);
+  s->xn = reinterpret_cast<__nv_bfloat16*>(b + L.xn);
+  s->q = reinterpret_cast<__nv_bfloat16*>(b + L.q);
+  s->opart = reinterpret_cast<float*>(b + L.opart);
+  s->ml = reinterpret_cast<float*>(b + L.ml);
+  s->attn = reinterpret_cast<__nv_bfloat16*>(b + L.attn);
+  s->rlog = reinterpret_cast<float*>(b + L.rlog);
+  s->sel = reinterpret_cast<int32_t*>(b + L.sel);
+  s->gate = reinterpret_cast<float*>(b + L.gate);
+  s->counts = reinterpret_cast<int32_t*>(b + L.counts);
+  s->offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  s->perm_gate = reinterpret_cast<float*>(b + L.perm_gate);
+  s->perm_tok = reinterpret_cast<int32_t*>(b + L.perm_tok);
+  s->slot = reinterpret_cast<int32_t*>(b + L.slot);
+  s->xp = reinterpret_cast<__nv_bfloat16*>(b + L.xp);
+  s->hb = reinterpret_cast<__nv_bfloat16*>(b + L.hb);
+  s->y = reinterpret_cast<float*>(b + L.y);
+  s->logits = reinterpret_cast<float*>(b + L.logits);
+  s->samp = reinterpret_cast<float*>(b + L.samp);
+  s->rope = reinterpret_cast<float2*>(b + L.rope);
+  s->cids = reinterpret_cast<int32_t*>(b + L.cids);
+  s->ccommit = b + L.ccommit;
+  s->cH = reinterpret_cast<float*>(b + L.cH);
+  s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
+  s->P.assign(n_seq, 0);
+  s->step = 0;
+  s->block_open = false;
+  for (int k = 0; k < DG_K_COUNT; ++k) {
+    s->launches[k] = 0;
+    s->ms[k] = 0.0;
+  }
+  s->timing = false;
+  s->next_pair = 0;
+  s->max_splits = kMaxSplits;
+  if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
+
+  const uint64_t d = c.d_model, R = L.R, A = L.A;
+  const uint64_t zdim = (uint64_t)c.n_layers * n_seq * c.n_kv;
+  dg_status st = DG_OK;
+  if (st == DG_OK) st = map_2d(&s->xn_map, s->xn, R, d, 128);
+  if (st == DG_OK) st = map_2d(&s->attn_map, s->attn, R, (uint64_t)c.n_q * c.d_head, 128);
+  if (st == DG_OK) st = map_2d(&s->xp_map, s->xp, A, d, 32);
+  if (st == DG_OK) st = map_2d(&s->hb_map, s->hb, A, c.d_ff, 32);
+  if (st == DG_OK) st = map_2d(&s->q_map, s->q, (uint64_t)n_seq * c.n_q * kCanvas, c.d_head, 128);
+  if (st == DG_OK) st = map_3d(&s->k_map, s->kc, c.d_head, max_ctx, zdim, 128);
+  if (st == DG_OK) st = map_3d(&s->v_map, s->vt, max_ctx, c.d_head, zdim, c.d_head);
+  if (st != DG_OK) {
+    delete s;
+    return st;
+  }
+  // clear the cache and the buffers whose stale contents a masked lane may read, build the table
+  cudaError_t e = cudaMemsetAsync(kv, 0, need_kv, s->st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(s->ws, 0, L.rope, s->st);
+  if (e == cudaSuccess) e = rope_table(s->rope, max_ctx, c.d_head, c.rope_theta, s->st);
+  if (e != cudaSuccess) {
+    delete s;
+    return fail(DG_ERR_CUDA, "seqs init: %s", cudaGetErrorString(e));
+  }
+  *out = s;
+  return DG_OK;
+}
+
+DG_API void dg_seqs_destroy(dg_seqs* s) { delete s; }
+
+DG_API dg_status dg_seqs_get_state(const dg_seqs* s, int* h_P, int* h_step) {
+  if (!s) return fail(DG_ERR_INVALID_ARG, "seqs is null");
+  if (h_P)
+    for (int i = 0; i < s->n_seq; ++i) h_P[i] = s->P[i];
+  if (h_step) *h_step = s->step;
+  return DG_OK;
+}
+
+DG_API float dg_temperature(const dg_sampler_params* p, int step) {
+  if (!p) return 0.f;
+  const double frac = p->max_steps > 1 ? (double)step / (double)(p->max_steps - 1) : 0.0;
+  return (float)((double)p->t_start - ((double)p->t_start - (double)p->t_end) * frac);
+}
+
+// ---------------------------------------------------------------------------------------------
+// layer stack
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+size_t layer_kv_elems(const dg_seqs* s) {
+  return (size_t)s->n_seq * s->m->cfg.n_kv * s->max_ctx * s->m->cfg.d_head;
+}
+
+// One decoder layer on `rows` rows of x.  n_local sequences starting at cache sequence seq_base,
+// Tq rows per sequence (rows == n_local * 256 for a canvas, rows == Tq for a prefill chunk).
+dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_base, int Tq, bool causal,
+                    float* x_mid, float* rlog_out) {
+  const dg_model_config& c = s->m->cfg;
+  const dg_layer_weights& W = s->m->layers[l];
+  const LayerMaps& M = s->m->maps[l];
+  cudaStream_t st = s->st;
+  const int d = c.d_model, dh = c.d_head;
+
+  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.attn_norm), rows, d, c.rms_eps, s->xn, st));
+  EpiParams ep{};
+  ep.q = s->q;
+  ep.kc = s->kc + (size_t)l * layer_kv_elems(s);
+  ep.vt = s->vt + (size_t)l * layer_kv_elems(s);
+  ep.rope = s->rope;
+  ep.seq_P = s->seqP;
+  ep.n_q = c.n_q;
+  ep.n_kv = c.n_kv;
+  ep.dh = dh;
+  ep.rows_per_seq = kCanvas;
+  ep.max_ctx = s->max_ctx;
+  ep.seq_base = seq_base;
+  LAUNCH(s, DG_K_QKV, 1, gemm_dense(128, EPI_QKV, s->xn_map, M.wqkv, rows, (c.n_q + 2 * c.n_kv) * dh, d, ep, s->err, st));
+
+  // attention over cache [0, P) + the Tq new rows
+  int Pmax = 0;
+  for (int i = 0; i < n_local; ++i) Pmax = std::max(Pmax, s->P[seq_base + i]);
+  const int ntiles = (Pmax + Tq + 127) / 128;
+  AttnParams ap{};
+  ap.n_q = c.n_q;
+  ap.n_kv = c.n_kv;
+  ap.dh = dh;
+  ap.rows_per_seq = kCanvas;
+  ap.Tq = Tq;
+  ap.max_ctx = s->max_ctx;
+  ap.causal = causal ? 1 : 0;
+  ap.seq_base = seq_base;
+  ap.cache_seq_stride = s->n_seq * c.n_kv;
+  ap.layer = l;
+  const int sp = std::min(std::min(s->L.split_cap, s->max_splits), ntiles);
+  ap.tiles_per_split = (ntiles + sp - 1) / sp;
+  ap.n_splits = (ntiles + ap.tiles_per_split - 1) / ap.tiles_per_split;
+  ap.seq_P = s->seqP;
+  ap.opart = s->opart;
+  ap.ml = s->ml;
+  LAUNCH(s, DG_K_ATTN, 1, attention_partial(s->q_map, s->k_map, s->v_map, ap, n_local, s->err, st));
+  LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
+
+  EpiParams eo{};
+  eo.x = x;
+  eo.ldo = d;
+  LAUNCH(s, DG_K_OPROJ, 1, gemm_dense(64, EPI_RESID, s->attn_map, M.wo, rows, d, c.n_q * dh, eo, s->err, st));
+  if (x_mid) CK(cudaMemcpyAsync(x_mid, x, sizeof(float) * (size_t)rows * d, cudaMemcpyDeviceToDevice, st));
+
+  // mixture of experts
+  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.ffn_norm), rows, d, c.rms_eps, s->xn, st));
+  EpiParams er{};
+  er.out = s->rlog;
+  er.ldo = c.n_exp;
+  LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
+  if (rlog_out)
+    CK(cudaMemcpyAsync(rlog_out, s->rlog, sizeof(float) * (size_t)rows * c.n_exp, cudaMemcpyDeviceToDevice, st));
+  CK(cudaMemsetAsync(s->counts, 0, sizeof(int32_t) * c.n_exp, st));
+  LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));
+  LAUNCH(s, DG_K_BUCKET, 1,
+         bucket_gather(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->xn, d, s->offsets, s->perm_gate,
+                       s->perm_tok, s->slot, s->xp, st));
+  ExpertParams xp{};
+  xp.counts = s->counts;
+  xp.offsets = s->offsets;
+  xp.perm_gate = s->perm_gate;
+  xp.h_out = s->hb;
+  xp.y_out = s->y;
+  xp.d = d;
+  xp.F = c.d_ff;
+  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->err, st));
+  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->err, st));
+  LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, rows, c.top_k, d, x, st));
+  return DG_OK;
+}
+
+// Embedding + all layers on the n_seq canvases (rows n_seq*256).  hidden: nullable debug dump.
+dg_status run_canvas_stack(dg_seqs* s, const int32_t* d_ids, float* hidden) {
+  const dg_model_config& c = s->m->cfg;
+  const int R = s->L.R;
+  const size_t plane = (size_t)R * c.d_model;
+  LAUNCH(s, DG_K_EMBED, 1, embed_rows(s->m->emb, d_ids, R, c.d_model, c.vocab, s->x, s->err, s->st));
+  if (hidden) CK(cudaMemcpyAsync(hidden, s->x, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s->st));
+  for (int l = 0; l < c.n_layers; ++l) {
+    dg_status r = run_layer(s, l, s->x, R, s->n_seq, 0, kCanvas, false, nullptr, nullptr);
+    if (r != DG_OK) return r;
+    if (hidden)
+      CK(cudaMemcpyAsync(hidden + (size_t)(l + 1) * plane, s->x, sizeof(float) * plane, cudaMemcpyDeviceToDevice,
+                         s->st));
+  }
+  return DG_OK;
+}
+
+dg_status check_params(const dg_seqs* s, const dg_sampler_params* p) {
+  if (!p) return fail(DG_ERR_INVALID_ARG, "sampler params are null");
+  if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "canvas_len must be 256");
+  if (p->max_steps <= 0 || p->fixed_steps < 0) return fail(DG_ERR_INVALID_ARG, "bad step budget");
+  if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
+  (void)s;
+  return DG_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// public calls
+// ---------------------------------------------------------------------------------------------
+DG_API dg_status dg_load_prefix(dg_seqs* s, int seq, int P, const void* const* h_k, const void* const* h_v) {
+  if (!s || !h_k || !h_v) return fail(DG_ERR_INVALID_ARG, "null argument");
+  if (seq < 0 || seq >= s->n_seq) return fail(DG_ERR_INVALID_ARG, "seq %d out of range", seq);
+  if (P < 0 || P + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "prefix %d + canvas exceeds max_ctx", P);
+  const dg_model_config& c = s->m->cfg;
+  const size_t per_seq = (size_t)c.n_kv * s->max_ctx * c.d_head;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (!h_k[l] || !h_v[l]) return fail(DG_ERR_INVALID_ARG, "layer %d prefix pointer is null", l);
+    __nv_bfloat16* kc = s->kc + (size_t)l * layer_kv_elems(s) + (size_t)seq * per_seq;
+    __nv_bfloat16* vt = s->vt + (size_t)l * layer_kv_elems(s) + (size_t)seq * per_seq;
+    CK(load_prefix(static_cast<const __nv_bfloat16*>(h_k[l]), static_cast<const __nv_bfloat16*>(h_v[l]), P, c.n_kv,
+                   c.d_head, s->max_ctx, kc, vt, s->st));
+  }
+  CK(add_to_P(s->seqP, seq, 1, P - s->P[seq], s->st));
+  s->P[seq] = P;
+  return DG_OK;
+}
+
+DG_API dg_status dg_prefill(dg_seqs* s, const int32_t* d_ids, const int32_t* h_lens) {
+  if (!s || !d_ids || !h_lens) return fail(DG_ERR_INVALID_ARG, "null argument");
+  const dg_model_config& c = s->m->cfg;
+  for (int i = 0; i < s->n_seq; ++i)
+    if (h_lens[i] < 0 || s->P[i] + h_lens[i] + kCanvas > s->max_ctx)
+      return fail(DG_ERR_CAPACITY, "sequence %d: prompt of %d tokens does not fit (P=%d, max_ctx=%d)", i, h_lens[i],
+                  s->P[i], s->max_ctx);
+  size_t off = 0;
+  for (int i = 0; i < s->n_seq; ++i) {
+    for (int c0 = 0; c0 < h_lens[i]; c0 += kCanvas) {
+      const int n = std::min(kCanvas, h_lens[i] - c0);
+      LAUNCH(s, DG_K_EMBED, 1, embed_rows(s->m->emb, d_ids + off + c0, n, c.d_model, c.vocab, s->x, s->err, s->st));
+      for (int l = 0; l < c.n_layers; ++l) {
+        dg_status r = run_layer(s, l, s->x, n, 1, i, n, true, nullptr, nullptr);
+        if (r != DG_OK) return r;
+      }
+      LAUNCH(s, DG_K_MISC, 1, add_to_P(s->seqP, i, 1, n, s->st));
+      s->P[i] += n;
+    }
+    off += h_lens[i];
+  }
+  s->block_open = false;
+  return DG_OK;
+}
+
+DG_API dg_status dg_canvas_init(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit) {
+  if (!s || !d_ids || !d_commit) return fail(DG_ERR_INVALID_ARG, "null argument");
+  dg_status r = check_params(s, p);
+  if (r != DG_OK) return r;
+  for (int i = 0; i < s->n_seq; ++i)
+    if (s->P[i] + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "sequence %d: no room for a canvas", i);
+  LAUNCH(s, DG_K_MISC, 1, canvas_init_ids(s->seqP, s->n_seq, kCanvas, p->seed, s->m->cfg.vocab, d_ids, d_commit, s->st));
+  s->step = 0;
+  s->block_open = true;
+  return DG_OK;
+}
+
+DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit,
+                                float* d_entropy, int32_t* d_stop, float* d_hidden, float* d_logits_out) {
+  if (!s || !d_ids || !d_commit || !d_entropy || !d_stop) return fail(DG_ERR_INVALID_ARG, "null argument");
+  dg_status r = check_params(s, p);
+  if (r != DG_OK) return r;
+  if (!s->block_open) return fail(DG_ERR_STATE, "no open canvas: call dg_canvas_init first");
+  const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
+  if (s->step >= budget) return fail(DG_ERR_STATE, "step budget of %d already used", budget);
+  const dg_model_config& c = s->m->cfg;
+  r = run_canvas_stack(s, d_ids, d_hidden);
+  if (r != DG_OK) return r;
+  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(s->x, s->m->final_norm, s->L.R, c.d_model, c.rms_eps, s->xn, s->st));
+  EpiParams eh{};
+  eh.out = s->logits;
+  eh.ldo = c.vocab;
+  LAUNCH(s, DG_K_HEAD, 1, gemm_dense(256, EPI_F32, s->xn_map, s->m->head_map, s->L.R, c.vocab, c.d_model, eh, s->err, s->st));
+  if (d_logits_out)
+    CK(cudaMemcpyAsync(d_logits_out, s->logits, sizeof(float) * (size_t)s->L.R * c.vocab, cudaMemcpyDeviceToDevice,
+                       s->st));
+  SamplerArgs a{};
+  a.logits = s->logits;
+  a.n_seq = s->n_seq;
+  a.canvas = kCanvas;
+  a.vocab = c.vocab;
+  a.n_chunks = s->L.chunks;
+  a.seq_P = s->seqP;
+  a.ids_in = d_ids;
+  a.commit_in = d_commit;
+  a.ids_out = d_ids;
+  a.commit_out = d_commit;
+  a.entropy = d_entropy;
+  a.stop = d_stop;
+  a.partial = s->samp;
+  a.inv_temp = 1.0f / dg_temperature(p, s->step);
+  a.seed = p->seed;
+  a.step = s->step;
+  a.max_steps = p->max_steps;
+  a.fixed_steps = p->fixed_steps;
+  a.entropy_bound = p->entropy_bound;
+  a.stop_mean_entropy = p->stop_mean_entropy;
+  a.rerand_entropy = p->rerand_entropy;
+  LAUNCH(s, DG_K_SAMPLER, 2, sampler_run(a, s->st));
+  s->step += 1;
+  return DG_OK;
+}
+
+DG_API dg_status dg_block_commit(dg_seqs* s, const int32_t* d_ids) {
+  if (!s || !d_ids) return fail(DG_ERR_INVALID_ARG, "null argument");
+  for (int i = 0; i < s->n_seq; ++i)
+    if (s->P[i] + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "sequence %d: cache full", i);
+  dg_status r = run_canvas_stack(s, d_ids, nullptr);
+  if (r != DG_OK) return r;
+  LAUNCH(s, DG_K_MISC, 1, add_to_P(s->seqP, 0, s->n_seq, kCanvas, s->st));
+  for (int i = 0; i < s->n_seq; ++i) s->P[i] += kCanvas;
+  s->block_open = false;
+  return DG_OK;
+}
+
+DG_API dg_status dg_layer_forward(dg_seqs* s, int layer, int n_rows, int causal, float* d_x, float* d_x_mid,
+                                  float* d_router_logits) {
+  if (!s || !d_x) return fail(DG_ERR_INVALID_ARG, "null argument");
+  if (layer < 0 || layer >= s->m->cfg.n_layers) return fail(DG_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (n_rows <= 0 || n_rows > kCanvas) return fail(DG_ERR_INVALID_ARG, "n_rows must be in [1, 256]");
+  const bool canvas = (n_rows == kCanvas && !causal);
+  if (!canvas && s->n_seq != 1) return fail(DG_ERR_UNSUPPORTED, "partial or causal rows need n_seq == 1");
+  for (int i = 0; i < s->n_seq; ++i)
+    if (s->P[i] + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "sequence %d: no room for a canvas", i);
+  if (canvas) return run_layer(s, layer, d_x, s->L.R, s->n_seq, 0, kCanvas, false, d_x_mid, d_router_logits);
+  return run_layer(s, layer, d_x, n_rows, 1, 0, n_rows, causal != 0, d_x_mid, d_router_logits);
+}
+
+DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_blocks, int32_t* d_out, int32_t* h_n_out,
+                           int32_t* h_steps) {
+  if (!s || !d_out || !h_n_out || max_blocks <= 0) return fail(DG_ERR_INVALID_ARG, "bad argument");
+  dg_status r = check_params(s, p);
+  if (r != DG_OK) return r;
+  const int n = s->n_seq;
+  const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
+  const size_t out_stride = (size_t)max_blocks * kCanvas;
+  for (int i = 0; i < n; ++i)
+    if (s->P[i] + max_blocks * kCanvas > s->max_ctx)
+      return fail(DG_ERR_CAPACITY, "sequence %d: %d blocks do not fit (P=%d, max_ctx=%d)", i, max_blocks, s->P[i],
+                  s->max_ctx);
+  std::vector<int32_t> h_stop(n), h_ids((size_t)n * kCanvas);
+  std::vector<int> done(n, 0);
+  for (int i = 0; i < n; ++i) h_n_out[i] = 0;
+  for (int b = 0; b < max_blocks; ++b) {
+    r = dg_canvas_init(s, p, s->cids, s->ccommit);
+    if (r != DG_OK) return r;
+    int steps = 0;
+    for (;;) {
+      r = dg_canvas_step(s, p, s->cids, s->ccommit, s->cH, s->cstop, nullptr, nullptr);
+      if (r != DG_OK) return r;
+      ++steps;
+      CK(cudaMemcpyAsync(h_stop.data(), s->cstop, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s->st));
+      CK(cudaStreamSynchronize(s->st));
+      bool all = true;
+      for (int i = 0; i < n; ++i) all = all && h_stop[i] != 0;
+      if (all || steps >= budget) break;
+    }
+    if (h_steps) h_steps[b] = steps;
+    r = dg_block_commit(s, s->cids);
+    if (r != DG_OK) return r;
+    CK(cudaMemcpy2DAsync(d_out + (size_t)b * kCanvas, out_stride * sizeof(int32_t), s->cids,
+                         kCanvas * sizeof(int32_t), kCanvas * sizeof(int32_t), n, cudaMemcpyDeviceToDevice, s->st));
+    bool all_done = true;
+    if (p->eos_id >= 0) {
+      CK(cudaMemcpyAsync(h_ids.data(), s->cids, sizeof(int32_t) * h_ids.size(), cudaMemcpyDeviceToHost, s->st));
+      CK(cudaStreamSynchronize(s->st));
+    }
+    for (int i = 0; i < n; ++i) {
+      if (done[i]) continue;
+      int take = kCanvas;
+      if (p->eos_id >= 0)
+        for (int j = 0; j < kCanvas; ++j)
+          if (h_ids[(size_t)i * kCanvas + j] == p->eos_id) {
+            take = j + 1;
+            done[i] = 1;
+            break;
+          }
+      h_n_out[i] += take;
+      all_done = all_done && done[i];
+    }
+    if (all_done) break;
+  }
+  CK(cudaStreamSynchronize(s->st));
+  return DG_OK;
+}
+
+DG_API size_t dg_sample_workspace_bytes(int n_rows, int vocab) {
+  if (n_rows <= 0 || vocab <= 0) return 0;
+  return (size_t)4 * 8 * n_rows * sampler_chunks(vocab) + 1024;
+}
+
+DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg_sampler_params* p, int step,
+                           const int32_t* d_seq_P, int32_t* d_ids, uint8_t* d_commit, float* d_entropy, int32_t* d_stop,
+                           void* ws, size_t ws_bytes, void* stream) {
+  if (!d_logits || !p || !d_ids || !d_commit || !d_entropy || !d_stop || !ws)
+    return fail(DG_ERR_INVALID_ARG, "null argument");
+  if (n_seq <= 0 || vocab <= 0 || vocab % 1024) return fail(DG_ERR_INVALID_ARG, "bad n_seq / vocab");
+  if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "canvas_len must be 256");
+  if (step < 0 || p->max_steps <= 0) return fail(DG_ERR_INVALID_ARG, "bad step");
+  const int rows = n_seq * kCanvas;
+  if (ws_bytes < dg_sample_workspace_bytes(rows, vocab)) return fail(DG_ERR_CAPACITY, "sampler workspace too small");
+  SamplerArgs a{};
+  a.logits = d_logits;
+  a.n_seq = n_seq;
+  a.canvas = kCanvas;
+  a.vocab = vocab;
+  a.n_chunks = sampler_chunks(vocab);
+  a.seq_P = d_seq_P;
+  a.ids_in = d_ids;
+  a.commit_in = d_commit;
+  a.ids_out = d_ids;
+  a.commit_out = d_commit;
+  a.entropy = d_entropy;
+  a.stop = d_stop;
+  a.partial = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  a.inv_temp = 1.0f / dg_temperature(p, step);
+  a.seed = p->seed;
+  a.step = step;
+  a.max_steps = p->max_steps;
+  a.fixed_steps = p->fixed_steps;
+  a.entropy_bound = p->entropy_bound;
+  a.stop_mean_entropy = p->stop_mean_entropy;
+  a.rerand_entropy = p->rerand_entropy;
+  CK(sampler_run(a, static_cast<cudaStream_t>(stream)));
+  return DG_OK;
+}
+
+DG_API dg_status dg_device_error(dg_seqs* s, int* h_code) {
+  if (!s || !h_code) return fail(DG_ERR_INVALID_ARG, "null argument");
+  CK(cudaStreamSynchronize(s->st));
+  int code = 0;
+  CK(cudaMemcpy(&code, s->err, sizeof(int), cudaMemcpyDeviceToHost));
+  CK(cudaMemset(s->err, 0, sizeof(int)));
+  *h_code = code;
+  if (code) return fail(DG_ERR_DEVICE, "device-side error code %d", code);
+  return DG_OK;
+}
+
+DG_API dg_status dg_stats_reset(dg_seqs* s, int timing) {
+  if (!s) return fail(DG_ERR_INVALID_ARG, "seqs is null");
+  CK(stats_fold(s));
+  for (int k = 0; k < DG_K_COUNT; ++k) {
+    s->launches[k] = 0;
+    s->ms[k] = 0.0;
+  }
+  if (timing && s->events.empty()) {
+    s->events.resize(2 * kEventPairs);
+    for (auto& e : s->events) CK(cudaEventCreate(&e));
+  }
+  s->timing = timing != 0;
+  s->next_pair = 0;
+  return DG_OK;
+}
+
+DG_API dg_status dg_stats_read(dg_seqs* s, long long* h_launches, double* h_ms) {
+  if (!s || !h_launches) return fail(DG_ERR_INVALID_ARG, "null argument");
+  CK(stats_fold(s));
+  for (int k = 0; k < DG_K_COUNT; ++k) {
+    h_launches[k] = s->launches[k];
+    if (h_ms) h_ms[k] = s->ms[k];
+  }
+  return DG_OK;
+}

@@ -1,0 +1,97 @@
+// dg_kernels.h -- internal launch interface between the C ABI runtime (dg_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dg {
+
+enum { EPI_QKV = 0, EPI_RESID = 1, EPI_F32 = 2 };
+
+struct EpiParams {
+  float* out;            // EPI_F32: out[row * ldo + col]
+  float* x;              // EPI_RESID: x[row * ldo + col] += acc
+  int ldo;
+  __nv_bfloat16* q;      // EPI_QKV: query buffer [seq][n_q][rows_per_seq][dh]
+  __nv_bfloat16* kc;     // key cache of this layer [seq][n_kv][max_ctx][dh] (post-rotary)
+  __nv_bfloat16* vt;     // value cache of this layer, transposed [seq][n_kv][dh][max_ctx]
+  const float2* rope;    // (cos, sin) table [max_ctx][dh/2]
+  const int* seq_P;      // committed length of each sequence (device)
+  int n_q, n_kv, dh, rows_per_seq, max_ctx, seq_base;
+};
+
+struct ExpertParams {
+  const int* counts;     // [E] tokens routed to each expert
+  const int* offsets;    // [E+1] first bucketed row of each expert
+  const float* perm_gate;  // [A] gate weight of each bucketed row
+  __nv_bfloat16* h_out;  // MODE 1: SwiGLU rows [A][F]
+  float* y_out;          // MODE 2: gate-scaled expert outputs [A][d]
+  int d, F;
+};
+
+struct AttnParams {
+  int n_q, n_kv, dh;
+  int rows_per_seq;      // query-buffer rows per head (256)
+  int Tq;                // query rows present per head (256 for a canvas, n for a prefill chunk)
+  int max_ctx;
+  int causal;            // 0: canvas (all keys visible), 1: prefill (key <= own position)
+  int seq_base;          // cache sequence index of local sequence 0
+  int cache_seq_stride;  // layer offset inside the 3-D cache maps, in (seq, head) units
+  int layer;
+  int n_splits, tiles_per_split;
+  const int* seq_P;
+  float* opart;          // [split][seq][n_q][rows_per_seq][dh] un-normalised partial outputs
+  float* ml;             // [split][seq][n_q][rows_per_seq][2] (running max in log2 units, sum)
+};
+
+cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
+                       const EpiParams& ep, int* err, cudaStream_t st);
+cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
+                        int* err, cudaStream_t st);
+cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const AttnParams& p, int n_seq, int* err, cudaStream_t st);
+cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st);
+
+// elementwise / routing kernels (misc.cu)
+cudaError_t embed_rows(const __nv_bfloat16* emb, const int32_t* ids, int n_rows, int d, int vocab, float* x,
+                       int* err, cudaStream_t st);
+cudaError_t rmsnorm_rows(const float* x, const float* g, int n_rows, int d, float eps, __nv_bfloat16* out,
+                         cudaStream_t st);
+cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st);
+cudaError_t router_topk(const float* logits, int n_rows, int n_exp, int top_k, int32_t* sel, float* gate,
+                        int32_t* counts, cudaStream_t st);
+cudaError_t bucket_gather(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k,
+                          int n_exp, const __nv_bfloat16* xn, int d, int32_t* offsets, float* perm_gate,
+                          int32_t* perm_tok, int32_t* slot, __nv_bfloat16* xp, cudaStream_t st);
+cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x,
+                        cudaStream_t st);
+cudaError_t add_to_P(int* seq_P, int first, int count, int delta, cudaStream_t st);
+cudaError_t load_prefix(const __nv_bfloat16* k_in, const __nv_bfloat16* v_in, int P, int n_kv, int dh, int max_ctx,
+                        __nv_bfloat16* kc, __nv_bfloat16* vt, cudaStream_t st);
+cudaError_t canvas_init_ids(const int* seq_P, int n_seq, int canvas, uint64_t seed, int vocab, int32_t* ids,
+                            uint8_t* commit, cudaStream_t st);
+
+// sampler (sampler.cu)
+struct SamplerArgs {
+  const float* logits;   // [n_seq * canvas][vocab]
+  int n_seq, canvas, vocab, n_chunks;
+  const int* seq_P;      // absolute position of row 0 of each sequence (nullptr -> 0)
+  const int32_t* ids_in;
+  const uint8_t* commit_in;
+  int32_t* ids_out;
+  uint8_t* commit_out;
+  float* entropy;        // [n_seq * canvas]
+  int32_t* stop;         // [n_seq]
+  float* partial;        // [n_seq * canvas][n_chunks][8]
+  float inv_temp;
+  uint64_t seed;
+  int step, max_steps, fixed_steps;
+  float entropy_bound, stop_mean_entropy, rerand_entropy;
+};
+cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st);
+int sampler_chunks(int vocab);
+
+}  // namespace dg

@@ -1,0 +1,269 @@
+// sampler.cu -- the uniform-state canvas sampler (entropy-bound commit, self-correcting
+// re-randomisation, adaptive stop) over fp32 vocabulary logits.
+//
+// Constants and rules from the pages: canvas of 256, at most 48 steps, temperature linear 0.8 ->
+// 0.4, adaptive-stop threshold 0.005 ("Composition of DiffusionGemma", sampler settings, in the
+// technical-report summary); the entropy_bound sampler with bound 0.1 ("Serving with vLLM" in the
+// diffusion-gemma developer guide); random placeholder start and re-randomisation of positions
+// whose confidence dropped ("Uniform State Diffusion", same guide).  The precise rule (which
+// entropy, which threshold re-randomises, what ends a block) is the build's written reading:
+//   H = entropy (nats) of softmax(l / T);  y = argmax_v (l_v / T + Gumbel_v);
+//   commit iff H <= entropy_bound; else re-randomise iff H > rerand_entropy, else take y;
+//   stop iff all committed, or mean H over the canvas (committed = 0) <= stop_mean_entropy, or the
+//   step budget is reached (fixed_steps > 0: exactly fixed_steps steps); on stop the remaining
+//   positions take y and commit.
+//
+// sampler_partial_kernel: grid (vocab chunk, row).  One pass over the chunk with 16-byte loads;
+// each thread keeps (m, S, A) of the tempered softmax in the exp2 domain with one rescale per 16
+// elements, and the best perturbed score.  A group of four logits whose largest tempered value
+// cannot beat the running best even with the largest possible Gumbel draw skips the Philox call
+// and the two logarithms (exact pruning).
+// sampler_finalize_kernel: one CTA per sequence, one thread per canvas position.
+#include <math.h>
+
+#include "dg_device.cuh"
+#include "dg_kernels.h"
+#include "philox.cuh"
+
+namespace dg {
+
+constexpr int kSampThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct SoftStats {
+  float m;   // running max of z * log2(e)
+  float S;   // sum 2^(z2 - m)
+  float A;   // sum 2^(z2 - m) * (z2 - m)
+};
+
+__device__ __forceinline__ SoftStats stats_merge(SoftStats a, SoftStats b) {
+  if (a.m == -INFINITY) return b;
+  if (b.m == -INFINITY) return a;
+  const float M = fmaxf(a.m, b.m);
+  const float fa = fast_exp2(a.m - M), fb = fast_exp2(b.m - M);
+  SoftStats r;
+  r.m = M;
+  r.S = fa * a.S + fb * b.S;
+  r.A = fa * (a.A + a.S * (a.m - M)) + fb * (b.A + b.S * (b.m - M));
+  return r;
+}
+
+__device__ __forceinline__ void best_merge(float& bs, int& bi, float os, int oi) {
+  if (os > bs || (os == bs && oi < bi)) {
+    bs = os;
+    bi = oi;
+  }
+}
+
+__global__ void __launch_bounds__(kSampThreads)
+    sampler_partial_kernel(const float* __restrict__ logits, int canvas, int vocab, int n_chunks,
+                           const int* __restrict__ seq_P, const uint8_t* __restrict__ commit_in, float inv_temp,
+                           uint64_t seed, int step, float* __restrict__ partial) {
+  const int row = blockIdx.y, chunk = blockIdx.x;
+  if (commit_in[row]) return;
+  const int seq = row / canvas, j = row % canvas;
+  const uint32_t pos = (uint32_t)((seq_P ? seq_P[seq] : 0) + j);
+  const uint64_t sd = seed + (uint64_t)seq;
+  const uint32_t k0 = (uint32_t)sd, k1 = (uint32_t)(sd >> 32);
+  const int vchunk = vocab / n_chunks;
+  const int g0 = (chunk * vchunk) >> 2, g1 = ((chunk + 1) * vchunk) >> 2;   // float4 groups
+  const float4* lr = reinterpret_cast<const float4*>(logits + (size_t)row * vocab);
+  const float s2 = inv_temp * kLog2e;
+
+  SoftStats st = {-INFINITY, 0.f, 0.f};
+  float best = -INFINITY;
+  int bidx = 0x7fffffff;
+
+  for (int gb = g0 + threadIdx.x; gb < g1; gb += 4 * kSampThreads) {
+    float4 q[4];
+    bool have[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = gb + u * kSampThreads;
+      have[u] = g < g1;
+      q[u] = have[u] ? __ldcs(lr + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    // batch max in the exp2 domain, then one rescale of (S, A)
+    float bm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) bm = fmaxf(bm, fmaxf(fmaxf(q[u].x, q[u].y), fmaxf(q[u].z, q[u].w)));
+    bm *= s2;
+    if (bm > st.m) {
+      if (st.m != -INFINITY) {
+        const float f = fast_exp2(st.m - bm);
+        st.A = f * (st.A + st.S * (st.m - bm));
+        st.S *= f;
+      }
+      st.m = bm;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!have[u]) continue;
+      const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+      float zmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float t2 = zz[i] * s2 - st.m;
+        const float e = fast_exp2(t2);
+        st.S += e;
+        st.A += e * t2;
+        zmax = fmaxf(zmax, zz[i]);
+      }
+      // Gumbel-max over the 4 elements of this group, unless none can beat the running best
+      if (zmax * inv_temp + kGumbelMax >= best) {
+        const int g = gb + u * kSampThreads;
+        const uint4 w = philox4x32_10(make_uint4((uint32_t)g, pos, (uint32_t)step, RNG_TAG_GUMBEL), k0, k1);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float sc = zz[i] * inv_temp + gumbel_from_word(ww[i]);
+          if (sc > best) {
+            best = sc;
+            bidx = 4 * g + i;
+          }
+        }
+      }
+    }
+  }
+
+  // block reduction: warp shuffles, then the 8 warp results through shared memory
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    SoftStats other = {__shfl_xor_sync(0xffffffffu, st.m, o), __shfl_xor_sync(0xffffffffu, st.S, o),
+                       __shfl_xor_sync(0xffffffffu, st.A, o)};
+    st = stats_merge(st, other);
+    best_merge(best, bidx, __shfl_xor_sync(0xffffffffu, best, o), __shfl_xor_sync(0xffffffffu, bidx, o));
+  }
+  __shared__ float red[kSampThreads / 32][5];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[w][0] = st.m;
+    red[w][1] = st.S;
+    red[w][2] = st.A;
+    red[w][3] = best;
+    red[w][4] = __int_as_float(bidx);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    SoftStats t = {red[0][0], red[0][1], red[0][2]};
+    float bb = red[0][3];
+    int bi = __float_as_int(red[0][4]);
+    for (int i = 1; i < kSampThreads / 32; ++i) {
+      t = stats_merge(t, SoftStats{red[i][0], red[i][1], red[i][2]});
+      best_merge(bb, bi, red[i][3], __float_as_int(red[i][4]));
+    }
+    float* out = partial + ((size_t)row * n_chunks + chunk) * 8;
+    out[0] = t.m;
+    out[1] = t.S;
+    out[2] = t.A;
+    out[3] = bb;
+    out[4] = __int_as_float(bi);
+  }
+}
+
+__global__ void sampler_finalize_kernel(SamplerArgs a) {
+  __shared__ float red_h[32];
+  __shared__ int red_c[32];
+  const int seq = blockIdx.x;
+  float Hsum_part = 0.f;
+  int all_part = 1;
+  // positions are strided over the block so any canvas length works with 256 threads
+  const int n_iter = (a.canvas + blockDim.x - 1) / blockDim.x;
+  // first pass: per-position decision without the stop override; remember (id, y, commit) locally
+  int my_id[4], my_y[4];
+  uint8_t my_c[4];
+  float my_H[4];
+  for (int it = 0; it < n_iter && it < 4; ++it) {
+    const int jj = threadIdx.x + it * blockDim.x;
+    my_id[it] = 0; my_y[it] = 0; my_c[it] = 1; my_H[it] = 0.f;
+    if (jj >= a.canvas) continue;
+    const int row = seq * a.canvas + jj;
+    if (a.commit_in[row]) {
+      my_id[it] = a.ids_in[row];
+      my_y[it] = my_id[it];
+      my_c[it] = 1;
+      my_H[it] = 0.f;
+      continue;
+    }
+    SoftStats st = {-INFINITY, 0.f, 0.f};
+    float best = -INFINITY;
+    int bidx = 0x7fffffff;
+    for (int c = 0; c < a.n_chunks; ++c) {
+      const float* pr = a.partial + ((size_t)row * a.n_chunks + c) * 8;
+      st = stats_merge(st, SoftStats{pr[0], pr[1], pr[2]});
+      best_merge(best, bidx, pr[3], __float_as_int(pr[4]));
+    }
+    const float H = logf(st.S) - kLn2 * st.A / st.S;
+    const uint32_t pos = (uint32_t)((a.seq_P ? a.seq_P[seq] : 0) + jj);
+    const uint4 w = rng_block(a.seed + (uint64_t)seq, 0u, pos, (uint32_t)a.step, RNG_TAG_RERAND);
+    const int rr = token_from_word(w.x, (uint32_t)a.vocab);
+    my_H[it] = H;
+    my_y[it] = bidx;
+    if (H <= a.entropy_bound) {
+      my_id[it] = bidx;
+      my_c[it] = 1;
+    } else {
+      my_id[it] = H > a.rerand_entropy ? rr : bidx;
+      my_c[it] = 0;
+      all_part = 0;
+    }
+    Hsum_part += H;
+  }
+  // canvas-mean entropy and the all-committed test
+  float hs = warp_sum(Hsum_part);
+  int al = __all_sync(0xffffffffu, all_part);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red_h[w] = hs;
+    red_c[w] = al;
+  }
+  __syncthreads();
+  float Hsum = 0.f;
+  int all = 1;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+    Hsum += red_h[i];
+    all &= red_c[i];
+  }
+  const float mean = Hsum / (float)a.canvas;
+  int stop;
+  if (a.fixed_steps > 0)
+    stop = (a.step + 1 >= a.fixed_steps);
+  else
+    stop = all || (mean <= a.stop_mean_entropy) || (a.step + 1 >= a.max_steps);
+  for (int it = 0; it < n_iter && it < 4; ++it) {
+    const int jj = threadIdx.x + it * blockDim.x;
+    if (jj >= a.canvas) continue;
+    const int row = seq * a.canvas + jj;
+    int id = my_id[it];
+    uint8_t c = my_c[it];
+    if (stop && !c) {
+      id = my_y[it];
+      c = 1;
+    }
+    a.ids_out[row] = id;
+    a.commit_out[row] = c;
+    a.entropy[row] = my_H[it];
+  }
+  if (threadIdx.x == 0) a.stop[seq] = stop;
+}
+
+int sampler_chunks(int vocab) {
+  int c = vocab / 32768;
+  if (c < 1) c = 1;
+  while (c > 1 && (vocab % (c * 4) != 0)) --c;
+  return c;
+}
+
+cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st) {
+  if (a.canvas > 4 * 256 || a.vocab % (4 * a.n_chunks) != 0) return cudaErrorInvalidValue;
+  dim3 grid(a.n_chunks, a.n_seq * a.canvas);
+  sampler_partial_kernel<<<grid, kSampThreads, 0, st>>>(a.logits, a.canvas, a.vocab, a.n_chunks, a.seq_P, a.commit_in,
+                                                        a.inv_temp, a.seed, a.step, a.partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sampler_finalize_kernel<<<a.n_seq, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dg

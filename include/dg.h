@@ -1,0 +1,223 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) block-diffusion canvas decoder.
+ *
+ * The decoder is block-autoregressive, uniform-state text diffusion over a Gemma-4-26B-A4B-shaped
+ * mixture-of-experts model.  Sources, cited by page title and section:
+ *   [guide]  "diffusion-gemma developer guide" (aisparkup.com wiki)
+ *   [report] "DiffusionGemma: a diffusion LLM that refines 256-token blocks in parallel"
+ *            (42jerrykim.github.io, summary of the technical report)
+ * The report's flowchart ("Composition of DiffusionGemma") is the call sequence of this ABI:
+ *   prompt -> KV cache            dg_prefill
+ *   256-token canvas of noise     dg_canvas_init
+ *   one bidirectional refinement  dg_canvas_step   (repeated until the adaptive-stop test passes)
+ *   block -> KV cache             dg_block_commit
+ *   loop until EOS                dg_decode
+ *
+ * Conventions
+ *  - Ownership: the caller owns every device buffer (weights, KV cache, workspace, inputs,
+ *    outputs), typically allocated through PyTorch.  The library allocates no device memory; its
+ *    handles are small host structures.  Every pointer named d_* is device memory; h_* is host.
+ *  - Asynchrony: every call is enqueued on the stream given to dg_seqs_create and returns without
+ *    waiting, except dg_decode (one 4-byte-per-sequence read of the stop flags per step) and
+ *    dg_device_error (synchronises the stream).
+ *  - Errors: arguments and state are checked on the host before any launch; nothing traps on the
+ *    device.  A kernel that sees a bad index or whose pipeline wait runs out records a code that
+ *    dg_device_error returns (DG_ERR_DEVICE).  dg_last_error() gives a message for the last non-OK
+ *    status of the calling thread.
+ *  - Determinism: outputs depend only on (weights, inputs, params, seed).
+ *  - Layouts are row-major; bf16 is IEEE bfloat16, fp32 is IEEE binary32.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,  /* a null pointer, a bad size, a shape the kernels do not support */
+  DG_ERR_CAPACITY = 2,     /* the KV cache or the workspace is too small */
+  DG_ERR_STATE = 3,        /* call out of order (e.g. a step after the block stopped) */
+  DG_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  DG_ERR_UNSUPPORTED = 5,  /* valid request this build does not implement */
+  DG_ERR_DEVICE = 6        /* a kernel recorded a device-side error (wait timeout, bad index) */
+} dg_status;
+
+typedef struct dg_model dg_model; /* opaque: config + borrowed weight pointers + TMA descriptors */
+typedef struct dg_seqs dg_seqs;   /* opaque: n sequences sharing one KV cache and one workspace */
+
+/* Model shape.  Requirements of this build: d_head in {64, 128}; d_model % 128 == 0;
+ * d_ff % 64 == 0; n_q % n_kv == 0; n_exp <= 256; top_k <= 32; vocab % 1024 == 0. */
+typedef struct {
+  int d_model, n_q, n_kv, d_head, n_exp, top_k, d_ff, n_layers, vocab;
+  float rms_eps;    /* RMSNorm epsilon (1e-6) */
+  float rope_theta; /* rotary base (10000) */
+} dg_model_config;
+
+/* One decoder layer's weights, device pointers, layouts [out_features][in_features]:
+ *   attn_norm  fp32 [d]                   RMSNorm gain before attention
+ *   w_qkv      bf16 [(n_q+2 n_kv) dh][d]  Q rows, then K rows, then V rows
+ *   w_o        bf16 [d][n_q dh]
+ *   ffn_norm   fp32 [d]                   RMSNorm gain before the MoE
+ *   w_router   bf16 [n_exp][d]
+ *   w_gate_up  bf16 [n_exp][2 d_ff][d]    per expert: d_ff gate rows, then d_ff up rows
+ *   w_down     bf16 [n_exp][d][d_ff]
+ * Buffers must be 16-byte aligned and stay valid while the model exists. */
+typedef struct {
+  const void *attn_norm, *w_qkv, *w_o, *ffn_norm, *w_router, *w_gate_up, *w_down;
+} dg_layer_weights;
+
+typedef struct {
+  const void *emb;                /* bf16 [vocab][d]  embedding table */
+  const void *final_norm;         /* fp32 [d]         final RMSNorm gain */
+  const void *head;               /* bf16 [vocab][d]  vocabulary projection (untied) */
+  const dg_layer_weights *layers; /* host array of n_layers entries, copied by dg_model_create */
+} dg_weights;
+
+/* Sampler settings.  Defaults from the pages: canvas 256, at most 48 steps, temperature linear
+ * 0.8 -> 0.4, adaptive stop at canvas-mean entropy 0.005 ([report] "Composition", sampler
+ * settings); entropy bound 0.1 ([guide] "Serving with vLLM").  rerand_entropy (re-randomise a
+ * non-committing position whose entropy exceeds it) has no value on the pages; 0.5 ln(vocab) is
+ * this build's default. */
+typedef struct {
+  int canvas_len;          /* must be 256 */
+  int max_steps;           /* step budget of the temperature schedule (48) */
+  int fixed_steps;         /* > 0: exactly this many steps per block, adaptive stop off; 0: adaptive */
+  float t_start, t_end;    /* 0.8, 0.4 */
+  float entropy_bound;     /* 0.1 */
+  float stop_mean_entropy; /* 0.005 */
+  float rerand_entropy;    /* 0.5 ln(vocab) */
+  uint64_t seed;           /* sequence i uses seed + i */
+  int eos_id;              /* -1: no EOS */
+} dg_sampler_params;
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char *dg_last_error(void);
+
+/* Model handle.  Checks the shape, copies the config and the per-layer pointer table, builds the
+ * weight TMA descriptors.  Weights are borrowed, not copied. */
+dg_status dg_model_create(const dg_model_config *cfg, const dg_weights *w, dg_model **out);
+void dg_model_destroy(dg_model *m);
+
+/* Bytes the caller must provide for the KV cache (all layers, n_seq sequences of max_ctx
+ * positions; max_ctx % 256 == 0) and for the workspace.  0 on invalid arguments.
+ * KV cache layout (bf16): the key half first, then the value half, each
+ * L * n_seq * n_kv * max_ctx * d_head elements:
+ *   K[l][seq][h][pos][c]   keys after rotary embedding, head-major
+ *   Vt[l][seq][h][c][pos]  values, transposed (positions contiguous) */
+size_t dg_kv_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
+size_t dg_workspace_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
+
+/* Sequence set: n_seq independent sequences (1 = batch 1) with max_ctx positions each.  kv and ws
+ * are caller device buffers of at least dg_kv_bytes / dg_workspace_bytes; both belong to this
+ * handle until dg_seqs_destroy.  The cache is cleared and every sequence starts empty (P = 0).
+ * stream is a cudaStream_t (NULL = legacy default stream). */
+dg_status dg_seqs_create(dg_model *m, int n_seq, int max_ctx, void *kv, size_t kv_bytes, void *ws,
+                         size_t ws_bytes, void *stream, dg_seqs **out);
+void dg_seqs_destroy(dg_seqs *s);
+
+/* Committed length P of every sequence (h_P[n_seq]) and the canvas step index of the current block. */
+dg_status dg_seqs_get_state(const dg_seqs *s, int *h_P, int *h_step);
+
+/* Install a ready-made committed prefix for sequence `seq` (replacing its cache content): per
+ * layer l, d_k[l] and d_v[l] are bf16 [P][n_kv][d_head] (K already rotated).  Sets that sequence's
+ * P.  h_k / h_v are host arrays of n_layers device pointers. */
+dg_status dg_load_prefix(dg_seqs *s, int seq, int P, const void *const *h_k, const void *const *h_v);
+
+/* Prompt -> KV cache ([report] flowchart, first box; causal attention over the prompt).
+ * d_ids: the prompts packed back to back (int32), h_lens[n_seq] their lengths.  Each sequence's
+ * tokens are appended at its current P, in chunks of 256 positions. */
+dg_status dg_prefill(dg_seqs *s, const int32_t *d_ids, const int32_t *h_lens);
+
+/* New canvas for every sequence: uniform random placeholder ids (Philox stream tag 2 at the
+ * absolute positions P..P+255), commit mask cleared, step index reset.  d_ids int32
+ * [n_seq][256], d_commit uint8 [n_seq][256]. */
+dg_status dg_canvas_init(dg_seqs *s, const dg_sampler_params *p, int32_t *d_ids, uint8_t *d_commit);
+
+/* One denoising step over all canvases: the full layer stack on the n_seq*256 canvas rows
+ * (bidirectional inside the canvas, full view of the committed prefix), vocabulary logits, and the
+ * sampler.  In/out: d_ids, d_commit.  Out: d_entropy fp32 [n_seq][256] (0 for positions committed
+ * before this step), d_stop int32 [n_seq].  d_hidden (nullable): fp32 [n_layers+1][n_seq*256][d],
+ * the residual stream before the first layer and after each layer.  d_logits_out (nullable): fp32
+ * [n_seq*256][vocab] copy of the logits.  The committed prefix [0, P) of the cache is not modified;
+ * the block's own cache rows [P, P+256) are used as scratch.  DG_ERR_STATE after the block has
+ * stopped (call dg_block_commit and dg_canvas_init first). */
+dg_status dg_canvas_step(dg_seqs *s, const dg_sampler_params *p, int32_t *d_ids, uint8_t *d_commit,
+                         float *d_entropy, int32_t *d_stop, float *d_hidden, float *d_logits_out);
+
+/* Append the finished canvases to the KV cache ([guide] "Block Autoregressive Diffusion", step 2):
+ * one pass of the layer stack over the final ids with the canvas mask writes every layer's K/V to
+ * cache rows [P, P+256), then P += 256.  DG_ERR_CAPACITY if P + 256 > max_ctx. */
+dg_status dg_block_commit(dg_seqs *s, const int32_t *d_ids);
+
+/* The whole block loop ([report] flowchart): for each of up to max_blocks blocks: dg_canvas_init,
+ * dg_canvas_step until every sequence's stop flag is set (sequences that stopped keep their ids),
+ * dg_block_commit; a sequence ends after the block that contains eos_id (its output cut after the
+ * first EOS).  d_out int32 [n_seq][max_blocks*256] receives the committed tokens, h_n_out[n_seq]
+ * their counts.  h_steps (nullable) [max_blocks] receives the step count of each block. */
+dg_status dg_decode(dg_seqs *s, const dg_sampler_params *p, int max_blocks, int32_t *d_out, int32_t *h_n_out,
+                    int32_t *h_steps);
+
+/* One decoder layer on caller hidden states (the attention block and the MoE block of a canvas
+ * step, without embedding, head or sampler).  n_rows = 256 with causal = 0: every sequence's canvas
+ * (d_x fp32 [n_seq*256][d] in/out) at positions P..P+255, bidirectional; n_rows < 256 or causal = 1
+ * (n_seq must be 1): n_rows rows at positions P..P+n_rows-1 attending to the cache and, causally
+ * or not, to each other (the mask of one prefill chunk).  The rows' K/V are written to cache rows
+ * [P, P+n_rows) (scratch; P is not advanced).  d_x_mid (nullable) receives x after the attention
+ * residual, d_router_logits (nullable) fp32 [rows][n_exp]. */
+dg_status dg_layer_forward(dg_seqs *s, int layer, int n_rows, int causal, float *d_x, float *d_x_mid,
+                           float *d_router_logits);
+
+/* Sampler alone over caller logits (fp32 [n_seq*canvas_len][vocab]): the entropy / Gumbel-argmax /
+ * commit / re-randomise / stop rule of one step.  d_seq_P (nullable, int32 [n_seq]): absolute
+ * position of each sequence's first canvas row (0 if NULL).  d_ids, d_commit in/out as in
+ * dg_canvas_step.  ws: device scratch of dg_sample_workspace_bytes(n_seq*canvas_len, vocab). */
+size_t dg_sample_workspace_bytes(int n_rows, int vocab);
+dg_status dg_sample(const float *d_logits, int n_seq, int vocab, const dg_sampler_params *p, int step,
+                    const int32_t *d_seq_P, int32_t *d_ids, uint8_t *d_commit, float *d_entropy, int32_t *d_stop,
+                    void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise the handle's stream and return the first device-side error code recorded since the
+ * last call (0 = none) in *h_code; the record is cleared.  Returns DG_ERR_DEVICE if non-zero. */
+dg_status dg_device_error(dg_seqs *s, int *h_code);
+
+/* Kernel classes counted by the statistics below (one class may launch more than one kernel). */
+typedef enum {
+  DG_K_EMBED = 0,     /* embedding gather */
+  DG_K_RMSNORM,       /* RMSNorm -> bf16 GEMM operand */
+  DG_K_QKV,           /* fused Q|K|V projection + rotary (tcgen05) */
+  DG_K_ATTN,          /* canvas attention partials (tcgen05) */
+  DG_K_ATTN_MERGE,    /* split-KV merge */
+  DG_K_OPROJ,         /* output projection + residual (tcgen05) */
+  DG_K_ROUTER,        /* router logits (tcgen05) */
+  DG_K_TOPK,          /* top-k selection, gates, expert counts */
+  DG_K_BUCKET,        /* expert bucketing + activation gather */
+  DG_K_EXPERT_UP,     /* grouped gate|up GEMM + SwiGLU (tcgen05) */
+  DG_K_EXPERT_DOWN,   /* grouped down GEMM x gate (tcgen05) */
+  DG_K_COMBINE,       /* top-k combine + residual */
+  DG_K_HEAD,          /* vocabulary logits (tcgen05) */
+  DG_K_SAMPLER,       /* sampler partial + finalize */
+  DG_K_MISC,          /* canvas init, cache bookkeeping */
+  DG_K_COUNT
+} dg_kernel_class;
+
+/* Reset the per-class counters of this handle.  timing != 0 also brackets every launch with CUDA
+ * events on the handle's stream (adds a small overhead per launch). */
+dg_status dg_stats_reset(dg_seqs *s, int timing);
+
+/* Synchronise the stream and read, per class, the kernels launched (h_launches[DG_K_COUNT]) and,
+ * when timing is on, the summed device milliseconds (h_ms[DG_K_COUNT], nullable). */
+dg_status dg_stats_read(dg_seqs *s, long long *h_launches, double *h_ms);
+
+/* Temperature of step s: fp32(t_start - (t_start - t_end) * s / (max_steps - 1)). */
+float dg_temperature(const dg_sampler_params *p, int step);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H */

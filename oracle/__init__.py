@@ -50,7 +50,7 @@ def lib():
         L.orc_router_topk.argtypes = [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
         L.orc_moe.argtypes = [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_layer_forward.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p,
-                                        c_void_p, c_int, c_void_p, c_void_p, c_void_p]
+                                        c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_layer_forward.restype = c_int
         L.orc_forward.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
                                   c_int, c_int, c_void_p, c_void_p, c_void_p]
@@ -238,9 +238,10 @@ class Model:
                       self._mat(L["w_down"], c.n_exp * c.d_model, c.d_ff))
 
 
-def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=None, causal=False):
+def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=None, causal=False, want_mid=False):
     """One decoder layer on rows x [n, d] (fp64, updated copy returned) at positions pos, keys =
-    cache[0:P] + the rows.  Returns (x_out, k_new, v_new, router_logits)."""
+    cache[0:P] + the rows.  Returns (x_out, k_new, v_new, router_logits) and, with want_mid, x after
+    the attention residual as a fifth item."""
     c = model.cfg
     x = _f64(x).copy()
     n = x.shape[0]
@@ -250,10 +251,12 @@ def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=N
     kn = np.empty((n, c.n_kv, c.d_head))
     vn = np.empty((n, c.n_kv, c.d_head))
     rl = np.empty((n, c.n_exp))
+    mid = np.empty_like(x) if want_mid else None
     rc = lib().orc_layer_forward(ctypes.byref(model.c_cfg), ctypes.byref(model.c_layers[layer]), n, _p(pos),
-                                 _p(x), P, _p(kc), _p(vc), int(causal), _p(kn), _p(vn), _p(rl))
+                                 _p(x), P, _p(kc), _p(vc), int(causal), _p(kn), _p(vn), _p(rl),
+                                 None if mid is None else _p(mid))
     assert rc == 0
-    return x, kn, vn, rl
+    return (x, kn, vn, rl, mid) if want_mid else (x, kn, vn, rl)
 
 
 def moe(model: Model, layer: int, h, sel, gate):

@@ -353,10 +353,11 @@ void orc_moe(const orc_config *c, const orc_layer_weights *w, int n, int k, cons
  * every key (canvas step: bidirectional inside the canvas, full view of the committed prefix;
  * guide "Dual attention of prefill and denoising", report "Composition", training recipe);
  * causal = 1: row i sees cache and rows j <= i (prompt prefill).
- * k_new/v_new receive the rows' post-RoPE K and V ([n][n_kv][dh]); router_logits is [n][E]. */
+ * k_new/v_new receive the rows' post-RoPE K and V ([n][n_kv][dh]); router_logits is [n][E];
+ * x_mid (nullable) receives x after the attention residual. */
 int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, const int32_t *pos,
                       double *x, int P, const double *k_cache, const double *v_cache, int causal,
-                      double *k_new, double *v_new, double *router_logits)
+                      double *k_new, double *v_new, double *router_logits, double *x_mid)
 {
     int d = c->d_model, nq = c->n_q, nkv = c->n_kv, dh = c->d_head, E = c->n_exp;
     int nqkv = (nq + 2 * nkv) * dh, nkeys = P + n;
@@ -395,6 +396,7 @@ int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, co
     orc_attention(n, nkeys, nq, nkv, dh, q, keys, vals, mask, att);
     mat_apply(&w->w_o, n, att, o, d);
     for (size_t i = 0; i < (size_t)n * d; ++i) x[i] += o[i];
+    if (x_mid) memcpy(x_mid, x, sizeof(double) * (size_t)n * d);
     if (k_new) memcpy(k_new, kn, sizeof(double) * (size_t)n * nkv * dh);
     if (v_new) memcpy(v_new, vn, sizeof(double) * (size_t)n * nkv * dh);
 
@@ -447,7 +449,7 @@ int orc_forward(const orc_config *c, const orc_model_weights *m, int n, const in
     if (hidden_dbg) memcpy(hidden_dbg, x, sizeof(double) * (size_t)n * d);
     for (int l = 0; l < c->n_layers; ++l) {
         double *rl = router_dbg ? router_dbg + (size_t)l * n * c->n_exp : NULL;
-        if (orc_layer_forward(c, &m->layers[l], n, pos, x, P, k_cache[l], v_cache[l], causal, kn, vn, rl))
+        if (orc_layer_forward(c, &m->layers[l], n, pos, x, P, k_cache[l], v_cache[l], causal, kn, vn, rl, NULL))
             return -1;
         if (write_cache) {
             memcpy(k_cache[l] + (size_t)P * kvw, kn, sizeof(double) * (size_t)n * kvw);

@@ -79,33 +79,49 @@ def _normal_bf16(shape, std, gen, device) -> torch.Tensor:
 
 
 def make_layer_weights(cfg: ModelConfig, gen: torch.Generator, device="cpu", w_std=0.02,
-                       router_std=None) -> dict:
+                       router_std=None, out_std=None) -> dict:
+    """One layer.  ``out_std`` is the std of the two residual-branch output matrices (w_o, w_down);
+    it defaults to w_std."""
     d, E, F = cfg.d_model, cfg.n_exp, cfg.d_ff
     if router_std is None:
         router_std = w_std
+    if out_std is None:
+        out_std = w_std
     return {
         "attn_norm": torch.ones(d, dtype=torch.float32, device=device),
         "w_qkv": _normal_bf16((cfg.qkv_rows, d), w_std, gen, device),
-        "w_o": _normal_bf16((d, cfg.n_q * cfg.d_head), w_std, gen, device),
+        "w_o": _normal_bf16((d, cfg.n_q * cfg.d_head), out_std, gen, device),
         "ffn_norm": torch.ones(d, dtype=torch.float32, device=device),
         "w_router": _normal_bf16((E, d), router_std, gen, device),
         "w_gate_up": _normal_bf16((E, 2 * F, d), w_std, gen, device),
-        "w_down": _normal_bf16((E, d, F), w_std, gen, device),
+        "w_down": _normal_bf16((E, d, F), out_std, gen, device),
     }
 
 
 def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, router_std=None,
-                       head_scale=1.0) -> dict:
+                       head_scale=1.0, emb_std=None, out_std=None) -> dict:
     """Random-init weights N(0, w_std^2) rounded to bf16 (round-to-nearest-even), norm gains 1.
-    ``head_scale`` multiplies the LM head's std (a larger head gives confident rows that commit)."""
+    ``head_scale`` multiplies the LM head's std (a larger head gives confident rows that commit);
+    ``emb_std`` / ``out_std`` override the embedding std and the residual-output std."""
     gen = _gen(seed, device)
     w = {
-        "emb": _normal_bf16((cfg.vocab, cfg.d_model), w_std, gen, device),
-        "layers": [make_layer_weights(cfg, gen, device, w_std, router_std) for _ in range(cfg.n_layers)],
+        "emb": _normal_bf16((cfg.vocab, cfg.d_model), w_std if emb_std is None else emb_std, gen, device),
+        "layers": [make_layer_weights(cfg, gen, device, w_std, router_std, out_std) for _ in range(cfg.n_layers)],
         "final_norm": torch.ones(cfg.d_model, dtype=torch.float32, device=device),
     }
     w["head"] = _normal_bf16((cfg.vocab, cfg.d_model), w_std * head_scale, gen, device)
     return w
+
+
+def full_stack_init(cfg: ModelConfig) -> dict:
+    """Keyword arguments of make_model_weights for the full-depth benchmark model: router logits of
+    unit-RMS inputs ~ N(0, 1) (router std d^-1/2), unit-variance embeddings, and residual-branch
+    output matrices scaled by 1/sqrt(2L) (the scaled init of deep pre-norm transformers).  With all
+    matrices at N(0, 0.02^2) the random residual stream of the 30-layer model collapses onto one
+    direction after the first layer (cross-token cosine ~0.97) and the router sends the whole canvas
+    to ~12 of the 128 experts; a trained MoE routes a 256-token canvas to nearly all of them, which
+    sets the weight traffic this workload has to model."""
+    return {"router_std": cfg.d_model ** -0.5, "emb_std": 1.0, "out_std": 0.02 / math.sqrt(2 * cfg.n_layers)}
 
 
 def make_ids(n: int, vocab: int, seed: int, device="cpu") -> torch.Tensor:

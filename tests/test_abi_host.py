@@ -1,0 +1,100 @@
+"""The C ABI library without a GPU: it builds, loads, exports every entry point include/dg.h
+declares, and its host-side logic (sizes, argument checks, temperature schedule) is right.
+No compute call is made here."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import oracle
+import synthetic
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dg():
+    from block_discrete_diffusion_b200 import build, dg as dgmod
+    build.build()
+    return dgmod
+
+
+def _declared_entry_points():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", txt))
+    return names
+
+
+def test_library_exports_every_declared_entry_point(dg):
+    declared = _declared_entry_points()
+    assert "dg_canvas_step" in declared and "dg_prefill" in declared and "dg_decode" in declared
+    L = ctypes.CDLL(dg.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+    assert declared == set(dg.ENTRY_POINTS), declared ^ set(dg.ENTRY_POINTS)
+
+
+def test_kv_and_workspace_sizes(dg):
+    for cfg in (synthetic.TINY, synthetic.FULL):
+        kv = dg.dg_kv_bytes(cfg, 2, 4096)
+        assert kv == 2 * cfg.n_layers * 2 * cfg.n_kv * 4096 * cfg.d_head * 2
+        ws = dg.dg_workspace_bytes(cfg, 2, 4096)
+        # the workspace holds at least the fp32 logits of both canvases and the expert buffers
+        R, A = 2 * 256, 2 * 256 * cfg.top_k
+        assert ws >= 4 * R * cfg.vocab + 4 * A * cfg.d_model + 2 * A * cfg.d_model
+        assert dg.dg_kv_bytes(cfg, 1, 1000) == 0           # max_ctx must be a multiple of 256
+        assert dg.dg_workspace_bytes(cfg, 0, 4096) == 0
+    assert dg.dg_sample_workspace_bytes(256, 262144) >= 4 * 8 * 256 * 8
+
+
+@pytest.mark.parametrize("field,value", [("d_head", 96), ("d_model", 200), ("n_q", 5), ("top_k", 0),
+                                         ("vocab", 1000), ("n_exp", 300), ("d_ff", 100)])
+def test_model_create_rejects_unsupported_shapes_on_the_host(dg, field, value):
+    import dataclasses
+    cfg = dataclasses.replace(synthetic.TINY, **{field: value})
+    c = dg.make_config(cfg)
+    w = dg.dg_weights()
+    h = ctypes.c_void_p()
+    st = dg.lib().dg_model_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h))
+    assert st == dg.DG_ERR_INVALID_ARG
+    assert dg.lib().dg_last_error().decode()
+
+
+def test_null_weights_rejected(dg):
+    c = dg.make_config(synthetic.TINY)
+    w = dg.dg_weights()
+    h = ctypes.c_void_p()
+    assert dg.lib().dg_model_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib().dg_model_create(ctypes.byref(c), None, ctypes.byref(h)) == dg.DG_ERR_INVALID_ARG
+
+
+def test_temperature_schedule_matches_oracle(dg):
+    prm = dg.sampler_params(4096)
+    for s in range(48):
+        assert dg.dg_temperature(prm, s) == oracle.temperature(s)
+    assert math.isclose(dg.dg_temperature(prm, 0), 0.8, rel_tol=1e-7)
+
+
+def test_sampler_params_defaults(dg):
+    p = dg.sampler_params(262144, seed=7)
+    assert (p.canvas_len, p.max_steps, p.fixed_steps) == (256, 48, 0)
+    assert math.isclose(p.t_start, 0.8, rel_tol=1e-7) and math.isclose(p.t_end, 0.4, rel_tol=1e-7)
+    assert math.isclose(p.entropy_bound, 0.1, rel_tol=1e-7)
+    assert math.isclose(p.stop_mean_entropy, 0.005, rel_tol=1e-6)
+    assert math.isclose(p.rerand_entropy, 0.5 * math.log(262144), rel_tol=1e-6)
+    assert ctypes.sizeof(dg.dg_sampler_params) == 48
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "block_discrete_diffusion_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt and "dg_oracle" not in txt, f

@@ -1,0 +1,333 @@
+"""CUDA path (libdg.so through the C ABI) vs the oracle, element by element, on seeded inputs.
+
+Marked gpu: they need an sm_100a device.  Shapes: the tiny model (several tiles plus ragged tails),
+the full-width single layer, and the full-size sampler workload; full-size cases compare sampled
+rows the oracle computes one by one plus properties that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from dg_testutil import (ENTROPY_TOL, HIDDEN_TOL, judge_step, kv_views, rel_err, router_tie_tokens, to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg(cuda_ok):
+    from block_discrete_diffusion_b200 import build, dg as dgmod
+    build.build()
+    return dgmod
+
+
+def _oracle_sample(logits_cpu, commit, ids, pos, prm, step, vocab):
+    T = oracle.temperature(step, prm.max_steps, prm.t_start, prm.t_end)
+    smp = oracle.sample_rows(logits_cpu, commit, pos, T, prm.seed, step)
+    rule = oracle.step_rule(commit, ids, smp["H"], smp["y"], smp["rr"], step, prm.entropy_bound, prm.rerand_entropy,
+                            prm.stop_mean_entropy, prm.max_steps, prm.fixed_steps)
+    out = dict(smp)
+    out.update(rule)
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# sampler alone
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("vocab,spike,step,rows_checked", [
+    (4096, 12.0, 0, None),
+    (4096, 40.0, 47, None),
+    (262144, 12.0, 12, None),          # the full-size sampler workload, every row
+    (262144, 40.0, 0, 48),             # spike +40 rows commit; sampled rows
+    (262144, 12.0, 47, 48),
+])
+def test_sampler_matches_oracle(dg, vocab, spike, step, rows_checked):
+    n_seq, canvas = 1, 256
+    logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, spike=spike)
+    prm_o = oracle.SamplerParams(vocab, seed=7)
+    prm = dg.sampler_params(vocab, seed=7)
+    rng = np.random.default_rng(step)
+    commit0 = (rng.random(canvas) < 0.2).astype(np.uint8)      # some positions already committed
+    ids0 = rng.integers(0, vocab, canvas).astype(np.int32)
+    d_logits = logits.cuda()
+    ids = torch.from_numpy(ids0).cuda()
+    commit = torch.from_numpy(commit0).cuda()
+    H = torch.empty(canvas, device="cuda")
+    stop = torch.empty(n_seq, dtype=torch.int32, device="cuda")
+    ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device="cuda")
+    dg.dg_sample(d_logits, n_seq, vocab, prm, step, None, ids, commit, H, stop, ws)
+    torch.cuda.synchronize()
+    g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(), "stop": int(stop.item())}
+    lg = logits.numpy()
+    rows = np.arange(canvas) if rows_checked is None else np.unique(
+        np.concatenate([np.arange(0, canvas, 10)[: rows_checked // 2], rng.choice(canvas, rows_checked // 2)]))
+    if rows_checked is None:
+        o = _oracle_sample(lg, commit0, ids0, np.arange(canvas), prm_o, step, vocab)
+        fails, judged = judge_step(g, o, prm_o, commit0)
+        assert not fails, fails[:10]
+        assert judged > canvas // 2
+    else:
+        # per-row decisions on a sample of rows (the stop flag needs every row and is checked above)
+        sub = np.ascontiguousarray(lg[rows])
+        T = oracle.temperature(step)
+        smp = oracle.sample_rows(sub, commit0[rows], rows, T, 7, step)
+        assert np.abs(g["H"][rows] - smp["H"]).max() <= ENTROPY_TOL
+        for k, r in enumerate(rows):
+            if commit0[r]:
+                assert g["ids"][r] == ids0[r] and g["commit"][r] == 1
+                continue
+            Hk = smp["H"][k]
+            if abs(Hk - 0.1) <= 1e-3 or abs(Hk - prm_o.rerand_entropy) <= 1e-3:
+                continue
+            if Hk <= 0.1:
+                assert g["commit"][r] == 1 and (smp["margin"][k] <= 1e-2 or g["ids"][r] == smp["y"][k])
+            elif not g["stop"]:
+                assert g["commit"][r] == 0
+                if Hk > prm_o.rerand_entropy:
+                    assert g["ids"][r] == smp["rr"][k]
+                elif smp["margin"][k] > 1e-2:
+                    assert g["ids"][r] == smp["y"][k]
+    if spike == 40.0:
+        spiked = np.arange(0, canvas, 10)
+        assert g["commit"][spiked].all()       # near-one-hot rows commit
+
+
+def test_sampler_is_deterministic(dg):
+    vocab, canvas = 262144, 256
+    logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=3)
+    d_logits = logits.cuda()
+    prm = dg.sampler_params(vocab, seed=3)
+    ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        ids = torch.zeros(canvas, dtype=torch.int32, device="cuda")
+        commit = torch.zeros(canvas, dtype=torch.uint8, device="cuda")
+        H = torch.empty(canvas, device="cuda")
+        stop = torch.empty(1, dtype=torch.int32, device="cuda")
+        dg.dg_sample(d_logits, 1, vocab, prm, 5, None, ids, commit, H, stop, ws)
+        outs.append((ids.cpu(), commit.cpu(), H.cpu()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------------------------------------
+# one decoder layer (attention block + MoE block)
+# ------------------------------------------------------------------------------------------------
+
+def _layer_case(dg, cfg, P, seed, router_std=None):
+    w = synthetic.make_model_weights(cfg, seed, router_std=router_std)
+    wd = to_device(w)
+    model = dg.dg_model_create(cfg, wd)
+    max_ctx = ((P + 256 + 255) // 256) * 256
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    ks, vs = synthetic.make_prefix_kv(cfg.n_layers, P, cfg.n_kv, cfg.d_head, seed + 1)
+    if P > 0:
+        dg.dg_load_prefix(seqs, 0, P, [k.cuda() for k in ks], [v.cuda() for v in vs])
+    x = synthetic.make_hidden(256, cfg.d_model, seed + 2)
+    return w, model, seqs, ks, vs, x
+
+
+@pytest.mark.parametrize("cfg_name,P", [("tiny", 0), ("tiny", 128), ("tiny", 300), ("one_layer", 4096)])
+def test_layer_matches_oracle(dg, cfg_name, P):
+    if cfg_name == "tiny":
+        cfg, router_std = synthetic.TINY, None
+    else:
+        import dataclasses
+        cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024)   # the layer does not read the vocabulary
+        router_std = cfg.d_model ** -0.5                            # router logits ~ N(0, 1)
+    w, model, seqs, ks, vs, x = _layer_case(dg, cfg, P, 11, router_std)
+    xd = x.cuda()
+    mid = torch.empty_like(xd)
+    rl = torch.empty(256, cfg.n_exp, device="cuda")
+    dg.dg_layer_forward(seqs, 0, xd, mid, rl)
+    torch.cuda.synchronize()
+    assert dg.dg_device_error(seqs) == 0
+    M = oracle.Model(cfg, w)
+    kc = ks[0].double().numpy() if P else None
+    vc = vs[0].double().numpy() if P else None
+    xo, kn, vn, rlo, mido = oracle.layer_forward(M, 0, x.double().numpy(), np.arange(P, P + 256), P, kc, vc,
+                                                 want_mid=True)
+    e_mid = rel_err(mid.cpu().numpy(), mido)
+    assert e_mid <= HIDDEN_TOL, f"attention block rel err {e_mid}"
+    e_rl = rel_err(rl.cpu().numpy(), rlo)
+    assert e_rl <= HIDDEN_TOL, f"router logits rel err {e_rl}"
+    keep = ~router_tie_tokens(rlo, cfg.top_k)
+    e_out = rel_err(xd.cpu().numpy()[keep], xo[keep])
+    assert e_out <= HIDDEN_TOL, f"layer output rel err {e_out} ({keep.sum()} tokens judged)"
+    # the canvas rows' K/V went to cache rows [P, P+256); the prefix rows are unchanged
+    K, Vt = kv_views(seqs.kv, cfg, 1, seqs.max_ctx)
+    Kg = K[0, 0, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
+    Vg = Vt[0, 0, :, :, P:P + 256].permute(2, 0, 1).float().cpu().numpy()
+    assert rel_err(Kg, kn) <= HIDDEN_TOL and rel_err(Vg, vn) <= HIDDEN_TOL
+    if P:
+        assert torch.equal(K[0, 0, :, :P].permute(1, 0, 2).cpu(), ks[0])
+        assert torch.equal(Vt[0, 0, :, :, :P].permute(2, 0, 1).cpu(), vs[0])
+
+
+# ------------------------------------------------------------------------------------------------
+# full tiny model: prefill, canvas steps (resynchronised to the oracle), block commit, decode
+# ------------------------------------------------------------------------------------------------
+
+def _tiny_model_pair(dg, head_scale=1.0, seed=0):
+    cfg = synthetic.TINY
+    w = synthetic.make_model_weights(cfg, seed, head_scale=head_scale)
+    model = dg.dg_model_create(cfg, to_device(w))
+    return cfg, w, model, oracle.Model(cfg, w)
+
+
+@pytest.mark.parametrize("head_scale,prompt_len,n_steps", [(1.0, 128, 4), (50.0, 128, 48), (50.0, 300, 6)])
+def test_canvas_steps_match_oracle(dg, head_scale, prompt_len, n_steps):
+    cfg, w, model, M = _tiny_model_pair(dg, head_scale)
+    max_ctx = 1024
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    prompt = synthetic.make_ids(prompt_len, cfg.vocab, 0)
+    dg.dg_prefill(seqs, prompt.cuda(), [prompt_len])
+    oseq = oracle.Sequence(M, max_ctx)
+    oseq.prefill(prompt.numpy())
+    # prefill K/V match
+    K, Vt = kv_views(seqs.kv, cfg, 1, max_ctx)
+    for l in range(cfg.n_layers):
+        kg = K[l, 0, :, :prompt_len].permute(1, 0, 2).float().cpu().numpy()
+        vg = Vt[l, 0, :, :, :prompt_len].permute(2, 0, 1).float().cpu().numpy()
+        assert rel_err(kg, oseq.k[l][:prompt_len]) <= HIDDEN_TOL, f"prefill K layer {l}"
+        assert rel_err(vg, oseq.v[l][:prompt_len]) <= HIDDEN_TOL, f"prefill V layer {l}"
+
+    prm = dg.sampler_params(cfg.vocab, seed=0)
+    prm_o = oracle.SamplerParams(cfg.vocab, seed=0)
+    ids = torch.empty(256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    oids, ocommit = oseq.canvas_init(prm_o)
+    np.testing.assert_array_equal(ids.cpu().numpy(), oids)          # Philox stream, bit-exact
+    assert commit.sum().item() == 0
+
+    H = torch.empty(256, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+    hidden = torch.empty(cfg.n_layers + 1, 256, cfg.d_model, device="cuda")
+    logits = torch.empty(256, cfg.vocab, device="cuda")
+    prefix_before = seqs.kv.clone()
+    n_cache = cfg.n_layers * cfg.n_kv * max_ctx * cfg.d_head
+    total_judged = 0
+    for s in range(n_steps):
+        # resynchronise: the GPU starts each step from the oracle's state
+        ids.copy_(torch.from_numpy(oids))
+        commit.copy_(torch.from_numpy(ocommit))
+        dg.dg_canvas_step(seqs, prm, ids, commit, H, stop, hidden, logits)
+        torch.cuda.synchronize()
+        r = oseq.canvas_step(prm_o, oids, ocommit, want_hidden=True, want_router=True)
+        keep = ~router_tie_tokens(r["router"], cfg.top_k)
+        hg = hidden.cpu().numpy()
+        for l in range(cfg.n_layers + 1):
+            e = rel_err(hg[l][keep], r["hidden"][l][keep])
+            assert e <= HIDDEN_TOL, f"step {s} hidden {l} rel err {e}"
+        el = rel_err(logits.cpu().numpy()[keep], r["logits"][keep])
+        assert el <= HIDDEN_TOL, f"step {s} logits rel err {el}"
+        g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(), "stop": int(stop.item())}
+        fails, judged = judge_step(g, r, prm_o, ocommit)
+        assert not fails, (s, fails[:10])
+        total_judged += judged
+        oids, ocommit = r["ids"], r["commit"]
+        if r["stop"]:
+            break
+    assert total_judged > 0
+    # the committed prefix [0, P) is untouched by canvas steps
+    P = prompt_len
+    Kb, Vb = kv_views(prefix_before, cfg, 1, max_ctx)
+    assert torch.equal(K[:, :, :, :P], Kb[:, :, :, :P]) and torch.equal(Vt[..., :P], Vb[..., :P])
+    assert n_cache > 0
+    # block commit of the final ids: cache rows [P, P+256) hold the K/V of a canvas forward
+    ids.copy_(torch.from_numpy(oids))
+    dg.dg_block_commit(seqs, ids)
+    oseq.block_commit(oids)
+    torch.cuda.synchronize()
+    Pn, _ = dg.dg_seqs_get_state(seqs)
+    assert Pn[0] == P + 256 == oseq.P
+    for l in range(cfg.n_layers):
+        kg = K[l, 0, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
+        vg = Vt[l, 0, :, :, P:P + 256].permute(2, 0, 1).float().cpu().numpy()
+        assert rel_err(kg, oseq.k[l][P:P + 256]) <= HIDDEN_TOL and rel_err(vg, oseq.v[l][P:P + 256]) <= HIDDEN_TOL
+    assert dg.dg_device_error(seqs) == 0
+
+
+def test_canvas_step_without_prompt_and_determinism(dg):
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=4)
+    seqs = dg.dg_seqs_create(model, 1, 512)
+    prm = dg.sampler_params(cfg.vocab, seed=9, fixed_steps=2)
+    outs = []
+    for rep in range(2):
+        ids = torch.empty(256, dtype=torch.int32, device="cuda")
+        commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+        H = torch.empty(256, device="cuda")
+        stop = torch.empty(1, dtype=torch.int32, device="cuda")
+        dg.dg_canvas_init(seqs, prm, ids, commit)
+        for s in range(2):
+            dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+        outs.append((ids.cpu(), commit.cpu(), H.cpu(), stop.cpu()))
+        with pytest.raises(dg.DGError) as ei:                    # budget used: state error, no launch
+            dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+        assert ei.value.status == dg.DG_ERR_STATE
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+    assert outs[0][3].item() == 1 and outs[0][1].all()
+    # oracle: P = 0, two fixed steps
+    oseq = oracle.Sequence(M, 512)
+    prm_o = oracle.SamplerParams(cfg.vocab, seed=9, fixed_steps=2)
+    oids, oc = oseq.canvas_init(prm_o)
+    for s in range(2):
+        r = oseq.canvas_step(prm_o, oids, oc)
+        oids, oc = r["ids"], r["commit"]
+    judged = r["margin"] > 1e-2
+    np.testing.assert_array_equal(outs[0][0].numpy()[judged], oids[judged])
+
+
+def test_decode_matches_oracle_tiny(dg):
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=1)
+    max_ctx = 1024
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    prompt = synthetic.make_ids(128, cfg.vocab, 1)
+    dg.dg_prefill(seqs, prompt.cuda(), [128])
+    prm = dg.sampler_params(cfg.vocab, seed=5, fixed_steps=3)
+    out = torch.full((1, 2 * 256), -1, dtype=torch.int32, device="cuda")
+    n_out, steps = dg.dg_decode(seqs, prm, 2, out)
+    assert n_out == [512] and steps == [3, 3]
+    oseq = oracle.Sequence(M, max_ctx)
+    oseq.prefill(prompt.numpy())
+    otoks = oseq.decode(oracle.SamplerParams(cfg.vocab, seed=5, fixed_steps=3), 2)
+    g = out.cpu().numpy()[0]
+    agree = (g == otoks).mean()
+    assert agree > 0.97, agree           # ids agree except at near-ties the oracle does not judge
+    P, _ = dg.dg_seqs_get_state(seqs)
+    assert P == [128 + 512]
+
+
+def test_capacity_and_argument_errors(dg):
+    cfg, w, model, M = _tiny_model_pair(dg)
+    seqs = dg.dg_seqs_create(model, 1, 256)
+    prm = dg.sampler_params(cfg.vocab)
+    ids = torch.zeros(256, dtype=torch.int32, device="cuda")
+    with pytest.raises(dg.DGError) as ei:
+        dg.dg_prefill(seqs, ids, [10])            # 10 + 256 > 256
+    assert ei.value.status == dg.DG_ERR_CAPACITY
+    commit = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    dg.dg_block_commit(seqs, ids)
+    with pytest.raises(dg.DGError) as ei:
+        dg.dg_block_commit(seqs, ids)             # cache full
+    assert ei.value.status == dg.DG_ERR_CAPACITY
+    bad = dg.sampler_params(cfg.vocab, canvas_len=128)
+    seqs2 = dg.dg_seqs_create(model, 1, 512)
+    with pytest.raises(dg.DGError) as ei:
+        dg.dg_canvas_init(seqs2, bad, ids, commit)
+    assert ei.value.status == dg.DG_ERR_UNSUPPORTED
+    # an out-of-range id is recorded as a device-side error, not a fault
+    ids_bad = torch.full((256,), cfg.vocab + 5, dtype=torch.int32, device="cuda")
+    dg.dg_canvas_init(seqs2, prm, ids, commit)
+    H = torch.empty(256, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+    dg.dg_canvas_step(seqs2, prm, ids_bad, commit, H, stop)
+    assert dg.dg_device_error(seqs2) != 0
+    assert dg.dg_device_error(seqs2) == 0         # the record is cleared by reading it
