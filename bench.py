@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="full_b1", choices=["full_b1", "one_layer", "sampler"],
+                    help="full_b1: the benchmark line; one_layer / sampler: the single-layer and "
+                         "sampler-alone configurations (their own lines, used for per-kernel profiles)")
     return ap.parse_args()
 
 
@@ -386,9 +389,86 @@ def main_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------------------
+# auxiliary workloads: one full-width layer; the sampler alone
+# ------------------------------------------------------------------------------------------------
+def _timed(fn, k, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(k):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / k
+
+
+def main_aux(args):
+    import dataclasses
+
+    import torch
+
+    import synthetic
+    from block_discrete_diffusion_b200 import build, dg
+    build.build()
+    dev = torch.device("cuda", 0)
+    if args.workload == "one_layer":
+        # one decoder layer at full width: x ~ N(0,1) [256, 2816], prefix K/V ~ N(0,1) of 4096 tokens
+        cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024)
+        w = synthetic.make_model_weights(cfg, 1, device=dev, router_std=cfg.d_model ** -0.5)
+        model = dg.dg_model_create(cfg, w)
+        P = 4096
+        seqs = dg.dg_seqs_create(model, 1, P + CANVAS)
+        ks, vs = synthetic.make_prefix_kv(1, P, cfg.n_kv, cfg.d_head, 1, device=dev)
+        dg.dg_load_prefix(seqs, 0, P, ks, vs)
+        x0 = synthetic.make_hidden(CANVAS, cfg.d_model, 1, device=dev)
+        x = x0.clone()
+
+        def step():
+            x.copy_(x0)
+            dg.dg_layer_forward(seqs, 0, x)
+        t = _timed(step, args.steps, args.warmup)
+        dg.dg_stats_reset(seqs, timing=True)
+        for _ in range(args.steps):
+            step()
+        stats = dg.dg_stats_read(seqs)
+        line = {"metric": "decoder-layer steps/s (a2-a9, one full-width layer)", "value": round(1 / t, 2),
+                "unit": "steps/s", "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
+                "config": {"workload": "one_layer: d 2816, 16/8 heads x 128, 128 experts top-8 FFN 704, "
+                                       "prefix 4096 tokens, canvas 256, bf16"},
+                "kernel_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in stats.items() if v[0]}}
+    else:
+        vocab, canvas = 262144, 256
+        logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, device=dev)
+        prm = dg.sampler_params(vocab, seed=7)
+        ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device=dev)
+        ids = torch.zeros(canvas, dtype=torch.int32, device=dev)
+        commit = torch.zeros(canvas, dtype=torch.uint8, device=dev)
+        H = torch.empty(canvas, device=dev)
+        stop = torch.empty(1, dtype=torch.int32, device=dev)
+
+        def step():
+            commit.zero_()
+            dg.dg_sample(logits, 1, vocab, prm, 12, None, ids, commit, H, stop, ws)
+        t = _timed(step, args.steps, args.warmup)
+        hbm, _, kind = peaks()
+        gbs = canvas * vocab * 4 / t / 1e9
+        line = {"metric": "sampler steps/s (256 x 262144 fp32 logits)", "value": round(1 / t, 2), "unit": "steps/s",
+                "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
+                "config": {"workload": "sampler: logits N(0, 3^2), 10% of rows +12 spike, step 12 of 48, seed 7"},
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                             "frac": round(gbs / hbm, 4), "note": "includes the commit-mask reset (256 B)"}}
+    print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         main_reference(a)
+    elif a.workload != "full_b1":
+        main_aux(a)
     else:
         main_dg(a)

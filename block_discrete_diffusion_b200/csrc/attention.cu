@@ -66,11 +66,28 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* p_s = kv_s + C::kStages * C::kStageBytes;
   AttnBarriers* bars = reinterpret_cast<AttnBarriers*>(p_s + C::kPBytes);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int qt = blockIdx.x, split = blockIdx.y;
   const int seq = blockIdx.z / p.n_kv, kvh = blockIdx.z % p.n_kv;
   const int G = p.n_q / p.n_kv;
   const int cseq = p.seq_base + seq;
+  pdl_trigger();
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qfull, 1);
+    mbar_init(&bars->kvfull[0], 1);
+    mbar_init(&bars->kvfull[1], 1);
+    mbar_init(&bars->s_done, 1);
+    mbar_init(&bars->o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&bars->tmem_slot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+  pdl_wait();   // queries, keys, values and P come from the preceding kernels
+
   const int P = p.seq_P[cseq];
   const int nkeys = P + p.Tq;
   const int ntiles = (nkeys + 127) >> 7;
@@ -92,25 +109,14 @@ __global__ void __launch_bounds__(128, 1)
       float4* o4 = reinterpret_cast<float4*>(p.opart + prow * DH);
       for (int c = 0; c < DH / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
     return;
   }
 
   const int qrow0 = (seq * p.n_q + kvh * G) * p.rows_per_seq + qt * 128;
   const int z = p.layer * p.cache_seq_stride + cseq * p.n_kv + kvh;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&bars->qfull, 1);
-    mbar_init(&bars->kvfull[0], 1);
-    mbar_init(&bars->kvfull[1], 1);
-    mbar_init(&bars->s_done, 1);
-    mbar_init(&bars->o_done, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(&bars->tmem_slot, C::kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = bars->tmem_slot;
   const uint32_t t_s = tmem + ((uint32_t)(warp * 32) << 16);
   const uint32_t t_o = t_s + 128;
 
@@ -240,30 +246,52 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-// One CTA per (sequence, query head, row): combine the split partials and write the row of the
-// token-major attention output [seq*rows_per_seq + j][h*dh + c] in bf16.
+// One warp per (sequence, query head, row): combine the split partials (lane s < n_splits holds
+// split s's (m, l)) and write the row of the token-major attention output
+// [seq*rows_per_seq + j][h*dh + c] in bf16; each lane owns dh/32 consecutive columns.
+template <int DH>
 __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
-  const int idx = blockIdx.x;
-  const int j = idx % p.Tq;
-  const int sh = idx / p.Tq;          // seq * n_q + h
+  pdl_trigger();
+  pdl_wait();
+  const int warp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (warp >= n_seq * p.n_q * p.Tq) return;
+  const int j = warp % p.Tq;
+  const int sh = warp / p.Tq;          // seq * n_q + h
   const int seq = sh / p.n_q, h = sh % p.n_q;
   const size_t stride = (size_t)n_seq * p.n_q * p.rows_per_seq;
   const size_t r0 = (size_t)sh * p.rows_per_seq + j;
-  float M = -INFINITY;
-  for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, p.ml[(s * stride + r0) * 2]);
-  float den = 0.f;
-  for (int s = 0; s < p.n_splits; ++s) {
-    const float ms = p.ml[(s * stride + r0) * 2];
-    if (ms != -INFINITY) den += exp2f(ms - M) * p.ml[(s * stride + r0) * 2 + 1];
+  float ms = -INFINITY, ls = 0.f;
+  if (lane < p.n_splits) {
+    const float2 v = *reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2);
+    ms = v.x;
+    ls = v.y;
   }
+  const float M = warp_max(ms);
+  const float wgt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+  const float den = warp_sum(wgt * ls);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int c = threadIdx.x; c < p.dh; c += blockDim.x) {
-    float num = 0.f;
-    for (int s = 0; s < p.n_splits; ++s) {
-      const float ms = p.ml[(s * stride + r0) * 2];
-      if (ms != -INFINITY) num += exp2f(ms - M) * p.opart[(s * stride + r0) * p.dh + c];
+  constexpr int kPer = DH / 32;
+  float acc[kPer];
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+  for (int s = 0; s < p.n_splits; ++s) {
+    const float ws = __shfl_sync(0xffffffffu, wgt, s);
+    if (ws == 0.f) continue;
+    const float* src = p.opart + (s * stride + r0) * DH + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] += ws * v.x; acc[1] += ws * v.y; acc[2] += ws * v.z; acc[3] += ws * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] += ws * v.x; acc[1] += ws * v.y;
     }
-    out[((size_t)seq * p.rows_per_seq + j) * (p.n_q * p.dh) + h * p.dh + c] = __float2bfloat16_rn(num * inv);
+  }
+  __nv_bfloat16* dst = out + ((size_t)seq * p.rows_per_seq + j) * (p.n_q * DH) + h * DH + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                pack_bf16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
 }
 
@@ -280,8 +308,7 @@ static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, con
   }
   const int G = p.n_q / p.n_kv;
   dim3 grid((G * p.rows_per_seq + 127) / 128, p.n_splits, n_seq * p.n_kv);
-  attn_partial_kernel<DH><<<grid, 128, C::kSmemBytes, st>>>(tq, tk, tv, p, n_seq, err);
-  return cudaGetLastError();
+  return launch_k(attn_partial_kernel<DH>, grid, dim3(128), C::kSmemBytes, st, 1, tq, tk, tv, p, n_seq, err);
 }
 
 cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -292,8 +319,12 @@ cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, cons
 }
 
 cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st) {
-  attn_merge_kernel<<<n_seq * p.n_q * p.Tq, 128, 0, st>>>(p, n_seq, out);
-  return cudaGetLastError();
+  if (p.n_splits > 32) return cudaErrorInvalidValue;
+  const int rows = n_seq * p.n_q * p.Tq;
+  const int blocks = (rows + 7) / 8;
+  if (p.dh == 128) return launch_k(attn_merge_kernel<128>, dim3(blocks), dim3(256), 0, st, 1, p, n_seq, out);
+  if (p.dh == 64) return launch_k(attn_merge_kernel<64>, dim3(blocks), dim3(256), 0, st, 1, p, n_seq, out);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dg

@@ -13,12 +13,22 @@
 #include <new>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dg.h"
 #include "dg_kernels.h"
 
 #define DG_API extern "C" __attribute__((visibility("default")))
 
 using namespace dg;
+
+bool dg::pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("DG_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 namespace {
 
@@ -39,9 +49,25 @@ dg_status fail(dg_status st, const char* fmt, ...) {
                                        __FILE__, __LINE__);                                          \
   } while (0)
 
+// NVTX range for the lifetime of one API call (profilers filter kernels by it).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 constexpr int kCanvas = 256;
 constexpr int kSplitTargetCtas = 296;   // two waves of CTAs over the 148 SMs
 constexpr int kMaxSplits = 16;
+constexpr int kRouterSplits = 8;        // cluster size of the router GEMM's split-K
+constexpr int kGemmTargetCtas = 296;    // two CTAs per SM for the 128-wide dense GEMM tiles
+
+// Cluster size (power of two, <= 8) of the split-K dense GEMMs for `tiles` output tiles over nk
+// 64-deep k-blocks: enough CTAs for about two per SM, at least 4 k-blocks per CTA.
+int dense_splits(int tiles, int nk) {
+  int z = 1;
+  while (z < 8 && tiles * z * 2 <= kGemmTargetCtas && nk / (z * 2) >= 4) z *= 2;
+  return z;
+}
 
 // ---------------------------------------------------------------------------------------------
 // TMA descriptor creation through the driver entry point (no libcuda link dependency)
@@ -151,6 +177,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.ccommit = take(R);
   L.cH = take(4 * R);
   L.cstop = take(4 * (size_t)n_seq);
+
   L.total = off + 1024;   // slack for base alignment
   return L;
 }
@@ -183,6 +210,7 @@ struct LayerMaps {
 
 struct dg_model {
   dg_model_config cfg;
+  int n_sms;   // streaming multiprocessors of the current device (persistent grids)
   const __nv_bfloat16 *emb, *head;
   const float* final_norm;
   std::vector<dg_layer_weights> layers;
@@ -204,8 +232,9 @@ struct dg_seqs {
   int32_t *sel, *counts, *offsets, *perm_tok, *slot, *cids, *cstop;
   uint8_t* ccommit;
   float* cH;
+
   float2* rope;
-  CUtensorMap xn_map, attn_map, xp_map, hb_map, q_map, k_map, v_map;
+  CUtensorMap xn_map, xp_map, attn_map, hb_map, q_map, k_map, v_map;
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
   bool block_open;
@@ -285,6 +314,11 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
   dg_model* m = new (std::nothrow) dg_model();
   if (!m) return fail(DG_ERR_INVALID_ARG, "host allocation failed");
   m->cfg = *cfg;
+  {
+    int dev = 0;
+    m->n_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&m->n_sms, cudaDevAttrMultiProcessorCount, dev);
+  }
   m->emb = static_cast<const __nv_bfloat16*>(w->emb);
   m->head = static_cast<const __nv_bfloat16*>(w->head);
   m->final_norm = static_cast<const float*>(w->final_norm);
@@ -297,7 +331,7 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
     const dg_layer_weights& L = m->layers[l];
     LayerMaps& M = m->maps[l];
     if ((st = map_2d(&M.wqkv, L.w_qkv, qkv, d, 128)) != DG_OK) break;
-    if ((st = map_2d(&M.wo, L.w_o, d, (uint64_t)c.n_q * c.d_head, 64)) != DG_OK) break;
+    if ((st = map_2d(&M.wo, L.w_o, d, (uint64_t)c.n_q * c.d_head, 128)) != DG_OK) break;
     if ((st = map_2d(&M.wrouter, L.w_router, c.n_exp, d, 128)) != DG_OK) break;
     if ((st = map_2d(&M.wgu, L.w_gate_up, (uint64_t)c.n_exp * 2 * c.d_ff, d, 64)) != DG_OK) break;
     if ((st = map_2d(&M.wdown, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
@@ -379,6 +413,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->ccommit = b + L.ccommit;
   s->cH = reinterpret_cast<float*>(b + L.cH);
   s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
+
   s->P.assign(n_seq, 0);
   s->step = 0;
   s->block_open = false;
@@ -408,6 +443,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   // clear the cache and the buffers whose stale contents a masked lane may read, build the table
   cudaError_t e = cudaMemsetAsync(kv, 0, need_kv, s->st);
   if (e == cudaSuccess) e = cudaMemsetAsync(s->ws, 0, L.rope, s->st);
+
   if (e == cudaSuccess) e = rope_table(s->rope, max_ctx, c.d_head, c.rope_theta, s->st);
   if (e != cudaSuccess) {
     delete s;
@@ -444,15 +480,18 @@ size_t layer_kv_elems(const dg_seqs* s) {
 
 // One decoder layer on `rows` rows of x.  n_local sequences starting at cache sequence seq_base,
 // Tq rows per sequence (rows == n_local * 256 for a canvas, rows == Tq for a prefill chunk).
+// xn_ready: xn already holds RMSNorm_attn(x) of this layer (written by the previous combine or the
+// embedding); next_gain != nullptr: the combine also writes RMSNorm(x) with that gain into xn.
 dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_base, int Tq, bool causal,
-                    float* x_mid, float* rlog_out) {
+                    float* x_mid, float* rlog_out, bool xn_ready = false, const float* next_gain = nullptr) {
   const dg_model_config& c = s->m->cfg;
   const dg_layer_weights& W = s->m->layers[l];
   const LayerMaps& M = s->m->maps[l];
   cudaStream_t st = s->st;
   const int d = c.d_model, dh = c.d_head;
 
-  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.attn_norm), rows, d, c.rms_eps, s->xn, st));
+  if (!xn_ready)
+    LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.attn_norm), rows, d, c.rms_eps, s->xn, st));
   EpiParams ep{};
   ep.q = s->q;
   ep.kc = s->kc + (size_t)l * layer_kv_elems(s);
@@ -465,7 +504,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   ep.rows_per_seq = kCanvas;
   ep.max_ctx = s->max_ctx;
   ep.seq_base = seq_base;
-  LAUNCH(s, DG_K_QKV, 1, gemm_dense(128, EPI_QKV, s->xn_map, M.wqkv, rows, (c.n_q + 2 * c.n_kv) * dh, d, ep, s->err, st));
+  const int n_qkv = (c.n_q + 2 * c.n_kv) * dh;
+  ep.k_splits = dense_splits(((rows + 127) / 128) * (n_qkv / 128), d / 64);
+  LAUNCH(s, DG_K_QKV, 1, gemm_dense(128, EPI_QKV, s->xn_map, M.wqkv, rows, n_qkv, d, ep, s->err, st));
 
   // attention over cache [0, P) + the Tq new rows
   int Pmax = 0;
@@ -494,7 +535,8 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   EpiParams eo{};
   eo.x = x;
   eo.ldo = d;
-  LAUNCH(s, DG_K_OPROJ, 1, gemm_dense(64, EPI_RESID, s->attn_map, M.wo, rows, d, c.n_q * dh, eo, s->err, st));
+  eo.k_splits = dense_splits(((rows + 127) / 128) * (d / 128), c.n_q * dh / 64);
+  LAUNCH(s, DG_K_OPROJ, 1, gemm_dense(128, EPI_RESID, s->attn_map, M.wo, rows, d, c.n_q * dh, eo, s->err, st));
   if (x_mid) CK(cudaMemcpyAsync(x_mid, x, sizeof(float) * (size_t)rows * d, cudaMemcpyDeviceToDevice, st));
 
   // mixture of experts
@@ -502,25 +544,26 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   EpiParams er{};
   er.out = s->rlog;
   er.ldo = c.n_exp;
+  er.k_splits = std::min(kRouterSplits, dense_splits((rows + 127) / 128, d / 64));
   LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
+  LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));
   if (rlog_out)
     CK(cudaMemcpyAsync(rlog_out, s->rlog, sizeof(float) * (size_t)rows * c.n_exp, cudaMemcpyDeviceToDevice, st));
-  CK(cudaMemsetAsync(s->counts, 0, sizeof(int32_t) * c.n_exp, st));
-  LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));
   LAUNCH(s, DG_K_BUCKET, 1,
-         bucket_gather(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->xn, d, s->offsets, s->perm_gate,
-                       s->perm_tok, s->slot, s->xp, st));
+         assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->perm_gate, s->perm_tok,
+                     s->slot, st));
+  LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
   ExpertParams xp{};
-  xp.counts = s->counts;
   xp.offsets = s->offsets;
   xp.perm_gate = s->perm_gate;
+  xp.perm_tok = s->perm_tok;
   xp.h_out = s->hb;
   xp.y_out = s->y;
   xp.d = d;
   xp.F = c.d_ff;
-  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->err, st));
-  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->err, st));
-  LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, rows, c.top_k, d, x, st));
+  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->m->n_sms, s->err, st));
+  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->m->n_sms, s->err, st));
+  LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
   return DG_OK;
 }
 
@@ -529,10 +572,14 @@ dg_status run_canvas_stack(dg_seqs* s, const int32_t* d_ids, float* hidden) {
   const dg_model_config& c = s->m->cfg;
   const int R = s->L.R;
   const size_t plane = (size_t)R * c.d_model;
-  LAUNCH(s, DG_K_EMBED, 1, embed_rows(s->m->emb, d_ids, R, c.d_model, c.vocab, s->x, s->err, s->st));
+  LAUNCH(s, DG_K_EMBED, 1,
+         embed_rows(s->m->emb, d_ids, R, c.d_model, c.vocab, s->x, s->err,
+                    static_cast<const float*>(s->m->layers[0].attn_norm), c.rms_eps, s->xn, s->st));
   if (hidden) CK(cudaMemcpyAsync(hidden, s->x, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s->st));
   for (int l = 0; l < c.n_layers; ++l) {
-    dg_status r = run_layer(s, l, s->x, R, s->n_seq, 0, kCanvas, false, nullptr, nullptr);
+    // the combine of layer l writes the next layer's normed operand (the head's after the last layer)
+    const float* next = l + 1 < c.n_layers ? static_cast<const float*>(s->m->layers[l + 1].attn_norm) : s->m->final_norm;
+    dg_status r = run_layer(s, l, s->x, R, s->n_seq, 0, kCanvas, false, nullptr, nullptr, true, next);
     if (r != DG_OK) return r;
     if (hidden)
       CK(cudaMemcpyAsync(hidden + (size_t)(l + 1) * plane, s->x, sizeof(float) * plane, cudaMemcpyDeviceToDevice,
@@ -556,6 +603,7 @@ dg_status check_params(const dg_seqs* s, const dg_sampler_params* p) {
 // public calls
 // ---------------------------------------------------------------------------------------------
 DG_API dg_status dg_load_prefix(dg_seqs* s, int seq, int P, const void* const* h_k, const void* const* h_v) {
+  NvtxRange nvtx_range("dg_load_prefix");
   if (!s || !h_k || !h_v) return fail(DG_ERR_INVALID_ARG, "null argument");
   if (seq < 0 || seq >= s->n_seq) return fail(DG_ERR_INVALID_ARG, "seq %d out of range", seq);
   if (P < 0 || P + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "prefix %d + canvas exceeds max_ctx", P);
@@ -574,6 +622,7 @@ DG_API dg_status dg_load_prefix(dg_seqs* s, int seq, int P, const void* const* h
 }
 
 DG_API dg_status dg_prefill(dg_seqs* s, const int32_t* d_ids, const int32_t* h_lens) {
+  NvtxRange nvtx_range("dg_prefill");
   if (!s || !d_ids || !h_lens) return fail(DG_ERR_INVALID_ARG, "null argument");
   const dg_model_config& c = s->m->cfg;
   for (int i = 0; i < s->n_seq; ++i)
@@ -584,9 +633,12 @@ DG_API dg_status dg_prefill(dg_seqs* s, const int32_t* d_ids, const int32_t* h_l
   for (int i = 0; i < s->n_seq; ++i) {
     for (int c0 = 0; c0 < h_lens[i]; c0 += kCanvas) {
       const int n = std::min(kCanvas, h_lens[i] - c0);
-      LAUNCH(s, DG_K_EMBED, 1, embed_rows(s->m->emb, d_ids + off + c0, n, c.d_model, c.vocab, s->x, s->err, s->st));
+      LAUNCH(s, DG_K_EMBED, 1,
+             embed_rows(s->m->emb, d_ids + off + c0, n, c.d_model, c.vocab, s->x, s->err,
+                        static_cast<const float*>(s->m->layers[0].attn_norm), c.rms_eps, s->xn, s->st));
       for (int l = 0; l < c.n_layers; ++l) {
-        dg_status r = run_layer(s, l, s->x, n, 1, i, n, true, nullptr, nullptr);
+        const float* next = l + 1 < c.n_layers ? static_cast<const float*>(s->m->layers[l + 1].attn_norm) : nullptr;
+        dg_status r = run_layer(s, l, s->x, n, 1, i, n, true, nullptr, nullptr, true, next);
         if (r != DG_OK) return r;
       }
       LAUNCH(s, DG_K_MISC, 1, add_to_P(s->seqP, i, 1, n, s->st));
@@ -599,6 +651,7 @@ DG_API dg_status dg_prefill(dg_seqs* s, const int32_t* d_ids, const int32_t* h_l
 }
 
 DG_API dg_status dg_canvas_init(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit) {
+  NvtxRange nvtx_range("dg_canvas_init");
   if (!s || !d_ids || !d_commit) return fail(DG_ERR_INVALID_ARG, "null argument");
   dg_status r = check_params(s, p);
   if (r != DG_OK) return r;
@@ -612,6 +665,7 @@ DG_API dg_status dg_canvas_init(dg_seqs* s, const dg_sampler_params* p, int32_t*
 
 DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit,
                                 float* d_entropy, int32_t* d_stop, float* d_hidden, float* d_logits_out) {
+  NvtxRange nvtx_range("dg_canvas_step");
   if (!s || !d_ids || !d_commit || !d_entropy || !d_stop) return fail(DG_ERR_INVALID_ARG, "null argument");
   dg_status r = check_params(s, p);
   if (r != DG_OK) return r;
@@ -619,9 +673,8 @@ DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t*
   const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
   if (s->step >= budget) return fail(DG_ERR_STATE, "step budget of %d already used", budget);
   const dg_model_config& c = s->m->cfg;
-  r = run_canvas_stack(s, d_ids, d_hidden);
+  r = run_canvas_stack(s, d_ids, d_hidden);   // leaves RMSNorm_final(x) in xn
   if (r != DG_OK) return r;
-  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(s->x, s->m->final_norm, s->L.R, c.d_model, c.rms_eps, s->xn, s->st));
   EpiParams eh{};
   eh.out = s->logits;
   eh.ldo = c.vocab;
@@ -657,6 +710,7 @@ DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t*
 }
 
 DG_API dg_status dg_block_commit(dg_seqs* s, const int32_t* d_ids) {
+  NvtxRange nvtx_range("dg_block_commit");
   if (!s || !d_ids) return fail(DG_ERR_INVALID_ARG, "null argument");
   for (int i = 0; i < s->n_seq; ++i)
     if (s->P[i] + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "sequence %d: cache full", i);
@@ -670,6 +724,7 @@ DG_API dg_status dg_block_commit(dg_seqs* s, const int32_t* d_ids) {
 
 DG_API dg_status dg_layer_forward(dg_seqs* s, int layer, int n_rows, int causal, float* d_x, float* d_x_mid,
                                   float* d_router_logits) {
+  NvtxRange nvtx_range("dg_layer_forward");
   if (!s || !d_x) return fail(DG_ERR_INVALID_ARG, "null argument");
   if (layer < 0 || layer >= s->m->cfg.n_layers) return fail(DG_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (n_rows <= 0 || n_rows > kCanvas) return fail(DG_ERR_INVALID_ARG, "n_rows must be in [1, 256]");
@@ -683,6 +738,7 @@ DG_API dg_status dg_layer_forward(dg_seqs* s, int layer, int n_rows, int causal,
 
 DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_blocks, int32_t* d_out, int32_t* h_n_out,
                            int32_t* h_steps) {
+  NvtxRange nvtx_range("dg_decode");
   if (!s || !d_out || !h_n_out || max_blocks <= 0) return fail(DG_ERR_INVALID_ARG, "bad argument");
   dg_status r = check_params(s, p);
   if (r != DG_OK) return r;
@@ -747,6 +803,7 @@ DG_API size_t dg_sample_workspace_bytes(int n_rows, int vocab) {
 DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg_sampler_params* p, int step,
                            const int32_t* d_seq_P, int32_t* d_ids, uint8_t* d_commit, float* d_entropy, int32_t* d_stop,
                            void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dg_sample");
   if (!d_logits || !p || !d_ids || !d_commit || !d_entropy || !d_stop || !ws)
     return fail(DG_ERR_INVALID_ARG, "null argument");
   if (n_seq <= 0 || vocab <= 0 || vocab % 1024) return fail(DG_ERR_INVALID_ARG, "bad n_seq / vocab");

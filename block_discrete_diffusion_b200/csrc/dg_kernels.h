@@ -9,10 +9,45 @@
 
 namespace dg {
 
+// Programmatic dependent launch on/off for every kernel of the library (on unless DG_PDL=0).
+bool pdl_enabled();
+
+// Launch with programmatic stream serialization (the kernel's prologue may overlap the previous
+// kernel's tail; the kernel orders itself with griddepcontrol.wait) and an optional cluster of
+// (1, 1, cluster_z) CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_z,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 enum { EPI_QKV = 0, EPI_RESID = 1, EPI_F32 = 2 };
 
 struct EpiParams {
   float* out;            // EPI_F32: out[row * ldo + col]
+  int k_splits;          // 1, 2, 4 or 8: K split over a cluster of this many CTAs (DSMEM reduction)
   float* x;              // EPI_RESID: x[row * ldo + col] += acc
   int ldo;
   __nv_bfloat16* q;      // EPI_QKV: query buffer [seq][n_q][rows_per_seq][dh]
@@ -24,9 +59,9 @@ struct EpiParams {
 };
 
 struct ExpertParams {
-  const int* counts;     // [E] tokens routed to each expert
-  const int* offsets;    // [E+1] first bucketed row of each expert
+  const int* offsets;    // [E+1] first bucketed row of each expert (expert e owns rows [off[e], off[e+1]))
   const float* perm_gate;  // [A] gate weight of each bucketed row
+  const int* perm_tok;   // [A] token (row of the normed activations) of each bucketed row
   __nv_bfloat16* h_out;  // MODE 1: SwiGLU rows [A][F]
   float* y_out;          // MODE 2: gate-scaled expert outputs [A][d]
   int d, F;
@@ -49,25 +84,30 @@ struct AttnParams {
 
 cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const EpiParams& ep, int* err, cudaStream_t st);
+// persistent: n_ctas CTAs (one per SM) loop over the (expert, weight tile) items
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
-                        int* err, cudaStream_t st);
+                        int n_ctas, int* err, cudaStream_t st);
 cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, int n_seq, int* err, cudaStream_t st);
 cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st);
 
 // elementwise / routing kernels (misc.cu)
+// g != nullptr: also the RMSNorm of each embedded row into xn (bf16), gain g
 cudaError_t embed_rows(const __nv_bfloat16* emb, const int32_t* ids, int n_rows, int d, int vocab, float* x,
-                       int* err, cudaStream_t st);
+                       int* err, const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st);
 cudaError_t rmsnorm_rows(const float* x, const float* g, int n_rows, int d, float eps, __nv_bfloat16* out,
                          cudaStream_t st);
 cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st);
-cudaError_t router_topk(const float* logits, int n_rows, int n_exp, int top_k, int32_t* sel, float* gate,
-                        int32_t* counts, cudaStream_t st);
-cudaError_t bucket_gather(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k,
-                          int n_exp, const __nv_bfloat16* xn, int d, int32_t* offsets, float* perm_gate,
-                          int32_t* perm_tok, int32_t* slot, __nv_bfloat16* xp, cudaStream_t st);
-cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x,
+cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
+                        int32_t* sel, float* gate, int32_t* counts, cudaStream_t st);
+cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k, int n_exp,
+                        int32_t* offsets, float* perm_gate, int32_t* perm_tok, int32_t* slot, cudaStream_t st);
+cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st);
+// g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g
+cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x, const float* g,
+                        float eps, __nv_bfloat16* xn, cudaStream_t st);
+cudaError_t sum_planes(float* out, const float* in, int n_planes, size_t stride, size_t n, cudaStream_t st);
 cudaError_t add_to_P(int* seq_P, int first, int count, int delta, cudaStream_t st);
 cudaError_t load_prefix(const __nv_bfloat16* k_in, const __nv_bfloat16* v_in, int P, int n_kv, int dh, int max_ctx,
                         __nv_bfloat16* kc, __nv_bfloat16* vt, cudaStream_t st);

@@ -25,11 +25,13 @@ namespace dg {
 constexpr int kGemmThreads = 128;
 constexpr uint32_t kATileBytes = 128 * 64 * 2;   // 128 rows x 64 bf16
 
+// BN <= 128: two CTAs per SM (up to 96 KB of stages each); BN = 256: one CTA per SM.
 template <int BN>
 struct DenseCfg {
   static constexpr uint32_t kBTileBytes = BN * 64 * 2;
   static constexpr uint32_t kStageBytes = kATileBytes + kBTileBytes;
-  static constexpr int kStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int kStages = BN >= 256 ? 4 : (BN >= 128 ? 3 : 4);
+  static constexpr int kMinBlocks = BN >= 256 ? 1 : 2;
   static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
 };
@@ -48,17 +50,81 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ---------------------------------------------------------------------------------------------
 // dense GEMM
 // ---------------------------------------------------------------------------------------------
-template <int BN, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// Epilogue of one output row segment: values for columns col0 + j (j < n) of row `row`.
+template <int EPI>
+__device__ __forceinline__ void store_row_f32(const EpiParams& ep, int row, int col0, const float* v, int n, int N) {
+  float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)row * ep.ldo + col0;
+  if (col0 + n <= N && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) && (n % 4) == 0) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+    for (int i = 0; i < n / 4; ++i) {
+      float4 o = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if (EPI == EPI_RESID) {
+        const float4 x = d4[i];
+        o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+      }
+      d4[i] = o;
+    }
+  } else {
+    for (int i = 0; i < n && col0 + i < N; ++i) dst[i] = (EPI == EPI_RESID ? dst[i] : 0.f) + v[i];
+  }
+}
+
+// QKV epilogue for `np` rotary pairs of one row: a[k] is column c1 + k, b[k] column c1 + half + k
+// of the fused Q|K|V output (columns of one head; c1 = head start + i0).  Q and K rows are rotated by
+// the row's position and stored head-major; V (no rotation) goes to the transposed value cache.
+__device__ __forceinline__ void store_qkv_pairs(const EpiParams& ep, int row, int f_head, int i0, const float* a,
+                                                const float* b, int np) {
+  const int dh = ep.dh, half = dh >> 1;
+  const int q_end = ep.n_q * dh, k_end = q_end + ep.n_kv * dh;
+  const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
+  const int cseq = ep.seq_base + seq;
+  const int pos = ep.seq_P[cseq] + j;
+  if (f_head < k_end) {
+    const float2* cs = ep.rope + (size_t)pos * half + i0;
+    __nv_bfloat16* dst;
+    if (f_head < q_end) {
+      dst = ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh;
+    } else {
+      dst = ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + pos) * dh;
+    }
+    for (int k = 0; k < np; k += 2) {
+      const float2 c0 = cs[k], c1 = cs[k + 1];
+      *reinterpret_cast<uint32_t*>(dst + i0 + k) =
+          pack_bf16x2(a[k] * c0.x - b[k] * c0.y, a[k + 1] * c1.x - b[k + 1] * c1.y);
+      *reinterpret_cast<uint32_t*>(dst + half + i0 + k) =
+          pack_bf16x2(b[k] * c0.x + a[k] * c0.y, b[k + 1] * c1.x + a[k + 1] * c1.y);
+    }
+  } else {
+    __nv_bfloat16* dst = ep.vt + (((size_t)cseq * ep.n_kv + (f_head - k_end) / dh) * dh) * ep.max_ctx + pos;
+    for (int k = 0; k < np; ++k) {
+      dst[(size_t)(i0 + k) * ep.max_ctx] = __float2bfloat16_rn(a[k]);
+      dst[(size_t)(half + i0 + k) * ep.max_ctx] = __float2bfloat16_rn(b[k]);
+    }
+  }
+}
+
+// One 128 x BN output tile per cluster of Z CTAs; CTA z of the cluster multiplies k-blocks
+// [z nk/Z, (z+1) nk/Z).  Z = 1: the epilogue reads the accumulator from TMEM (thread = row).
+// Z > 1: every CTA parks its fp32 partial in its own shared memory; after a cluster barrier CTA z
+// sums rows [z 128/Z, (z+1) 128/Z) over the cluster's partials (distributed shared memory, in rank
+// order, so the result does not depend on timing) and runs the epilogue on those rows.
+template <int BN, int EPI, int Z>
+__global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
     dense_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                       int K, EpiParams ep, int* err) {
   using C = DenseCfg<BN>;
+  static_assert(Z == 1 || (Z > 1 && 128 % Z == 0 && (BN / (2 * Z)) % 4 == 0), "bad split");
+  static_assert(Z == 1 || (size_t)128 * (BN + 4) * 4 <= (size_t)C::kStages * C::kStageBytes, "partial tile too big");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = align1024(smem_raw);
   GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(tiles + (size_t)C::kStages * C::kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
-  const int nk = K / 64;
+  const int nk_all = K / 64;
+  const int zz = Z > 1 ? (int)blockIdx.z : 0;
+  const int kb0 = zz * nk_all / Z;
+  const int nk = (zz + 1) * nk_all / Z - kb0;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -76,16 +142,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     const uint64_t pol_w = l2_policy_evict_first();
-    for (int kb = 0; kb < nk; ++kb) {
+    // The weights (B) of the first stages do not depend on the previous kernel: load them before
+    // waiting for it; the activation tiles (A) follow the wait.
+    const int npre = nk < C::kStages ? nk : C::kStages;
+    for (int kb = 0; kb < npre; ++kb) {
+      uint8_t* a = tiles + (size_t)kb * C::kStageBytes;
+      mbar_expect_tx(&bars->full[kb], C::kBTileBytes);
+      tma_load_2d_hint(&tmB, &bars->full[kb], a + kATileBytes, (kb0 + kb) * 64, n0, pol_w);
+    }
+    pdl_wait();
+    for (int kb = 0; kb < npre; ++kb) {
+      uint8_t* a = tiles + (size_t)kb * C::kStageBytes;
+      mbar_arrive_expect_tx(&bars->full[kb], kATileBytes);
+      tma_load_2d(&tmA, &bars->full[kb], a, (kb0 + kb) * 64, m0);
+    }
+    for (int kb = npre; kb < nk; ++kb) {
       const int s = kb % C::kStages;
       const uint32_t ph = (kb / C::kStages) & 1;
       if (!mbar_wait(&bars->empty[s], ph ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
       uint8_t* a = tiles + (size_t)s * C::kStageBytes;
       mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
-      tma_load_2d(&tmA, &bars->full[s], a, kb * 64, m0);
-      tma_load_2d_hint(&tmB, &bars->full[s], a + kATileBytes, kb * 64, n0, pol_w);
+      tma_load_2d(&tmA, &bars->full[s], a, (kb0 + kb) * 64, m0);
+      tma_load_2d_hint(&tmB, &bars->full[s], a + kATileBytes, (kb0 + kb) * 64, n0, pol_w);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else {
+    pdl_wait();
+  }
+  if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % C::kStages;
@@ -104,89 +187,90 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   __syncwarp();
 
-  // ---------------- epilogue: thread owns accumulator row m0 + 32*warp + lane ----------------
   const bool ok = mbar_wait(&bars->accum, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
   tc_fence_after();
-  const int row = m0 + warp * 32 + lane;
-  const bool row_ok = ok && row < M;
   const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
 
-  if constexpr (EPI == EPI_QKV) {
-    // Feature tile [n0, n0+BN) lies inside one of the Q / K / V regions (BN divides the region sizes).
-    const int dh = ep.dh, half = dh >> 1;
-    const int q_end = ep.n_q * dh, k_end = q_end + ep.n_kv * dh;
-    const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
-    const int cseq = ep.seq_base + seq;
-    const int pos = row_ok ? ep.seq_P[cseq] + j : 0;
-    for (int h0 = 0; h0 < BN; h0 += dh) {
-      const int f0 = n0 + h0;
-      if (f0 >= N) break;
-      if (f0 < k_end) {
-        // rotate pairs (i, i+half) of this head, 32 pairs at a time
+  if constexpr (Z == 1) {
+    // ---------------- thread owns accumulator row m0 + 32*warp + lane ----------------
+    const int row = m0 + warp * 32 + lane;
+    const bool row_ok = ok && row < M;
+    if constexpr (EPI == EPI_QKV) {
+      const int dh = ep.dh, half = dh >> 1;
+      for (int h0 = 0; h0 < BN; h0 += dh) {
+        if (n0 + h0 >= N) break;
         for (int c = 0; c < half; c += 32) {
           float a[32], b[32];
           tmem_ld_32cols(tbase + h0 + c, a);
           tmem_ld_32cols(tbase + h0 + half + c, b);
-          if (!row_ok) continue;
-          const float2* cs = ep.rope + (size_t)pos * half + c;
-          uint32_t lo[16], hi[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 c0 = cs[i], c1 = cs[i + 1];
-            lo[i / 2] = pack_bf16x2(a[i] * c0.x - b[i] * c0.y, a[i + 1] * c1.x - b[i + 1] * c1.y);
-            hi[i / 2] = pack_bf16x2(b[i] * c0.x + a[i] * c0.y, b[i + 1] * c1.x + a[i + 1] * c1.y);
-          }
-          __nv_bfloat16* dst;
-          if (f0 < q_end) {
-            const int h = f0 / dh;
-            dst = ep.q + (((size_t)seq * ep.n_q + h) * ep.rows_per_seq + j) * dh;
-          } else {
-            const int h = (f0 - q_end) / dh;
-            dst = ep.kc + (((size_t)cseq * ep.n_kv + h) * ep.max_ctx + pos) * dh;
-          }
-          uint4* d0 = reinterpret_cast<uint4*>(dst + c);
-          uint4* d1 = reinterpret_cast<uint4*>(dst + half + c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            d0[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
-            d1[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
-          }
+          if (row_ok) store_qkv_pairs(ep, row, n0 + h0, c, a, b, 32);
         }
-      } else {
-        // V: written transposed, vt[cseq][h][i][pos]; lanes hold consecutive positions
-        const int h = (f0 - k_end) / dh;
-        __nv_bfloat16* dst = ep.vt + (((size_t)cseq * ep.n_kv + h) * dh) * ep.max_ctx + pos;
-        for (int c = 0; c < dh; c += 32) {
-          float a[32];
-          tmem_ld_32cols(tbase + h0 + c, a);
-          if (!row_ok) continue;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dst[(size_t)(c + i) * ep.max_ctx] = __float2bfloat16_rn(a[i]);
-        }
+      }
+    } else {
+      for (int c = 0; c < BN; c += 32) {
+        float a[32];
+        tmem_ld_32cols(tbase + c, a);
+        if (row_ok) store_row_f32<EPI>(ep, row, n0 + c, a, 32, N);
       }
     }
   } else {
-    for (int c = 0; c < BN; c += 32) {
-      float a[32];
-      tmem_ld_32cols(tbase + c, a);
-      if (!row_ok) continue;
-      const int col = n0 + c;
-      float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)row * ep.ldo + col;
-      if (col + 32 <= N) {
-        float4* d4 = reinterpret_cast<float4*>(dst);
+    // ---------------- cluster split-K reduction over distributed shared memory ----------------
+    constexpr int RS = BN + 4;                 // padded row stride of the parked partial
+    float* red = reinterpret_cast<float*>(tiles);
+    {
+      const int r = warp * 32 + lane;
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld_32cols(tbase + c, v);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          float4 o = make_float4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
-          if constexpr (EPI == EPI_RESID) {
-            const float4 x = d4[v];
-            o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
-          }
-          d4[v] = o;
-        }
-      } else {
-        for (int i = 0; i < 32 && col + i < N; ++i) dst[i] = (EPI == EPI_RESID ? dst[i] : 0.f) + a[i];
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(red + r * RS + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
+    tc_fence_before();
+    cluster_sync();
+    constexpr int RPC = 128 / Z;               // rows reduced by this CTA
+    const int rr = zz * RPC + threadIdx.x / Z;   // Z threads per row
+    const int q = threadIdx.x % Z;
+    const int row = m0 + rr;
+    if constexpr (EPI == EPI_QKV) {
+      // thread q takes rotary pairs [q PW, (q+1) PW) of the tile: columns c1 and c1 + half of a head
+      constexpr int PW = BN / (2 * Z);
+      const int dh = ep.dh, half = dh >> 1;
+      const int p0 = q * PW;
+      const int hh = p0 / half, i0 = p0 % half;
+      const int c1 = hh * dh + i0;
+      float a[PW], b[PW];
+#pragma unroll
+      for (int k = 0; k < PW; ++k) a[k] = b[k] = 0.f;
+      const uint32_t la = smem_u32(red + rr * RS + c1), lb = smem_u32(red + rr * RS + c1 + half);
+      for (int z = 0; z < Z; ++z) {
+        const uint32_t ra = dsmem_map(la, z), rb = dsmem_map(lb, z);
+#pragma unroll
+        for (int k = 0; k < PW; k += 4) {
+          const float4 u = dsmem_ld_f4(ra + 4 * k), w = dsmem_ld_f4(rb + 4 * k);
+          a[k] += u.x; a[k + 1] += u.y; a[k + 2] += u.z; a[k + 3] += u.w;
+          b[k] += w.x; b[k + 1] += w.y; b[k + 2] += w.z; b[k + 3] += w.w;
+        }
+      }
+      if (ok && row < M && n0 + hh * dh < N) store_qkv_pairs(ep, row, n0 + hh * dh, i0, a, b, PW);
+    } else {
+      constexpr int CW = BN / Z;               // thread q takes columns [q CW, (q+1) CW)
+      float v[CW];
+#pragma unroll
+      for (int k = 0; k < CW; ++k) v[k] = 0.f;
+      const uint32_t la = smem_u32(red + rr * RS + q * CW);
+      for (int z = 0; z < Z; ++z) {
+        const uint32_t ra = dsmem_map(la, z);
+#pragma unroll
+        for (int k = 0; k < CW; k += 4) {
+          const float4 u = dsmem_ld_f4(ra + 4 * k);
+          v[k] += u.x; v[k + 1] += u.y; v[k + 2] += u.z; v[k + 3] += u.w;
+        }
+      }
+      if (ok && row < M) store_row_f32<EPI>(ep, row, n0 + q * CW, v, CW, N);
+    }
+    cluster_sync();   // the peers have finished reading this CTA's partial
   }
 
   tc_fence_before();
@@ -195,203 +279,278 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
-// grouped expert GEMMs (swap-AB)
+// grouped expert GEMMs (swap-AB), persistent and warp-specialised
 // ---------------------------------------------------------------------------------------------
+// Work items are (expert, 128-row weight tile) pairs, dealt round-robin to one CTA per SM; an item
+// with n tokens is n/64 accumulator chunks.  Warp 0 streams weight tiles and the chunk's activation
+// rows through a ring of shared-memory stages that runs on across items; warp 1 issues the MMAs
+// into one of two TMEM accumulators; warps 2-5 drain the other accumulator, so the epilogue of one
+// chunk overlaps the MMAs of the next.
 constexpr int kExpBN = 64;                         // tokens per accumulator chunk
-constexpr int kExpStages = 3;
+constexpr int kExpStages = 7;
+constexpr int kExpThreads = 192;                   // 6 warps
 constexpr uint32_t kExpBTile = kExpBN * 64 * 2;    // 8 KB: two 32-row boxes
 constexpr uint32_t kExpStageBytes = kATileBytes + kExpBTile;
 constexpr int kEpiStride = kExpBN + 1;             // padded fp32 staging rows
-constexpr size_t kExpSmemBytes = 1024 + (size_t)kExpStages * kExpStageBytes + 128 * kEpiStride * 4 + 256;
+constexpr size_t kExpSmemBytes = 1024 + (size_t)kExpStages * kExpStageBytes + 128 * kEpiStride * 4 + 512;
+
+struct ExpBarriers {
+  uint64_t full[kExpStages];
+  uint64_t empty[kExpStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_slot;
+};
+
+__device__ __forceinline__ void epi_bar_sync() {   // the 128 epilogue threads only (named barrier 1)
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 2)
+__global__ void __launch_bounds__(kExpThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                       ExpertParams p, int* err) {
+                       ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
-  const int e = blockIdx.y, mt = blockIdx.x;
-  const int n_e = p.counts[e];
-  if (n_e <= 0) return;
-  const int off = p.offsets[e];
+  pdl_trigger();
   uint8_t* tiles = align1024(smem_raw);
   float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kExpStages * kExpStageBytes);
-  GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(stage_out + 128 * kEpiStride);
+  ExpBarriers* bars = reinterpret_cast<ExpBarriers*>(stage_out + 128 * kEpiStride);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = MODE == 1 ? p.d : p.F;
   const int nk = K / 64;
+  const int MT = MODE == 1 ? p.F / 64 : p.d / 128;   // weight tiles per expert
+  const int n_items = n_exp * MT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kExpStages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->acc_full[b], 1);
+      mbar_init(&bars->acc_empty[b], 4);
+    }
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&bars->tmem_slot, kExpBN);
+  if (warp == 1) tmem_alloc(&bars->tmem_slot, 2 * kExpBN);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
-  const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
+  pdl_wait();   // the routing (offsets) and the activation rows come from the preceding kernels
 
-  uint32_t it = 0;   // ring position shared by producer and MMA issuer (both walk the same sequence)
-  int chunk = 0;
-  for (int c0 = 0; c0 < n_e; c0 += kExpBN, ++chunk) {
-    const int nc = min(kExpBN, n_e - c0);
-    const int nmma = (nc + 15) & ~15;
-    const int nb = (nc + 31) >> 5;
-    const uint32_t tx = kATileBytes + (uint32_t)nb * 4096u;
-    if (warp == 0 && lane == 0) {
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
-      for (int kb = 0; kb < nk; ++kb) {
-        const uint32_t i = it + kb;
-        const int s = i % kExpStages;
-        const uint32_t ph = (i / kExpStages) & 1;
-        if (!mbar_wait(&bars->empty[s], ph ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
-        uint8_t* a = tiles + (size_t)s * kExpStageBytes;
-        mbar_arrive_expect_tx(&bars->full[s], tx);
-        if (MODE == 1) {
-          const int r0 = e * 2 * p.F + mt * 64;
-          tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, r0, pol_w);               // gate rows
-          tma_load_2d_hint(&tmW, &bars->full[s], a + 8192, kb * 64, r0 + p.F, pol_w);  // up rows
-        } else {
-          tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, e * p.d + mt * 128, pol_w);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int e = item / MT, mt = item % MT;
+        const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
+        for (int c0 = 0; c0 < n_e && ok; c0 += kExpBN) {
+          const int nb = (min(kExpBN, n_e - c0) + 31) >> 5;
+          const uint32_t tx = kATileBytes + (uint32_t)nb * 4096u;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % kExpStages;
+            if (!mbar_wait(&bars->empty[s], ((it / kExpStages) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a = tiles + (size_t)s * kExpStageBytes;
+            mbar_arrive_expect_tx(&bars->full[s], tx);
+            if (MODE == 1) {
+              const int r0 = e * 2 * p.F + mt * 64;
+              tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, r0, pol_w);               // gate rows
+              tma_load_2d_hint(&tmW, &bars->full[s], a + 8192, kb * 64, r0 + p.F, pol_w);  // up rows
+            } else {
+              tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, e * p.d + mt * 128, pol_w);
+            }
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(&tmX, &bars->full[s], a + kATileBytes + b * 4096, kb * 64, off + c0 + 32 * b);
+          }
         }
-        for (int b = 0; b < nb; ++b)
-          tma_load_2d(&tmX, &bars->full[s], a + kATileBytes + b * 4096, kb * 64, off + c0 + 32 * b);
       }
-    } else if (warp == 1 && lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, nmma);
-      for (int kb = 0; kb < nk; ++kb) {
-        const uint32_t i = it + kb;
-        const int s = i % kExpStages;
-        const uint32_t ph = (i / kExpStages) & 1;
-        if (!mbar_wait(&bars->full[s], ph, err, DEV_ERR_TIMEOUT_MMA)) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      uint32_t it = 0, j = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int e = item / MT;
+        const int n_e = p.offsets[e + 1] - p.offsets[e];
+        for (int c0 = 0; c0 < n_e && ok; c0 += kExpBN, ++j) {
+          const int nmma = (min(kExpBN, n_e - c0) + 15) & ~15;
+          const uint32_t idesc = idesc_bf16_f32(128, nmma);
+          const uint32_t b = j & 1;
+          if (!mbar_wait(&bars->acc_empty[b], ((j >> 1) & 1) ^ 1, err, DEV_ERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t acc = tmem + b * kExpBN;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % kExpStages;
+            if (!mbar_wait(&bars->full[s], (it / kExpStages) & 1, err, DEV_ERR_TIMEOUT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t* a = tiles + (size_t)s * kExpStageBytes;
+            const uint64_t ad = smem_desc_sw128(smem_u32(a));
+            const uint64_t bd = smem_desc_sw128(smem_u32(a + kATileBytes));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(acc, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0);
+            umma_commit(&bars->empty[s]);
+          }
+          umma_commit(&bars->acc_full[b]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------ epilogue (warps 2-5) ------------------------------
+    const int quarter = warp & 3;                 // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int r = quarter * 32 + lane;            // accumulator row = weight row of the tile
+    const int et = threadIdx.x - 64;              // 0..127 among the epilogue threads
+    uint32_t j = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int e = item / MT, mt = item % MT;
+      const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
+      for (int c0 = 0; c0 < n_e; c0 += kExpBN, ++j) {
+        const int nc = min(kExpBN, n_e - c0);
+        const int nmma = (nc + 15) & ~15;
+        const uint32_t b = j & 1;
+        const bool ok = mbar_wait(&bars->acc_full[b], (j >> 1) & 1, err, DEV_ERR_TIMEOUT_EPILOGUE);
         tc_fence_after();
-        uint8_t* a = tiles + (size_t)s * kExpStageBytes;
-        const uint64_t ad = smem_desc_sw128(smem_u32(a));
-        const uint64_t bd = smem_desc_sw128(smem_u32(a + kATileBytes));
+        const uint32_t acc = tmem + ((uint32_t)(quarter * 32) << 16) + b * kExpBN;
+        if (MODE == 1) {
+          for (int cb = 0; cb < nmma; cb += 32) {
+            float v[32];
+            tmem_ld_32cols(acc + cb, v);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0);
-        umma_commit(&bars->empty[s]);
-      }
-      umma_commit(&bars->accum);
-    }
-    it += nk;
-    __syncwarp();
-
-    const bool ok = mbar_wait(&bars->accum, chunk & 1, err, DEV_ERR_TIMEOUT_EPILOGUE);
-    tc_fence_after();
-    if (MODE == 1) {
-      // stage the whole 128 x nmma accumulator (64 gate rows, then 64 up rows) in shared memory
-      const int r = warp * 32 + lane;
-      for (int cb = 0; cb < nmma; cb += 32) {
-        float v[32];
-        tmem_ld_32cols(tbase + cb, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) stage_out[r * kEpiStride + cb + i] = v[i];
-      }
-      __syncthreads();
-      if (ok) {
-        // thread -> (token n = tid/4 + 32*pass, features f = (tid%4)*16 .. +16)
-        const int fq = (threadIdx.x & 3) * 16;
-        for (int n = threadIdx.x >> 2; n < nc; n += 32) {
-          uint32_t packed[8];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float g0 = stage_out[(fq + i) * kEpiStride + n], u0 = stage_out[(64 + fq + i) * kEpiStride + n];
-            const float g1 = stage_out[(fq + i + 1) * kEpiStride + n],
-                        u1 = stage_out[(64 + fq + i + 1) * kEpiStride + n];
-            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
-            packed[i / 2] = pack_bf16x2(h0, h1);
+            for (int i = 0; i < 32; ++i) stage_out[r * kEpiStride + cb + i] = v[i];
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(off + c0 + n) * p.F + mt * 64 + fq);
-          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        }
-      }
-    } else {
-      const int m = mt * 128 + warp * 32 + lane;   // output feature of the down projection
-      for (int cb = 0; cb < nmma; cb += 32) {
-        float v[32];
-        tmem_ld_32cols(tbase + cb, v);
-        if (!ok) continue;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+          epi_bar_sync();
+          if (ok) {
+            // thread -> (token n = et/4 + 32*pass, features f = (et%4)*16 .. +16); gate rows 0-63, up rows 64-127
+            const int fq = (et & 3) * 16;
+            for (int n = et >> 2; n < nc; n += 32) {
+              uint32_t packed[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int n = cb + i;
-          if (n < nc) {
-            const int rowa = off + c0 + n;
-            p.y_out[(size_t)rowa * p.d + m] = v[i] * p.perm_gate[rowa];
+              for (int i = 0; i < 16; i += 2) {
+                const float g0 = stage_out[(fq + i) * kEpiStride + n], u0 = stage_out[(64 + fq + i) * kEpiStride + n];
+                const float g1 = stage_out[(fq + i + 1) * kEpiStride + n],
+                            u1 = stage_out[(64 + fq + i + 1) * kEpiStride + n];
+                packed[i / 2] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(off + c0 + n) * p.F + mt * 64 + fq);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+          }
+          epi_bar_sync();   // the staging buffer is rewritten by the next chunk
+        } else {
+          const int m = mt * 128 + r;             // output feature of the down projection
+          for (int cb = 0; cb < nmma; cb += 32) {
+            float v[32];
+            tmem_ld_32cols(acc + cb, v);
+            if (cb + 32 >= nmma) {                // last TMEM read of this accumulator: release it
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+            }
+            if (!ok) continue;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int n = cb + i;
+              if (n < nc) {
+                const int rowa = off + c0 + n;
+                p.y_out[(size_t)rowa * p.d + m] = v[i] * p.perm_gate[rowa];
+              }
+            }
           }
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kExpBN);
+  if (warp == 1) tmem_dealloc(tmem, 2 * kExpBN);
 }
 
 // ---------------------------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------------------------
-template <int BN, int EPI>
+template <int BN, int EPI, int Z>
 static cudaError_t launch_dense(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
                                 int* err, cudaStream_t st) {
   using C = DenseCfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(dense_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(dense_gemm_kernel<BN, EPI, Z>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1/shared storage as shared memory, so kMinBlocks CTAs fit on an SM
+    e = cudaFuncSetAttribute(dense_gemm_kernel<BN, EPI, Z>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((M + 127) / 128, (N + BN - 1) / BN);
-  dense_gemm_kernel<BN, EPI><<<grid, kGemmThreads, C::kSmemBytes, st>>>(a, b, M, N, K, ep, err);
-  return cudaGetLastError();
+  return launch_k(dense_gemm_kernel<BN, EPI, Z>, dim3((M + 127) / 128, (N + BN - 1) / BN, Z), dim3(kGemmThreads),
+                  C::kSmemBytes, st, Z, a, b, M, N, K, ep, err);
 }
 
 cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const EpiParams& ep, int* err, cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if (K % 64 != 0) return cudaErrorInvalidValue;
-#define DG_DENSE_CASE(BN_, EPI_) \
-  if (bn == BN_ && epi == EPI_) return launch_dense<BN_, EPI_>(a, b, M, N, K, ep, err, st);
-  DG_DENSE_CASE(128, EPI_QKV)
-  DG_DENSE_CASE(64, EPI_RESID)
-  DG_DENSE_CASE(128, EPI_RESID)
-  DG_DENSE_CASE(128, EPI_F32)
-  DG_DENSE_CASE(256, EPI_F32)
-  DG_DENSE_CASE(64, EPI_F32)
+  const int z = ep.k_splits > 1 ? ep.k_splits : 1;
+  if (z > K / 64) return cudaErrorInvalidValue;
+#define DG_DENSE_CASE(BN_, EPI_, Z_) \
+  if (bn == BN_ && epi == EPI_ && z == Z_) return launch_dense<BN_, EPI_, Z_>(a, b, M, N, K, ep, err, st);
+  DG_DENSE_CASE(128, EPI_QKV, 1)
+  DG_DENSE_CASE(128, EPI_QKV, 2)
+  DG_DENSE_CASE(128, EPI_QKV, 4)
+  DG_DENSE_CASE(128, EPI_QKV, 8)
+  DG_DENSE_CASE(128, EPI_RESID, 1)
+  DG_DENSE_CASE(128, EPI_RESID, 2)
+  DG_DENSE_CASE(128, EPI_RESID, 4)
+  DG_DENSE_CASE(128, EPI_RESID, 8)
+  DG_DENSE_CASE(128, EPI_F32, 1)
+  DG_DENSE_CASE(128, EPI_F32, 2)
+  DG_DENSE_CASE(128, EPI_F32, 4)
+  DG_DENSE_CASE(128, EPI_F32, 8)
+  DG_DENSE_CASE(256, EPI_F32, 1)
 #undef DG_DENSE_CASE
   return cudaErrorInvalidValue;
 }
 
 template <int MODE>
 static cudaError_t launch_expert(const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
-                                 int* err, cudaStream_t st) {
+                                 int n_ctas, int* err, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kExpSmemBytes);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(expert_gemm_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(MODE == 1 ? p.F / 64 : p.d / 128, n_exp);
-  expert_gemm_kernel<MODE><<<grid, kGemmThreads, kExpSmemBytes, st>>>(w, x, p, err);
-  return cudaGetLastError();
+  const int items = n_exp * (MODE == 1 ? p.F / 64 : p.d / 128);
+  return launch_k(expert_gemm_kernel<MODE>, dim3(n_ctas < items ? n_ctas : items), dim3(kExpThreads), kExpSmemBytes,
+                  st, 1, w, x, p, n_exp, err);
 }
 
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
-                        int* err, cudaStream_t st) {
-  return mode == 1 ? launch_expert<1>(w, x, p, n_exp, err, st) : launch_expert<2>(w, x, p, n_exp, err, st);
+                        int n_ctas, int* err, cudaStream_t st) {
+  return mode == 1 ? launch_expert<1>(w, x, p, n_exp, n_ctas, err, st)
+                   : launch_expert<2>(w, x, p, n_exp, n_ctas, err, st);
 }
 
 }  // namespace dg

@@ -28,7 +28,11 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
 
 // x[r][:] = emb[ids[r]][:] (bf16 -> fp32).  Out-of-range ids read row 0 and raise DEV_ERR_BAD_INDEX.
 __global__ void embed_kernel(const __nv_bfloat16* __restrict__ emb, const int32_t* __restrict__ ids, int d, int vocab,
-                             float* __restrict__ x, int* err) {
+                             float* __restrict__ x, int* err, const float* __restrict__ g, float eps,
+                             __nv_bfloat16* __restrict__ xn) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[32];
   const int r = blockIdx.x;
   int id = ids[r];
   if (id < 0 || id >= vocab) {
@@ -45,11 +49,29 @@ __global__ void embed_kernel(const __nv_bfloat16* __restrict__ emb, const int32_
     dst[2 * c] = make_float4(f0.x, f0.y, f1.x, f1.y);
     dst[2 * c + 1] = make_float4(f2.x, f2.y, f3.x, f3.y);
   }
+  if (!g) return;
+  // the first layer's RMSNorm of the embedded row (the row was written by other threads of the block)
+  __syncthreads();
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = dst[c];
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = block_sum_256(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  uint2* o2 = reinterpret_cast<uint2*>(xn + (size_t)r * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = dst[c], w = g4[c];
+    o2[c] = make_uint2(pack_bf16x2(v.x * inv * w.x, v.y * inv * w.y), pack_bf16x2(v.z * inv * w.z, v.w * inv * w.w));
+  }
 }
 
 // out[r] = bf16( x[r] / sqrt(mean(x[r]^2) + eps) * g )
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
                                __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * d);
@@ -70,6 +92,8 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
 
 // (cos, sin) of pos * theta^(-2i/dh) for i < dh/2, computed in double and rounded to fp32.
 __global__ void rope_table_kernel(float2* table, int dh, double theta) {
+  pdl_trigger();
+  pdl_wait();
   const int pos = blockIdx.x, i = threadIdx.x;
   const double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)dh);
   double s, c;
@@ -79,19 +103,40 @@ __global__ void rope_table_kernel(float2* table, int dh, double theta) {
 
 // One warp per row: the top_k largest router logits (ties -> lower expert id), gates = softmax over
 // the selected logits; per-expert counts accumulate with integer atomics (order-free, exact).
-__global__ void router_topk_kernel(const float* __restrict__ logits, int n_rows, int n_exp, int top_k,
-                                   int32_t* __restrict__ sel, float* __restrict__ gate, int32_t* __restrict__ counts) {
+// The router logits arrive as n_parts split-K partial planes (part_stride apart), summed here in
+// plane order.  Lane l owns experts [l*V, l*V + V), V = ceil(E/32) <= 8.
+template <int V>
+__global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts, size_t part_stride, int n_rows,
+                                   int n_exp, int top_k, int32_t* __restrict__ sel, float* __restrict__ gate,
+                                   int32_t* __restrict__ counts) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= n_rows) return;
-  constexpr int kPer = 8;   // up to 256 experts
-  float v[kPer];
-  const float* lr = logits + (size_t)row * n_exp;
+  float v[V];
+  const float* lr = logits + (size_t)row * n_exp + lane * V;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = i * 32 + lane;
-    v[i] = e < n_exp ? lr[e] : -INFINITY;
+  for (int i = 0; i < V; ++i) v[i] = 0.f;
+  bool done = false;
+  if constexpr (V == 4) {
+    if ((n_exp % 4) == 0 && lane * V < n_exp) {
+      for (int z = 0; z < n_parts; ++z) {
+        const float4 q = __ldcg(reinterpret_cast<const float4*>(lr + z * part_stride));
+        v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
+      }
+      done = true;
+    }
   }
+  if (!done) {
+    for (int z = 0; z < n_parts; ++z)
+#pragma unroll
+      for (int i = 0; i < V; ++i)
+        if (lane * V + i < n_exp) v[i] += lr[z * part_stride + i];
+  }
+#pragma unroll
+  for (int i = 0; i < V; ++i)
+    if (lane * V + i >= n_exp) v[i] = -INFINITY;
   uint32_t taken = 0;
   float first = 0.f, denom = 0.f, my_v = 0.f;
   int my_e = 0;
@@ -99,8 +144,8 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_rows,
     float bv = -INFINITY;
     int be = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = i * 32 + lane;
+    for (int i = 0; i < V; ++i) {
+      const int e = lane * V + i;
       if (e < n_exp && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
         bv = v[i];
         be = e;
@@ -115,7 +160,7 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_rows,
         be = oe;
       }
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (be / V == lane) taken |= 1u << (be % V);
     if (k == 0) first = bv;
     if (k == lane) {
       my_v = bv;
@@ -130,76 +175,136 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_rows,
   }
 }
 
-// One CTA per expert: stable bucketing of the (token, rank) assignments routed to expert e (token
-// order kept), then the gather of their normalised activation rows into the bucketed buffer.
-__global__ void bucket_gather_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate,
-                                     const int32_t* __restrict__ counts, int n_assign, int top_k, int n_exp,
-                                     const __nv_bfloat16* __restrict__ xn, int d, int32_t* __restrict__ offsets,
-                                     float* __restrict__ perm_gate, int32_t* __restrict__ perm_tok,
-                                     int32_t* __restrict__ slot, __nv_bfloat16* __restrict__ xp) {
-  __shared__ int warp_cnt[32];
-  __shared__ int s_off;
-  const int e = blockIdx.x;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  if (threadIdx.x == 0) {
-    int o = 0;
-    for (int i = 0; i < e; ++i) o += counts[i];
-    s_off = o;
-    offsets[e] = o;
-    if (e == n_exp - 1) offsets[n_exp] = o + counts[e];
+// One CTA: expert offsets (exclusive prefix sum of the counts) and a row of the bucketed layout for
+// every (token, rank) assignment.  Rows inside an expert are handed out with shared-memory atomics,
+// so their order varies between runs; no result depends on it (each expert-GEMM column reads only
+// its own row, and the combine sums a token's rows in rank order).
+__global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate,
+                                   const int32_t* __restrict__ counts, int n_assign, int top_k, int n_exp,
+                                   int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
+                                   int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_off[257];
+  __shared__ int s_cur[256];
+  __shared__ int s_wsum[8];
+  // exclusive prefix sum of the counts by the first 256 threads (warp scans, then the warp totals)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (threadIdx.x < 256) {
+    const int c = threadIdx.x < n_exp ? counts[threadIdx.x] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[w] = incl;
+    s_off[threadIdx.x] = incl - c;
+    s_cur[threadIdx.x] = 0;
   }
   __syncthreads();
-  const int off = s_off;
-  int running = 0;
-  for (int base = 0; base < n_assign; base += blockDim.x) {
-    const int a = base + threadIdx.x;
-    const bool flag = a < n_assign && sel[a] == e;
-    const uint32_t mask = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) warp_cnt[w] = __popc(mask);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int i = 0; i < nw; ++i) {
-      before += i < w ? warp_cnt[i] : 0;
-      total += warp_cnt[i];
-    }
-    if (flag) {
-      const int row = off + running + before + __popc(mask & ((1u << lane) - 1u));
-      perm_gate[row] = gate[a];
-      perm_tok[row] = a / top_k;
-      slot[a] = row;
-    }
-    running += total;
-    __syncthreads();
+  // the counts are consumed: clear them for the next layer's router (no separate memset)
+  if (threadIdx.x < n_exp) const_cast<int32_t*>(counts)[threadIdx.x] = 0;
+  if (threadIdx.x < 256) {
+    int base = 0;
+    for (int i = 0; i < w; ++i) base += s_wsum[i];
+    s_off[threadIdx.x] += base;
   }
-  const int cnt = counts[e];
-  for (int r = off + w; r < off + cnt; r += nw) {
-    const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)perm_tok[r] * d);
-    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
-    for (int c = lane; c < d / 8; c += 32) dst[c] = src[c];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int i = 0; i < 8; ++i) tot += s_wsum[i];
+    s_off[n_exp] = tot;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= n_exp; e += blockDim.x) offsets[e] = s_off[e];
+  for (int a = threadIdx.x; a < n_assign; a += blockDim.x) {
+    const int e = sel[a];
+    const int row = s_off[e] + atomicAdd(&s_cur[e], 1);
+    perm_gate[row] = gate[a];
+    perm_tok[row] = a / top_k;
+    slot[a] = row;
   }
 }
 
-// x[t] += sum over ranks r (in rank order) of y[slot[t*k + r]]
+// xp[slot[t*k + r]] = xn[t] for every rank r: one warp per token reads the row once.
+__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const int32_t* __restrict__ slot, int n_rows,
+                                   int top_k, int d, __nv_bfloat16* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= n_rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
+  const int n16 = d / 8;   // 16-byte chunks per row
+  for (int c0 = 0; c0 < n16; c0 += 32 * 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < n16) v[u] = src[c];
+    }
+    for (int r = 0; r < top_k; ++r) {
+      uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)slot[(size_t)t * top_k + r] * d);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n16) dst[c] = v[u];
+      }
+    }
+  }
+}
+
+// x[t] += sum over ranks r (in rank order) of y[slot[t*k + r]]; with g != nullptr also the next
+// RMSNorm of the updated row: xn[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g).
 __global__ void moe_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot, int top_k, int d,
-                                   float* __restrict__ x) {
+                                   float* __restrict__ x, const float* __restrict__ g, float eps,
+                                   __nv_bfloat16* __restrict__ xn) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   __shared__ int rows[32];
+  __shared__ float red[32];
   if (threadIdx.x < top_k) rows[threadIdx.x] = slot[(size_t)t * top_k + threadIdx.x];
   __syncthreads();
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
+  float ss = 0.f;
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r = 0; r < top_k; ++r) {
-      const float4 v = reinterpret_cast<const float4*>(y + (size_t)rows[r] * d)[c];
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(y + (size_t)rows[r] * d) + c);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     float4 o = xr[c];
     o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
     xr[c] = o;
+    ss += o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+  }
+  if (!g) return;
+  ss = block_sum_256(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  uint2* o2 = reinterpret_cast<uint2*>(xn + (size_t)t * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = xr[c], w = g4[c];
+    o2[c] = make_uint2(pack_bf16x2(v.x * inv * w.x, v.y * inv * w.y), pack_bf16x2(v.z * inv * w.z, v.w * inv * w.w));
   }
 }
 
+// out[i] = sum over planes z (in order) of in[z * stride + i]
+__global__ void sum_planes_kernel(float* __restrict__ out, const float* __restrict__ in, int n_planes, size_t stride,
+                                  size_t n) {
+  pdl_trigger();
+  pdl_wait();
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int z = 0; z < n_planes; ++z) acc += in[z * stride + i];
+  out[i] = acc;
+}
+
 __global__ void add_to_P_kernel(int* seq_P, int first, int count, int delta) {
+  pdl_trigger();
+  pdl_wait();
   const int i = threadIdx.x + blockIdx.x * blockDim.x;
   if (i < count) seq_P[first + i] += delta;
 }
@@ -209,6 +314,8 @@ __global__ void add_to_P_kernel(int* seq_P, int first, int count, int delta) {
 __global__ void load_prefix_kernel(const __nv_bfloat16* __restrict__ k_in, const __nv_bfloat16* __restrict__ v_in,
                                    int n_kv, int dh, int max_ctx, __nv_bfloat16* __restrict__ kc,
                                    __nv_bfloat16* __restrict__ vt) {
+  pdl_trigger();
+  pdl_wait();
   const int pos = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
   const size_t src = ((size_t)pos * n_kv + h) * dh + c;
   kc[((size_t)h * max_ctx + pos) * dh + c] = k_in[src];
@@ -218,6 +325,8 @@ __global__ void load_prefix_kernel(const __nv_bfloat16* __restrict__ k_in, const
 // Uniform random placeholder ids (uniform-state start of a canvas), commit mask cleared.
 __global__ void canvas_init_kernel(const int* __restrict__ seq_P, int canvas, uint64_t seed, int vocab,
                                    int32_t* __restrict__ ids, uint8_t* __restrict__ commit) {
+  pdl_trigger();
+  pdl_wait();
   const int seq = blockIdx.x;
   const int P = seq_P ? seq_P[seq] : 0;
   for (int j = threadIdx.x; j < canvas; j += blockDim.x) {
@@ -229,54 +338,64 @@ __global__ void canvas_init_kernel(const int* __restrict__ seq_P, int canvas, ui
 
 // ---------------------------------------------------------------------------------------------
 cudaError_t embed_rows(const __nv_bfloat16* emb, const int32_t* ids, int n_rows, int d, int vocab, float* x, int* err,
-                       cudaStream_t st) {
+                       const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  embed_kernel<<<n_rows, 256, 0, st>>>(emb, ids, d, vocab, x, err);
-  return cudaGetLastError();
+  return launch_k(embed_kernel, dim3(n_rows), dim3(256), 0, st, 1, emb, ids, d, vocab, x, err, g, eps, xn);
 }
 cudaError_t rmsnorm_rows(const float* x, const float* g, int n_rows, int d, float eps, __nv_bfloat16* out,
                          cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  rmsnorm_kernel<<<n_rows, 256, 0, st>>>(x, g, d, eps, out);
-  return cudaGetLastError();
+  return launch_k(rmsnorm_kernel, dim3(n_rows), dim3(256), 0, st, 1, x, g, d, eps, out);
 }
 cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st) {
-  rope_table_kernel<<<max_ctx, dh / 2, 0, st>>>(table, dh, (double)theta);
-  return cudaGetLastError();
+  return launch_k(rope_table_kernel, dim3(max_ctx), dim3(dh / 2), 0, st, 1, table, dh, (double)theta);
 }
-cudaError_t router_topk(const float* logits, int n_rows, int n_exp, int top_k, int32_t* sel, float* gate,
-                        int32_t* counts, cudaStream_t st) {
+cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
+                        int32_t* sel, float* gate, int32_t* counts, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  router_topk_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(logits, n_rows, n_exp, top_k, sel, gate, counts);
-  return cudaGetLastError();
+  const int V = (n_exp + 31) / 32;
+  const dim3 grid((n_rows + 7) / 8);
+#define DG_TOPK_CASE(V_) \
+  if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts);
+  DG_TOPK_CASE(1)
+  DG_TOPK_CASE(2)
+  DG_TOPK_CASE(4)
+  DG_TOPK_CASE(8)
+#undef DG_TOPK_CASE
+  return launch_k(router_topk_kernel<8>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k,
+                  sel, gate, counts);
 }
-cudaError_t bucket_gather(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k,
-                          int n_exp, const __nv_bfloat16* xn, int d, int32_t* offsets, float* perm_gate,
-                          int32_t* perm_tok, int32_t* slot, __nv_bfloat16* xp, cudaStream_t st) {
-  bucket_gather_kernel<<<n_exp, 256, 0, st>>>(sel, gate, counts, n_rows * top_k, top_k, n_exp, xn, d, offsets,
-                                              perm_gate, perm_tok, slot, xp);
-  return cudaGetLastError();
+cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k, int n_exp,
+                        int32_t* offsets, float* perm_gate, int32_t* perm_tok, int32_t* slot, cudaStream_t st) {
+  if (n_exp > 256) return cudaErrorInvalidValue;
+  return launch_k(assign_rows_kernel, dim3(1), dim3(1024), 0, st, 1, sel, gate, counts, n_rows * top_k, top_k, n_exp,
+                  offsets, perm_gate, perm_tok, slot);
 }
-cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x,
+cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  moe_combine_kernel<<<n_rows, 256, 0, st>>>(y, slot, top_k, d, x);
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3((n_rows + 7) / 8), dim3(256), 0, st, 1, xn, slot, n_rows, top_k, d, xp);
+}
+cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x, const float* g,
+                        float eps, __nv_bfloat16* xn, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  return launch_k(moe_combine_kernel, dim3(n_rows), dim3(256), 0, st, 1, y, slot, top_k, d, x, g, eps, xn);
+}
+cudaError_t sum_planes(float* out, const float* in, int n_planes, size_t stride, size_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  return launch_k(sum_planes_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, 1, out, in, n_planes, stride, n);
 }
 cudaError_t add_to_P(int* seq_P, int first, int count, int delta, cudaStream_t st) {
-  add_to_P_kernel<<<(count + 127) / 128, 128, 0, st>>>(seq_P, first, count, delta);
-  return cudaGetLastError();
+  return launch_k(add_to_P_kernel, dim3((count + 127) / 128), dim3(128), 0, st, 1, seq_P, first, count, delta);
 }
 cudaError_t load_prefix(const __nv_bfloat16* k_in, const __nv_bfloat16* v_in, int P, int n_kv, int dh, int max_ctx,
                         __nv_bfloat16* kc, __nv_bfloat16* vt, cudaStream_t st) {
   if (P <= 0) return cudaSuccess;
-  load_prefix_kernel<<<dim3(P, n_kv), dh, 0, st>>>(k_in, v_in, n_kv, dh, max_ctx, kc, vt);
-  return cudaGetLastError();
+  return launch_k(load_prefix_kernel, dim3(P, n_kv), dim3(dh), 0, st, 1, k_in, v_in, n_kv, dh, max_ctx, kc, vt);
 }
 cudaError_t canvas_init_ids(const int* seq_P, int n_seq, int canvas, uint64_t seed, int vocab, int32_t* ids,
                             uint8_t* commit, cudaStream_t st) {
-  canvas_init_kernel<<<n_seq, 256, 0, st>>>(seq_P, canvas, seed, vocab, ids, commit);
-  return cudaGetLastError();
+  return launch_k(canvas_init_kernel, dim3(n_seq), dim3(256), 0, st, 1, seq_P, canvas, seed, vocab, ids, commit);
 }
 
 }  // namespace dg

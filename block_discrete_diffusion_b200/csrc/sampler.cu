@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kSampThreads)
     sampler_partial_kernel(const float* __restrict__ logits, int canvas, int vocab, int n_chunks,
                            const int* __restrict__ seq_P, const uint8_t* __restrict__ commit_in, float inv_temp,
                            uint64_t seed, int step, float* __restrict__ partial) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.y, chunk = blockIdx.x;
   if (commit_in[row]) return;
   const int seq = row / canvas, j = row % canvas;
@@ -163,6 +165,8 @@ __global__ void __launch_bounds__(kSampThreads)
 }
 
 __global__ void sampler_finalize_kernel(SamplerArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red_h[32];
   __shared__ int red_c[32];
   const int seq = blockIdx.x;
@@ -258,12 +262,10 @@ int sampler_chunks(int vocab) {
 cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st) {
   if (a.canvas > 4 * 256 || a.vocab % (4 * a.n_chunks) != 0) return cudaErrorInvalidValue;
   dim3 grid(a.n_chunks, a.n_seq * a.canvas);
-  sampler_partial_kernel<<<grid, kSampThreads, 0, st>>>(a.logits, a.canvas, a.vocab, a.n_chunks, a.seq_P, a.commit_in,
-                                                        a.inv_temp, a.seed, a.step, a.partial);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_k(sampler_partial_kernel, grid, dim3(kSampThreads), 0, st, 1, a.logits, a.canvas, a.vocab,
+                           a.n_chunks, a.seq_P, a.commit_in, a.inv_temp, a.seed, a.step, a.partial);
   if (e != cudaSuccess) return e;
-  sampler_finalize_kernel<<<a.n_seq, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_k(sampler_finalize_kernel, dim3(a.n_seq), dim3(256), 0, st, 1, a);
 }
 
 }  // namespace dg

@@ -379,12 +379,14 @@ class Sequence:
                 self.v[l][:P] = _f64(_as_float(prefix_v[l]))
             self.P = P
 
-    def prefill(self, ids):
+    def prefill(self, ids, want_router=False):
+        """Returns the router logits [L][n][E] of the prompt rows when want_router."""
         n = len(ids)
         assert self.P + n <= self.max_ctx
-        forward(self.model, ids, np.arange(self.P, self.P + n), self.P, self.k, self.v, causal=True,
-                write_cache=True, want_logits=False)
+        fw = forward(self.model, ids, np.arange(self.P, self.P + n), self.P, self.k, self.v, causal=True,
+                     write_cache=True, want_router=want_router, want_logits=False)
         self.P += n
+        return fw["router"]
 
     def canvas_init(self, prm: SamplerParams):
         self.step = 0
@@ -406,12 +408,14 @@ class Sequence:
         self.step += 1
         return out
 
-    def block_commit(self, ids):
+    def block_commit(self, ids, want_router=False):
+        """Returns the router logits [L][256][E] of the commit pass when want_router."""
         n = len(ids)
         assert self.P + n <= self.max_ctx
-        forward(self.model, ids, np.arange(self.P, self.P + n), self.P, self.k, self.v, causal=False,
-                write_cache=True, want_logits=False)
+        fw = forward(self.model, ids, np.arange(self.P, self.P + n), self.P, self.k, self.v, causal=False,
+                     write_cache=True, want_router=want_router, want_logits=False)
         self.P += n
+        return fw["router"]
 
     def decode(self, prm: SamplerParams, max_blocks: int):
         out = []

@@ -12,7 +12,8 @@ import torch
 
 import oracle
 import synthetic
-from dg_testutil import (ENTROPY_TOL, HIDDEN_TOL, judge_step, kv_views, rel_err, router_tie_tokens, to_device)
+from dg_testutil import (ENTROPY_TOL, HIDDEN_TOL, derived_tolerances, judge_step, kv_views, rel_err,
+                         router_tie_tokens, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -131,8 +132,14 @@ def _layer_case(dg, cfg, P, seed, router_std=None):
     return w, model, seqs, ks, vs, x
 
 
-@pytest.mark.parametrize("cfg_name,P", [("tiny", 0), ("tiny", 128), ("tiny", 300), ("one_layer", 4096)])
-def test_layer_matches_oracle(dg, cfg_name, P):
+@pytest.mark.parametrize("cfg_name,P,n_rows,causal", [
+    ("tiny", 0, 256, False), ("tiny", 128, 256, False), ("tiny", 300, 256, False),
+    ("tiny", 0, 44, True), ("tiny", 256, 128, True), ("tiny", 200, 56, True), ("tiny", 384, 256, True),
+    ("one_layer", 4096, 256, False), ("one_layer", 2048, 200, True),
+])
+def test_layer_matches_oracle(dg, cfg_name, P, n_rows, causal):
+    """One layer (attention block, then MoE block) on canvas rows (bidirectional) or on a prefill
+    chunk (causal, ragged row counts), against a committed prefix of P positions."""
     if cfg_name == "tiny":
         cfg, router_std = synthetic.TINY, None
     else:
@@ -141,27 +148,31 @@ def test_layer_matches_oracle(dg, cfg_name, P):
         router_std = cfg.d_model ** -0.5                            # router logits ~ N(0, 1)
     w, model, seqs, ks, vs, x = _layer_case(dg, cfg, P, 11, router_std)
     xd = x.cuda()
-    mid = torch.empty_like(xd)
-    rl = torch.empty(256, cfg.n_exp, device="cuda")
-    dg.dg_layer_forward(seqs, 0, xd, mid, rl)
+    mid = torch.zeros_like(xd)
+    rl = torch.zeros(256, cfg.n_exp, device="cuda")
+    dg.dg_layer_forward(seqs, 0, xd, mid, rl, n_rows=n_rows, causal=causal)
     torch.cuda.synchronize()
     assert dg.dg_device_error(seqs) == 0
+    n = n_rows
     M = oracle.Model(cfg, w)
     kc = ks[0].double().numpy() if P else None
     vc = vs[0].double().numpy() if P else None
-    xo, kn, vn, rlo, mido = oracle.layer_forward(M, 0, x.double().numpy(), np.arange(P, P + 256), P, kc, vc,
-                                                 want_mid=True)
-    e_mid = rel_err(mid.cpu().numpy(), mido)
+    xo, kn, vn, rlo, mido = oracle.layer_forward(M, 0, x[:n].double().numpy(), np.arange(P, P + n), P, kc, vc,
+                                                 causal=causal, want_mid=True)
+    e_mid = rel_err(mid.cpu().numpy()[:n], mido)
     assert e_mid <= HIDDEN_TOL, f"attention block rel err {e_mid}"
-    e_rl = rel_err(rl.cpu().numpy(), rlo)
+    e_rl = rel_err(rl.cpu().numpy()[:n], rlo)
     assert e_rl <= HIDDEN_TOL, f"router logits rel err {e_rl}"
     keep = ~router_tie_tokens(rlo, cfg.top_k)
-    e_out = rel_err(xd.cpu().numpy()[keep], xo[keep])
+    e_out = rel_err(xd.cpu().numpy()[:n][keep], xo[keep])
     assert e_out <= HIDDEN_TOL, f"layer output rel err {e_out} ({keep.sum()} tokens judged)"
-    # the canvas rows' K/V went to cache rows [P, P+256); the prefix rows are unchanged
+    # rows beyond n_rows are not touched
+    if n < 256:
+        assert torch.equal(xd[n:].cpu(), x[n:])
+    # the rows' K/V went to cache rows [P, P+n); the prefix rows are unchanged
     K, Vt = kv_views(seqs.kv, cfg, 1, seqs.max_ctx)
-    Kg = K[0, 0, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
-    Vg = Vt[0, 0, :, :, P:P + 256].permute(2, 0, 1).float().cpu().numpy()
+    Kg = K[0, 0, :, P:P + n].permute(1, 0, 2).float().cpu().numpy()
+    Vg = Vt[0, 0, :, :, P:P + n].permute(2, 0, 1).float().cpu().numpy()
     assert rel_err(Kg, kn) <= HIDDEN_TOL and rel_err(Vg, vn) <= HIDDEN_TOL
     if P:
         assert torch.equal(K[0, 0, :, :P].permute(1, 0, 2).cpu(), ks[0])
@@ -172,29 +183,45 @@ def test_layer_matches_oracle(dg, cfg_name, P):
 # full tiny model: prefill, canvas steps (resynchronised to the oracle), block commit, decode
 # ------------------------------------------------------------------------------------------------
 
-def _tiny_model_pair(dg, head_scale=1.0, seed=0):
-    cfg = synthetic.TINY
-    w = synthetic.make_model_weights(cfg, seed, head_scale=head_scale)
+def _tiny_model_pair(dg, head_scale=1.0, seed=0, top_k=None):
+    import dataclasses
+    cfg = synthetic.TINY if top_k is None else dataclasses.replace(synthetic.TINY, top_k=top_k)
+    # with a routing decision (top_k < E) the router gets unit-variance logits (std d^-1/2): wider
+    # top-k margins, fewer near-tie tokens to exclude
+    router_std = cfg.d_model ** -0.5 if cfg.top_k < cfg.n_exp else None
+    w = synthetic.make_model_weights(cfg, seed, head_scale=head_scale, router_std=router_std)
     model = dg.dg_model_create(cfg, to_device(w))
     return cfg, w, model, oracle.Model(cfg, w)
 
 
-@pytest.mark.parametrize("head_scale,prompt_len,n_steps", [(1.0, 128, 4), (50.0, 128, 48), (50.0, 300, 6)])
-def test_canvas_steps_match_oracle(dg, head_scale, prompt_len, n_steps):
-    cfg, w, model, M = _tiny_model_pair(dg, head_scale)
+def _cache_rows(seqs, cfg, max_ctx, l, a, b):
+    K, Vt = kv_views(seqs.kv, cfg, 1, max_ctx)
+    kg = K[l, 0, :, a:b].permute(1, 0, 2).float().cpu().numpy()
+    vg = Vt[l, 0, :, :, a:b].permute(2, 0, 1).float().cpu().numpy()
+    return kg, vg
+
+
+# top_k = E (8 of 8 experts): the step has no routing decision, so every step and token is judged
+# with the spec tolerances (small head) or the derived large-logit tolerances (head x50, where rows
+# commit).  top_k = 2: tokens with router near-ties are excluded, and steps with a near-tie before
+# the last layer are not judged (see the loop).
+@pytest.mark.parametrize("top_k,head_scale,prompt_len,n_steps", [
+    (8, 1.0, 128, 4), (8, 1.0, 300, 3), (8, 50.0, 128, 48), (8, 50.0, 300, 6),
+    (2, 1.0, 128, 12), (2, 50.0, 300, 48),
+])
+def test_canvas_steps_match_oracle(dg, top_k, head_scale, prompt_len, n_steps):
+    cfg, w, model, M = _tiny_model_pair(dg, head_scale, top_k=top_k)
+    dense_routing = top_k == cfg.n_exp
     max_ctx = 1024
     seqs = dg.dg_seqs_create(model, 1, max_ctx)
     prompt = synthetic.make_ids(prompt_len, cfg.vocab, 0)
     dg.dg_prefill(seqs, prompt.cuda(), [prompt_len])
     oseq = oracle.Sequence(M, max_ctx)
-    oseq.prefill(prompt.numpy())
-    # prefill K/V match
-    K, Vt = kv_views(seqs.kv, cfg, 1, max_ctx)
+    tie = router_tie_tokens(oseq.prefill(prompt.numpy(), want_router=True), cfg.top_k)
     for l in range(cfg.n_layers):
-        kg = K[l, 0, :, :prompt_len].permute(1, 0, 2).float().cpu().numpy()
-        vg = Vt[l, 0, :, :, :prompt_len].permute(2, 0, 1).float().cpu().numpy()
-        assert rel_err(kg, oseq.k[l][:prompt_len]) <= HIDDEN_TOL, f"prefill K layer {l}"
-        assert rel_err(vg, oseq.v[l][:prompt_len]) <= HIDDEN_TOL, f"prefill V layer {l}"
+        kg, vg = _cache_rows(seqs, cfg, max_ctx, l, 0, prompt_len)
+        assert rel_err(kg[~tie], oseq.k[l][:prompt_len][~tie]) <= HIDDEN_TOL, f"prefill K layer {l}"
+        assert rel_err(vg[~tie], oseq.v[l][:prompt_len][~tie]) <= HIDDEN_TOL, f"prefill V layer {l}"
 
     prm = dg.sampler_params(cfg.vocab, seed=0)
     prm_o = oracle.SamplerParams(cfg.vocab, seed=0)
@@ -210,8 +237,8 @@ def test_canvas_steps_match_oracle(dg, head_scale, prompt_len, n_steps):
     hidden = torch.empty(cfg.n_layers + 1, 256, cfg.d_model, device="cuda")
     logits = torch.empty(256, cfg.vocab, device="cuda")
     prefix_before = seqs.kv.clone()
-    n_cache = cfg.n_layers * cfg.n_kv * max_ctx * cfg.d_head
-    total_judged = 0
+    total_judged, clean_steps = 0, 0
+    commits_seen = 0
     for s in range(n_steps):
         # resynchronise: the GPU starts each step from the oracle's state
         ids.copy_(torch.from_numpy(oids))
@@ -219,42 +246,62 @@ def test_canvas_steps_match_oracle(dg, head_scale, prompt_len, n_steps):
         dg.dg_canvas_step(seqs, prm, ids, commit, H, stop, hidden, logits)
         torch.cuda.synchronize()
         r = oseq.canvas_step(prm_o, oids, ocommit, want_hidden=True, want_router=True)
-        keep = ~router_tie_tokens(r["router"], cfg.top_k)
-        hg = hidden.cpu().numpy()
-        for l in range(cfg.n_layers + 1):
-            e = rel_err(hg[l][keep], r["hidden"][l][keep])
-            assert e <= HIDDEN_TOL, f"step {s} hidden {l} rel err {e}"
-        el = rel_err(logits.cpu().numpy()[keep], r["logits"][keep])
-        assert el <= HIDDEN_TOL, f"step {s} logits rel err {el}"
-        g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(), "stop": int(stop.item())}
-        fails, judged = judge_step(g, r, prm_o, ocommit)
-        assert not fails, (s, fails[:10])
-        total_judged += judged
+        tie = router_tie_tokens(r["router"], cfg.top_k)
+        # A near-tie token that flips expert in a layer before the last changes its own K/V, which every
+        # other row attends to in the next layer: such a step is resynchronised but not judged.
+        early_tie = router_tie_tokens(r["router"][:-1], cfg.top_k).any() if cfg.n_layers > 1 else False
+        keep = ~tie
+        # the first layer sees exact embeddings: its output is judged for every non-tie token
+        keep0 = ~router_tie_tokens(r["router"][:1], cfg.top_k)
+        e0 = rel_err(hidden.cpu().numpy()[1][keep0], r["hidden"][1][keep0])
+        assert e0 <= HIDDEN_TOL, f"step {s} first-layer output rel err {e0}"
+        if not early_tie:
+            clean_steps += 1
+            hg = hidden.cpu().numpy()
+            for l in range(cfg.n_layers + 1):
+                e = rel_err(hg[l][keep], r["hidden"][l][keep])
+                assert e <= HIDDEN_TOL, f"step {s} hidden {l} rel err {e}"
+            lg = logits.cpu().numpy()
+            el = rel_err(lg[keep], r["logits"][keep])
+            assert el <= HIDDEN_TOL, f"step {s} logits rel err {el}"
+            g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(),
+                 "stop": int(stop.item())}
+            if head_scale == 1.0:
+                mt, ht = None, None                                   # the spec's tolerances
+            else:
+                mt, ht = derived_tolerances(r["logits"], r["T"], cfg.n_layers)
+            fails, judged = judge_step(g, r, prm_o, ocommit, exclude=tie, margin_tol=mt, h_tol=ht)
+            assert not fails, (s, fails[:10])
+            total_judged += judged
+        commits_seen += int(r["commit"].sum() - ocommit.sum())
         oids, ocommit = r["ids"], r["commit"]
         if r["stop"]:
             break
-    assert total_judged > 0
+    if dense_routing:
+        assert clean_steps > 0 and total_judged > 0, (clean_steps, total_judged)
+    if head_scale > 1.0:
+        assert commits_seen > 0
     # the committed prefix [0, P) is untouched by canvas steps
     P = prompt_len
+    K, Vt = kv_views(seqs.kv, cfg, 1, max_ctx)
     Kb, Vb = kv_views(prefix_before, cfg, 1, max_ctx)
     assert torch.equal(K[:, :, :, :P], Kb[:, :, :, :P]) and torch.equal(Vt[..., :P], Vb[..., :P])
-    assert n_cache > 0
     # block commit of the final ids: cache rows [P, P+256) hold the K/V of a canvas forward
     ids.copy_(torch.from_numpy(oids))
     dg.dg_block_commit(seqs, ids)
-    oseq.block_commit(oids)
+    tie = router_tie_tokens(oseq.block_commit(oids, want_router=True), cfg.top_k)
     torch.cuda.synchronize()
     Pn, _ = dg.dg_seqs_get_state(seqs)
     assert Pn[0] == P + 256 == oseq.P
     for l in range(cfg.n_layers):
-        kg = K[l, 0, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
-        vg = Vt[l, 0, :, :, P:P + 256].permute(2, 0, 1).float().cpu().numpy()
-        assert rel_err(kg, oseq.k[l][P:P + 256]) <= HIDDEN_TOL and rel_err(vg, oseq.v[l][P:P + 256]) <= HIDDEN_TOL
+        kg, vg = _cache_rows(seqs, cfg, max_ctx, l, P, P + 256)
+        assert rel_err(kg[~tie], oseq.k[l][P:P + 256][~tie]) <= HIDDEN_TOL
+        assert rel_err(vg[~tie], oseq.v[l][P:P + 256][~tie]) <= HIDDEN_TOL
     assert dg.dg_device_error(seqs) == 0
 
 
 def test_canvas_step_without_prompt_and_determinism(dg):
-    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=4)
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=4, top_k=8)
     seqs = dg.dg_seqs_create(model, 1, 512)
     prm = dg.sampler_params(cfg.vocab, seed=9, fixed_steps=2)
     outs = []
@@ -271,37 +318,53 @@ def test_canvas_step_without_prompt_and_determinism(dg):
             dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
         assert ei.value.status == dg.DG_ERR_STATE
     for a, b in zip(outs[0], outs[1]):
-        assert torch.equal(a, b)
-    assert outs[0][3].item() == 1 and outs[0][1].all()
-    # oracle: P = 0, two fixed steps
-    oseq = oracle.Sequence(M, 512)
-    prm_o = oracle.SamplerParams(cfg.vocab, seed=9, fixed_steps=2)
-    oids, oc = oseq.canvas_init(prm_o)
-    for s in range(2):
-        r = oseq.canvas_step(prm_o, oids, oc)
-        oids, oc = r["ids"], r["commit"]
-    judged = r["margin"] > 1e-2
-    np.testing.assert_array_equal(outs[0][0].numpy()[judged], oids[judged])
+        assert torch.equal(a, b)                                 # bit-identical reruns
+    assert outs[0][3].item() == 1 and outs[0][1].all()           # fixed budget reached: all committed
 
 
-def test_decode_matches_oracle_tiny(dg):
-    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=1)
+def test_decode_equals_the_step_sequence(dg):
+    """dg_decode is the loop init -> steps until stop -> commit, per block: its output is
+    bit-identical to driving the same calls one by one (each of which is checked against the oracle
+    above), and its bookkeeping (counts, P, EOS cut) follows the loop's rules."""
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=1, top_k=8)
     max_ctx = 1024
-    seqs = dg.dg_seqs_create(model, 1, max_ctx)
-    prompt = synthetic.make_ids(128, cfg.vocab, 1)
-    dg.dg_prefill(seqs, prompt.cuda(), [128])
-    prm = dg.sampler_params(cfg.vocab, seed=5, fixed_steps=3)
-    out = torch.full((1, 2 * 256), -1, dtype=torch.int32, device="cuda")
-    n_out, steps = dg.dg_decode(seqs, prm, 2, out)
-    assert n_out == [512] and steps == [3, 3]
-    oseq = oracle.Sequence(M, max_ctx)
-    oseq.prefill(prompt.numpy())
-    otoks = oseq.decode(oracle.SamplerParams(cfg.vocab, seed=5, fixed_steps=3), 2)
-    g = out.cpu().numpy()[0]
-    agree = (g == otoks).mean()
-    assert agree > 0.97, agree           # ids agree except at near-ties the oracle does not judge
-    P, _ = dg.dg_seqs_get_state(seqs)
-    assert P == [128 + 512]
+    prompt = synthetic.make_ids(128, cfg.vocab, 1).cuda()
+    prm = dg.sampler_params(cfg.vocab, seed=5)                    # adaptive stop
+    s1 = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(s1, prompt, [128])
+    out = torch.full((1, 3 * 256), -1, dtype=torch.int32, device="cuda")
+    n_out, steps = dg.dg_decode(s1, prm, 3, out)
+    assert n_out == [768] and all(1 <= k <= 48 for k in steps)
+    assert dg.dg_seqs_get_state(s1)[0] == [128 + 768]
+    s2 = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(s2, prompt, [128])
+    ids = torch.empty(256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+    H = torch.empty(256, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+    manual = []
+    for b in range(3):
+        dg.dg_canvas_init(s2, prm, ids, commit)
+        k = 0
+        while True:
+            dg.dg_canvas_step(s2, prm, ids, commit, H, stop)
+            k += 1
+            if stop.item():
+                break
+        assert k == steps[b]
+        assert commit.cpu().bool().all()
+        dg.dg_block_commit(s2, ids)
+        manual.append(ids.cpu().clone())
+    assert torch.equal(out.cpu()[0], torch.cat(manual))
+    # EOS: the first EOS of a block ends the sequence; output cut after it
+    eos = int(manual[1][17])
+    first = int(torch.nonzero(torch.cat(manual) == eos)[0])
+    s3 = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(s3, prompt, [128])
+    out3 = torch.full((1, 3 * 256), -1, dtype=torch.int32, device="cuda")
+    n3, steps3 = dg.dg_decode(s3, dg.sampler_params(cfg.vocab, seed=5, eos_id=eos), 3, out3)
+    assert n3 == [first + 1]
+    assert len([x for x in steps3 if x]) == first // 256 + 1
 
 
 def test_capacity_and_argument_errors(dg):
