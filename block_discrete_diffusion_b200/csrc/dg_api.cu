@@ -201,6 +201,11 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 
 }  // namespace
 
+dg_status dg::record_error(dg_status st, const char* msg) {
+  snprintf(g_err, sizeof g_err, "%s", msg);
+  return st;
+}
+
 // ---------------------------------------------------------------------------------------------
 // handles
 // ---------------------------------------------------------------------------------------------

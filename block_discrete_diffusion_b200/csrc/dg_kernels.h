@@ -7,7 +7,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "dg.h"
+
 namespace dg {
+
+// Set the calling thread's dg_last_error() message; returns st.
+dg_status record_error(dg_status st, const char* msg);
 
 // Programmatic dependent launch on/off for every kernel of the library (on unless DG_PDL=0).
 bool pdl_enabled();

@@ -23,7 +23,7 @@ ENTRY_POINTS = (
     "dg_last_error", "dg_model_create", "dg_model_destroy", "dg_kv_bytes", "dg_workspace_bytes", "dg_seqs_create",
     "dg_seqs_destroy", "dg_seqs_get_state", "dg_load_prefix", "dg_prefill", "dg_canvas_init", "dg_canvas_step",
     "dg_block_commit", "dg_decode", "dg_layer_forward", "dg_sample_workspace_bytes", "dg_sample", "dg_device_error",
-    "dg_temperature", "dg_stats_reset", "dg_stats_read",
+    "dg_temperature", "dg_stats_reset", "dg_stats_read", "dg_sample_noalloc", "dg_sample_noalloc_max_rows",
 )
 
 # dg_kernel_class, in order
@@ -103,6 +103,10 @@ def lib():
         L.dg_sample_workspace_bytes.restype = c_size_t
         L.dg_sample.argtypes = [c_void_p, c_int, c_int, P(dg_sampler_params), c_int, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+        L.dg_sample_noalloc.argtypes = [c_void_p, c_int, c_int, P(dg_sampler_params), c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p]
+        L.dg_sample_noalloc_max_rows.argtypes = [c_int]
+        L.dg_sample_noalloc_max_rows.restype = c_size_t
         L.dg_device_error.argtypes = [c_void_p, P(c_int)]
         L.dg_stats_reset.argtypes = [c_void_p, c_int]
         L.dg_stats_read.argtypes = [c_void_p, c_void_p, c_void_p]
@@ -251,6 +255,17 @@ def dg_sample(logits, n_seq, vocab, params, step, seq_P, ids, commit, entropy, s
     _check("dg_sample", lib().dg_sample(_ptr(logits), n_seq, vocab, ctypes.byref(params), step, _ptr(seq_P),
                                         _ptr(ids), _ptr(commit), _ptr(entropy), _ptr(stop), _ptr(ws), ws.numel(),
                                         _stream_handle(stream)))
+
+
+def dg_sample_noalloc(logits, n_seq, vocab, params, step, seq_P, ids, commit, entropy, stop, stream=None):
+    """dg_sample with its scratch in the library's static device array (no workspace argument)."""
+    _check("dg_sample_noalloc", lib().dg_sample_noalloc(_ptr(logits), n_seq, vocab, ctypes.byref(params), step,
+                                                        _ptr(seq_P), _ptr(ids), _ptr(commit), _ptr(entropy),
+                                                        _ptr(stop), _stream_handle(stream)))
+
+
+def dg_sample_noalloc_max_rows(vocab) -> int:
+    return int(lib().dg_sample_noalloc_max_rows(vocab))
 
 
 def dg_device_error(seqs: Seqs) -> int:

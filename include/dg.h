@@ -181,6 +181,23 @@ dg_status dg_sample(const float *d_logits, int n_seq, int vocab, const dg_sample
                     const int32_t *d_seq_P, int32_t *d_ids, uint8_t *d_commit, float *d_entropy, int32_t *d_stop,
                     void *ws, size_t ws_bytes, void *stream);
 
+/* dg_sample without a workspace argument.  The paper has no counterpart of this entry point: it is
+ * an interface of this library only.  For callers that cannot allocate device memory -- a server whose pool owns all
+ * free HBM, a real-time loop that must not allocate, a C component with no CUDA allocator -- the
+ * sampler's per-(row, vocabulary chunk) partial results live in a static device array of the
+ * library (1 MiB, held on every GPU that loads the library until the process exits).  Limit:
+ * n_seq * 256 * chunks <= 32768 records, chunks = max(1, vocab / 32768) (16 canvases at vocab
+ * 262144); larger requests return DG_ERR_CAPACITY.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current): make it before any
+ * stream capture.  It allocates nothing (no cudaMalloc / cudaFree).  All calls on a device share
+ * the array and it keeps the last call's contents (nothing in it needs to start at zero); calls
+ * that may overlap on the GPU race and must not be issued.  Arguments and outputs as dg_sample. */
+dg_status dg_sample_noalloc(const float *d_logits, int n_seq, int vocab, const dg_sampler_params *p, int step,
+                            const int32_t *d_seq_P, int32_t *d_ids, uint8_t *d_commit, float *d_entropy,
+                            int32_t *d_stop, void *stream);
+/* Largest n_seq * 256 that dg_sample_noalloc accepts for this vocabulary size. */
+size_t dg_sample_noalloc_max_rows(int vocab);
+
 /* Synchronise the handle's stream and return the first device-side error code recorded since the
  * last call (0 = none) in *h_code; the record is cleared.  Returns DG_ERR_DEVICE if non-zero. */
 dg_status dg_device_error(dg_seqs *s, int *h_code);
