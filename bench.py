@@ -65,29 +65,44 @@ def peaks():
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 50 ms; summary() keeps the samples taken
+    between mark_start() and mark_end() (host clock around the timed region, which ends with a
+    device synchronize, so it covers the GPU work)."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_ms=50):
         self.idx = gpu_index
+        self.period_ms = period_ms
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.idx), "-lms", "200"], stdout=subprocess.PIPE,
+                                          "-i", str(self.idx), "-lms", str(self.period_ms)], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            deadline = time.monotonic() + 10.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+        time.sleep(2.5 * self.period_ms / 1e3)   # let the sample that covers the end arrive
 
     def __exit__(self, *a):
         if self.proc:
@@ -100,7 +115,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lo = self.t0 if self.t0 is not None else -math.inf
+        hi = (self.t1 + self.period_ms / 1e3) if self.t1 is not None else math.inf
+        for ts, ln in self.lines:
+            if not lo <= ts <= hi:
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -117,6 +136,30 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
+# replicas: one independent batch-1 sequence per rank; the timing is the max over ranks
+# ------------------------------------------------------------------------------------------------
+def replica_seed(rank):
+    """Seed of rank `rank`'s weights, prompt and sampler stream (independent replicas)."""
+    return 2 + 1000 * rank
+
+
+def max_over_ranks(t, device, world):
+    """The slowest rank's time: every rank takes part (same collective on every rank)."""
+    if world <= 1:
+        return float(t)
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([float(t)], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(world, units_per_rank, t_max):
+    """Units all ranks processed divided by the slowest rank's time."""
+    return world * units_per_rank / t_max
+
+
+# ------------------------------------------------------------------------------------------------
 # the CUDA path
 # ------------------------------------------------------------------------------------------------
 def setup_full(rank, device):
@@ -126,13 +169,13 @@ def setup_full(rank, device):
     from block_discrete_diffusion_b200 import dg
 
     cfg = synthetic.FULL
-    w = synthetic.make_model_weights(cfg, seed=2 + 1000 * rank, device=device, **synthetic.full_stack_init(cfg))
+    w = synthetic.make_model_weights(cfg, seed=replica_seed(rank), device=device, **synthetic.full_stack_init(cfg))
     model = dg.dg_model_create(cfg, w)
     max_ctx = PROMPT + BLOCKS * CANVAS
     seqs = dg.dg_seqs_create(model, 1, max_ctx)
-    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=2 + 1000 * rank, device=device)
+    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=replica_seed(rank), device=device)
     dg.dg_prefill(seqs, prompt, [PROMPT])
-    prm = dg.sampler_params(cfg.vocab, seed=2 + 1000 * rank, fixed_steps=FIXED_STEPS)
+    prm = dg.sampler_params(cfg.vocab, seed=replica_seed(rank), fixed_steps=FIXED_STEPS)
     st = {
         "ids": torch.empty(CANVAS, dtype=torch.int32, device=device),
         "commit": torch.empty(CANVAS, dtype=torch.uint8, device=device),
@@ -192,19 +235,18 @@ def main_dg(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        clk.mark_start()
         e0.record(stream)
         run_steps(dg, seqs, prm, st, args.steps, state)
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         if world > 1:
             dist.barrier()
     t = e0.elapsed_time(e1) / 1e3
     launches = sum(v[0] for v in dg.dg_stats_read(seqs).values())
-    if world > 1:
-        tt = torch.tensor([t], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    value = world * args.steps / t
+    t = max_over_ranks(t, device, world)
+    value = whole_job_rate(world, args.steps, t)
     ms_per_step = 1e3 * t / args.steps
 
     # ---- per-kernel device time (CUDA events around each launch, same stream), separate pass ----
@@ -249,19 +291,15 @@ def main_dg(args):
         h_stop.copy_(st["stop"], non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    te = f0.elapsed_time(f1) / 1e3
-    if world > 1:
-        tt = torch.tensor([te], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        te = float(tt.item())
+    te = max_over_ranks(f0.elapsed_time(f1) / 1e3, device, world)
     state["step"] = 0
-    e2e = {"value": round(world * k_e2e / te, 3), "unit": "steps/s", "h2d_bytes_per_step": CANVAS * 4 + CANVAS,
+    e2e = {"value": round(whole_job_rate(world, k_e2e, te), 3), "unit": "steps/s", "h2d_bytes_per_step": CANVAS * 4 + CANVAS,
            "d2h_bytes_per_step": CANVAS * 4 + CANVAS + CANVAS * 4 + 4}
 
     # ---- committed tokens/s: dg_decode of 4 blocks x 12 fixed steps with a commit pass per block ----
     seqs2 = dg.dg_seqs_create(model, 1, PROMPT + BLOCKS * CANVAS)
     import synthetic
-    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=2 + 1000 * rank, device=device)
+    prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=replica_seed(rank), device=device)
     dg.dg_prefill(seqs2, prompt, [PROMPT])
     out = torch.empty(1, BLOCKS * CANVAS, dtype=torch.int32, device=device)
     torch.cuda.synchronize()
@@ -271,8 +309,8 @@ def main_dg(args):
     n_out, steps_per_block = dg.dg_decode(seqs2, prm, BLOCKS, out)
     d1.record(stream)
     torch.cuda.synchronize()
-    td = d0.elapsed_time(d1) / 1e3
-    committed_tok_s = sum(n_out) / td
+    td = max_over_ranks(d0.elapsed_time(d1) / 1e3, device, world)
+    committed_tok_s = whole_job_rate(world, sum(n_out), td)
     code = dg.dg_device_error(seqs)
     assert code == 0, f"device error {code}"
 
