@@ -46,9 +46,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="full_b1", choices=["full_b1", "one_layer", "sampler"],
+    ap.add_argument("--workload", default="full_b1", choices=["full_b1", "one_layer", "sampler", "fp8_b32"],
                     help="full_b1: the benchmark line; one_layer / sampler: the single-layer and "
-                         "sampler-alone configurations (their own lines, used for per-kernel profiles)")
+                         "sampler-alone configurations (their own lines, used for per-kernel profiles); "
+                         "fp8_b32: the 30-layer FP8 stack on 32 sequences behind 32768-token prefixes")
+    ap.add_argument("--seqs", type=int, default=32, help="fp8_b32: number of sequences")
+    ap.add_argument("--prefix", type=int, default=32768, help="fp8_b32: prefix length of every sequence")
     return ap.parse_args()
 
 
@@ -502,10 +505,112 @@ def main_aux(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------------------
+# FP8 weights, 32 sequences behind 32768-token prefixes
+# ------------------------------------------------------------------------------------------------
+def attention_flops(cfg, n_seq, P):
+    """Algorithmic FLOPs of one canvas attention launch: QK^T and PV over P + 256 keys for every
+    query head of every sequence (2 FLOPs per multiply-add)."""
+    return 4 * cfg.n_q * CANVAS * (P + CANVAS) * cfg.d_head * n_seq
+
+
+def main_fp8_b32(args):
+    import dataclasses
+
+    import torch
+
+    import synthetic
+    from block_discrete_diffusion_b200 import build, dg
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n_seq, P = args.seqs, args.prefix
+    cfg = dataclasses.replace(synthetic.FULL, wdtype=1)
+    t0 = time.perf_counter()
+    w = synthetic.make_model_weights(cfg, 3, device=dev, **synthetic.full_stack_init(cfg))
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    model = dg.dg_model_create(cfg, w)
+    max_ctx = P + CANVAS
+    seqs = dg.dg_seqs_create(model, n_seq, max_ctx)
+    for i in range(n_seq):
+        ks, vs = synthetic.make_prefix_kv(cfg.n_layers, P, cfg.n_kv, cfg.d_head, 3 + i, device=dev)
+        dg.dg_load_prefix(seqs, i, P, ks, vs)
+        del ks, vs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    t_setup = time.perf_counter() - t0
+    prm = dg.sampler_params(cfg.vocab, seed=3, fixed_steps=FIXED_STEPS)
+    ids = torch.empty(n_seq, CANVAS, dtype=torch.int32, device=dev)
+    commit = torch.empty(n_seq, CANVAS, dtype=torch.uint8, device=dev)
+    H = torch.empty(n_seq, CANVAS, device=dev)
+    stop = torch.empty(n_seq, dtype=torch.int32, device=dev)
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    for _ in range(args.warmup):
+        dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+    torch.cuda.synchronize()
+    assert dg.dg_device_error(seqs) == 0
+    k = min(args.steps, FIXED_STEPS - args.warmup)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dg.dg_stats_reset(seqs, timing=False)
+    with ClockSampler(0) as clk:
+        torch.cuda.synchronize()
+        clk.mark_start()
+        e0.record()
+        for _ in range(k):
+            dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+        e1.record()
+        torch.cuda.synchronize()
+        clk.mark_end()
+    t = e0.elapsed_time(e1) / 1e3
+    launches = sum(v[0] for v in dg.dg_stats_read(seqs).values())
+    # per-kernel device time in a second pass (a new canvas: the step budget is 12)
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    dg.dg_stats_reset(seqs, timing=True)
+    for _ in range(k):
+        dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+    stats = dg.dg_stats_read(seqs)
+    dg.dg_stats_reset(seqs, timing=False)
+    # one block through dg_decode: init, 12 steps, commit pass (committed tokens/s of the batch)
+    out = torch.empty(n_seq, CANVAS, dtype=torch.int32, device=dev)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record()
+    n_out, steps_per_block = dg.dg_decode(seqs, prm, 1, out)
+    d1.record()
+    torch.cuda.synchronize()
+    td = d0.elapsed_time(d1) / 1e3
+    assert dg.dg_device_error(seqs) == 0
+    hbm, tflops, kind = peaks()
+    attn_s = stats["attn"][1] / 1e3 / max(stats["attn"][0], 1)
+    fl = attention_flops(cfg, n_seq, P)
+    line = {"metric": "canvas denoise steps/s", "value": round(k / t, 4), "unit": "steps/s",
+            "ms_per_step": round(1e3 * t / k, 2), "steps": k, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "bf16 arithmetic, fp8 e4m3 weights", "data": "synthetic",
+            "config": {"workload": f"fp8_b{n_seq}: 30-layer stack, FP8 e4m3 per-layer matrices (fp32 scale per "
+                                   f"128x128 tile), {n_seq} sequences each behind a {P}-token prefix (N(0,1) "
+                                   f"K/V), 256-token canvases, 12 fixed steps per block", "global_batch": n_seq,
+                       "seq_len": CANVAS, "prefix": P},
+            "committed_tok_s": round(sum(n_out) / td, 1),
+            "decode": {"blocks": 1, "steps_per_block": steps_per_block, "tokens": sum(n_out),
+                       "seconds": round(td, 3)},
+            "gpu_launches": launches,
+            "roofline": {"kernel": "attn_partial (canvas attention)", "bound": "tensor",
+                         "achieved": round(fl / attn_s / 1e12, 1), "peak": tflops, "unit": "TFLOP/s",
+                         "frac": round(fl / attn_s / 1e12 / tflops, 4), "traffic": None,
+                         "algorithmic_flops_per_launch": fl, "launch_ms": round(attn_s * 1e3, 3),
+                         "peak_source": f"{kind} bf16_tflops"},
+            "kernel_ms_per_step": {kk: round(v[1] / k, 3) for kk, v in stats.items() if v[0]},
+            "clocks": clk.summary(), "setup_seconds": round(t_setup, 1),
+            "device_memory_gb": round(torch.cuda.max_memory_allocated() / 1e9, 1)}
+    print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         main_reference(a)
+    elif a.workload == "fp8_b32":
+        main_fp8_b32(a)
     elif a.workload != "full_b1":
         main_aux(a)
     else:

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdg.so")
-SOURCES = ["dg_api.cu", "gemm.cu", "attention.cu", "misc.cu", "sampler.cu", "sampler_noalloc.cu"]
+SOURCES = ["dg_api.cu", "gemm.cu", "attention.cu", "misc.cu", "sampler.cu", "sampler_noalloc.cu", "dequant.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

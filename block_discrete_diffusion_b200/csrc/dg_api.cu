@@ -60,6 +60,7 @@ constexpr int kSplitTargetCtas = 296;   // two waves of CTAs over the 148 SMs
 constexpr int kMaxSplits = 16;
 constexpr int kRouterSplits = 8;        // cluster size of the router GEMM's split-K
 constexpr int kGemmTargetCtas = 296;    // two CTAs per SM for the 128-wide dense GEMM tiles
+constexpr int kSplitKSlots = kGemmTargetCtas;   // split-K partial tiles: tiles x splits <= this (dense_splits)
 
 // Cluster size (power of two, <= 8) of the split-K dense GEMMs for `tiles` output tiles over nk
 // 64-deep k-blocks: enough CTAs for about two per SM, at least 4 k-blocks per CTA.
@@ -128,8 +129,19 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
-      y, logits, samp, rope, cids, ccommit, cH, cstop, total;
+      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, total;
+  size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
+
+// Elements of the five per-layer matrices, in the order qkv, o, router, gate_up, down.
+void layer_matrix_shapes(const dg_model_config& c, uint64_t rows[5], uint64_t cols[5]) {
+  const uint64_t d = c.d_model;
+  rows[0] = (uint64_t)(c.n_q + 2 * c.n_kv) * c.d_head; cols[0] = d;
+  rows[1] = d;                                       cols[1] = (uint64_t)c.n_q * c.d_head;
+  rows[2] = c.n_exp;                                 cols[2] = d;
+  rows[3] = (uint64_t)c.n_exp * 2 * c.d_ff;          cols[3] = d;
+  rows[4] = (uint64_t)c.n_exp * d;                   cols[4] = c.d_ff;
+}
 
 int attn_split_cap(const dg_model_config& c, int n_seq) {
   const int G = c.n_q / c.n_kv;
@@ -177,6 +189,12 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.ccommit = take(R);
   L.cH = take(4 * R);
   L.cstop = take(4 * (size_t)n_seq);
+  L.splitk = take(4 * (size_t)kSplitKSlots * 128 * 128);
+  if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
+    uint64_t rows[5], cols[5];
+    layer_matrix_shapes(c, rows, cols);
+    for (int i = 0; i < 5; ++i) L.wq[i] = take(2 * rows[i] * cols[i]);
+  }
 
   L.total = off + 1024;   // slack for base alignment
   return L;
@@ -194,6 +212,9 @@ bool shape_ok(const dg_model_config* c, const char** why) {
   if (c->top_k <= 0 || c->top_k > 32 || c->top_k > c->n_exp) return (*why = "top_k must be in [1, min(32, n_exp)]", false);
   if (c->n_layers <= 0) return (*why = "n_layers must be positive", false);
   if (c->vocab <= 0 || c->vocab % 1024) return (*why = "vocab must be a positive multiple of 1024", false);
+  if (c->wdtype != DG_WDTYPE_BF16 && c->wdtype != DG_WDTYPE_FP8_BLOCK128) return (*why = "unknown wdtype", false);
+  if (c->wdtype == DG_WDTYPE_FP8_BLOCK128 && (2 * c->d_ff) % 128)
+    return (*why = "FP8 weights need 2 d_ff % 128 == 0", false);
   return true;
 }
 
@@ -221,6 +242,7 @@ struct dg_model {
   std::vector<dg_layer_weights> layers;
   std::vector<LayerMaps> maps;
   CUtensorMap head_map;
+  bool fp8;   // per-layer matrices in the FP8 block-scaled form (expanded per layer into the workspace)
 };
 
 struct dg_seqs {
@@ -232,7 +254,7 @@ struct dg_seqs {
   uint8_t* ws;
   // typed workspace views
   int *err, *seqP;
-  float *x, *opart, *ml, *rlog, *gate, *perm_gate, *y, *logits, *samp;
+  float *x, *opart, *ml, *rlog, *gate, *perm_gate, *y, *logits, *samp, *splitk;
   __nv_bfloat16 *xn, *q, *attn, *xp, *hb;
   int32_t *sel, *counts, *offsets, *perm_tok, *slot, *cids, *cstop;
   uint8_t* ccommit;
@@ -240,6 +262,8 @@ struct dg_seqs {
 
   float2* rope;
   CUtensorMap xn_map, xp_map, attn_map, hb_map, q_map, k_map, v_map;
+  LayerMaps wmaps;              // FP8 form: descriptors of the bf16 scratch matrices
+  __nv_bfloat16* wq[5];         // FP8 form: the scratch matrices (qkv, o, router, gate_up, down)
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
   bool block_open;
@@ -310,15 +334,22 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
   if (!shape_ok(cfg, &why)) return fail(DG_ERR_INVALID_ARG, "model config: %s", why);
   if (!w || !w->layers || !aligned16(w->emb) || !aligned16(w->head) || !aligned16(w->final_norm))
     return fail(DG_ERR_INVALID_ARG, "weights: null or unaligned emb/head/final_norm/layers");
+  const bool fp8 = cfg->wdtype == DG_WDTYPE_FP8_BLOCK128;
   for (int l = 0; l < cfg->n_layers; ++l) {
     const dg_layer_weights& L = w->layers[l];
     if (!aligned16(L.attn_norm) || !aligned16(L.w_qkv) || !aligned16(L.w_o) || !aligned16(L.ffn_norm) ||
         !aligned16(L.w_router) || !aligned16(L.w_gate_up) || !aligned16(L.w_down))
       return fail(DG_ERR_INVALID_ARG, "layer %d: null or unaligned weight pointer", l);
+    if (fp8 && (!L.s_qkv || !L.s_o || !L.s_router || !L.s_gate_up || !L.s_down ||
+                ((reinterpret_cast<uintptr_t>(L.s_qkv) | reinterpret_cast<uintptr_t>(L.s_o) |
+                  reinterpret_cast<uintptr_t>(L.s_router) | reinterpret_cast<uintptr_t>(L.s_gate_up) |
+                  reinterpret_cast<uintptr_t>(L.s_down)) & 3)))
+      return fail(DG_ERR_INVALID_ARG, "layer %d: null or unaligned FP8 scale pointer", l);
   }
   dg_model* m = new (std::nothrow) dg_model();
   if (!m) return fail(DG_ERR_INVALID_ARG, "host allocation failed");
   m->cfg = *cfg;
+  m->fp8 = fp8;
   {
     int dev = 0;
     m->n_sms = 148;
@@ -332,7 +363,7 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
   const dg_model_config& c = *cfg;
   const uint64_t d = c.d_model, qkv = (uint64_t)(c.n_q + 2 * c.n_kv) * c.d_head;
   dg_status st = DG_OK;
-  for (int l = 0; l < c.n_layers && st == DG_OK; ++l) {
+  for (int l = 0; l < c.n_layers && st == DG_OK && !fp8; ++l) {
     const dg_layer_weights& L = m->layers[l];
     LayerMaps& M = m->maps[l];
     if ((st = map_2d(&M.wqkv, L.w_qkv, qkv, d, 128)) != DG_OK) break;
@@ -418,6 +449,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->ccommit = b + L.ccommit;
   s->cH = reinterpret_cast<float*>(b + L.cH);
   s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
+  s->splitk = reinterpret_cast<float*>(b + L.splitk);
+  for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
   s->step = 0;
@@ -441,6 +474,16 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (st == DG_OK) st = map_2d(&s->q_map, s->q, (uint64_t)n_seq * c.n_q * kCanvas, c.d_head, 128);
   if (st == DG_OK) st = map_3d(&s->k_map, s->kc, c.d_head, max_ctx, zdim, 128);
   if (st == DG_OK) st = map_3d(&s->v_map, s->vt, max_ctx, c.d_head, zdim, c.d_head);
+  if (st == DG_OK && m->fp8) {
+    uint64_t rows[5], cols[5];
+    layer_matrix_shapes(c, rows, cols);
+    LayerMaps& W = s->wmaps;
+    st = map_2d(&W.wqkv, s->wq[0], rows[0], cols[0], 128);
+    if (st == DG_OK) st = map_2d(&W.wo, s->wq[1], rows[1], cols[1], 128);
+    if (st == DG_OK) st = map_2d(&W.wrouter, s->wq[2], rows[2], cols[2], 128);
+    if (st == DG_OK) st = map_2d(&W.wgu, s->wq[3], rows[3], cols[3], 64);
+    if (st == DG_OK) st = map_2d(&W.wdown, s->wq[4], rows[4], cols[4], 128);
+  }
   if (st != DG_OK) {
     delete s;
     return st;
@@ -491,9 +534,23 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
                     float* x_mid, float* rlog_out, bool xn_ready = false, const float* next_gain = nullptr) {
   const dg_model_config& c = s->m->cfg;
   const dg_layer_weights& W = s->m->layers[l];
-  const LayerMaps& M = s->m->maps[l];
+  const bool fp8 = s->m->fp8;
+  const LayerMaps& M = fp8 ? s->wmaps : s->m->maps[l];
   cudaStream_t st = s->st;
   const int d = c.d_model, dh = c.d_head;
+
+  if (fp8) {
+    // expand this layer's FP8 matrices into the bf16 scratch the GEMM descriptors point at
+    uint64_t mr[5], mc[5];
+    layer_matrix_shapes(c, mr, mc);
+    const void* q[5] = {W.w_qkv, W.w_o, W.w_router, W.w_gate_up, W.w_down};
+    const float* sc[5] = {W.s_qkv, W.s_o, W.s_router, W.s_gate_up, W.s_down};
+    DequantArgs da{};
+    da.n = 5;
+    for (int i = 0; i < 5; ++i)
+      da.mat[i] = DequantMat{static_cast<const uint8_t*>(q[i]), sc[i], s->wq[i], (long long)mr[i], (int)mc[i]};
+    LAUNCH(s, DG_K_DEQUANT, 1, dequant_fp8(da, s->m->n_sms, st));
+  }
 
   if (!xn_ready)
     LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.attn_norm), rows, d, c.rms_eps, s->xn, st));
@@ -509,6 +566,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   ep.rows_per_seq = kCanvas;
   ep.max_ctx = s->max_ctx;
   ep.seq_base = seq_base;
+  ep.late_weights = fp8;
+  ep.part = s->splitk;
+  ep.part_slots = kSplitKSlots;
   const int n_qkv = (c.n_q + 2 * c.n_kv) * dh;
   ep.k_splits = dense_splits(((rows + 127) / 128) * (n_qkv / 128), d / 64);
   LAUNCH(s, DG_K_QKV, 1, gemm_dense(128, EPI_QKV, s->xn_map, M.wqkv, rows, n_qkv, d, ep, s->err, st));
@@ -540,6 +600,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   EpiParams eo{};
   eo.x = x;
   eo.ldo = d;
+  eo.late_weights = fp8;
+  eo.part = s->splitk;
+  eo.part_slots = kSplitKSlots;
   eo.k_splits = dense_splits(((rows + 127) / 128) * (d / 128), c.n_q * dh / 64);
   LAUNCH(s, DG_K_OPROJ, 1, gemm_dense(128, EPI_RESID, s->attn_map, M.wo, rows, d, c.n_q * dh, eo, s->err, st));
   if (x_mid) CK(cudaMemcpyAsync(x_mid, x, sizeof(float) * (size_t)rows * d, cudaMemcpyDeviceToDevice, st));
@@ -549,6 +612,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   EpiParams er{};
   er.out = s->rlog;
   er.ldo = c.n_exp;
+  er.late_weights = fp8;
+  er.part = s->splitk;
+  er.part_slots = kSplitKSlots;
   er.k_splits = std::min(kRouterSplits, dense_splits((rows + 127) / 128, d / 64));
   LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
   LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));

@@ -61,6 +61,23 @@ struct EpiParams {
   const float2* rope;    // (cos, sin) table [max_ctx][dh/2]
   const int* seq_P;      // committed length of each sequence (device)
   int n_q, n_kv, dh, rows_per_seq, max_ctx, seq_base;
+  int late_weights;      // 1: the weights are written by a preceding kernel (FP8 scratch): load them
+                         // only after the grid-dependency wait
+  float* part;           // k_splits > 1: fp32 scratch of part_slots [128][BN] partial tiles
+  int part_slots;
+};
+
+// One FP8 block-scaled matrix to expand: e4m3 q [rows][cols], scales s [ceil(rows/128)][ceil(cols/128)].
+struct DequantMat {
+  const uint8_t* q;
+  const float* s;
+  __nv_bfloat16* out;
+  long long rows;
+  int cols;              // multiple of 16
+};
+struct DequantArgs {
+  DequantMat mat[5];
+  int n;
 };
 
 struct ExpertParams {
@@ -102,6 +119,7 @@ cudaError_t embed_rows(const __nv_bfloat16* emb, const int32_t* ids, int n_rows,
                        int* err, const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st);
 cudaError_t rmsnorm_rows(const float* x, const float* g, int n_rows, int d, float eps, __nv_bfloat16* out,
                          cudaStream_t st);
+cudaError_t dequant_fp8(const DequantArgs& a, int n_sms, cudaStream_t st);
 cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st);
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
                         int32_t* sel, float* gate, int32_t* counts, cudaStream_t st);

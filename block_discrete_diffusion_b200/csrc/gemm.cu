@@ -103,11 +103,82 @@ __device__ __forceinline__ void store_qkv_pairs(const EpiParams& ep, int row, in
   }
 }
 
+// Epilogue of nr finished rows held in shared memory (t[r * rs + c], rows row0.., columns n0..),
+// laid out so that global stores are coalesced: F32 / RESID rows by one warp each (lane = 4
+// columns); Q and K heads rotated pairwise by one warp per row (lane = rotary pair), stored
+// head-major; V heads by one warp per channel (lane = row, positions contiguous in the
+// transposed value cache).
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const float* t, int rs, int row0, int nr,
+                                                   int n0, int M, int N) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = kGemmThreads / 32;
+  if constexpr (EPI == EPI_QKV) {
+    const int dh = ep.dh, half = dh >> 1;
+    const int q_end = ep.n_q * dh, k_end = q_end + ep.n_kv * dh;
+    for (int h0 = 0; h0 < BN; h0 += dh) {
+      const int f_head = n0 + h0;
+      if (f_head >= N) break;
+      if (f_head < k_end) {
+        for (int r = warp; r < nr; r += NW) {
+          const int row = row0 + r;
+          if (row >= M) break;
+          const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
+          const int cseq = ep.seq_base + seq;
+          const int pos = ep.seq_P[cseq] + j;
+          __nv_bfloat16* dst =
+              f_head < q_end ? ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh
+                             : ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + pos) * dh;
+          const float2* cs = ep.rope + (size_t)pos * half;
+          const float* tr = t + r * rs + h0;
+          for (int i = lane; i < half; i += 32) {
+            const float a = tr[i], b = tr[half + i];
+            const float2 c = cs[i];
+            dst[i] = __float2bfloat16_rn(a * c.x - b * c.y);
+            dst[half + i] = __float2bfloat16_rn(b * c.x + a * c.y);
+          }
+        }
+      } else {
+        const int vh = (f_head - k_end) / dh;
+        for (int c = warp; c < dh; c += NW) {
+          for (int r = lane; r < nr; r += 32) {
+            const int row = row0 + r;
+            if (row >= M) break;
+            const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
+            const int cseq = ep.seq_base + seq;
+            const int pos = ep.seq_P[cseq] + j;
+            ep.vt[(((size_t)cseq * ep.n_kv + vh) * dh + c) * ep.max_ctx + pos] = __float2bfloat16_rn(t[r * rs + h0 + c]);
+          }
+        }
+      }
+    }
+  } else {
+    for (int r = warp; r < nr; r += NW) {
+      const int row = row0 + r;
+      if (row >= M) break;
+      float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)row * ep.ldo + n0;
+      const float* tr = t + r * rs;
+      for (int c = lane * 4; c < BN; c += 128) {
+        if (n0 + c + 4 <= N) {
+          float4 v = *reinterpret_cast<const float4*>(tr + c);
+          if (EPI == EPI_RESID) {
+            const float4 x = *reinterpret_cast<const float4*>(dst + c);
+            v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+          }
+          *reinterpret_cast<float4*>(dst + c) = v;
+        } else {
+          for (int k = 0; k < 4 && n0 + c + k < N; ++k) dst[c + k] = (EPI == EPI_RESID ? dst[c + k] : 0.f) + tr[c + k];
+        }
+      }
+    }
+  }
+}
+
 // One 128 x BN output tile per cluster of Z CTAs; CTA z of the cluster multiplies k-blocks
 // [z nk/Z, (z+1) nk/Z).  Z = 1: the epilogue reads the accumulator from TMEM (thread = row).
-// Z > 1: every CTA parks its fp32 partial in its own shared memory; after a cluster barrier CTA z
-// sums rows [z 128/Z, (z+1) 128/Z) over the cluster's partials (distributed shared memory, in rank
-// order, so the result does not depend on timing) and runs the epilogue on those rows.
+// Z > 1: every CTA writes its fp32 partial to its slot of an L2-resident scratch (coalesced); after
+// a cluster barrier CTA z sums rows [z 128/Z, (z+1) 128/Z) over the Z slots in rank order (so the
+// result does not depend on timing) and runs the epilogue on those rows from shared memory.
 template <int BN, int EPI, int Z>
 __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
     dense_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
@@ -142,15 +213,16 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
 
   if (warp == 0 && lane == 0) {
     const uint64_t pol_w = l2_policy_evict_first();
-    // The weights (B) of the first stages do not depend on the previous kernel: load them before
-    // waiting for it; the activation tiles (A) follow the wait.
+    // The weights (B) of the first stages do not depend on the previous kernel (unless a preceding
+    // kernel writes them): load them before waiting for it; the activation tiles (A) follow the wait.
     const int npre = nk < C::kStages ? nk : C::kStages;
+    if (ep.late_weights) pdl_wait();
     for (int kb = 0; kb < npre; ++kb) {
       uint8_t* a = tiles + (size_t)kb * C::kStageBytes;
       mbar_expect_tx(&bars->full[kb], C::kBTileBytes);
       tma_load_2d_hint(&tmB, &bars->full[kb], a + kATileBytes, (kb0 + kb) * 64, n0, pol_w);
     }
-    pdl_wait();
+    if (!ep.late_weights) pdl_wait();
     for (int kb = 0; kb < npre; ++kb) {
       uint8_t* a = tiles + (size_t)kb * C::kStageBytes;
       mbar_arrive_expect_tx(&bars->full[kb], kATileBytes);
@@ -214,8 +286,10 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       }
     }
   } else {
-    // ---------------- cluster split-K reduction over distributed shared memory ----------------
-    constexpr int RS = BN + 4;                 // padded row stride of the parked partial
+    // ---------------- split-K: partials through an L2-resident scratch, summed in rank order ----------------
+    constexpr int RS = BN + 4;                 // padded row stride of the shared-memory tiles
+    constexpr int F4 = BN / 4;                 // float4 per row
+    constexpr int RPC = 128 / Z;               // rows finished by this CTA
     float* red = reinterpret_cast<float*>(tiles);
     {
       const int r = warp * 32 + lane;
@@ -227,50 +301,28 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
           *reinterpret_cast<float4*>(red + r * RS + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
-    tc_fence_before();
-    cluster_sync();
-    constexpr int RPC = 128 / Z;               // rows reduced by this CTA
-    const int rr = zz * RPC + threadIdx.x / Z;   // Z threads per row
-    const int q = threadIdx.x % Z;
-    const int row = m0 + rr;
-    if constexpr (EPI == EPI_QKV) {
-      // thread q takes rotary pairs [q PW, (q+1) PW) of the tile: columns c1 and c1 + half of a head
-      constexpr int PW = BN / (2 * Z);
-      const int dh = ep.dh, half = dh >> 1;
-      const int p0 = q * PW;
-      const int hh = p0 / half, i0 = p0 % half;
-      const int c1 = hh * dh + i0;
-      float a[PW], b[PW];
-#pragma unroll
-      for (int k = 0; k < PW; ++k) a[k] = b[k] = 0.f;
-      const uint32_t la = smem_u32(red + rr * RS + c1), lb = smem_u32(red + rr * RS + c1 + half);
-      for (int z = 0; z < Z; ++z) {
-        const uint32_t ra = dsmem_map(la, z), rb = dsmem_map(lb, z);
-#pragma unroll
-        for (int k = 0; k < PW; k += 4) {
-          const float4 u = dsmem_ld_f4(ra + 4 * k), w = dsmem_ld_f4(rb + 4 * k);
-          a[k] += u.x; a[k + 1] += u.y; a[k + 2] += u.z; a[k + 3] += u.w;
-          b[k] += w.x; b[k + 1] += w.y; b[k + 2] += w.z; b[k + 3] += w.w;
-        }
-      }
-      if (ok && row < M && n0 + hh * dh < N) store_qkv_pairs(ep, row, n0 + hh * dh, i0, a, b, PW);
-    } else {
-      constexpr int CW = BN / Z;               // thread q takes columns [q CW, (q+1) CW)
-      float v[CW];
-#pragma unroll
-      for (int k = 0; k < CW; ++k) v[k] = 0.f;
-      const uint32_t la = smem_u32(red + rr * RS + q * CW);
-      for (int z = 0; z < Z; ++z) {
-        const uint32_t ra = dsmem_map(la, z);
-#pragma unroll
-        for (int k = 0; k < CW; k += 4) {
-          const float4 u = dsmem_ld_f4(ra + 4 * k);
-          v[k] += u.x; v[k + 1] += u.y; v[k + 2] += u.z; v[k + 3] += u.w;
-        }
-      }
-      if (ok && row < M) store_row_f32<EPI>(ep, row, n0 + q * CW, v, CW, N);
+    __syncthreads();
+    // slot zz of this tile: [128][BN] fp32, written with coalesced 16-byte stores
+    float* slots = ep.part + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * Z * 128 * BN;
+    {
+      float4* dst = reinterpret_cast<float4*>(slots + (size_t)zz * 128 * BN);
+      for (int i = threadIdx.x; i < 128 * F4; i += kGemmThreads)
+        __stcg(dst + i, *reinterpret_cast<const float4*>(red + (i / F4) * RS + 4 * (i % F4)));
     }
-    cluster_sync();   // the peers have finished reading this CTA's partial
+    __threadfence();
+    cluster_sync();   // every slot of the tile is written (and this CTA's shared tile is free again)
+    for (int i = threadIdx.x; i < RPC * F4; i += kGemmThreads) {
+      const size_t off = (size_t)(zz * RPC + i / F4) * BN + 4 * (i % F4);
+      float4 acc = __ldcg(reinterpret_cast<const float4*>(slots + off));
+#pragma unroll
+      for (int z = 1; z < Z; ++z) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(slots + (size_t)z * 128 * BN + off));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      *reinterpret_cast<float4*>(red + (i / F4) * RS + 4 * (i % F4)) = acc;
+    }
+    __syncthreads();
+    if (ok) epilogue_from_smem<BN, EPI>(ep, red, RS, m0 + zz * RPC, RPC, n0, M, N);
   }
 
   tc_fence_before();
@@ -511,6 +563,8 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
   if (K % 64 != 0) return cudaErrorInvalidValue;
   const int z = ep.k_splits > 1 ? ep.k_splits : 1;
   if (z > K / 64) return cudaErrorInvalidValue;
+  if (z > 1 && (!ep.part || (long long)((M + 127) / 128) * ((N + bn - 1) / bn) * z > ep.part_slots || bn != 128))
+    return cudaErrorInvalidValue;   // the split-K scratch holds part_slots [128][128] tiles
 #define DG_DENSE_CASE(BN_, EPI_, Z_) \
   if (bn == BN_ && epi == EPI_ && z == Z_) return launch_dense<BN_, EPI_, Z_>(a, b, M, N, K, ep, err, st);
   DG_DENSE_CASE(128, EPI_QKV, 1)

@@ -28,7 +28,9 @@ ENTRY_POINTS = (
 
 # dg_kernel_class, in order
 KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attn", "attn_merge", "oproj", "router", "topk", "bucket", "expert_up",
-                  "expert_down", "combine", "head", "sampler", "misc")
+                  "expert_down", "combine", "head", "sampler", "misc", "dequant")
+WDTYPE_BF16, WDTYPE_FP8_BLOCK128 = 0, 1
+MATRICES = ("w_qkv", "w_o", "w_router", "w_gate_up", "w_down")
 
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_CAPACITY, DG_ERR_STATE, DG_ERR_CUDA, DG_ERR_UNSUPPORTED, DG_ERR_DEVICE = range(7)
 
@@ -41,11 +43,12 @@ class DGError(RuntimeError):
 
 class dg_model_config(ctypes.Structure):
     _fields_ = [(n, c_int) for n in ("d_model", "n_q", "n_kv", "d_head", "n_exp", "top_k", "d_ff", "n_layers",
-                                     "vocab")] + [("rms_eps", c_float), ("rope_theta", c_float)]
+                                     "vocab")] + [("rms_eps", c_float), ("rope_theta", c_float), ("wdtype", c_int)]
 
 
 class dg_layer_weights(ctypes.Structure):
-    _fields_ = [(n, c_void_p) for n in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate_up", "w_down")]
+    _fields_ = [(n, c_void_p) for n in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate_up", "w_down",
+                                        "s_qkv", "s_o", "s_router", "s_gate_up", "s_down")]
 
 
 class dg_weights(ctypes.Structure):
@@ -136,7 +139,16 @@ def _stream_handle(stream):
 
 def make_config(cfg) -> dg_model_config:
     return dg_model_config(cfg.d_model, cfg.n_q, cfg.n_kv, cfg.d_head, cfg.n_exp, cfg.top_k, cfg.d_ff, cfg.n_layers,
-                           cfg.vocab, cfg.rms_eps, cfg.rope_theta)
+                           cfg.vocab, cfg.rms_eps, cfg.rope_theta, getattr(cfg, "wdtype", WDTYPE_BF16))
+
+
+def _layer_struct(L: dict) -> "dg_layer_weights":
+    """A layer dict of device tensors; in the FP8 form each matrix is {"e4m3": uint8, "scale": fp32}."""
+    def mat(k):
+        t = L[k]
+        return (_ptr(t["e4m3"]), _ptr(t["scale"])) if isinstance(t, dict) else (_ptr(t), None)
+    (q, sq), (o, so), (r, sr), (gu, sgu), (dn, sdn) = (mat(k) for k in MATRICES)
+    return dg_layer_weights(_ptr(L["attn_norm"]), q, o, _ptr(L["ffn_norm"]), r, gu, dn, sq, so, sr, sgu, sdn)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -158,8 +170,7 @@ def dg_model_create(cfg, weights: dict) -> Model:
     c = make_config(cfg)
     layers = (dg_layer_weights * cfg.n_layers)()
     for i, L in enumerate(weights["layers"]):
-        layers[i] = dg_layer_weights(*[_ptr(L[k]) for k in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router",
-                                                             "w_gate_up", "w_down")])
+        layers[i] = _layer_struct(L)
     w = dg_weights(_ptr(weights["emb"]), _ptr(weights["final_norm"]), _ptr(weights["head"]),
                    ctypes.cast(layers, ctypes.POINTER(dg_layer_weights)))
     h = c_void_p()

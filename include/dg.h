@@ -50,25 +50,38 @@ typedef enum {
 typedef struct dg_model dg_model; /* opaque: config + borrowed weight pointers + TMA descriptors */
 typedef struct dg_seqs dg_seqs;   /* opaque: n sequences sharing one KV cache and one workspace */
 
+/* Storage form of the per-layer matrices (w_qkv, w_o, w_router, w_gate_up, w_down). */
+#define DG_WDTYPE_BF16 0          /* bf16 */
+#define DG_WDTYPE_FP8_BLOCK128 1  /* OCP FP8 E4M3 bytes, one fp32 scale per 128 x 128 tile (w = q * s) */
+
 /* Model shape.  Requirements of this build: d_head in {64, 128}; d_model % 128 == 0;
- * d_ff % 64 == 0; n_q % n_kv == 0; n_exp <= 256; top_k <= 32; vocab % 1024 == 0. */
+ * d_ff % 64 == 0; n_q % n_kv == 0; n_exp <= 256; top_k <= 32; vocab % 1024 == 0; with
+ * DG_WDTYPE_FP8_BLOCK128 also 2 d_ff % 128 == 0 (128-row tiles never straddle two experts). */
 typedef struct {
   int d_model, n_q, n_kv, d_head, n_exp, top_k, d_ff, n_layers, vocab;
   float rms_eps;    /* RMSNorm epsilon (1e-6) */
   float rope_theta; /* rotary base (10000) */
+  int wdtype;       /* DG_WDTYPE_BF16 or DG_WDTYPE_FP8_BLOCK128 */
 } dg_model_config;
 
 /* One decoder layer's weights, device pointers, layouts [out_features][in_features]:
  *   attn_norm  fp32 [d]                   RMSNorm gain before attention
- *   w_qkv      bf16 [(n_q+2 n_kv) dh][d]  Q rows, then K rows, then V rows
- *   w_o        bf16 [d][n_q dh]
+ *   w_qkv      [(n_q+2 n_kv) dh][d]       Q rows, then K rows, then V rows
+ *   w_o        [d][n_q dh]
  *   ffn_norm   fp32 [d]                   RMSNorm gain before the MoE
- *   w_router   bf16 [n_exp][d]
- *   w_gate_up  bf16 [n_exp][2 d_ff][d]    per expert: d_ff gate rows, then d_ff up rows
- *   w_down     bf16 [n_exp][d][d_ff]
- * Buffers must be 16-byte aligned and stay valid while the model exists. */
+ *   w_router   [n_exp][d]
+ *   w_gate_up  [n_exp][2 d_ff][d]         per expert: d_ff gate rows, then d_ff up rows
+ *   w_down     [n_exp][d][d_ff]
+ * The five matrices are bf16 (DG_WDTYPE_BF16) or e4m3 bytes (DG_WDTYPE_FP8_BLOCK128).  In the FP8
+ * form s_* are their fp32 scales, one per 128 x 128 tile of the matrix viewed as 2-D
+ * ([n_exp 2 d_ff][d] for w_gate_up, [n_exp d][d_ff] for w_down), row-major over
+ * [ceil(rows/128)][ceil(cols/128)] tiles; the weight is q * s exactly.  The GEMMs compute with the
+ * weights rounded to bf16 (one rounding of q * s), activations in bf16, accumulation in fp32.
+ * s_* are ignored in the bf16 form.  Buffers must be 16-byte aligned and stay valid while the model
+ * exists. */
 typedef struct {
   const void *attn_norm, *w_qkv, *w_o, *ffn_norm, *w_router, *w_gate_up, *w_down;
+  const float *s_qkv, *s_o, *s_router, *s_gate_up, *s_down;
 } dg_layer_weights;
 
 typedef struct {
@@ -110,6 +123,8 @@ void dg_model_destroy(dg_model *m);
  *   K[l][seq][h][pos][c]   keys after rotary embedding, head-major
  *   Vt[l][seq][h][c][pos]  values, transposed (positions contiguous) */
 size_t dg_kv_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
+/* With DG_WDTYPE_FP8_BLOCK128 the workspace also holds one layer's matrices in bf16 (each layer is
+ * expanded there just before it runs). */
 size_t dg_workspace_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
 
 /* Sequence set: n_seq independent sequences (1 = batch 1) with max_ctx positions each.  kv and ws
@@ -219,6 +234,7 @@ typedef enum {
   DG_K_HEAD,          /* vocabulary logits (tcgen05) */
   DG_K_SAMPLER,       /* sampler partial + finalize */
   DG_K_MISC,          /* canvas init, cache bookkeeping */
+  DG_K_DEQUANT,       /* FP8 block-scaled weights -> bf16 (DG_WDTYPE_FP8_BLOCK128 only) */
   DG_K_COUNT
 } dg_kernel_class;
 

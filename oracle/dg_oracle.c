@@ -59,6 +59,16 @@ double orc_e4m3_to_double(uint8_t q)
     return sign ? -v : v;
 }
 
+/* The 256 decoded e4m3 values, filled once when the library loads (a table of orc_e4m3_to_double,
+ * so that expanding FP8 weight rows costs a lookup per element). */
+static double e4m3_value[256];
+
+__attribute__((constructor)) static void fill_e4m3_table(void)
+{
+    for (int q = 0; q < 256; ++q)
+        e4m3_value[q] = orc_e4m3_to_double((uint8_t)q);
+}
+
 /* A weight matrix [rows][cols], row-major: bf16 bits, or e4m3 bytes with one fp32 scale per
  * 128x128 tile (scale index [r/128][c/128], row-major over ceil(cols/128) tiles). */
 typedef struct {
@@ -78,7 +88,7 @@ static void mat_row(const orc_mat *w, int r, double *out)
         const uint8_t *p = w->e4m3 + (size_t)r * w->cols;
         int tiles_c = (w->cols + 127) / 128;
         for (int c = 0; c < w->cols; ++c)
-            out[c] = orc_e4m3_to_double(p[c]) * (double)w->scale[(size_t)(r / 128) * tiles_c + c / 128];
+            out[c] = e4m3_value[p[c]] * (double)w->scale[(size_t)(r / 128) * tiles_c + c / 128];
     }
 }
 

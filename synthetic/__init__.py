@@ -39,6 +39,7 @@ class ModelConfig:
     vocab: int
     rms_eps: float = 1e-6
     rope_theta: float = 10000.0
+    wdtype: int = 0   # per-layer matrices: 0 bf16; 1 FP8 e4m3 with one fp32 scale per 128 x 128 tile
 
     @property
     def qkv_rows(self) -> int:
@@ -78,24 +79,69 @@ def _normal_bf16(shape, std, gen, device) -> torch.Tensor:
     return t.to(torch.bfloat16)
 
 
+FP8_E4M3_MAX = 448.0
+
+
+def quantize_fp8_block128(w: torch.Tensor) -> dict:
+    """FP8 storage form of a random weight matrix [rows, cols] (an expert stack [E, rows, cols] is
+    viewed as [E rows, cols]): per 128 x 128 tile the scale s = amax / 448 (1 for an all-zero
+    tile) and the bytes q = w / s cast to e4m3 (torch's round-to-nearest-even cast, clamped to
+    +-448).  The stored weight is q * s.  Returns {"e4m3": uint8 [same shape], "scale": fp32
+    [ceil(rows/128), ceil(cols/128)]}."""
+    shape = w.shape
+    w2 = w.reshape(-1, shape[-1]).float()
+    R, C = w2.shape
+    tr, tc = -(-R // 128), -(-C // 128)
+    pad = torch.zeros((tr * 128, tc * 128), dtype=torch.float32, device=w.device)
+    pad[:R, :C] = w2
+    del w2
+    tiles = pad.view(tr, 128, tc, 128)
+    amax = tiles.abs().amax(dim=(1, 3))
+    scale = torch.where(amax > 0, amax / FP8_E4M3_MAX, torch.ones_like(amax))
+    tiles.div_(scale[:, None, :, None]).clamp_(-FP8_E4M3_MAX, FP8_E4M3_MAX)
+    q = pad.to(torch.float8_e4m3fn)
+    del pad, tiles
+    q = q[:R, :C].contiguous().view(torch.uint8).reshape(shape)
+    return {"e4m3": q, "scale": scale.contiguous()}
+
+
+def _matrix(shape, std, gen, device, wdtype):
+    if wdtype == 0:
+        return _normal_bf16(shape, std, gen, device)
+    t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    t.mul_(std)
+    return quantize_fp8_block128(t)
+
+
 def make_layer_weights(cfg: ModelConfig, gen: torch.Generator, device="cpu", w_std=0.02,
                        router_std=None, out_std=None) -> dict:
     """One layer.  ``out_std`` is the std of the two residual-branch output matrices (w_o, w_down);
-    it defaults to w_std."""
+    it defaults to w_std.  With cfg.wdtype == 1 the five matrices come in the FP8 form of
+    quantize_fp8_block128 (same random draws, no bf16 rounding before the quantisation)."""
     d, E, F = cfg.d_model, cfg.n_exp, cfg.d_ff
     if router_std is None:
         router_std = w_std
     if out_std is None:
         out_std = w_std
+    wd = cfg.wdtype
     return {
         "attn_norm": torch.ones(d, dtype=torch.float32, device=device),
-        "w_qkv": _normal_bf16((cfg.qkv_rows, d), w_std, gen, device),
-        "w_o": _normal_bf16((d, cfg.n_q * cfg.d_head), out_std, gen, device),
+        "w_qkv": _matrix((cfg.qkv_rows, d), w_std, gen, device, wd),
+        "w_o": _matrix((d, cfg.n_q * cfg.d_head), out_std, gen, device, wd),
         "ffn_norm": torch.ones(d, dtype=torch.float32, device=device),
-        "w_router": _normal_bf16((E, d), router_std, gen, device),
-        "w_gate_up": _normal_bf16((E, 2 * F, d), w_std, gen, device),
-        "w_down": _normal_bf16((E, d, F), out_std, gen, device),
+        "w_router": _matrix((E, d), router_std, gen, device, wd),
+        "w_gate_up": _matrix((E, 2 * F, d), w_std, gen, device, wd),
+        "w_down": _matrix((E, d, F), out_std, gen, device, wd),
     }
+
+
+def dequantize_fp8_block128(m: dict) -> torch.Tensor:
+    """fp64 weights q * s of the FP8 form (for building test inputs only)."""
+    q = m["e4m3"]
+    shape = q.shape
+    v = q.reshape(-1, shape[-1]).view(torch.float8_e4m3fn).double()
+    s = m["scale"].double().repeat_interleave(128, 0).repeat_interleave(128, 1)[:v.shape[0], :v.shape[1]]
+    return (v * s).reshape(shape)
 
 
 def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, router_std=None,

@@ -17,9 +17,9 @@ Judging rules.
   step's sequential GEMM inputs.  Each rounding adds a relative error of rms 2^-9/sqrt(3) to its
   products; with 2L+1 sequential roundings the rms relative error of z is about
   sqrt(2L+1) * 2^-9 / sqrt(3).  Judging at 4 sigma gives c_z = 4 sqrt(2L+1) 2^-9 / sqrt(3)
-  (1.0e-2 for L = 2).  Where c_z * std(z_row) exceeds the spec margin, ids are judged where the
-  oracle margin exceeds c_z * std(z_row), and entropies within c_z * (std(z) std_p(z) + Var_p(z))
-  (the first-order change of the entropy under a perturbation of that size: random part
+  (1.0e-2 for L = 2; FP8 weights add 5L roundings, see c_z).  Where c_z * std(z_row) exceeds
+  the spec margin, ids are judged where the oracle margin exceeds c_z * std(z_row), and
+  entropies within c_z * (std(z) std_p(z) + Var_p(z)) (the first-order change of the entropy under a perturbation of that size: random part
   std(dz) std_p(z), scale part Var_p(z) c_z).  These derived bounds reduce to the spec's at small
   logits and are only used by the tests that say so.
 """
@@ -29,14 +29,20 @@ import numpy as np
 import torch
 
 HIDDEN_TOL = 2e-2
+HIDDEN_TOL_FP8 = 6e-2      # hidden states with FP8 block-scaled weights
 ENTROPY_TOL = 1e-3
 MARGIN = 1e-2
 DECISION_BAND = 1e-3
 
 
+def _dev(v, device):
+    return {k: t.to(device) for k, t in v.items()} if isinstance(v, dict) else v.to(device)
+
+
 def to_device(w: dict, device="cuda") -> dict:
+    """Weights to the device; FP8 matrices ({"e4m3", "scale"}) move as pairs."""
     out = {k: v.to(device) for k, v in w.items() if k != "layers"}
-    out["layers"] = [{k: v.to(device) for k, v in L.items()} for L in w["layers"]]
+    out["layers"] = [{k: _dev(v, device) for k, v in L.items()} for L in w["layers"]]
     return out
 
 
@@ -70,15 +76,20 @@ def router_tie_tokens(router_logits, top_k, margin=MARGIN):
     return bad
 
 
-def c_z(n_layers):
-    return 4.0 * math.sqrt(2 * n_layers + 1) * 2.0 ** -9 / math.sqrt(3.0)
+def c_z(n_layers, fp8=False):
+    """4-sigma relative error of the tempered scores after n_r sequential bf16 roundings:
+    n_r = 2L+1 activation roundings; with FP8 weights each of the five per-layer matrices is also
+    rounded once (the kernels multiply bf16(q*s), the oracle q*s), 5L more roundings of the same
+    size, independent of the others."""
+    n_r = 2 * n_layers + 1 + (5 * n_layers if fp8 else 0)
+    return 4.0 * math.sqrt(n_r) * 2.0 ** -9 / math.sqrt(3.0)
 
 
-def derived_tolerances(logits, T, n_layers):
+def derived_tolerances(logits, T, n_layers, fp8=False):
     """Per-row (margin, entropy) judging tolerances for end-to-end steps at large logits (see the
     module docstring); never below the spec's 1e-2 / 1e-3."""
     z = np.asarray(logits, np.float64) / T
-    cz = c_z(n_layers)
+    cz = c_z(n_layers, fp8)
     std_z = z.std(axis=1)
     zs = z - z.max(axis=1, keepdims=True)
     p = np.exp(zs)

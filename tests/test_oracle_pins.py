@@ -466,3 +466,65 @@ def test_decode_invariants_with_confident_head():
             break
     assert r["stop"] == 1 and commit.all()
     assert 0 < s < 47            # some positions commit early and the block stops before the budget
+
+
+# ------------------------------------------------------------------------------------------------
+# FP8 weight form (e4m3 bytes with one fp32 scale per 128 x 128 tile)
+# ------------------------------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_float8_e4m3fn():
+    """Every one of the 256 codes decodes as torch's float8_e4m3fn (an independent implementation
+    of the OCP E4M3 format: subnormals, the 448 maximum, the two NaN codes, signed zero)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_double(int(q)) for q in range(256)])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and np.array_equal(nan, np.isnan(got))
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    np.testing.assert_array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    assert oracle.e4m3_to_double(0x7E) == 448.0 and oracle.e4m3_to_double(0x01) == 2.0 ** -9
+
+
+def _fp8_pow2_layer(cfg, seed):
+    """A layer in the FP8 form whose tile scales are distinct powers of two (so q * s is exactly a
+    bf16 value) together with the same layer as bf16 tensors holding q * s."""
+    rng = np.random.default_rng(seed)
+    shapes = {"w_qkv": (cfg.qkv_rows, cfg.d_model), "w_o": (cfg.d_model, cfg.n_q * cfg.d_head),
+              "w_router": (cfg.n_exp, cfg.d_model), "w_gate_up": (cfg.n_exp, 2 * cfg.d_ff, cfg.d_model),
+              "w_down": (cfg.n_exp, cfg.d_model, cfg.d_ff)}
+    fp8 = {"attn_norm": torch.ones(cfg.d_model), "ffn_norm": torch.ones(cfg.d_model)}
+    bf = dict(fp8)
+    for k, shp in shapes.items():
+        codes = rng.integers(0, 256, size=shp).astype(np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x38          # no NaN codes (0x38 = 1.0)
+        R, C = int(np.prod(shp[:-1])), shp[-1]
+        tr, tc = -(-R // 128), -(-C // 128)
+        expo = -(4 + (np.arange(tr)[:, None] * 3 + np.arange(tc)[None, :] * 5) % 7)
+        scale = np.ldexp(1.0, expo).astype(np.float32)
+        q = torch.from_numpy(codes)
+        fp8[k] = {"e4m3": q, "scale": torch.from_numpy(scale)}
+        s_full = torch.from_numpy(scale).double().repeat_interleave(128, 0).repeat_interleave(128, 1)[:R, :C]
+        w = q.view(torch.float8_e4m3fn).double().reshape(R, C) * s_full
+        wb = w.to(torch.bfloat16)
+        assert torch.equal(wb.double(), w)              # exactly representable
+        bf[k] = wb.reshape(shp)
+    return fp8, bf
+
+
+def test_fp8_layer_equals_bf16_layer_holding_q_times_s():
+    """The oracle's FP8 matrices are q * s with the scale of tile [r / 128][c / 128]: a layer in the
+    FP8 form equals, bit for bit, the layer given as bf16 weights q * s (distinct per-tile scales
+    catch a transposed or shifted tile index, in every matrix including the expert stacks)."""
+    cfg = synthetic.TINY
+    fp8, bf = _fp8_pow2_layer(cfg, 11)
+    M8 = oracle.Model(cfg, {"layers": [fp8]}, layers=[fp8])
+    Mb = oracle.Model(cfg, {"layers": [bf]}, layers=[bf])
+    rng = np.random.default_rng(12)
+    n, P = 10, 7
+    x = rng.normal(size=(n, cfg.d_model))
+    kc, vc = rng.normal(size=(P, cfg.n_kv, cfg.d_head)), rng.normal(size=(P, cfg.n_kv, cfg.d_head))
+    pos = np.arange(P, P + n)
+    a = oracle.layer_forward(M8, 0, x, pos, P, kc, vc)
+    b = oracle.layer_forward(Mb, 0, x, pos, P, kc, vc)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
