@@ -6,15 +6,20 @@
 // developer guide; the block-diagonal training mask in "Composition of DiffusionGemma" of the
 // technical-report summary).  Prompt prefill uses the same kernel with a causal mask.
 //
-// Grid: (query tile, key split, sequence x KV head).  A CTA owns 128 query rows of one GQA group
-// (the n_q/n_kv query heads that share a KV head are adjacent in the head-major query buffer, so a
-// 128-row tile is one TMA box) and a contiguous run of 128-key tiles.  Per key tile:
-//   S = Q K^T            (tcgen05, M=128 queries, N=128 keys, K=dh) -> TMEM
-//   online softmax       (one thread per query row, exp2 domain, fp32) -> P bf16 in swizzled smem
-//   O_t = P V            (tcgen05, M=128, N=dh, K=128 keys; V is cached transposed so both
-//                         operands are K-major) -> TMEM, folded into fp32 registers with the
-//                         running rescale.
-// Splits write un-normalised (O, m, l) partials; attn_merge_kernel combines them.
+// Grid: (query-tile pair, key split, sequence x KV head).  A CTA owns two 128-row query tiles of
+// one GQA group (the n_q/n_kv query heads that share a KV head are adjacent in the head-major query
+// buffer) and a contiguous run of 128-key tiles, so every K/V tile it loads serves 256 query rows.
+// Warp roles (320 threads):
+//   warp 8      TMA producer: both Q tiles once, then K(t), V(t), K(t+1), ... through a 3-buffer ring
+//   warp 9      MMA issuer:   S_x = Q_x K^T into TMEM, O_x += P_x V into TMEM, in the order
+//               S_0(0) S_1(0) | PV_0(t) S_0(t+1) PV_1(t) S_1(t+1) ..., so the tensor core works on
+//               one tile's products while the other tile's softmax runs
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1 (thread = query row): S from TMEM,
+//               row max, P = exp2(S - m) in bf16 to swizzled shared memory, running sum
+// The running max is updated lazily: O (in TMEM) and the sum are rescaled only when a row's max
+// grows by more than 2^8, so P stays below 256 and most tiles need no rescale; the final O / l is
+// the same.  With one key split the normalised row is written straight to the attention output;
+// otherwise un-normalised (O, m, l) partials go to attn_merge_kernel.
 #include <math.h>
 
 #include "dg_device.cuh"
@@ -24,226 +29,312 @@ namespace dg {
 
 template <int DH>
 struct AttnCfg {
-  static constexpr uint32_t kQBytes = 128u * DH * 2u;
-  static constexpr uint32_t kKBytes = 128u * DH * 2u;
-  static constexpr uint32_t kVBytes = (uint32_t)DH * 128u * 2u;
-  static constexpr uint32_t kPBytes = 128u * 128u * 2u;
-  static constexpr int kStages = 2;
-  static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
-  static constexpr uint32_t kTmemCols = 256;   // S in [0,128), O in [128, 128+DH)
-  static constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kPBytes + 256;
+  static constexpr uint32_t kTileBytes = 128u * DH * 2u;   // a Q tile, a K tile or a V tile (DH x 128 keys)
+  static constexpr uint32_t kPBytes = 128u * 128u * 2u;    // P: 128 rows x 128 keys, bf16
+  static constexpr int kBufs = 3;                          // K / V ring
+  static constexpr uint32_t kTmemCols = 512;               // S0 [0,128) S1 [128,256) O0 [256,..) O1 [384,..)
+  static constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kBufs * kTileBytes + 2 * kPBytes + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+constexpr int kAttnThreads = 320;
+constexpr float kLazyRescale = 8.f;   // log2 units: rescale O only when the max grows by more than this
 
 struct AttnBarriers {
-  uint64_t qfull;
-  uint64_t kvfull[2];
-  uint64_t s_done;
-  uint64_t o_done;
+  uint64_t q_full;
+  uint64_t kv_full[3], kv_empty[3];
+  uint64_t s_full[2], s_free[2], p_ready[2], pv_done[2];
   uint32_t tmem_slot;
 };
 
-template <int DH>
-__device__ __forceinline__ void attn_issue_kv(const CUtensorMap* tk, const CUtensorMap* tv, AttnBarriers* b,
-                                              uint8_t* stage, int s, int tile, int z) {
-  using C = AttnCfg<DH>;
-  mbar_arrive_expect_tx(&b->kvfull[s], C::kStageBytes);
-#pragma unroll
-  for (int h = 0; h < DH / 64; ++h) tma_load_3d(tk, &b->kvfull[s], stage + h * 16384, h * 64, tile * 128, z);
-#pragma unroll
-  for (int hk = 0; hk < 2; ++hk)
-    tma_load_3d(tv, &b->kvfull[s], stage + C::kKBytes + hk * (DH * 128), tile * 128 + hk * 64, 0, z);
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
 }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int DH>
-__global__ void __launch_bounds__(128, 1)
-    attn_partial_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, AttnParams p, int n_seq, int* err) {
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, AttnParams p, int n_seq, __nv_bfloat16* out, int* err) {
   using C = AttnCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = base;
-  uint8_t* kv_s = q_s + C::kQBytes;
-  uint8_t* p_s = kv_s + C::kStages * C::kStageBytes;
-  AttnBarriers* bars = reinterpret_cast<AttnBarriers*>(p_s + C::kPBytes);
+  uint8_t* q_s = base;                                  // 2 tiles
+  uint8_t* kv_s = q_s + 2 * C::kTileBytes;              // kBufs tiles
+  uint8_t* p_s = kv_s + C::kBufs * C::kTileBytes;       // 2 P tiles
+  AttnBarriers* bars = reinterpret_cast<AttnBarriers*>(p_s + 2 * C::kPBytes);
 
-  const int warp = threadIdx.x >> 5;
-  const int qt = blockIdx.x, split = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, split = blockIdx.y;
   const int seq = blockIdx.z / p.n_kv, kvh = blockIdx.z % p.n_kv;
   const int G = p.n_q / p.n_kv;
   const int cseq = p.seq_base + seq;
   pdl_trigger();
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->qfull, 1);
-    mbar_init(&bars->kvfull[0], 1);
-    mbar_init(&bars->kvfull[1], 1);
-    mbar_init(&bars->s_done, 1);
-    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->q_full, 1);
+    for (int b = 0; b < C::kBufs; ++b) {
+      mbar_init(&bars->kv_full[b], 1);
+      mbar_init(&bars->kv_empty[b], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_free[x], 4);
+      mbar_init(&bars->p_ready[x], 4);
+      mbar_init(&bars->pv_done[x], 1);
+    }
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&bars->tmem_slot, C::kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
-  pdl_wait();   // queries, keys, values and P come from the preceding kernels
+  pdl_wait();   // queries and the canvas keys / values come from the preceding kernels
 
   const int P = p.seq_P[cseq];
   const int nkeys = P + p.Tq;
   const int ntiles = (nkeys + 127) >> 7;
   const int t0 = split * p.tiles_per_split;
   const int t1 = min(ntiles, t0 + p.tiles_per_split);
-
-  // this thread's query row
-  const int rr = qt * 128 + threadIdx.x;
-  const int g = rr / p.rows_per_seq, j = rr % p.rows_per_seq;
-  const int h = kvh * G + g;
-  const bool row_valid = (g < G) && (j < p.Tq);
-  const int qpos = P + j;
-  const size_t prow = ((size_t)(split * n_seq + seq) * p.n_q + h) * p.rows_per_seq + j;
-
-  if (t0 >= t1) {   // empty split: neutral partial
-    if (row_valid) {
-      p.ml[prow * 2 + 0] = -INFINITY;
-      p.ml[prow * 2 + 1] = 0.f;
-      float4* o4 = reinterpret_cast<float4*>(p.opart + prow * DH);
-      for (int c = 0; c < DH / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
-    return;
-  }
-
-  const int qrow0 = (seq * p.n_q + kvh * G) * p.rows_per_seq + qt * 128;
+  const int T = t1 > t0 ? t1 - t0 : 0;
   const int z = p.layer * p.cache_seq_stride + cseq * p.n_kv + kvh;
-  const uint32_t t_s = tmem + ((uint32_t)(warp * 32) << 16);
-  const uint32_t t_o = t_s + 128;
+  const int qrow0 = (seq * p.n_q + kvh * G) * p.rows_per_seq + pair * 256;
 
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&bars->qfull, C::kQBytes);
+  if (warp == 8) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0 && T > 0) {
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+      for (int x = 0; x < 2; ++x)
 #pragma unroll
-    for (int hh = 0; hh < DH / 64; ++hh) tma_load_2d(&tq, &bars->qfull, q_s + hh * 16384, hh * 64, qrow0);
-    for (int t = t0; t < min(t1, t0 + C::kStages); ++t)
-      attn_issue_kv<DH>(&tk, &tv, bars, kv_s + (size_t)((t - t0) % C::kStages) * C::kStageBytes,
-                        (t - t0) % C::kStages, t, z);
-  }
-
-  const float sl2 = 1.4426950408889634f * rsqrtf((float)DH);
-  float o[DH];
+        for (int hh = 0; hh < DH / 64; ++hh)
+          tma_load_2d(&tq, &bars->q_full, q_s + x * C::kTileBytes + hh * 16384, hh * 64, qrow0 + x * 128);
+      for (int i = 0; i < 2 * T; ++i) {
+        const int b = i % C::kBufs;
+        if (!mbar_wait(&bars->kv_empty[b], ((i / C::kBufs) & 1) ^ 1, err, DEV_ERR_TIMEOUT_ATTN)) break;
+        uint8_t* dst = kv_s + (size_t)b * C::kTileBytes;
+        const int t = t0 + (i >> 1);
+        mbar_arrive_expect_tx(&bars->kv_full[b], C::kTileBytes);
+        if ((i & 1) == 0) {
 #pragma unroll
-  for (int c = 0; c < DH; ++c) o[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  bool ok = true;
-
-  for (int t = t0; t < t1; ++t) {
-    const int it = t - t0;
-    const int s = it % C::kStages;
-    uint8_t* stage = kv_s + (size_t)s * C::kStageBytes;
-    if (threadIdx.x == 0 && ok) {
-      if (it == 0) ok = mbar_wait(&bars->qfull, 0, err, DEV_ERR_TIMEOUT_ATTN);
-      if (ok) ok = mbar_wait(&bars->kvfull[s], (it / C::kStages) & 1, err, DEV_ERR_TIMEOUT_ATTN);
-      tc_fence_after();
-      if (ok) {
-        const uint32_t idesc = idesc_bf16_f32(128, 128);
+          for (int h = 0; h < DH / 64; ++h) tma_load_3d(&tk, &bars->kv_full[b], dst + h * 16384, h * 64, t * 128, z);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint64_t ad = desc_advance(smem_desc_sw128(smem_u32(q_s + (kk / 4) * 16384)), (kk % 4) * 32);
-          const uint64_t bd = desc_advance(smem_desc_sw128(smem_u32(stage + (kk / 4) * 16384)), (kk % 4) * 32);
-          umma_bf16(tmem, ad, bd, idesc, kk != 0);
+          for (int hk = 0; hk < 2; ++hk)
+            tma_load_3d(&tv, &bars->kv_full[b], dst + hk * (DH * 128), t * 128 + hk * 64, 0, z);
         }
       }
-      umma_commit(&bars->s_done);
     }
-    __syncwarp();
-    ok = mbar_wait(&bars->s_done, it & 1, err, DEV_ERR_TIMEOUT_ATTN) && ok;
-    tc_fence_after();
-
-    // ---- online softmax of this thread's row over the 128 keys of tile t ----
-    const int key0 = t * 128;
-    int kmax = nkeys - key0;                       // keys [key0, key0 + kmax) exist
-    if (p.causal) kmax = min(kmax, qpos - key0 + 1);
-    float tmax = -INFINITY;
+  } else if (warp == 9) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, DH);
+      bool ok = mbar_wait(&bars->q_full, 0, err, DEV_ERR_TIMEOUT_ATTN);
+      auto issue_s = [&](int x, int tt) {
+        const int i = 2 * tt, b = i % C::kBufs;
+        ok = ok && mbar_wait(&bars->kv_full[b], (i / C::kBufs) & 1, err, DEV_ERR_TIMEOUT_ATTN);
+        ok = ok && mbar_wait(&bars->s_free[x], (tt & 1) ^ 1, err, DEV_ERR_TIMEOUT_ATTN);
+        tc_fence_after();
+        if (ok) {
+          const uint8_t* kb = kv_s + (size_t)b * C::kTileBytes;
 #pragma unroll
-    for (int cb = 0; cb < 128; cb += 32) {
-      float v[32];
-      tmem_ld_32cols(t_s + cb, v);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint64_t ad =
+                desc_advance(smem_desc_sw128(smem_u32(q_s + x * C::kTileBytes + (kk / 4) * 16384)), (kk % 4) * 32);
+            const uint64_t bd = desc_advance(smem_desc_sw128(smem_u32(kb + (kk / 4) * 16384)), (kk % 4) * 32);
+            umma_bf16(tmem + x * 128, ad, bd, idesc_s, kk != 0);
+          }
+        }
+        umma_commit(&bars->s_full[x]);
+        if (x == 1) umma_commit(&bars->kv_empty[b]);   // both S products of K(t) issued
+      };
+      auto issue_pv = [&](int x, int tt) {
+        const int i = 2 * tt + 1, b = i % C::kBufs;
+        ok = ok && mbar_wait(&bars->kv_full[b], (i / C::kBufs) & 1, err, DEV_ERR_TIMEOUT_ATTN);
+        ok = ok && mbar_wait(&bars->p_ready[x], tt & 1, err, DEV_ERR_TIMEOUT_ATTN);
+        tc_fence_after();
+        if (ok) {
+          const uint8_t* vb = kv_s + (size_t)b * C::kTileBytes;
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (cb + i < kmax) tmax = fmaxf(tmax, v[i] * sl2);
-    }
-    const float m_new = fmaxf(m, tmax);
-    const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m - m_new);
-    float lt = 0.f;
-#pragma unroll
-    for (int cb = 0; cb < 128; cb += 32) {
-      float v[32];
-      tmem_ld_32cols(t_s + cb, v);
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float p0 = (cb + i < kmax) ? fast_exp2(v[i] * sl2 - m_new) : 0.f;
-        float p1 = (cb + i + 1 < kmax) ? fast_exp2(v[i + 1] * sl2 - m_new) : 0.f;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        lt += __low2float(b2) + __high2float(b2);
-        pk[i / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad =
+                desc_advance(smem_desc_sw128(smem_u32(p_s + x * C::kPBytes + (kk / 4) * 16384)), (kk % 4) * 32);
+            const uint64_t bd = desc_advance(smem_desc_sw128(smem_u32(vb + (kk / 4) * (DH * 128))), (kk % 4) * 32);
+            umma_bf16(tmem + 256 + x * 128, ad, bd, idesc_o, (tt | kk) != 0);
+          }
+        }
+        umma_commit(&bars->pv_done[x]);
+        if (x == 1) umma_commit(&bars->kv_empty[b]);   // both PV products of V(t) issued
+      };
+      issue_s(0, 0);
+      issue_s(1, 0);
+      for (int tt = 0; tt < T; ++tt) {
+        issue_pv(0, tt);
+        if (tt + 1 < T) issue_s(0, tt + 1);
+        issue_pv(1, tt);
+        if (tt + 1 < T) issue_s(1, tt + 1);
       }
-      // keys [cb, cb+32) of row threadIdx.x -> 4 swizzled 16-byte chunks
-      const int r = threadIdx.x;
-      uint8_t* prow_s = p_s + (cb / 64) * 16384 + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int chunk = ((cb % 64) / 8) + ch;
-        *reinterpret_cast<uint4*>(prow_s + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      }
     }
-    l = l * alpha + lt;
-    m = m_new;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    if (threadIdx.x == 0) {
+  } else {
+    // ------------------------------ softmax (warps 0-3: tile 0, warps 4-7: tile 1) ------------------------------
+    const int x = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + x * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + x * 128;
+    const int rr = pair * 256 + x * 128 + r;       // query row inside the GQA group
+    const int g = rr / p.rows_per_seq, j = rr % p.rows_per_seq;
+    const int h = kvh * G + g;
+    const bool row_valid = (g < G) && (j < p.Tq);
+    const int qpos = P + j;
+    const float sl2 = 1.4426950408889634f * rsqrtf((float)DH);
+    uint8_t* prow = p_s + x * C::kPBytes + r * 128;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int tt = 0; tt < T; ++tt) {
+      ok = ok && mbar_wait(&bars->s_full[x], tt & 1, err, DEV_ERR_TIMEOUT_ATTN);
       tc_fence_after();
-      if (ok) {
-        const uint32_t idesc = idesc_bf16_f32(128, DH);
+      const int key0 = (t0 + tt) * 128;
+      int kmax = nkeys - key0;                        // keys [key0, key0 + kmax) exist (and are visible)
+      if (p.causal) kmax = min(kmax, qpos - key0 + 1);
+      // pass 1 over S (TMEM): the row max of this tile
+      float tmax = -INFINITY;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = desc_advance(smem_desc_sw128(smem_u32(p_s + (kk / 4) * 16384)), (kk % 4) * 32);
-          const uint64_t bd =
-              desc_advance(smem_desc_sw128(smem_u32(stage + C::kKBytes + (kk / 4) * (DH * 128))), (kk % 4) * 32);
-          umma_bf16(tmem + 128, ad, bd, idesc, kk != 0);
+      for (int cb = 0; cb < 128; cb += 64) {
+        float s[64];
+        tmem_ld32_nowait(t_s + cb, s);
+        tmem_ld32_nowait(t_s + cb + 32, s + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (cb + i < kmax) tmax = fmaxf(tmax, s[i] * sl2);
+      }
+      // lazy max: O and l are rescaled only when this row's max grows by more than kLazyRescale
+      const bool grow = tmax > m_used + kLazyRescale;
+      const float m_new = grow ? tmax : m_used;
+      const float alpha = (grow && m_used != -INFINITY) ? fast_exp2(m_used - m_new) : 1.f;
+      l *= alpha;
+      m_used = m_new;
+      // PV(tt-1) of this tile completed before S(tt) (tensor-core operations complete in order), so O
+      // and this tile's P buffer are free here
+      if (tt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int cb = 0; cb < DH; cb += 32) {
+          float o[32];
+          tmem_ld32_nowait(t_o + cb, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_o + cb, o);
+        }
+        tmem_wait_st();
+      }
+      // pass 2: P = exp2(S - m) in bf16 to this tile's swizzled P buffer (4 x 16-byte chunks per 32 keys)
+      float lt = 0.f;
+#pragma unroll
+      for (int cb = 0; cb < 128; cb += 32) {
+        float s[32];
+        tmem_ld32_nowait(t_s + cb, s);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = cb + i < kmax ? fast_exp2(s[i] * sl2 - m_used) : 0.f;   // masked keys: 0
+          const float p1 = cb + i + 1 < kmax ? fast_exp2(s[i + 1] * sl2 - m_used) : 0.f;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          lt += __low2float(b2) + __high2float(b2);
+          pk[i / 2] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        uint8_t* prow_c = prow + (cb / 64) * 16384;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = ((cb % 64) / 8) + ch;
+          *reinterpret_cast<uint4*>(prow_c + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
       }
-      umma_commit(&bars->o_done);
+      l += lt;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->s_free[x]);    // S(tt) is read: S(tt+1) may overwrite it
+        mbar_arrive(&bars->p_ready[x]);
+      }
     }
-    __syncwarp();
-    ok = mbar_wait(&bars->o_done, it & 1, err, DEV_ERR_TIMEOUT_ATTN) && ok;
-    tc_fence_after();
-#pragma unroll
-    for (int cb = 0; cb < DH; cb += 32) {
-      float v[32];
-      tmem_ld_32cols(t_o + cb, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[cb + i] = o[cb + i] * alpha + v[i];
+    // ---- output ----
+    if (T > 0) {
+      ok = ok && mbar_wait(&bars->pv_done[x], (T - 1) & 1, err, DEV_ERR_TIMEOUT_ATTN);
+      tc_fence_after();
     }
-    tc_fence_before();
-    __syncthreads();
-    // stage s is free again (both MMAs that read it have completed): prefetch tile t + kStages
-    if (threadIdx.x == 0 && ok && t + C::kStages < t1) attn_issue_kv<DH>(&tk, &tv, bars, stage, s, t + C::kStages, z);
-  }
-
-  if (row_valid && ok) {
-    p.ml[prow * 2 + 0] = m;
-    p.ml[prow * 2 + 1] = l;
-    float4* o4 = reinterpret_cast<float4*>(p.opart + prow * DH);
+    const size_t prw = ((size_t)(split * n_seq + seq) * p.n_q + h) * p.rows_per_seq + j;
+    if (p.n_splits == 1) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = out + ((size_t)seq * p.rows_per_seq + j) * (p.n_q * DH) + h * DH;
 #pragma unroll
-    for (int c = 0; c < DH / 4; ++c) o4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+      for (int cb = 0; cb < DH; cb += 32) {
+        float o[32];
+        tmem_ld32_nowait(t_o + cb, o);
+        tmem_wait_ld();
+        if (row_valid && ok && T > 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+            *reinterpret_cast<uint4*>(dst + cb + i) =
+                make_uint4(pack_bf16x2(o[i] * inv, o[i + 1] * inv), pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv),
+                           pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv), pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv));
+        }
+      }
+    } else if (T == 0) {   // empty split: neutral partial
+      if (row_valid) {
+        p.ml[prw * 2 + 0] = -INFINITY;
+        p.ml[prw * 2 + 1] = 0.f;
+        float4* o4 = reinterpret_cast<float4*>(p.opart + prw * DH);
+        for (int c = 0; c < DH / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    } else {
+      float4* o4 = reinterpret_cast<float4*>(p.opart + prw * DH);
+#pragma unroll
+      for (int cb = 0; cb < DH; cb += 32) {
+        float o[32];
+        tmem_ld32_nowait(t_o + cb, o);
+        tmem_wait_ld();
+        if (row_valid && ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) o4[(cb + i) / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        }
+      }
+      if (row_valid && ok) {
+        p.ml[prw * 2 + 0] = m_used;
+        p.ml[prw * 2 + 1] = l;
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // One warp per (sequence, query head, row): combine the split partials (lane s < n_splits holds
@@ -297,24 +388,27 @@ __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
 
 template <int DH>
 static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                               const AttnParams& p, int n_seq, int* err, cudaStream_t st) {
+                               const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
   using C = AttnCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_partial_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int G = p.n_q / p.n_kv;
-  dim3 grid((G * p.rows_per_seq + 127) / 128, p.n_splits, n_seq * p.n_kv);
-  return launch_k(attn_partial_kernel<DH>, grid, dim3(128), C::kSmemBytes, st, 1, tq, tk, tv, p, n_seq, err);
+  dim3 grid((G * p.rows_per_seq + 255) / 256, p.n_splits, n_seq * p.n_kv);
+  return launch_k(attn_fwd_kernel<DH>, grid, dim3(kAttnThreads), C::kSmemBytes, st, 1, tq, tk, tv, p, n_seq, out,
+                  err);
 }
 
+// n_splits == 1: the attention output is written directly to `out`; otherwise the partials are
+// left for attention_merge.
 cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const AttnParams& p, int n_seq, int* err, cudaStream_t st) {
-  if (p.dh == 128) return launch_attn<128>(tq, tk, tv, p, n_seq, err, st);
-  if (p.dh == 64) return launch_attn<64>(tq, tk, tv, p, n_seq, err, st);
+                              const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
+  if (p.dh == 128) return launch_attn<128>(tq, tk, tv, p, n_seq, out, err, st);
+  if (p.dh == 64) return launch_attn<64>(tq, tk, tv, p, n_seq, out, err, st);
   return cudaErrorInvalidValue;
 }
 

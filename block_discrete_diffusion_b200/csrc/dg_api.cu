@@ -56,7 +56,7 @@ struct NvtxRange {
 };
 
 constexpr int kCanvas = 256;
-constexpr int kSplitTargetCtas = 296;   // two waves of CTAs over the 148 SMs
+constexpr int kAttnTargetCtas = 148;    // attention CTAs hold a whole SM (all of TMEM)
 constexpr int kMaxSplits = 16;
 constexpr int kRouterSplits = 8;        // cluster size of the router GEMM's split-K
 constexpr int kGemmTargetCtas = 296;    // two CTAs per SM for the 128-wide dense GEMM tiles
@@ -143,11 +143,12 @@ void layer_matrix_shapes(const dg_model_config& c, uint64_t rows[5], uint64_t co
   rows[4] = (uint64_t)c.n_exp * d;                   cols[4] = c.d_ff;
 }
 
+// Key splits of the attention: one CTA (a pair of 128-row query tiles) per SM, about one wave.
 int attn_split_cap(const dg_model_config& c, int n_seq) {
   const int G = c.n_q / c.n_kv;
-  const int qtiles = (G * kCanvas + 127) / 128;
-  const int base = qtiles * n_seq * c.n_kv;
-  return std::max(1, std::min(kMaxSplits, (kSplitTargetCtas + base - 1) / base));
+  const int pairs = (G * kCanvas + 255) / 256;
+  const int base = pairs * n_seq * c.n_kv;
+  return std::max(1, std::min(kMaxSplits, (kAttnTargetCtas + base - 1) / base));
 }
 
 WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
@@ -594,8 +595,8 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   ap.seq_P = s->seqP;
   ap.opart = s->opart;
   ap.ml = s->ml;
-  LAUNCH(s, DG_K_ATTN, 1, attention_partial(s->q_map, s->k_map, s->v_map, ap, n_local, s->err, st));
-  LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
+  LAUNCH(s, DG_K_ATTN, 1, attention_partial(s->q_map, s->k_map, s->v_map, ap, n_local, s->attn, s->err, st));
+  if (ap.n_splits > 1) LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
 
   EpiParams eo{};
   eo.x = x;
