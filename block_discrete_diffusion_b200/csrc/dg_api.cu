@@ -633,8 +633,10 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   xp.y_out = s->y;
   xp.d = d;
   xp.F = c.d_ff;
-  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->m->n_sms, s->err, st));
-  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->m->n_sms, s->err, st));
+  // many tokens per expert on average (several canvases): 256-token accumulator chunks
+  const int wide = rows * c.top_k >= 128 * c.n_exp ? 1 : 0;
+  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
+  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
   LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
   return DG_OK;
 }

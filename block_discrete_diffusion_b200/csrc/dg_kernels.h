@@ -106,9 +106,10 @@ struct AttnParams {
 
 cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const EpiParams& ep, int* err, cudaStream_t st);
-// persistent: n_ctas CTAs (one per SM) loop over the (expert, weight tile) items
+// persistent: n_ctas CTAs (one per SM) loop over the (expert, weight tile) items; wide selects
+// 256-token (else 64-token) accumulator chunks
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
-                        int n_ctas, int* err, cudaStream_t st);
+                        int n_ctas, int wide, int* err, cudaStream_t st);
 cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st);
 cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st);

@@ -12,7 +12,7 @@
 //                Gemma-style layer, read from "same architecture as Gemma 4 26B A4B").
 //     EPI_RESID  x += D (attention output projection + residual).
 //     EPI_F32    out = D (router logits, vocabulary logits).
-//   expert_gemm_kernel<MODE>     grouped, swap-AB (weights are the 128-row M side, the few tokens
+//   expert_gemm_kernel<MODE, BN> grouped, swap-AB (weights are the 128-row M side, the few tokens
 //                routed to one expert are the N side):
 //     MODE 1     [gate | up] rows of expert e times its gathered tokens; SwiGLU in the epilogue.
 //     MODE 2     down-projection rows of expert e times its SwiGLU rows, scaled by each
@@ -338,17 +338,23 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
 // rows through a ring of shared-memory stages that runs on across items; warp 1 issues the MMAs
 // into one of two TMEM accumulators; warps 2-5 drain the other accumulator, so the epilogue of one
 // chunk overlaps the MMAs of the next.
-constexpr int kExpBN = 64;                         // tokens per accumulator chunk
-constexpr int kExpStages = 7;
+// BN = tokens per accumulator chunk: 64 when a few tokens reach each expert (batch 1), 256 when
+// hundreds do (several canvases), so that a weight tile is streamed once per 256 tokens.
+template <int BN>
+struct ExpCfg {
+  static constexpr int kStages = BN >= 256 ? 4 : 7;
+  static constexpr uint32_t kBTile = BN * 64 * 2;            // BN token rows x 64 k (32-row boxes)
+  static constexpr uint32_t kStageBytes = kATileBytes + kBTile;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 128 * 65 * 4 + 512;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 constexpr int kExpThreads = 192;                   // 6 warps
-constexpr uint32_t kExpBTile = kExpBN * 64 * 2;    // 8 KB: two 32-row boxes
-constexpr uint32_t kExpStageBytes = kATileBytes + kExpBTile;
-constexpr int kEpiStride = kExpBN + 1;             // padded fp32 staging rows
-constexpr size_t kExpSmemBytes = 1024 + (size_t)kExpStages * kExpStageBytes + 128 * kEpiStride * 4 + 512;
+constexpr int kEpiCols = 64;                       // MODE 1 epilogue slice (accumulator columns)
+constexpr int kEpiStride = kEpiCols + 1;           // padded fp32 staging rows
 
 struct ExpBarriers {
-  uint64_t full[kExpStages];
-  uint64_t empty[kExpStages];
+  uint64_t full[8];
+  uint64_t empty[8];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_slot;
@@ -358,13 +364,17 @@ __device__ __forceinline__ void epi_bar_sync() {   // the 128 epilogue threads o
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-template <int MODE>
+template <int MODE, int BN>
 __global__ void __launch_bounds__(kExpThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
   uint8_t* tiles = align1024(smem_raw);
+  using C = ExpCfg<BN>;
+  constexpr int kExpStages = C::kStages;
+  constexpr uint32_t kExpStageBytes = C::kStageBytes;
+  constexpr int kExpBN = BN;
   float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kExpStages * kExpStageBytes);
   ExpBarriers* bars = reinterpret_cast<ExpBarriers*>(stage_out + 128 * kEpiStride);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -478,34 +488,41 @@ __global__ void __launch_bounds__(kExpThreads, 1)
         tc_fence_after();
         const uint32_t acc = tmem + ((uint32_t)(quarter * 32) << 16) + b * kExpBN;
         if (MODE == 1) {
-          for (int cb = 0; cb < nmma; cb += 32) {
-            float v[32];
-            tmem_ld_32cols(acc + cb, v);
+          // slices of kEpiCols tokens: accumulator -> staging rows -> SwiGLU of (gate row f, up row 64 + f)
+          for (int cs = 0; cs < nmma; cs += kEpiCols) {
+            const int ncs = min(kEpiCols, nmma - cs);
+            for (int cb = 0; cb < ncs; cb += 32) {
+              float v[32];
+              tmem_ld_32cols(acc + cs + cb, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) stage_out[r * kEpiStride + cb + i] = v[i];
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
-          epi_bar_sync();
-          if (ok) {
-            // thread -> (token n = et/4 + 32*pass, features f = (et%4)*16 .. +16); gate rows 0-63, up rows 64-127
-            const int fq = (et & 3) * 16;
-            for (int n = et >> 2; n < nc; n += 32) {
-              uint32_t packed[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                const float g0 = stage_out[(fq + i) * kEpiStride + n], u0 = stage_out[(64 + fq + i) * kEpiStride + n];
-                const float g1 = stage_out[(fq + i + 1) * kEpiStride + n],
-                            u1 = stage_out[(64 + fq + i + 1) * kEpiStride + n];
-                packed[i / 2] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(off + c0 + n) * p.F + mt * 64 + fq);
-              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              for (int i = 0; i < 32; ++i) stage_out[r * kEpiStride + cb + i] = v[i];
             }
+            if (cs + kEpiCols >= nmma) {          // last TMEM read of this accumulator: release it
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+            }
+            epi_bar_sync();
+            if (ok) {
+              // thread -> (token n = et/4 + 32*pass, features f = (et%4)*16 .. +16); gate rows 0-63, up rows 64-127
+              const int fq = (et & 3) * 16;
+              const int ncv = min(ncs, nc - cs);
+              for (int n = et >> 2; n < ncv; n += 32) {
+                uint32_t packed[8];
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                  const float g0 = stage_out[(fq + i) * kEpiStride + n], u0 = stage_out[(64 + fq + i) * kEpiStride + n];
+                  const float g1 = stage_out[(fq + i + 1) * kEpiStride + n],
+                              u1 = stage_out[(64 + fq + i + 1) * kEpiStride + n];
+                  packed[i / 2] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(off + c0 + cs + n) * p.F + mt * 64 + fq);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              }
+            }
+            epi_bar_sync();   // the staging buffer is rewritten by the next slice
           }
-          epi_bar_sync();   // the staging buffer is rewritten by the next chunk
         } else {
           const int m = mt * 128 + r;             // output feature of the down projection
           for (int cb = 0; cb < nmma; cb += 32) {
@@ -584,27 +601,32 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
   return cudaErrorInvalidValue;
 }
 
-template <int MODE>
+template <int MODE, int BN>
 static cudaError_t launch_expert(const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                                  int n_ctas, int* err, cudaStream_t st) {
+  using C = ExpCfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kExpSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(expert_gemm_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int items = n_exp * (MODE == 1 ? p.F / 64 : p.d / 128);
-  return launch_k(expert_gemm_kernel<MODE>, dim3(n_ctas < items ? n_ctas : items), dim3(kExpThreads), kExpSmemBytes,
-                  st, 1, w, x, p, n_exp, err);
+  return launch_k(expert_gemm_kernel<MODE, BN>, dim3(n_ctas < items ? n_ctas : items), dim3(kExpThreads),
+                  C::kSmemBytes, st, 1, w, x, p, n_exp, err);
 }
 
+// wide = 1: 256-token accumulator chunks (many tokens per expert); 0: 64-token chunks.
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
-                        int n_ctas, int* err, cudaStream_t st) {
-  return mode == 1 ? launch_expert<1>(w, x, p, n_exp, n_ctas, err, st)
-                   : launch_expert<2>(w, x, p, n_exp, n_ctas, err, st);
+                        int n_ctas, int wide, int* err, cudaStream_t st) {
+  if (wide)
+    return mode == 1 ? launch_expert<1, 256>(w, x, p, n_exp, n_ctas, err, st)
+                     : launch_expert<2, 256>(w, x, p, n_exp, n_ctas, err, st);
+  return mode == 1 ? launch_expert<1, 64>(w, x, p, n_exp, n_ctas, err, st)
+                   : launch_expert<2, 64>(w, x, p, n_exp, n_ctas, err, st);
 }
 
 }  // namespace dg
