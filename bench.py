@@ -41,6 +41,7 @@ WORKLOAD = ("full_b1: 30-layer Gemma-4-26B-A4B-shaped MoE (d 2816, 16/8 heads x 
 
 def parse():
     ap = argparse.ArgumentParser()
+    seqs_given = any(a == "--seqs" or a.startswith("--seqs=") for a in sys.argv[1:])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=24)
     ap.add_argument("--warmup", type=int, default=3)
@@ -52,7 +53,10 @@ def parse():
                          "fp8_b32: the 30-layer FP8 stack on 32 sequences behind 32768-token prefixes")
     ap.add_argument("--seqs", type=int, default=32, help="fp8_b32: number of sequences")
     ap.add_argument("--prefix", type=int, default=32768, help="fp8_b32: prefix length of every sequence")
-    return ap.parse_args()
+    ap.add_argument("--fp8", action="store_true", help="one_layer: FP8 block-scaled weights")
+    a = ap.parse_args()
+    a.seqs_given = seqs_given
+    return a
 
 
 def peaks():
@@ -458,14 +462,17 @@ def main_aux(args):
     dev = torch.device("cuda", 0)
     if args.workload == "one_layer":
         # one decoder layer at full width: x ~ N(0,1) [256, 2816], prefix K/V ~ N(0,1) of 4096 tokens
-        cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024)
+        # --seqs n (default 1) canvases each behind a 4096-token prefix; --fp8: FP8 block-scaled weights
+        cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024, wdtype=1 if args.fp8 else 0)
+        n_seq = args.seqs if args.seqs_given else 1
         w = synthetic.make_model_weights(cfg, 1, device=dev, router_std=cfg.d_model ** -0.5)
         model = dg.dg_model_create(cfg, w)
         P = 4096
-        seqs = dg.dg_seqs_create(model, 1, P + CANVAS)
-        ks, vs = synthetic.make_prefix_kv(1, P, cfg.n_kv, cfg.d_head, 1, device=dev)
-        dg.dg_load_prefix(seqs, 0, P, ks, vs)
-        x0 = synthetic.make_hidden(CANVAS, cfg.d_model, 1, device=dev)
+        seqs = dg.dg_seqs_create(model, n_seq, P + CANVAS)
+        for i in range(n_seq):
+            ks, vs = synthetic.make_prefix_kv(1, P, cfg.n_kv, cfg.d_head, 1 + i, device=dev)
+            dg.dg_load_prefix(seqs, i, P, ks, vs)
+        x0 = synthetic.make_hidden(n_seq * CANVAS, cfg.d_model, 1, device=dev)
         x = x0.clone()
 
         def step():
@@ -478,8 +485,9 @@ def main_aux(args):
         stats = dg.dg_stats_read(seqs)
         line = {"metric": "decoder-layer steps/s (a2-a9, one full-width layer)", "value": round(1 / t, 2),
                 "unit": "steps/s", "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
-                "config": {"workload": "one_layer: d 2816, 16/8 heads x 128, 128 experts top-8 FFN 704, "
-                                       "prefix 4096 tokens, canvas 256, bf16"},
+                "config": {"workload": f"one_layer: d 2816, 16/8 heads x 128, 128 experts top-8 FFN 704, "
+                                       f"{n_seq} canvas(es) of 256 each behind a 4096-token prefix, "
+                                       f"{'fp8 e4m3 block-scaled' if args.fp8 else 'bf16'} weights"},
                 "kernel_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in stats.items() if v[0]}}
     else:
         vocab, canvas = 262144, 256

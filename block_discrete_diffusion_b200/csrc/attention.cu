@@ -220,61 +220,92 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int key0 = (t0 + tt) * 128;
       int kmax = nkeys - key0;                        // keys [key0, key0 + kmax) exist (and are visible)
       if (p.causal) kmax = min(kmax, qpos - key0 + 1);
-      // pass 1 over S (TMEM): the row max of this tile
-      float tmax = -INFINITY;
+      const bool full = kmax >= 128;                  // no masked key in this tile for this row
+      // P pass: P = exp2(S scale - m_ref) in bf16 to this tile's swizzled P buffer (4 x 16-byte chunks
+      // per 32 keys); returns the fp32 sum and the raw max of the visible scores
+      auto p_pass = [&](float m_ref, float& rmax) {
+        float lt = 0.f;
+        rmax = -INFINITY;
 #pragma unroll
-      for (int cb = 0; cb < 128; cb += 64) {
-        float s[64];
-        tmem_ld32_nowait(t_s + cb, s);
-        tmem_ld32_nowait(t_s + cb + 32, s + 32);
-        tmem_wait_ld();
+        for (int cb = 0; cb < 128; cb += 32) {
+          float s[32];
+          tmem_ld32_nowait(t_s + cb, s);
+          tmem_wait_ld();
+          uint32_t pk[16];
+          if (full) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (cb + i < kmax) tmax = fmaxf(tmax, s[i] * sl2);
-      }
-      // lazy max: O and l are rescaled only when this row's max grows by more than kLazyRescale
-      const bool grow = tmax > m_used + kLazyRescale;
-      const float m_new = grow ? tmax : m_used;
-      const float alpha = (grow && m_used != -INFINITY) ? fast_exp2(m_used - m_new) : 1.f;
-      l *= alpha;
-      m_used = m_new;
+            for (int i = 0; i < 32; i += 2) {
+              rmax = fmaxf(rmax, fmaxf(s[i], s[i + 1]));
+              const float p0 = fast_exp2(fmaf(s[i], sl2, -m_ref));
+              const float p1 = fast_exp2(fmaf(s[i + 1], sl2, -m_ref));
+              lt += p0 + p1;
+              pk[i / 2] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const bool v0 = cb + i < kmax, v1 = cb + i + 1 < kmax;   // masked keys: p = 0
+              if (v0) rmax = fmaxf(rmax, s[i]);
+              if (v1) rmax = fmaxf(rmax, s[i + 1]);
+              const float p0 = v0 ? fast_exp2(fmaf(s[i], sl2, -m_ref)) : 0.f;
+              const float p1 = v1 ? fast_exp2(fmaf(s[i + 1], sl2, -m_ref)) : 0.f;
+              lt += p0 + p1;
+              pk[i / 2] = pack_bf16x2(p0, p1);
+            }
+          }
+          uint8_t* prow_c = prow + (cb / 64) * 16384;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int chunk = ((cb % 64) / 8) + ch;
+            *reinterpret_cast<uint4*>(prow_c + ((chunk ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          }
+        }
+        return lt;
+      };
       // PV(tt-1) of this tile completed before S(tt) (tensor-core operations complete in order), so O
-      // and this tile's P buffer are free here
-      if (tt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      // and this tile's P buffer are free here.  Optimistic single pass against the running max; a
+      // warp redoes the tile when one of its rows' max grew by more than kLazyRescale (or has none yet).
+      float rmax = -INFINITY, lt = 0.f;
+      bool redo = m_used == -INFINITY;
+      if (!__any_sync(0xffffffffu, redo)) {
+        lt = p_pass(m_used, rmax);
+        redo = rmax * sl2 > m_used + kLazyRescale;
+      }
+      if (__any_sync(0xffffffffu, redo)) {
+        // the row max of this tile (raw scores; the scale is positive); every lane of the warp takes
+        // part in the collective TMEM loads, also lanes whose row needs no redo
+        rmax = -INFINITY;
 #pragma unroll
-        for (int cb = 0; cb < DH; cb += 32) {
-          float o[32];
-          tmem_ld32_nowait(t_o + cb, o);
+        for (int cb = 0; cb < 128; cb += 64) {
+          float s[64];
+          tmem_ld32_nowait(t_s + cb, s);
+          tmem_ld32_nowait(t_s + cb + 32, s + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(t_o + cb, o);
+          for (int i = 0; i < 64; ++i)
+            if (cb + i < kmax) rmax = fmaxf(rmax, s[i]);
         }
-        tmem_wait_st();
-      }
-      // pass 2: P = exp2(S - m) in bf16 to this tile's swizzled P buffer (4 x 16-byte chunks per 32 keys)
-      float lt = 0.f;
+        // lazy max: O and l are rescaled only when this row's max grows by more than kLazyRescale
+        const float tmax = rmax * sl2;
+        const bool grow = redo && tmax > m_used + kLazyRescale;
+        const float m_new = grow ? tmax : m_used;
+        const float alpha = (grow && m_used != -INFINITY) ? fast_exp2(m_used - m_new) : 1.f;
+        l *= alpha;
+        m_used = m_new;
+        if (tt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) {
-        float s[32];
-        tmem_ld32_nowait(t_s + cb, s);
-        tmem_wait_ld();
-        uint32_t pk[16];
+          for (int cb = 0; cb < DH; cb += 32) {
+            float o[32];
+            tmem_ld32_nowait(t_o + cb, o);
+            tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = cb + i < kmax ? fast_exp2(s[i] * sl2 - m_used) : 0.f;   // masked keys: 0
-          const float p1 = cb + i + 1 < kmax ? fast_exp2(s[i + 1] * sl2 - m_used) : 0.f;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          lt += __low2float(b2) + __high2float(b2);
-          pk[i / 2] = *reinterpret_cast<uint32_t*>(&b2);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(t_o + cb, o);
+          }
+          tmem_wait_st();
         }
-        uint8_t* prow_c = prow + (cb / 64) * 16384;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = ((cb % 64) / 8) + ch;
-          *reinterpret_cast<uint4*>(prow_c + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        }
+        lt = p_pass(m_used, rmax);   // rows without a redo recompute the values they already wrote
       }
       l += lt;
       fence_proxy_async_smem();

@@ -143,12 +143,26 @@ void layer_matrix_shapes(const dg_model_config& c, uint64_t rows[5], uint64_t co
   rows[4] = (uint64_t)c.n_exp * d;                   cols[4] = c.d_ff;
 }
 
-// Key splits of the attention: one CTA (a pair of 128-row query tiles) per SM, about one wave.
+// Key splits of the attention.  A CTA (a pair of 128-row query tiles) holds a whole SM.  Few
+// CTAs: split the keys until about one wave is busy.  Many CTAs: at most 4 splits, the count that
+// wastes the least of the last wave (a split costs one merge pass, so 1 wins near-ties).
 int attn_split_cap(const dg_model_config& c, int n_seq) {
   const int G = c.n_q / c.n_kv;
   const int pairs = (G * kCanvas + 255) / 256;
   const int base = pairs * n_seq * c.n_kv;
-  return std::max(1, std::min(kMaxSplits, (kAttnTargetCtas + base - 1) / base));
+  if (base < kAttnTargetCtas) return std::max(1, std::min(kMaxSplits, (kAttnTargetCtas + base - 1) / base));
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= 4; ++sp) {
+    const int ctas = base * sp;
+    const int waves = (ctas + kAttnTargetCtas - 1) / kAttnTargetCtas;
+    const double eff = (double)ctas / ((double)waves * kAttnTargetCtas) - 0.02 * (sp > 1);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = sp;
+    }
+  }
+  return best;
 }
 
 WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
@@ -637,7 +651,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   const int wide = rows * c.top_k >= 128 * c.n_exp ? 1 : 0;
   LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
   LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
-  LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
+  LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
   return DG_OK;
 }
 

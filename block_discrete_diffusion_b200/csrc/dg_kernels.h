@@ -129,7 +129,7 @@ cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* co
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st);
 // g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g
-cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x, const float* g,
+cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x, const float* g,
                         float eps, __nv_bfloat16* xn, cudaStream_t st);
 cudaError_t sum_planes(float* out, const float* in, int n_planes, size_t stride, size_t n, cudaStream_t st);
 cudaError_t add_to_P(int* seq_P, int first, int count, int delta, cudaStream_t st);

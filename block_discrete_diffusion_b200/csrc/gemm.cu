@@ -15,8 +15,8 @@
 //   expert_gemm_kernel<MODE, BN> grouped, swap-AB (weights are the 128-row M side, the few tokens
 //                routed to one expert are the N side):
 //     MODE 1     [gate | up] rows of expert e times its gathered tokens; SwiGLU in the epilogue.
-//     MODE 2     down-projection rows of expert e times its SwiGLU rows, scaled by each
-//                assignment's gate weight (top-k routed MoE of the 26B-A4B model, 3.8B active).
+//     MODE 2     down-projection rows of expert e times its SwiGLU rows (the combine applies the
+//                gate weights; top-k routed MoE of the 26B-A4B model, 3.8B active).
 #include "dg_device.cuh"
 #include "dg_kernels.h"
 
@@ -404,7 +404,9 @@ __global__ void __launch_bounds__(kExpThreads, 1)
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
+      // narrow chunks read every weight tile once: evict first; wide chunks read it once per 256
+      // tokens, a few microseconds apart: keep the normal policy so the re-read hits L2
+      const uint64_t pol_w = BN >= 256 ? l2_policy_evict_normal() : l2_policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -539,7 +541,7 @@ __global__ void __launch_bounds__(kExpThreads, 1)
               const int n = cb + i;
               if (n < nc) {
                 const int rowa = off + c0 + n;
-                p.y_out[(size_t)rowa * p.d + m] = v[i] * p.perm_gate[rowa];
+                p.y_out[(size_t)rowa * p.d + m] = v[i];
               }
             }
           }

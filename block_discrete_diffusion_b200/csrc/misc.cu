@@ -254,17 +254,21 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const i
   }
 }
 
-// x[t] += sum over ranks r (in rank order) of y[slot[t*k + r]]; with g != nullptr also the next
+// x[t] += sum over ranks r (in rank order) of gate[t][r] * y[slot[t*k + r]]; with g != nullptr also the next
 // RMSNorm of the updated row: xn[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g).
-__global__ void moe_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot, int top_k, int d,
-                                   float* __restrict__ x, const float* __restrict__ g, float eps,
-                                   __nv_bfloat16* __restrict__ xn) {
+__global__ void moe_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot,
+                                   const float* __restrict__ gate, int top_k, int d, float* __restrict__ x,
+                                   const float* __restrict__ g, float eps, __nv_bfloat16* __restrict__ xn) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x;
   __shared__ int rows[32];
+  __shared__ float gw[32];
   __shared__ float red[32];
-  if (threadIdx.x < top_k) rows[threadIdx.x] = slot[(size_t)t * top_k + threadIdx.x];
+  if (threadIdx.x < top_k) {
+    rows[threadIdx.x] = slot[(size_t)t * top_k + threadIdx.x];
+    gw[threadIdx.x] = gate[(size_t)t * top_k + threadIdx.x];
+  }
   __syncthreads();
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
   float ss = 0.f;
@@ -272,7 +276,8 @@ __global__ void moe_combine_kernel(const float* __restrict__ y, const int32_t* _
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r = 0; r < top_k; ++r) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(y + (size_t)rows[r] * d) + c);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      const float w = gw[r];
+      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
     }
     float4 o = xr[c];
     o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
@@ -376,10 +381,10 @@ cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows
   if (n_rows <= 0) return cudaSuccess;
   return launch_k(gather_rows_kernel, dim3((n_rows + 7) / 8), dim3(256), 0, st, 1, xn, slot, n_rows, top_k, d, xp);
 }
-cudaError_t moe_combine(const float* y, const int32_t* slot, int n_rows, int top_k, int d, float* x, const float* g,
-                        float eps, __nv_bfloat16* xn, cudaStream_t st) {
+cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x,
+                        const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  return launch_k(moe_combine_kernel, dim3(n_rows), dim3(256), 0, st, 1, y, slot, top_k, d, x, g, eps, xn);
+  return launch_k(moe_combine_kernel, dim3(n_rows), dim3(256), 0, st, 1, y, slot, gate, top_k, d, x, g, eps, xn);
 }
 cudaError_t sum_planes(float* out, const float* in, int n_planes, size_t stride, size_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
