@@ -39,6 +39,10 @@ WORKLOAD = ("full_b1: 30-layer Gemma-4-26B-A4B-shaped MoE (d 2816, 16/8 heads x 
             "128 experts of every layer), batch 1, 2048-token prompt, 256-token canvas, 12 fixed steps per block")
 
 
+WORKLOAD_FP8 = WORKLOAD.replace("bf16 random-init", "FP8 e4m3 per-layer matrices (fp32 scale per 128x128 tile; "
+                                                   "embedding and head bf16) random-init")
+
+
 def parse():
     ap = argparse.ArgumentParser()
     seqs_given = any(a == "--seqs" or a.startswith("--seqs=") for a in sys.argv[1:])
@@ -53,7 +57,7 @@ def parse():
                          "fp8_b32: the 30-layer FP8 stack on 32 sequences behind 32768-token prefixes")
     ap.add_argument("--seqs", type=int, default=32, help="fp8_b32: number of sequences")
     ap.add_argument("--prefix", type=int, default=32768, help="fp8_b32: prefix length of every sequence")
-    ap.add_argument("--fp8", action="store_true", help="one_layer: FP8 block-scaled weights")
+    ap.add_argument("--fp8", action="store_true", help="full_b1 / one_layer: FP8 block-scaled per-layer weights")
     a = ap.parse_args()
     a.seqs_given = seqs_given
     return a
@@ -169,13 +173,15 @@ def whole_job_rate(world, units_per_rank, t_max):
 # ------------------------------------------------------------------------------------------------
 # the CUDA path
 # ------------------------------------------------------------------------------------------------
-def setup_full(rank, device):
+def setup_full(rank, device, fp8=False):
+    import dataclasses
+
     import torch
 
     import synthetic
     from block_discrete_diffusion_b200 import dg
 
-    cfg = synthetic.FULL
+    cfg = dataclasses.replace(synthetic.FULL, wdtype=1 if fp8 else 0)
     w = synthetic.make_model_weights(cfg, seed=replica_seed(rank), device=device, **synthetic.full_stack_init(cfg))
     model = dg.dg_model_create(cfg, w)
     max_ctx = PROMPT + BLOCKS * CANVAS
@@ -203,11 +209,14 @@ def run_steps(dg, seqs, prm, st, k, state):
 
 
 def expert_up_bytes(cfg):
-    """Algorithmic bytes of one grouped gate|up launch at batch 1: every expert's [2F x d] bf16
-    weights (all 128 experts are routed to with probability 1 - 128*(120/128)^256 > 0.99999), the
-    gathered activations read once, the SwiGLU rows written once."""
+    """Algorithmic bytes of one grouped gate|up launch at batch 1: every expert's [2F x d] weights
+    (bf16, or e4m3 bytes plus one fp32 scale per 128x128 tile; all 128 experts are routed to with
+    probability 1 - 128*(120/128)^256 > 0.99999), the gathered activations read once, the SwiGLU
+    rows written once."""
     A = CANVAS * cfg.top_k
-    return cfg.n_exp * 2 * cfg.d_ff * cfg.d_model * 2 + A * cfg.d_model * 2 + A * cfg.d_ff * 2
+    n_w = cfg.n_exp * 2 * cfg.d_ff * cfg.d_model
+    w_bytes = n_w + 4 * (n_w // (128 * 128)) if getattr(cfg, "wdtype", 0) == 1 else 2 * n_w
+    return w_bytes + A * cfg.d_model * 2 + A * cfg.d_ff * 2
 
 
 def main_dg(args):
@@ -227,7 +236,7 @@ def main_dg(args):
         build.build()
     if world > 1:
         dist.barrier()
-    cfg, w, model, seqs, prm, st = setup_full(rank, device)
+    cfg, w, model, seqs, prm, st = setup_full(rank, device, fp8=args.fp8)
     state = {"step": 0}
     run_steps(dg, seqs, prm, st, args.warmup, state)
     torch.cuda.synchronize()
@@ -322,16 +331,18 @@ def main_dg(args):
     assert code == 0, f"device error {code}"
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         cpu = cpu_baseline_sample(cfg, w, sample_rows_layer=256, head_rows=32, samp_rows=256)
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "steps/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CANVAS,
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 arithmetic, fp8 e4m3 per-layer weights" if args.fp8 else "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD_FP8 if args.fp8 else WORKLOAD, "global_batch": world, "seq_len": CANVAS,
                            "parallelism": f"replicas x{world} (independent sequences, no exchange)",
-                           "l2": "inputs larger than L2: 48.2 GB of weights streamed per step"},
+                           "l2": "inputs larger than L2: " + ("25 GB" if args.fp8 else "48.2 GB")
+                                 + " of weights streamed per step"},
                 "committed_tok_s": round(committed_tok_s, 1),
                 "decode": {"blocks": BLOCKS, "steps_per_block": steps_per_block, "tokens": sum(n_out),
                            "seconds": round(td, 4), "includes": "canvas init, 12 steps and a commit pass per block"},

@@ -108,6 +108,26 @@ dg_status map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, 
   return DG_OK;
 }
 
+// 2-D bytes [rows][cols] (e4m3 weights), box box_rows x 64 bytes, no swizzle (rows land 64 bytes
+// apart; the expert kernel's converter warps lay them out for the tensor cores).
+dg_status map_2d_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || cols % 16)
+    return fail(DG_ERR_INVALID_ARG, "FP8 TMA operand not 16-byte aligned (ptr %p, row bytes %llu)", ptr,
+                (unsigned long long)cols);
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (2d u8, %llux%llu box %u) failed: %d",
+                                     (unsigned long long)rows, (unsigned long long)cols, box_rows, (int)r);
+  return DG_OK;
+}
+
 // 3-D bf16 [d2][d1][d0] (d0 contiguous), box {64, box1, 1}, 128-byte swizzle.
 dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
   EncodeTiledFn f = encode_fn();
@@ -208,7 +228,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
-    for (int i = 0; i < 5; ++i) L.wq[i] = take(2 * rows[i] * cols[i]);
+    for (int i = 0; i < 3; ++i) L.wq[i] = take(2 * rows[i] * cols[i]);   // the expert GEMMs read e4m3 directly
   }
 
   L.total = off + 1024;   // slack for base alignment
@@ -230,6 +250,8 @@ bool shape_ok(const dg_model_config* c, const char** why) {
   if (c->wdtype != DG_WDTYPE_BF16 && c->wdtype != DG_WDTYPE_FP8_BLOCK128) return (*why = "unknown wdtype", false);
   if (c->wdtype == DG_WDTYPE_FP8_BLOCK128 && (2 * c->d_ff) % 128)
     return (*why = "FP8 weights need 2 d_ff % 128 == 0", false);
+  if (c->wdtype == DG_WDTYPE_FP8_BLOCK128 && (c->d_model > 32 * 128 || c->d_ff > 32 * 128))
+    return (*why = "FP8 weights need d_model, d_ff <= 4096 (32 scale blocks per row)", false);
   return true;
 }
 
@@ -378,6 +400,13 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
   const dg_model_config& c = *cfg;
   const uint64_t d = c.d_model, qkv = (uint64_t)(c.n_q + 2 * c.n_kv) * c.d_head;
   dg_status st = DG_OK;
+  for (int l = 0; l < c.n_layers && st == DG_OK && fp8; ++l) {
+    // FP8: the expert GEMMs read e4m3 bytes directly (64-row boxes for gate|up halves, 128 for down)
+    const dg_layer_weights& L = m->layers[l];
+    LayerMaps& M = m->maps[l];
+    if ((st = map_2d_u8(&M.wgu, L.w_gate_up, (uint64_t)c.n_exp * 2 * c.d_ff, d, 64)) != DG_OK) break;
+    if ((st = map_2d_u8(&M.wdown, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
+  }
   for (int l = 0; l < c.n_layers && st == DG_OK && !fp8; ++l) {
     const dg_layer_weights& L = m->layers[l];
     LayerMaps& M = m->maps[l];
@@ -465,7 +494,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->cH = reinterpret_cast<float*>(b + L.cH);
   s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
   s->splitk = reinterpret_cast<float*>(b + L.splitk);
-  for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
+  for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 && i < 3 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
   s->step = 0;
@@ -496,8 +525,6 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
     st = map_2d(&W.wqkv, s->wq[0], rows[0], cols[0], 128);
     if (st == DG_OK) st = map_2d(&W.wo, s->wq[1], rows[1], cols[1], 128);
     if (st == DG_OK) st = map_2d(&W.wrouter, s->wq[2], rows[2], cols[2], 128);
-    if (st == DG_OK) st = map_2d(&W.wgu, s->wq[3], rows[3], cols[3], 64);
-    if (st == DG_OK) st = map_2d(&W.wdown, s->wq[4], rows[4], cols[4], 128);
   }
   if (st != DG_OK) {
     delete s;
@@ -561,8 +588,8 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
     const void* q[5] = {W.w_qkv, W.w_o, W.w_router, W.w_gate_up, W.w_down};
     const float* sc[5] = {W.s_qkv, W.s_o, W.s_router, W.s_gate_up, W.s_down};
     DequantArgs da{};
-    da.n = 5;
-    for (int i = 0; i < 5; ++i)
+    da.n = 3;   // qkv, o, router; the expert GEMMs expand their e4m3 tiles on the fly
+    for (int i = 0; i < 3; ++i)
       da.mat[i] = DequantMat{static_cast<const uint8_t*>(q[i]), sc[i], s->wq[i], (long long)mr[i], (int)mc[i]};
     LAUNCH(s, DG_K_DEQUANT, 1, dequant_fp8(da, s->m->n_sms, st));
   }
@@ -649,8 +676,16 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   xp.F = c.d_ff;
   // many tokens per expert on average (several canvases): 256-token accumulator chunks
   const int wide = rows * c.top_k >= 128 * c.n_exp ? 1 : 0;
-  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, M.wgu, s->xp_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
-  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, M.wdown, s->hb_map, xp, c.n_exp, s->m->n_sms, wide, s->err, st));
+  const LayerMaps& ME = s->m->maps[l];   // expert weight descriptors: bf16, or e4m3 bytes in the FP8 form
+  ExpertParams xu = xp, xd = xp;
+  if (fp8) {
+    xu.w_scale = W.s_gate_up;
+    xu.w_scale_cols = (d + 127) / 128;
+    xd.w_scale = W.s_down;
+    xd.w_scale_cols = (c.d_ff + 127) / 128;
+  }
+  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, ME.wgu, s->xp_map, xu, c.n_exp, s->m->n_sms, wide, s->err, st));
+  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, ME.wdown, s->hb_map, xd, c.n_exp, s->m->n_sms, wide, s->err, st));
   LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
   return DG_OK;
 }
@@ -681,6 +716,7 @@ dg_status check_params(const dg_seqs* s, const dg_sampler_params* p) {
   if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "canvas_len must be 256");
   if (p->max_steps <= 0 || p->fixed_steps < 0) return fail(DG_ERR_INVALID_ARG, "bad step budget");
   if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
+  if (p->commit_mode != 0 && p->commit_mode != 1) return fail(DG_ERR_INVALID_ARG, "commit_mode must be 0 or 1");
   (void)s;
   return DG_OK;
 }
@@ -810,6 +846,18 @@ DG_API dg_status dg_block_commit(dg_seqs* s, const int32_t* d_ids) {
   return DG_OK;
 }
 
+DG_API dg_status dg_block_commit_last_kv(dg_seqs* s) {
+  NvtxRange nvtx_range("dg_block_commit_last_kv");
+  if (!s) return fail(DG_ERR_INVALID_ARG, "null argument");
+  if (!s->block_open || s->step == 0) return fail(DG_ERR_STATE, "no canvas step since dg_canvas_init");
+  for (int i = 0; i < s->n_seq; ++i)
+    if (s->P[i] + kCanvas > s->max_ctx) return fail(DG_ERR_CAPACITY, "sequence %d: cache full", i);
+  LAUNCH(s, DG_K_MISC, 1, add_to_P(s->seqP, 0, s->n_seq, kCanvas, s->st));
+  for (int i = 0; i < s->n_seq; ++i) s->P[i] += kCanvas;
+  s->block_open = false;
+  return DG_OK;
+}
+
 DG_API dg_status dg_layer_forward(dg_seqs* s, int layer, int n_rows, int causal, float* d_x, float* d_x_mid,
                                   float* d_router_logits) {
   NvtxRange nvtx_range("dg_layer_forward");
@@ -855,7 +903,7 @@ DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_block
       if (all || steps >= budget) break;
     }
     if (h_steps) h_steps[b] = steps;
-    r = dg_block_commit(s, s->cids);
+    r = p->commit_mode == 1 ? dg_block_commit_last_kv(s) : dg_block_commit(s, s->cids);
     if (r != DG_OK) return r;
     CK(cudaMemcpy2DAsync(d_out + (size_t)b * kCanvas, out_stride * sizeof(int32_t), s->cids,
                          kCanvas * sizeof(int32_t), kCanvas * sizeof(int32_t), n, cudaMemcpyDeviceToDevice, s->st));

@@ -85,8 +85,10 @@ struct ExpertParams {
   const float* perm_gate;  // [A] gate weight of each bucketed row
   const int* perm_tok;   // [A] token (row of the normed activations) of each bucketed row
   __nv_bfloat16* h_out;  // MODE 1: SwiGLU rows [A][F]
-  float* y_out;          // MODE 2: gate-scaled expert outputs [A][d]
+  float* y_out;          // MODE 2: expert outputs [A][d] (the combine applies the gates)
   int d, F;
+  const float* w_scale;  // FP8 weights: fp32 scale per 128 x 128 tile of the weight matrix viewed as
+  int w_scale_cols;      // 2-D, w_scale_cols tiles per row; nullptr for bf16 weights
 };
 
 struct AttnParams {

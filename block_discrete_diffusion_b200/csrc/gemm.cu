@@ -17,6 +17,9 @@
 //     MODE 1     [gate | up] rows of expert e times its gathered tokens; SwiGLU in the epilogue.
 //     MODE 2     down-projection rows of expert e times its SwiGLU rows (the combine applies the
 //                gate weights; top-k routed MoE of the 26B-A4B model, 3.8B active).
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "dg_device.cuh"
 #include "dg_kernels.h"
 
@@ -340,21 +343,33 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
 // chunk overlaps the MMAs of the next.
 // BN = tokens per accumulator chunk: 64 when a few tokens reach each expert (batch 1), 256 when
 // hundreds do (several canvases), so that a weight tile is streamed once per 256 tokens.
-template <int BN>
+// bf16 weights: a ring of kStages (weight tile 16 KB + token tile) stages.
+// FP8 weights: a ring of kStages load slots (e4m3 weight tile 8 KB + token tile) and, apart from
+// it, kConv bf16 weight tiles that the converter warps fill; the deeper load ring keeps about as
+// many weight bytes in flight from HBM as the bf16 ring does.
+template <int BN, bool FP8>
 struct ExpCfg {
-  static constexpr int kStages = BN >= 256 ? 4 : 7;
   static constexpr uint32_t kBTile = BN * 64 * 2;            // BN token rows x 64 k (32-row boxes)
-  static constexpr uint32_t kStageBytes = kATileBytes + kBTile;
-  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 128 * 65 * 4 + 512;
+  static constexpr uint32_t kAOff = FP8 ? kATileBytes / 2 : kATileBytes;   // token tile offset in a slot
+  static constexpr uint32_t kStageBytes = kAOff + kBTile;
+  static constexpr int kStages = FP8 ? (BN >= 256 ? 4 : 13) : (BN >= 256 ? 4 : 7);
+  static constexpr int kConv = FP8 ? (BN >= 256 ? 2 : 3) : 0;
+  static constexpr int kEpiCols = BN < 64 ? BN : 64;         // MODE 1 epilogue slice (accumulator columns)
+  static constexpr int kEpiStride = kEpiCols + 1;            // padded fp32 staging rows
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + (size_t)kConv * kATileBytes +
+                                       128 * kEpiStride * 4 + 512;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages <= 16 && kConv <= 4, "barrier arrays");
 };
-constexpr int kExpThreads = 192;                   // 6 warps
-constexpr int kEpiCols = 64;                       // MODE 1 epilogue slice (accumulator columns)
-constexpr int kEpiStride = kEpiCols + 1;           // padded fp32 staging rows
+constexpr int kExpThreads = 192;                   // 6 warps (bf16 weights)
+constexpr int kConvWarps = 4;                      // FP8: converter warps
+constexpr int kExpThreadsFp8 = kExpThreads + 32 * kConvWarps;
 
 struct ExpBarriers {
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[16];
+  uint64_t empty[16];
+  uint64_t cfull[4];   // FP8: a bf16 weight tile has been expanded
+  uint64_t cempty[4];  // FP8: the MMAs reading a bf16 weight tile have completed
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_slot;
@@ -364,18 +379,33 @@ __device__ __forceinline__ void epi_bar_sync() {   // the 128 epilogue threads o
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-template <int MODE, int BN>
-__global__ void __launch_bounds__(kExpThreads, 1)
+// 4 e4m3 bytes times a scale -> 4 bf16: hardware e4m3x2 -> f16x2, fp32 multiply (the product's fp32
+// rounding), one round-to-nearest-even to bf16.
+__device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two, float sc) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x * sc, f.y * sc);
+}
+__device__ __forceinline__ uint2 e4m3x4_scaled(uint32_t w, float sc) {
+  return make_uint2(e4m3x2_scaled(w, sc), e4m3x2_scaled(w >> 16, sc));
+}
+
+// FP8: the weight operand arrives as e4m3 bytes (TMA into a load slot); kConvWarps converter warps
+// expand it to bf16(q * s) in one of two bf16 tiles, in the 128-byte-swizzled layout the MMA reads.
+template <int MODE, int BN, bool FP8>
+__global__ void __launch_bounds__(FP8 ? kExpThreadsFp8 : kExpThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
   uint8_t* tiles = align1024(smem_raw);
-  using C = ExpCfg<BN>;
+  using C = ExpCfg<BN, FP8>;
   constexpr int kExpStages = C::kStages;
   constexpr uint32_t kExpStageBytes = C::kStageBytes;
   constexpr int kExpBN = BN;
-  float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kExpStages * kExpStageBytes);
+  uint8_t* conv_tiles = tiles + (size_t)kExpStages * kExpStageBytes;   // FP8: kConv bf16 weight tiles
+  float* stage_out = reinterpret_cast<float*>(conv_tiles + (size_t)C::kConv * kATileBytes);
+  constexpr int kEpiCols = C::kEpiCols, kEpiStride = C::kEpiStride, kConv = C::kConv > 0 ? C::kConv : 1;
   ExpBarriers* bars = reinterpret_cast<ExpBarriers*>(stage_out + 128 * kEpiStride);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = MODE == 1 ? p.d : p.F;
@@ -387,6 +417,10 @@ __global__ void __launch_bounds__(kExpThreads, 1)
     for (int s = 0; s < kExpStages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
+    }
+    for (int c = 0; c < kConv; ++c) {
+      mbar_init(&bars->cfull[c], kConvWarps);
+      mbar_init(&bars->cempty[c], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->acc_full[b], 1);
@@ -404,9 +438,9 @@ __global__ void __launch_bounds__(kExpThreads, 1)
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
-      // narrow chunks read every weight tile once: evict first; wide chunks read it once per 256
-      // tokens, a few microseconds apart: keep the normal policy so the re-read hits L2
-      const uint64_t pol_w = BN >= 256 ? l2_policy_evict_normal() : l2_policy_evict_first();
+      // 64-token bf16 chunks read every weight tile once: evict first; wide chunks (and the 32-token
+      // FP8 chunks) may read it again a few microseconds later: normal policy, the re-read hits L2
+      const uint64_t pol_w = (BN >= 256 || FP8) ? l2_policy_evict_normal() : l2_policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -414,7 +448,7 @@ __global__ void __launch_bounds__(kExpThreads, 1)
         const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
         for (int c0 = 0; c0 < n_e && ok; c0 += kExpBN) {
           const int nb = (min(kExpBN, n_e - c0) + 31) >> 5;
-          const uint32_t tx = kATileBytes + (uint32_t)nb * 4096u;
+          const uint32_t tx = (FP8 ? kATileBytes / 2 : kATileBytes) + (uint32_t)nb * 4096u;
           for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = it % kExpStages;
             if (!mbar_wait(&bars->empty[s], ((it / kExpStages) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) {
@@ -423,7 +457,15 @@ __global__ void __launch_bounds__(kExpThreads, 1)
             }
             uint8_t* a = tiles + (size_t)s * kExpStageBytes;
             mbar_arrive_expect_tx(&bars->full[s], tx);
-            if (MODE == 1) {
+            if (FP8) {   // e4m3 rows of 64 bytes at the start of the slot
+              if (MODE == 1) {
+                const int r0 = e * 2 * p.F + mt * 64;
+                tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, r0, pol_w);
+                tma_load_2d_hint(&tmW, &bars->full[s], a + 4096, kb * 64, r0 + p.F, pol_w);
+              } else {
+                tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, e * p.d + mt * 128, pol_w);
+              }
+            } else if (MODE == 1) {
               const int r0 = e * 2 * p.F + mt * 64;
               tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, r0, pol_w);               // gate rows
               tma_load_2d_hint(&tmW, &bars->full[s], a + 8192, kb * 64, r0 + p.F, pol_w);  // up rows
@@ -431,7 +473,7 @@ __global__ void __launch_bounds__(kExpThreads, 1)
               tma_load_2d_hint(&tmW, &bars->full[s], a, kb * 64, e * p.d + mt * 128, pol_w);
             }
             for (int b = 0; b < nb; ++b)
-              tma_load_2d(&tmX, &bars->full[s], a + kATileBytes + b * 4096, kb * 64, off + c0 + 32 * b);
+              tma_load_2d(&tmX, &bars->full[s], a + C::kAOff + b * 4096, kb * 64, off + c0 + 32 * b);
           }
         }
       }
@@ -456,22 +498,81 @@ __global__ void __launch_bounds__(kExpThreads, 1)
           const uint32_t acc = tmem + b * kExpBN;
           for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = it % kExpStages;
-            if (!mbar_wait(&bars->full[s], (it / kExpStages) & 1, err, DEV_ERR_TIMEOUT_MMA)) {
+            const int cv = it % kConv;
+            if (!mbar_wait(&bars->full[s], (it / kExpStages) & 1, err, DEV_ERR_TIMEOUT_MMA) ||
+                (FP8 && !mbar_wait(&bars->cfull[cv], (it / kConv) & 1, err, DEV_ERR_TIMEOUT_MMA))) {
               ok = false;
               break;
             }
             tc_fence_after();
             uint8_t* a = tiles + (size_t)s * kExpStageBytes;
-            const uint64_t ad = smem_desc_sw128(smem_u32(a));
-            const uint64_t bd = smem_desc_sw128(smem_u32(a + kATileBytes));
+            const uint64_t ad = smem_desc_sw128(smem_u32(FP8 ? conv_tiles + cv * kATileBytes : a));
+            const uint64_t bd = smem_desc_sw128(smem_u32(a + C::kAOff));
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               umma_bf16(acc, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0);
             umma_commit(&bars->empty[s]);
+            if (FP8) umma_commit(&bars->cempty[cv]);
           }
           umma_commit(&bars->acc_full[b]);
         }
       }
+    }
+  } else if (FP8 && warp >= 6) {
+    // ------------------------------ FP8 converters (warps 6 ..) ------------------------------
+    // Lane l keeps the scales of 128-column block l of the item's two 64-row halves (MODE 1: gate,
+    // up) or of its 128-row tile (MODE 2); the next item's are loaded while this one is converted.
+    // Waits are made warp-uniform so that the shuffles always see all 32 lanes.
+    const int ct = threadIdx.x - kExpThreads;     // 0 .. 32 kConvWarps - 1
+    auto load_scales = [&](int item, float& s0, float& s1) {
+      const int e = item / MT, mt = item % MT;
+      const int sr0 = MODE == 1 ? (e * 2 * p.F + mt * 64) / 128 : (e * p.d + mt * 128) / 128;
+      const int sr1 = MODE == 1 ? (e * 2 * p.F + p.F + mt * 64) / 128 : sr0;
+      s0 = lane < p.w_scale_cols ? __ldg(p.w_scale + (size_t)sr0 * p.w_scale_cols + lane) : 0.f;
+      s1 = lane < p.w_scale_cols ? __ldg(p.w_scale + (size_t)sr1 * p.w_scale_cols + lane) : 0.f;
+    };
+    uint32_t it = 0;
+    bool ok = true;
+    float cur0 = 0.f, cur1 = 0.f;
+    if ((int)blockIdx.x < n_items) load_scales(blockIdx.x, cur0, cur1);
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int e = item / MT;
+      const int n_e = p.offsets[e + 1] - p.offsets[e];
+      float nxt0 = 0.f, nxt1 = 0.f;
+      if (item + (int)gridDim.x < n_items) load_scales(item + gridDim.x, nxt0, nxt1);
+      for (int c0 = 0; c0 < n_e && ok; c0 += kExpBN) {
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kExpStages;
+          const int cv = it % kConv;
+          const bool got = mbar_wait(&bars->full[s], (it / kExpStages) & 1, err, DEV_ERR_TIMEOUT_PRODUCER) &&
+                           mbar_wait(&bars->cempty[cv], ((it / kConv) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* a8 = tiles + (size_t)s * kExpStageBytes;     // e4m3 rows of 64 bytes
+          uint8_t* a = conv_tiles + cv * kATileBytes;                 // bf16, 128-byte swizzle
+          const float sc0 = __shfl_sync(0xffffffffu, cur0, kb >> 1);
+          const float sc1 = __shfl_sync(0xffffffffu, cur1, kb >> 1);
+          // 16-byte chunk g = ct + 32 kConvWarps i of the e4m3 tile: row g / 4, bytes 16 (g % 4) ..
+#pragma unroll
+          for (int i = 0; i < 512 / (32 * kConvWarps); ++i) {
+            const int g = ct + 32 * kConvWarps * i, row = g >> 2, qc = g & 3;
+            const uint4 q = *reinterpret_cast<const uint4*>(a8 + g * 16);
+            const float sc = row < 64 ? sc0 : sc1;
+            uint8_t* dst = a + row * 128;
+            const uint2 p0 = e4m3x4_scaled(q.x, sc), p1 = e4m3x4_scaled(q.y, sc);
+            const uint2 p2 = e4m3x4_scaled(q.z, sc), p3 = e4m3x4_scaled(q.w, sc);
+            *reinterpret_cast<uint4*>(dst + (((2 * qc) ^ (row & 7)) << 4)) = make_uint4(p0.x, p0.y, p1.x, p1.y);
+            *reinterpret_cast<uint4*>(dst + (((2 * qc + 1) ^ (row & 7)) << 4)) = make_uint4(p2.x, p2.y, p3.x, p3.y);
+          }
+          fence_proxy_async_smem();                 // generic-proxy writes -> tensor-core reads
+          __syncwarp();
+          if ((threadIdx.x & 31) == 0) mbar_arrive(&bars->cfull[cv]);
+        }
+      }
+      cur0 = nxt0;
+      cur1 = nxt1;
     }
   } else {
     // ------------------------------ epilogue (warps 2-5) ------------------------------
@@ -603,32 +704,44 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
   return cudaErrorInvalidValue;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool FP8>
 static cudaError_t launch_expert(const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                                  int n_ctas, int* err, cudaStream_t st) {
-  using C = ExpCfg<BN>;
+  using C = ExpCfg<BN, FP8>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN, FP8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BN, FP8>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int items = n_exp * (MODE == 1 ? p.F / 64 : p.d / 128);
-  return launch_k(expert_gemm_kernel<MODE, BN>, dim3(n_ctas < items ? n_ctas : items), dim3(kExpThreads),
-                  C::kSmemBytes, st, 1, w, x, p, n_exp, err);
+  return launch_k(expert_gemm_kernel<MODE, BN, FP8>, dim3(n_ctas < items ? n_ctas : items),
+                  dim3(FP8 ? kExpThreadsFp8 : kExpThreads), C::kSmemBytes, st, 1, w, x, p, n_exp, err);
 }
 
-// wide = 1: 256-token accumulator chunks (many tokens per expert); 0: 64-token chunks.
+// wide = 1: 256-token accumulator chunks (many tokens per expert); 0: 64-token chunks.  p.w_scale
+// != nullptr: the weights are e4m3 with one fp32 scale per 128 x 128 tile (w is a byte map).
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                         int n_ctas, int wide, int* err, cudaStream_t st) {
-  if (wide)
-    return mode == 1 ? launch_expert<1, 256>(w, x, p, n_exp, n_ctas, err, st)
-                     : launch_expert<2, 256>(w, x, p, n_exp, n_ctas, err, st);
-  return mode == 1 ? launch_expert<1, 64>(w, x, p, n_exp, n_ctas, err, st)
-                   : launch_expert<2, 64>(w, x, p, n_exp, n_ctas, err, st);
+  const bool f8 = p.w_scale != nullptr;
+  // chunk width: 256 (wide), else 64 tokens for bf16 weights and 32 for FP8 (smaller slots, so the
+  // e4m3 ring keeps enough weight bytes in flight)
+  const int bn = wide ? 256 : (f8 ? 32 : 64);
+#define DG_EXPERT_CASE(M_, BN_, F8_) \
+  if (mode == M_ && bn == BN_ && f8 == F8_) return launch_expert<M_, BN_, F8_>(w, x, p, n_exp, n_ctas, err, st);
+  DG_EXPERT_CASE(1, 64, false)
+  DG_EXPERT_CASE(2, 64, false)
+  DG_EXPERT_CASE(1, 256, false)
+  DG_EXPERT_CASE(2, 256, false)
+  DG_EXPERT_CASE(1, 32, true)
+  DG_EXPERT_CASE(2, 32, true)
+  DG_EXPERT_CASE(1, 256, true)
+  DG_EXPERT_CASE(2, 256, true)
+#undef DG_EXPERT_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dg

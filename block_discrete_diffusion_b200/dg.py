@@ -24,6 +24,7 @@ ENTRY_POINTS = (
     "dg_seqs_destroy", "dg_seqs_get_state", "dg_load_prefix", "dg_prefill", "dg_canvas_init", "dg_canvas_step",
     "dg_block_commit", "dg_decode", "dg_layer_forward", "dg_sample_workspace_bytes", "dg_sample", "dg_device_error",
     "dg_temperature", "dg_stats_reset", "dg_stats_read", "dg_sample_noalloc", "dg_sample_noalloc_max_rows",
+    "dg_block_commit_last_kv",
 )
 
 # dg_kernel_class, in order
@@ -59,15 +60,16 @@ class dg_weights(ctypes.Structure):
 class dg_sampler_params(ctypes.Structure):
     _fields_ = [("canvas_len", c_int), ("max_steps", c_int), ("fixed_steps", c_int), ("t_start", c_float),
                 ("t_end", c_float), ("entropy_bound", c_float), ("stop_mean_entropy", c_float),
-                ("rerand_entropy", c_float), ("seed", c_uint64), ("eos_id", c_int)]
+                ("rerand_entropy", c_float), ("seed", c_uint64), ("eos_id", c_int), ("commit_mode", c_int)]
 
 
 def sampler_params(vocab, seed=0, canvas_len=256, max_steps=48, fixed_steps=0, t_start=0.8, t_end=0.4,
-                   entropy_bound=0.1, stop_mean_entropy=0.005, rerand_entropy=None, eos_id=-1) -> dg_sampler_params:
+                   entropy_bound=0.1, stop_mean_entropy=0.005, rerand_entropy=None, eos_id=-1,
+                   commit_mode=0) -> dg_sampler_params:
     if rerand_entropy is None:
         rerand_entropy = 0.5 * math.log(vocab)
     return dg_sampler_params(canvas_len, max_steps, fixed_steps, t_start, t_end, entropy_bound, stop_mean_entropy,
-                             rerand_entropy, seed, eos_id)
+                             rerand_entropy, seed, eos_id, commit_mode)
 
 
 _LIB = None
@@ -100,6 +102,7 @@ def lib():
         L.dg_canvas_step.argtypes = [c_void_p, P(dg_sampler_params), c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p]
         L.dg_block_commit.argtypes = [c_void_p, c_void_p]
+        L.dg_block_commit_last_kv.argtypes = [c_void_p]
         L.dg_decode.argtypes = [c_void_p, P(dg_sampler_params), c_int, c_void_p, c_void_p, c_void_p]
         L.dg_layer_forward.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
         L.dg_sample_workspace_bytes.argtypes = [c_int, c_int]
@@ -244,6 +247,10 @@ def dg_canvas_step(seqs: Seqs, params, ids, commit, entropy, stop, hidden=None, 
 
 def dg_block_commit(seqs: Seqs, ids):
     _check("dg_block_commit", lib().dg_block_commit(seqs.handle, _ptr(ids)))
+
+
+def dg_block_commit_last_kv(seqs: Seqs):
+    _check("dg_block_commit_last_kv", lib().dg_block_commit_last_kv(seqs.handle))
 
 
 def dg_decode(seqs: Seqs, params, max_blocks, out):

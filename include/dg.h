@@ -106,6 +106,8 @@ typedef struct {
   float rerand_entropy;    /* 0.5 ln(vocab) */
   uint64_t seed;           /* sequence i uses seed + i */
   int eos_id;              /* -1: no EOS */
+  int commit_mode;         /* dg_decode's block commit: 0 dg_block_commit (recompute, default),
+                              1 dg_block_commit_last_kv (keep the last step's K/V) */
 } dg_sampler_params;
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
@@ -168,6 +170,14 @@ dg_status dg_canvas_step(dg_seqs *s, const dg_sampler_params *p, int32_t *d_ids,
  * one pass of the layer stack over the final ids with the canvas mask writes every layer's K/V to
  * cache rows [P, P+256), then P += 256.  DG_ERR_CAPACITY if P + 256 > max_ctx. */
 dg_status dg_block_commit(dg_seqs *s, const int32_t *d_ids);
+
+/* Append the finished canvases keeping the K/V that the block's last dg_canvas_step computed in
+ * cache rows [P, P+256): P += 256 without another pass of the layer stack.  The kept K/V are those
+ * of the ids that step read (one sampling older than the final ids).  The pages only say that the
+ * finished block is committed to the cache; dg_block_commit (recompute from the final ids) is this
+ * library's default reading and this call the cheaper alternative.  DG_ERR_STATE if no canvas step
+ * ran since dg_canvas_init; DG_ERR_CAPACITY if P + 256 > max_ctx. */
+dg_status dg_block_commit_last_kv(dg_seqs *s);
 
 /* The whole block loop ([report] flowchart): for each of up to max_blocks blocks: dg_canvas_init,
  * dg_canvas_step until every sequence's stop flag is set (sequences that stopped keep their ids),

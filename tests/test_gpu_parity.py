@@ -367,6 +367,62 @@ def test_decode_equals_the_step_sequence(dg):
     assert len([x for x in steps3 if x]) == first // 256 + 1
 
 
+def test_commit_keeping_the_last_steps_kv(dg):
+    """dg_block_commit_last_kv: the cache rows of the block keep the K/V of the ids the last step
+    read (the oracle's commit pass over those ids), the prefix is untouched, P advances; dg_decode
+    with commit_mode 1 equals the same calls made one by one; a commit before any step is a state
+    error."""
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=2, top_k=8)
+    max_ctx = 1024
+    prompt = synthetic.make_ids(128, cfg.vocab, 2)
+    prm = dg.sampler_params(cfg.vocab, seed=6, fixed_steps=3)
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(seqs, prompt.cuda(), [128])
+    ids = torch.empty(256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+    H = torch.empty(256, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    with pytest.raises(dg.DGError) as ei:
+        dg.dg_block_commit_last_kv(seqs)
+    assert ei.value.status == dg.DG_ERR_STATE
+    for _ in range(3):
+        last_in = ids.cpu().clone()
+        dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+    before = seqs.kv.clone()
+    dg.dg_block_commit_last_kv(seqs)
+    torch.cuda.synchronize()
+    assert dg.dg_seqs_get_state(seqs)[0] == [128 + 256]
+    assert torch.equal(seqs.kv, before)                        # nothing recomputed or moved
+    oseq = oracle.Sequence(M, max_ctx)
+    oseq.prefill(prompt.numpy())
+    oseq.block_commit(last_in.numpy())
+    for l in range(cfg.n_layers):
+        kg, vg = _cache_rows(seqs, cfg, max_ctx, l, 128, 384)
+        assert rel_err(kg, oseq.k[l][128:384]) <= HIDDEN_TOL and rel_err(vg, oseq.v[l][128:384]) <= HIDDEN_TOL
+        kp, vp = _cache_rows(seqs, cfg, max_ctx, l, 0, 128)
+        assert rel_err(kp, oseq.k[l][:128]) <= HIDDEN_TOL
+    # dg_decode with commit_mode 1 is the loop with this commit
+    prm1 = dg.sampler_params(cfg.vocab, seed=6, fixed_steps=3, commit_mode=1)
+    s1 = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(s1, prompt.cuda(), [128])
+    out = torch.full((1, 2 * 256), -1, dtype=torch.int32, device="cuda")
+    n_out, steps = dg.dg_decode(s1, prm1, 2, out)
+    assert n_out == [512] and steps == [3, 3]
+    s2 = dg.dg_seqs_create(model, 1, max_ctx)
+    dg.dg_prefill(s2, prompt.cuda(), [128])
+    manual = []
+    for b in range(2):
+        dg.dg_canvas_init(s2, prm1, ids, commit)
+        for _ in range(3):
+            dg.dg_canvas_step(s2, prm1, ids, commit, H, stop)
+        dg.dg_block_commit_last_kv(s2)
+        manual.append(ids.cpu().clone())
+    assert torch.equal(out.cpu()[0], torch.cat(manual))
+    assert torch.equal(s1.kv, s2.kv)
+    assert dg.dg_device_error(s1) == 0 and dg.dg_device_error(s2) == 0
+
+
 def test_capacity_and_argument_errors(dg):
     cfg, w, model, M = _tiny_model_pair(dg)
     seqs = dg.dg_seqs_create(model, 1, 256)
