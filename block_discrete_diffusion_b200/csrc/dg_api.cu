@@ -149,7 +149,7 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
-      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, total;
+      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, total;
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
 
@@ -170,7 +170,7 @@ int attn_split_cap(const dg_model_config& c, int n_seq) {
   const int G = c.n_q / c.n_kv;
   const int pairs = (G * kCanvas + 255) / 256;
   const int base = pairs * n_seq * c.n_kv;
-  if (base < kAttnTargetCtas) return std::max(1, std::min(kMaxSplits, (kAttnTargetCtas + base - 1) / base));
+  if (base < kAttnTargetCtas) return std::max(1, std::min(kMaxSplits, kAttnTargetCtas / base));   // one wave
   int best = 1;
   double best_eff = 0.0;
   for (int sp = 1; sp <= 4; ++sp) {
@@ -225,6 +225,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.cH = take(4 * R);
   L.cstop = take(4 * (size_t)n_seq);
   L.splitk = take(4 * (size_t)kSplitKSlots * 128 * 128);
+  L.head_off = take(8);
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
@@ -278,7 +279,8 @@ struct dg_model {
   const float* final_norm;
   std::vector<dg_layer_weights> layers;
   std::vector<LayerMaps> maps;
-  CUtensorMap head_map;
+  CUtensorMap head_map;      // 256-row boxes (dense head GEMM)
+  CUtensorMap head_map128;   // 128-row boxes (persistent swap-AB head GEMM)
   bool fp8;   // per-layer matrices in the FP8 block-scaled form (expanded per layer into the workspace)
 };
 
@@ -300,6 +302,8 @@ struct dg_seqs {
   float2* rope;
   CUtensorMap xn_map, xp_map, attn_map, hb_map, q_map, k_map, v_map;
   LayerMaps wmaps;              // FP8 form: descriptors of the bf16 scratch matrices
+  CUtensorMap xn32_map;         // xn in 32-row boxes (token operand of the persistent head GEMM)
+  int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   __nv_bfloat16* wq[5];         // FP8 form: the scratch matrices (qkv, o, router, gate_up, down)
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
@@ -417,6 +421,7 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
     if ((st = map_2d(&M.wdown, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
   }
   if (st == DG_OK) st = map_2d(&m->head_map, w->head, c.vocab, d, 256);
+  if (st == DG_OK) st = map_2d(&m->head_map128, w->head, c.vocab, d, 128);
   if (st != DG_OK) {
     delete m;
     return st;
@@ -494,6 +499,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->cH = reinterpret_cast<float*>(b + L.cH);
   s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
   s->splitk = reinterpret_cast<float*>(b + L.splitk);
+  s->head_off = reinterpret_cast<int32_t*>(b + L.head_off);
   for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 && i < 3 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
@@ -515,6 +521,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (st == DG_OK) st = map_2d(&s->attn_map, s->attn, R, (uint64_t)c.n_q * c.d_head, 128);
   if (st == DG_OK) st = map_2d(&s->xp_map, s->xp, A, d, 32);
   if (st == DG_OK) st = map_2d(&s->hb_map, s->hb, A, c.d_ff, 32);
+  if (st == DG_OK) st = map_2d(&s->xn32_map, s->xn, R, d, 32);
   if (st == DG_OK) st = map_2d(&s->q_map, s->q, (uint64_t)n_seq * c.n_q * kCanvas, c.d_head, 128);
   if (st == DG_OK) st = map_3d(&s->k_map, s->kc, c.d_head, max_ctx, zdim, 128);
   if (st == DG_OK) st = map_3d(&s->v_map, s->vt, max_ctx, c.d_head, zdim, c.d_head);
@@ -535,6 +542,11 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (e == cudaSuccess) e = cudaMemsetAsync(s->ws, 0, L.rope, s->st);
 
   if (e == cudaSuccess) e = rope_table(s->rope, max_ctx, c.d_head, c.rope_theta, s->st);
+  if (e == cudaSuccess) {
+    const int32_t h_off[2] = {0, (int32_t)L.R};
+    e = cudaMemcpyAsync(s->head_off, h_off, sizeof h_off, cudaMemcpyHostToDevice, s->st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s->st);   // h_off is on this stack frame
+  }
   if (e != cudaSuccess) {
     delete s;
     return fail(DG_ERR_CUDA, "seqs init: %s", cudaGetErrorString(e));
@@ -799,10 +811,23 @@ DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t*
   const dg_model_config& c = s->m->cfg;
   r = run_canvas_stack(s, d_ids, d_hidden);   // leaves RMSNorm_final(x) in xn
   if (r != DG_OK) return r;
-  EpiParams eh{};
-  eh.out = s->logits;
-  eh.ldo = c.vocab;
-  LAUNCH(s, DG_K_HEAD, 1, gemm_dense(256, EPI_F32, s->xn_map, s->m->head_map, s->L.R, c.vocab, c.d_model, eh, s->err, s->st));
+  if (s->L.R <= kCanvas) {
+    // one canvas: the head as a persistent swap-AB GEMM (vocabulary rows are the 128-row side, the
+    // 256 canvas rows one 256-wide chunk), one CTA per SM, epilogues overlapping the weight stream
+    ExpertParams hp{};
+    hp.offsets = s->head_off;
+    hp.y_out = s->logits;
+    hp.d = c.vocab;        // output rows of the weight (logit columns)
+    hp.F = c.d_model;      // reduction length
+    LAUNCH(s, DG_K_HEAD, 1,
+           gemm_expert(2, s->m->head_map128, s->xn32_map, hp, 1, s->m->n_sms, 1, s->err, s->st));
+  } else {
+    EpiParams eh{};
+    eh.out = s->logits;
+    eh.ldo = c.vocab;
+    LAUNCH(s, DG_K_HEAD, 1,
+           gemm_dense(256, EPI_F32, s->xn_map, s->m->head_map, s->L.R, c.vocab, c.d_model, eh, s->err, s->st));
+  }
   if (d_logits_out)
     CK(cudaMemcpyAsync(d_logits_out, s->logits, sizeof(float) * (size_t)s->L.R * c.vocab, cudaMemcpyDeviceToDevice,
                        s->st));
