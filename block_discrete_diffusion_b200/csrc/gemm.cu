@@ -111,66 +111,95 @@ __device__ __forceinline__ void store_qkv_pairs(const EpiParams& ep, int row, in
 // columns); Q and K heads rotated pairwise by one warp per row (lane = rotary pair), stored
 // head-major; V heads by one warp per channel (lane = row, positions contiguous in the
 // transposed value cache).
-template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const float* t, int rs, int row0, int nr,
-                                                   int n0, int M, int N) {
+template <int BN, int EPI, int RPC>
+__device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const float* t, int rs, int row0, int n0,
+                                                   int M, int N) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kGemmThreads / 32;
+  constexpr int RPW = (RPC + NW - 1) / NW;   // rows per warp
+  // A 128-row tile lies inside one sequence's rows_per_seq rows: one committed length for all rows.
+  // Global loads (length, rotary table, residual) are all issued before the stores that follow them.
+  const int seq = row0 / ep.rows_per_seq, j0 = row0 % ep.rows_per_seq;
   if constexpr (EPI == EPI_QKV) {
     const int dh = ep.dh, half = dh >> 1;
     const int q_end = ep.n_q * dh, k_end = q_end + ep.n_kv * dh;
+    const int cseq = ep.seq_base + seq;
+    const int P = __ldg(ep.seq_P + cseq);
     for (int h0 = 0; h0 < BN; h0 += dh) {
       const int f_head = n0 + h0;
       if (f_head >= N) break;
       if (f_head < k_end) {
-        for (int r = warp; r < nr; r += NW) {
-          const int row = row0 + r;
-          if (row >= M) break;
-          const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
-          const int cseq = ep.seq_base + seq;
-          const int pos = ep.seq_P[cseq] + j;
+        float2 cs[RPW][2];
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+          const int r = warp + NW * k;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int i = lane + 32 * u;
+            cs[k][u] = (r < RPC && row0 + r < M && i < half) ? __ldg(ep.rope + (size_t)(P + j0 + r) * half + i)
+                                                              : make_float2(0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+          const int r = warp + NW * k;
+          if (r >= RPC || row0 + r >= M) break;
+          const int j = j0 + r;
           __nv_bfloat16* dst =
               f_head < q_end ? ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh
-                             : ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + pos) * dh;
-          const float2* cs = ep.rope + (size_t)pos * half;
+                             : ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + P + j) * dh;
           const float* tr = t + r * rs + h0;
-          for (int i = lane; i < half; i += 32) {
-            const float a = tr[i], b = tr[half + i];
-            const float2 c = cs[i];
-            dst[i] = __float2bfloat16_rn(a * c.x - b * c.y);
-            dst[half + i] = __float2bfloat16_rn(b * c.x + a * c.y);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int i = lane + 32 * u;
+            if (i < half) {
+              const float a = tr[i], b = tr[half + i];
+              dst[i] = __float2bfloat16_rn(a * cs[k][u].x - b * cs[k][u].y);
+              dst[half + i] = __float2bfloat16_rn(b * cs[k][u].x + a * cs[k][u].y);
+            }
           }
         }
       } else {
-        const int vh = (f_head - k_end) / dh;
-        for (int c = warp; c < dh; c += NW) {
-          for (int r = lane; r < nr; r += 32) {
-            const int row = row0 + r;
-            if (row >= M) break;
-            const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
-            const int cseq = ep.seq_base + seq;
-            const int pos = ep.seq_P[cseq] + j;
-            ep.vt[(((size_t)cseq * ep.n_kv + vh) * dh + c) * ep.max_ctx + pos] = __float2bfloat16_rn(t[r * rs + h0 + c]);
-          }
-        }
+        // transposed value cache: one warp per channel, lanes along positions (contiguous)
+        __nv_bfloat16* vbase = ep.vt + (((size_t)cseq * ep.n_kv + (f_head - k_end) / dh) * dh) * ep.max_ctx + P + j0;
+        for (int c = warp; c < dh; c += NW)
+          for (int r = lane; r < RPC && row0 + r < M; r += 32)
+            vbase[(size_t)c * ep.max_ctx + r] = __float2bfloat16_rn(t[r * rs + h0 + c]);
       }
     }
   } else {
-    for (int r = warp; r < nr; r += NW) {
-      const int row = row0 + r;
-      if (row >= M) break;
-      float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)row * ep.ldo + n0;
+    constexpr int CG = BN / 128;             // 128-column groups (lane = 4 columns of each)
+    float4 xv[RPW][CG];
+    if constexpr (EPI == EPI_RESID) {
+#pragma unroll
+      for (int k = 0; k < RPW; ++k) {
+        const int r = warp + NW * k;
+#pragma unroll
+        for (int g = 0; g < CG; ++g) {
+          const int c = g * 128 + lane * 4;
+          xv[k][g] = (r < RPC && row0 + r < M && n0 + c + 4 <= N)
+                         ? *reinterpret_cast<const float4*>(ep.x + (size_t)(row0 + r) * ep.ldo + n0 + c)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+      const int r = warp + NW * k;
+      if (r >= RPC || row0 + r >= M) break;
+      float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)(row0 + r) * ep.ldo + n0;
       const float* tr = t + r * rs;
-      for (int c = lane * 4; c < BN; c += 128) {
+#pragma unroll
+      for (int g = 0; g < CG; ++g) {
+        const int c = g * 128 + lane * 4;
         if (n0 + c + 4 <= N) {
           float4 v = *reinterpret_cast<const float4*>(tr + c);
           if (EPI == EPI_RESID) {
-            const float4 x = *reinterpret_cast<const float4*>(dst + c);
-            v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+            v.x += xv[k][g].x; v.y += xv[k][g].y; v.z += xv[k][g].z; v.w += xv[k][g].w;
           }
           *reinterpret_cast<float4*>(dst + c) = v;
         } else {
-          for (int k = 0; k < 4 && n0 + c + k < N; ++k) dst[c + k] = (EPI == EPI_RESID ? dst[c + k] : 0.f) + tr[c + k];
+          for (int q = 0; q < 4 && n0 + c + q < N; ++q) dst[c + q] = (EPI == EPI_RESID ? dst[c + q] : 0.f) + tr[c + q];
         }
       }
     }
@@ -325,7 +354,7 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       *reinterpret_cast<float4*>(red + (i / F4) * RS + 4 * (i % F4)) = acc;
     }
     __syncthreads();
-    if (ok) epilogue_from_smem<BN, EPI>(ep, red, RS, m0 + zz * RPC, RPC, n0, M, N);
+    if (ok) epilogue_from_smem<BN, EPI, RPC>(ep, red, RS, m0 + zz * RPC, n0, M, N);
   }
 
   tc_fence_before();

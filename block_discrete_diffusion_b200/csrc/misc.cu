@@ -379,7 +379,8 @@ cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* co
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
-  return launch_k(gather_rows_kernel, dim3((n_rows + 7) / 8), dim3(256), 0, st, 1, xn, slot, n_rows, top_k, d, xp);
+  // two tokens (warps) per CTA: the copy of 256 tokens spreads over 128 SMs
+  return launch_k(gather_rows_kernel, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, xn, slot, n_rows, top_k, d, xp);
 }
 cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x,
                         const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st) {
