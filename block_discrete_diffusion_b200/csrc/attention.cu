@@ -396,16 +396,32 @@ __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
   float acc[kPer];
 #pragma unroll
   for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
-  for (int s = 0; s < p.n_splits; ++s) {
-    const float ws = __shfl_sync(0xffffffffu, wgt, s);
-    if (ws == 0.f) continue;
-    const float* src = p.opart + (s * stride + r0) * DH + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      acc[0] += ws * v.x; acc[1] += ws * v.y; acc[2] += ws * v.z; acc[3] += ws * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(src);
-      acc[0] += ws * v.x; acc[1] += ws * v.y;
+  // splits in groups of 8: the group's loads are all issued before they are summed (in split order)
+  for (int s0 = 0; s0 < p.n_splits; s0 += 8) {
+    float v[8][kPer];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      const float* src = p.opart + ((size_t)s * stride + r0) * DH + lane * kPer;
+#pragma unroll
+      for (int c = 0; c < kPer; ++c) v[u][c] = 0.f;
+      if (s < p.n_splits) {
+        if constexpr (kPer == 4) {
+          const float4 q = *reinterpret_cast<const float4*>(src);
+          v[u][0] = q.x; v[u][1] = q.y; v[u][2] = q.z; v[u][3] = q.w;
+        } else {
+          const float2 q = *reinterpret_cast<const float2*>(src);
+          v[u][0] = q.x; v[u][1] = q.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float ws = __shfl_sync(0xffffffffu, wgt, (s0 + u) & 31);
+      if (s0 + u < p.n_splits && ws != 0.f) {
+#pragma unroll
+        for (int c = 0; c < kPer; ++c) acc[c] += ws * v[u][c];
+      }
     }
   }
   __nv_bfloat16* dst = out + ((size_t)seq * p.rows_per_seq + j) * (p.n_q * DH) + h * DH + lane * kPer;
