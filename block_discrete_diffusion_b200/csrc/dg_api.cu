@@ -149,7 +149,7 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
-      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, total;
+      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, total;
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
 
@@ -226,6 +226,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.cstop = take(4 * (size_t)n_seq);
   L.splitk = take(4 * (size_t)kSplitKSlots * 128 * 128);
   L.head_off = take(8);
+  L.cursor = take(4 * 256);
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
@@ -304,6 +305,7 @@ struct dg_seqs {
   LayerMaps wmaps;              // FP8 form: descriptors of the bf16 scratch matrices
   CUtensorMap xn32_map;         // xn in 32-row boxes (token operand of the persistent head GEMM)
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
+  int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
   __nv_bfloat16* wq[5];         // FP8 form: the scratch matrices (qkv, o, router, gate_up, down)
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
@@ -500,6 +502,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->cstop = reinterpret_cast<int32_t*>(b + L.cstop);
   s->splitk = reinterpret_cast<float*>(b + L.splitk);
   s->head_off = reinterpret_cast<int32_t*>(b + L.head_off);
+  s->cursor = reinterpret_cast<int32_t*>(b + L.cursor);
   for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 && i < 3 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
@@ -674,9 +677,10 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));
   if (rlog_out)
     CK(cudaMemcpyAsync(rlog_out, s->rlog, sizeof(float) * (size_t)rows * c.n_exp, cudaMemcpyDeviceToDevice, st));
-  LAUNCH(s, DG_K_BUCKET, 1,
-         assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->perm_gate, s->perm_tok,
-                     s->slot, st));
+  int n_assign_k = 1;
+  LAUNCH(s, DG_K_BUCKET, n_assign_k,
+         assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->perm_gate,
+                     s->perm_tok, s->slot, &n_assign_k, st));
   LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
   ExpertParams xp{};
   xp.offsets = s->offsets;

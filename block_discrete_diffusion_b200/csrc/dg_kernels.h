@@ -126,8 +126,10 @@ cudaError_t dequant_fp8(const DequantArgs& a, int n_sms, cudaStream_t st);
 cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st);
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
                         int32_t* sel, float* gate, int32_t* counts, cudaStream_t st);
-cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k, int n_exp,
-                        int32_t* offsets, float* perm_gate, int32_t* perm_tok, int32_t* slot, cudaStream_t st);
+// expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
+cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
+                        int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,
+                        int* n_launched, cudaStream_t st);
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st);
 // g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g

@@ -227,6 +227,47 @@ __global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float*
   }
 }
 
+// Many assignments (several canvases): the offsets come from one small CTA (prefix sum; per-expert
+// cursors start at the offsets; counts cleared), then every assignment takes a row with a global
+// atomic on its expert's cursor (row order inside an expert is free, as above).
+__global__ void expert_offsets_kernel(int32_t* __restrict__ counts, int n_exp, int32_t* __restrict__ offsets,
+                                      int32_t* __restrict__ cursor) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_wsum[8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = threadIdx.x < n_exp ? counts[threadIdx.x] : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_wsum[w] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += s_wsum[i];
+  if (threadIdx.x < n_exp) {
+    offsets[threadIdx.x] = base + incl - c;
+    cursor[threadIdx.x] = base + incl - c;
+    counts[threadIdx.x] = 0;
+  }
+  if (threadIdx.x == n_exp - 1) offsets[n_exp] = base + incl;
+}
+
+__global__ void scatter_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate, int n_assign,
+                                    int top_k, int32_t* __restrict__ cursor, float* __restrict__ perm_gate,
+                                    int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+  pdl_trigger();
+  pdl_wait();
+  const int a = blockIdx.x * blockDim.x + threadIdx.x;
+  if (a >= n_assign) return;
+  const int row = atomicAdd(&cursor[sel[a]], 1);
+  perm_gate[row] = gate[a];
+  perm_tok[row] = a / top_k;
+  slot[a] = row;
+}
+
 // xp[slot[t*k + r]] = xn[t] for every rank r: one warp per token reads the row once.
 __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const int32_t* __restrict__ slot, int n_rows,
                                    int top_k, int d, __nv_bfloat16* __restrict__ xp) {
@@ -370,11 +411,21 @@ cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, in
   return launch_k(router_topk_kernel<8>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k,
                   sel, gate, counts);
 }
-cudaError_t assign_rows(const int32_t* sel, const float* gate, const int32_t* counts, int n_rows, int top_k, int n_exp,
-                        int32_t* offsets, float* perm_gate, int32_t* perm_tok, int32_t* slot, cudaStream_t st) {
+cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
+                        int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,
+                        int* n_launched, cudaStream_t st) {
   if (n_exp > 256) return cudaErrorInvalidValue;
-  return launch_k(assign_rows_kernel, dim3(1), dim3(1024), 0, st, 1, sel, gate, counts, n_rows * top_k, top_k, n_exp,
-                  offsets, perm_gate, perm_tok, slot);
+  const int n_assign = n_rows * top_k;
+  if (n_assign <= 8192) {   // one canvas: a single CTA does both (one launch)
+    *n_launched = 1;
+    return launch_k(assign_rows_kernel, dim3(1), dim3(1024), 0, st, 1, sel, gate, counts, n_assign, top_k, n_exp,
+                    offsets, perm_gate, perm_tok, slot);
+  }
+  *n_launched = 2;
+  cudaError_t e = launch_k(expert_offsets_kernel, dim3(1), dim3(256), 0, st, 1, counts, n_exp, offsets, cursor);
+  if (e != cudaSuccess) return e;
+  return launch_k(scatter_rows_kernel, dim3((n_assign + 255) / 256), dim3(256), 0, st, 1, sel, gate, n_assign, top_k,
+                  cursor, perm_gate, perm_tok, slot);
 }
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st) {
