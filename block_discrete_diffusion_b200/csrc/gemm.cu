@@ -53,60 +53,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ---------------------------------------------------------------------------------------------
 // dense GEMM
 // ---------------------------------------------------------------------------------------------
-// Epilogue of one output row segment: values for columns col0 + j (j < n) of row `row`.
-template <int EPI>
-__device__ __forceinline__ void store_row_f32(const EpiParams& ep, int row, int col0, const float* v, int n, int N) {
-  float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)row * ep.ldo + col0;
-  if (col0 + n <= N && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) && (n % 4) == 0) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-    for (int i = 0; i < n / 4; ++i) {
-      float4 o = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      if (EPI == EPI_RESID) {
-        const float4 x = d4[i];
-        o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
-      }
-      d4[i] = o;
-    }
-  } else {
-    for (int i = 0; i < n && col0 + i < N; ++i) dst[i] = (EPI == EPI_RESID ? dst[i] : 0.f) + v[i];
-  }
-}
-
-// QKV epilogue for `np` rotary pairs of one row: a[k] is column c1 + k, b[k] column c1 + half + k
-// of the fused Q|K|V output (columns of one head; c1 = head start + i0).  Q and K rows are rotated by
-// the row's position and stored head-major; V (no rotation) goes to the transposed value cache.
-__device__ __forceinline__ void store_qkv_pairs(const EpiParams& ep, int row, int f_head, int i0, const float* a,
-                                                const float* b, int np) {
-  const int dh = ep.dh, half = dh >> 1;
-  const int q_end = ep.n_q * dh, k_end = q_end + ep.n_kv * dh;
-  const int seq = row / ep.rows_per_seq, j = row % ep.rows_per_seq;
-  const int cseq = ep.seq_base + seq;
-  const int pos = ep.seq_P[cseq] + j;
-  if (f_head < k_end) {
-    const float2* cs = ep.rope + (size_t)pos * half + i0;
-    __nv_bfloat16* dst;
-    if (f_head < q_end) {
-      dst = ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh;
-    } else {
-      dst = ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + pos) * dh;
-    }
-    for (int k = 0; k < np; k += 2) {
-      const float2 c0 = cs[k], c1 = cs[k + 1];
-      *reinterpret_cast<uint32_t*>(dst + i0 + k) =
-          pack_bf16x2(a[k] * c0.x - b[k] * c0.y, a[k + 1] * c1.x - b[k + 1] * c1.y);
-      *reinterpret_cast<uint32_t*>(dst + half + i0 + k) =
-          pack_bf16x2(b[k] * c0.x + a[k] * c0.y, b[k + 1] * c1.x + a[k + 1] * c1.y);
-    }
-  } else {
-    __nv_bfloat16* dst = ep.vt + (((size_t)cseq * ep.n_kv + (f_head - k_end) / dh) * dh) * ep.max_ctx + pos;
-    for (int k = 0; k < np; ++k) {
-      dst[(size_t)(i0 + k) * ep.max_ctx] = __float2bfloat16_rn(a[k]);
-      dst[(size_t)(half + i0 + k) * ep.max_ctx] = __float2bfloat16_rn(b[k]);
-    }
-  }
-}
-
-// Epilogue of nr finished rows held in shared memory (t[r * rs + c], rows row0.., columns n0..),
+// Epilogue of RPC finished rows held in shared memory (t[r * rs + c], rows row0.., columns n0..),
 // laid out so that global stores are coalesced: F32 / RESID rows by one warp each (lane = 4
 // columns); Q and K heads rotated pairwise by one warp per row (lane = rotary pair), stored
 // head-major; V heads by one warp per channel (lane = row, positions contiguous in the
@@ -117,6 +64,7 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kGemmThreads / 32;
   constexpr int RPW = (RPC + NW - 1) / NW;   // rows per warp
+  constexpr int RB = RPW < 8 ? RPW : 8;      // rows whose loads are issued together
   // A 128-row tile lies inside one sequence's rows_per_seq rows: one committed length for all rows.
   // Global loads (length, rotary table, residual) are all issued before the stores that follow them.
   const int seq = row0 / ep.rows_per_seq, j0 = row0 % ep.rows_per_seq;
@@ -129,33 +77,36 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
       const int f_head = n0 + h0;
       if (f_head >= N) break;
       if (f_head < k_end) {
-        float2 cs[RPW][2];
+        for (int kb = 0; kb < RPW; kb += RB) {
+          float2 cs[RB][2];
 #pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-          const int r = warp + NW * k;
+          for (int k = 0; k < RB; ++k) {
+            const int r = warp + NW * (kb + k);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int i = lane + 32 * u;
-            cs[k][u] = (r < RPC && row0 + r < M && i < half) ? __ldg(ep.rope + (size_t)(P + j0 + r) * half + i)
-                                                              : make_float2(0.f, 0.f);
+            for (int u = 0; u < 2; ++u) {
+              const int i = lane + 32 * u;
+              cs[k][u] = (kb + k < RPW && r < RPC && row0 + r < M && i < half)
+                             ? __ldg(ep.rope + (size_t)(P + j0 + r) * half + i)
+                             : make_float2(0.f, 0.f);
+            }
           }
-        }
 #pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-          const int r = warp + NW * k;
-          if (r >= RPC || row0 + r >= M) break;
-          const int j = j0 + r;
-          __nv_bfloat16* dst =
-              f_head < q_end ? ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh
-                             : ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + P + j) * dh;
-          const float* tr = t + r * rs + h0;
+          for (int k = 0; k < RB; ++k) {
+            const int r = warp + NW * (kb + k);
+            if (kb + k >= RPW || r >= RPC || row0 + r >= M) break;
+            const int j = j0 + r;
+            __nv_bfloat16* dst =
+                f_head < q_end ? ep.q + (((size_t)seq * ep.n_q + f_head / dh) * ep.rows_per_seq + j) * dh
+                               : ep.kc + (((size_t)cseq * ep.n_kv + (f_head - q_end) / dh) * ep.max_ctx + P + j) * dh;
+            const float* tr = t + r * rs + h0;
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int i = lane + 32 * u;
-            if (i < half) {
-              const float a = tr[i], b = tr[half + i];
-              dst[i] = __float2bfloat16_rn(a * cs[k][u].x - b * cs[k][u].y);
-              dst[half + i] = __float2bfloat16_rn(b * cs[k][u].x + a * cs[k][u].y);
+            for (int u = 0; u < 2; ++u) {
+              const int i = lane + 32 * u;
+              if (i < half) {
+                const float a = tr[i], b = tr[half + i];
+                dst[i] = __float2bfloat16_rn(a * cs[k][u].x - b * cs[k][u].y);
+                dst[half + i] = __float2bfloat16_rn(b * cs[k][u].x + a * cs[k][u].y);
+              }
             }
           }
         }
@@ -169,37 +120,40 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
     }
   } else {
     constexpr int CG = BN / 128;             // 128-column groups (lane = 4 columns of each)
-    float4 xv[RPW][CG];
-    if constexpr (EPI == EPI_RESID) {
+    for (int kb = 0; kb < RPW; kb += RB) {
+      float4 xv[RB][CG];
+      if constexpr (EPI == EPI_RESID) {
 #pragma unroll
-      for (int k = 0; k < RPW; ++k) {
-        const int r = warp + NW * k;
+        for (int k = 0; k < RB; ++k) {
+          const int r = warp + NW * (kb + k);
+#pragma unroll
+          for (int g = 0; g < CG; ++g) {
+            const int c = g * 128 + lane * 4;
+            xv[k][g] = (kb + k < RPW && r < RPC && row0 + r < M && n0 + c + 4 <= N)
+                           ? *reinterpret_cast<const float4*>(ep.x + (size_t)(row0 + r) * ep.ldo + n0 + c)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        const int r = warp + NW * (kb + k);
+        if (kb + k >= RPW || r >= RPC || row0 + r >= M) break;
+        float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)(row0 + r) * ep.ldo + n0;
+        const float* tr = t + r * rs;
 #pragma unroll
         for (int g = 0; g < CG; ++g) {
           const int c = g * 128 + lane * 4;
-          xv[k][g] = (r < RPC && row0 + r < M && n0 + c + 4 <= N)
-                         ? *reinterpret_cast<const float4*>(ep.x + (size_t)(row0 + r) * ep.ldo + n0 + c)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < RPW; ++k) {
-      const int r = warp + NW * k;
-      if (r >= RPC || row0 + r >= M) break;
-      float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)(row0 + r) * ep.ldo + n0;
-      const float* tr = t + r * rs;
-#pragma unroll
-      for (int g = 0; g < CG; ++g) {
-        const int c = g * 128 + lane * 4;
-        if (n0 + c + 4 <= N) {
-          float4 v = *reinterpret_cast<const float4*>(tr + c);
-          if (EPI == EPI_RESID) {
-            v.x += xv[k][g].x; v.y += xv[k][g].y; v.z += xv[k][g].z; v.w += xv[k][g].w;
+          if (n0 + c + 4 <= N) {
+            float4 v = *reinterpret_cast<const float4*>(tr + c);
+            if (EPI == EPI_RESID) {
+              v.x += xv[k][g].x; v.y += xv[k][g].y; v.z += xv[k][g].z; v.w += xv[k][g].w;
+            }
+            *reinterpret_cast<float4*>(dst + c) = v;
+          } else {
+            for (int q = 0; q < 4 && n0 + c + q < N; ++q)
+              dst[c + q] = (EPI == EPI_RESID ? dst[c + q] : 0.f) + tr[c + q];
           }
-          *reinterpret_cast<float4*>(dst + c) = v;
-        } else {
-          for (int q = 0; q < 4 && n0 + c + q < N; ++q) dst[c + q] = (EPI == EPI_RESID ? dst[c + q] : 0.f) + tr[c + q];
         }
       }
     }
@@ -207,7 +161,8 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
 }
 
 // One 128 x BN output tile per cluster of Z CTAs; CTA z of the cluster multiplies k-blocks
-// [z nk/Z, (z+1) nk/Z).  Z = 1: the epilogue reads the accumulator from TMEM (thread = row).
+// [z nk/Z, (z+1) nk/Z).  Z = 1: the accumulator goes from TMEM (thread = row) to shared memory and
+// the epilogue runs from there.
 // Z > 1: every CTA writes its fp32 partial to its slot of an L2-resident scratch (coalesced); after
 // a cluster barrier CTA z sums rows [z 128/Z, (z+1) 128/Z) over the Z slots in rank order (so the
 // result does not depend on timing) and runs the epilogue on those rows from shared memory.
@@ -217,7 +172,7 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
                       int K, EpiParams ep, int* err) {
   using C = DenseCfg<BN>;
   static_assert(Z == 1 || (Z > 1 && 128 % Z == 0 && (BN / (2 * Z)) % 4 == 0), "bad split");
-  static_assert(Z == 1 || (size_t)128 * (BN + 4) * 4 <= (size_t)C::kStages * C::kStageBytes, "partial tile too big");
+  static_assert((size_t)128 * (BN + 4) * 4 <= (size_t)C::kStages * C::kStageBytes, "parked tile too big");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = align1024(smem_raw);
   GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(tiles + (size_t)C::kStages * C::kStageBytes);
@@ -296,27 +251,21 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
   const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
 
   if constexpr (Z == 1) {
-    // ---------------- thread owns accumulator row m0 + 32*warp + lane ----------------
-    const int row = m0 + warp * 32 + lane;
-    const bool row_ok = ok && row < M;
-    if constexpr (EPI == EPI_QKV) {
-      const int dh = ep.dh, half = dh >> 1;
-      for (int h0 = 0; h0 < BN; h0 += dh) {
-        if (n0 + h0 >= N) break;
-        for (int c = 0; c < half; c += 32) {
-          float a[32], b[32];
-          tmem_ld_32cols(tbase + h0 + c, a);
-          tmem_ld_32cols(tbase + h0 + half + c, b);
-          if (row_ok) store_qkv_pairs(ep, row, n0 + h0, c, a, b, 32);
-        }
-      }
-    } else {
+    // ---------------- accumulator -> shared memory (thread = row) -> coalesced epilogue ----------------
+    constexpr int RS = BN + 4;
+    float* red = reinterpret_cast<float*>(tiles);
+    {
+      const int r = warp * 32 + lane;
       for (int c = 0; c < BN; c += 32) {
-        float a[32];
-        tmem_ld_32cols(tbase + c, a);
-        if (row_ok) store_row_f32<EPI>(ep, row, n0 + c, a, 32, N);
+        float v[32];
+        tmem_ld_32cols(tbase + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(red + r * RS + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
+    __syncthreads();
+    if (ok) epilogue_from_smem<BN, EPI, 128>(ep, red, RS, m0, n0, M, N);
   } else {
     // ---------------- split-K: partials through an L2-resident scratch, summed in rank order ----------------
     constexpr int RS = BN + 4;                 // padded row stride of the shared-memory tiles
