@@ -74,6 +74,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// packed fp32 pairs (one 64-bit register, low word first)
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -224,26 +241,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // P pass: P = exp2(S scale - m_ref) in bf16 to this tile's swizzled P buffer (4 x 16-byte chunks
       // per 32 keys); returns the fp32 sum and the raw max of the visible scores
       auto p_pass = [&](float m_ref, float& rmax) {
-        float lt = 0.f;
+        uint64_t lt2 = 0;                               // two fp32 partial sums (packed)
+        const uint64_t sl2x2 = pack_f32x2(sl2, sl2), negm2 = pack_f32x2(-m_ref, -m_ref);
         rmax = -INFINITY;
 #pragma unroll
-        for (int cb = 0; cb < 128; cb += 32) {
-          float s[32];
+        for (int cb = 0; cb < 128; cb += 64) {
+          float s[64];
           tmem_ld32_nowait(t_s + cb, s);
+          tmem_ld32_nowait(t_s + cb + 32, s + 32);
           tmem_wait_ld();
-          uint32_t pk[16];
+          uint32_t pk[32];
           if (full) {
+            // packed fp32 pairs: one FMA and one add per two keys
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
+            for (int i = 0; i < 64; i += 2) {
               rmax = fmaxf(rmax, fmaxf(s[i], s[i + 1]));
-              const float p0 = fast_exp2(fmaf(s[i], sl2, -m_ref));
-              const float p1 = fast_exp2(fmaf(s[i + 1], sl2, -m_ref));
-              lt += p0 + p1;
+              const uint64_t x = ffma_f32x2(pack_f32x2(s[i], s[i + 1]), sl2x2, negm2);
+              const float p0 = fast_exp2(lo_f32(x)), p1 = fast_exp2(hi_f32(x));
+              lt2 = fadd_f32x2(lt2, pack_f32x2(p0, p1));
               pk[i / 2] = pack_bf16x2(p0, p1);
             }
           } else {
+            float lt = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
+            for (int i = 0; i < 64; i += 2) {
               const bool v0 = cb + i < kmax, v1 = cb + i + 1 < kmax;   // masked keys: p = 0
               if (v0) rmax = fmaxf(rmax, s[i]);
               if (v1) rmax = fmaxf(rmax, s[i + 1]);
@@ -252,16 +273,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               lt += p0 + p1;
               pk[i / 2] = pack_bf16x2(p0, p1);
             }
+            lt2 = fadd_f32x2(lt2, pack_f32x2(lt, 0.f));
           }
           uint8_t* prow_c = prow + (cb / 64) * 16384;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int chunk = ((cb % 64) / 8) + ch;
-            *reinterpret_cast<uint4*>(prow_c + ((chunk ^ (r & 7)) << 4)) =
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(prow_c + ((ch ^ (r & 7)) << 4)) =
                 make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          }
         }
-        return lt;
+        return lo_f32(lt2) + hi_f32(lt2);
       };
       // PV(tt-1) of this tile completed before S(tt) (tensor-core operations complete in order), so O
       // and this tile's P buffer are free here.  Optimistic single pass against the running max; a
