@@ -733,6 +733,7 @@ dg_status check_params(const dg_seqs* s, const dg_sampler_params* p) {
   if (p->max_steps <= 0 || p->fixed_steps < 0) return fail(DG_ERR_INVALID_ARG, "bad step budget");
   if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
   if (p->commit_mode != 0 && p->commit_mode != 1) return fail(DG_ERR_INVALID_ARG, "commit_mode must be 0 or 1");
+  if (p->commit_rule != 0 && p->commit_rule != 1) return fail(DG_ERR_INVALID_ARG, "commit_rule must be 0 or 1");
   (void)s;
   return DG_OK;
 }
@@ -857,6 +858,7 @@ DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t*
   a.entropy_bound = p->entropy_bound;
   a.stop_mean_entropy = p->stop_mean_entropy;
   a.rerand_entropy = p->rerand_entropy;
+  a.commit_rule = p->commit_rule;
   LAUNCH(s, DG_K_SAMPLER, 2, sampler_run(a, s->st));
   s->step += 1;
   return DG_OK;
@@ -998,6 +1000,7 @@ DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg
   a.entropy_bound = p->entropy_bound;
   a.stop_mean_entropy = p->stop_mean_entropy;
   a.rerand_entropy = p->rerand_entropy;
+  a.commit_rule = p->commit_rule;
   CK(sampler_run(a, static_cast<cudaStream_t>(stream)));
   return DG_OK;
 }

@@ -158,6 +158,7 @@ struct SamplerArgs {
   uint64_t seed;
   int step, max_steps, fixed_steps;
   float entropy_bound, stop_mean_entropy, rerand_entropy;
+  int commit_rule;       // 0 per-position entropy bound, 1 cumulative entropy bound
 };
 cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st);
 int sampler_chunks(int vocab);

@@ -14,10 +14,10 @@ enum : uint32_t { RNG_TAG_GUMBEL = 0, RNG_TAG_RERAND = 1, RNG_TAG_INIT = 2 };
 __device__ __forceinline__ uint4 philox4x32_10(uint4 ctr, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
-    const uint32_t a = ctr.x, c = ctr.z;
-    const uint32_t mul_a_hi = __umulhi(a, 0xD2511F53u), mul_a_lo = a * 0xD2511F53u;
-    const uint32_t mul_c_hi = __umulhi(c, 0xCD9E8D57u), mul_c_lo = c * 0xCD9E8D57u;
-    ctr = make_uint4(mul_c_hi ^ ctr.y ^ k0, mul_c_lo, mul_a_hi ^ ctr.w ^ k1, mul_a_lo);
+    // one 32 x 32 -> 64-bit product per multiplier gives both halves
+    const uint64_t pa = (uint64_t)ctr.x * 0xD2511F53u;
+    const uint64_t pc = (uint64_t)ctr.z * 0xCD9E8D57u;
+    ctr = make_uint4((uint32_t)(pc >> 32) ^ ctr.y ^ k0, (uint32_t)pc, (uint32_t)(pa >> 32) ^ ctr.w ^ k1, (uint32_t)pa);
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }

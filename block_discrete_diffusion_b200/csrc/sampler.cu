@@ -8,7 +8,9 @@
 // whose confidence dropped ("Uniform State Diffusion", same guide).  The precise rule (which
 // entropy, which threshold re-randomises, what ends a block) is the build's written reading:
 //   H = entropy (nats) of softmax(l / T);  y = argmax_v (l_v / T + Gumbel_v);
-//   commit iff H <= entropy_bound; else re-randomise iff H > rerand_entropy, else take y;
+//   commit iff H <= entropy_bound (or, with commit_rule 1, iff the entropies of the uncommitted
+//   positions at or before it in ascending (H, position) order sum to <= entropy_bound);
+//   else re-randomise iff H > rerand_entropy, else take y;
 //   stop iff all committed, or mean H over the canvas (committed = 0) <= stop_mean_entropy, or the
 //   step budget is reached (fixed_steps > 0: exactly fixed_steps steps); on stop the remaining
 //   positions take y and commit.
@@ -175,12 +177,13 @@ __global__ void sampler_finalize_kernel(SamplerArgs a) {
   // positions are strided over the block so any canvas length works with 256 threads
   const int n_iter = (a.canvas + blockDim.x - 1) / blockDim.x;
   // first pass: per-position decision without the stop override; remember (id, y, commit) locally
-  int my_id[4], my_y[4];
-  uint8_t my_c[4];
+  __shared__ float s_H[1024];   // cumulative rule: entropies of the uncommitted positions (canvas <= 1024)
+  int my_id[4], my_y[4], my_rr[4];
+  uint8_t my_c[4], my_unc[4];
   float my_H[4];
   for (int it = 0; it < n_iter && it < 4; ++it) {
     const int jj = threadIdx.x + it * blockDim.x;
-    my_id[it] = 0; my_y[it] = 0; my_c[it] = 1; my_H[it] = 0.f;
+    my_id[it] = 0; my_y[it] = 0; my_rr[it] = 0; my_c[it] = 1; my_unc[it] = 0; my_H[it] = 0.f;
     if (jj >= a.canvas) continue;
     const int row = seq * a.canvas + jj;
     if (a.commit_in[row]) {
@@ -204,15 +207,43 @@ __global__ void sampler_finalize_kernel(SamplerArgs a) {
     const int rr = token_from_word(w.x, (uint32_t)a.vocab);
     my_H[it] = H;
     my_y[it] = bidx;
-    if (H <= a.entropy_bound) {
-      my_id[it] = bidx;
+    my_rr[it] = rr;
+    my_unc[it] = 1;
+    Hsum_part += H;
+  }
+  // commit decisions: per position (H <= bound), or cumulative (ascending (H, position) order while
+  // the running entropy sum stays <= bound: position i commits iff the entropies of the uncommitted
+  // positions ordered at or before it sum to <= bound)
+  if (a.commit_rule == 1) {
+    for (int jj = threadIdx.x; jj < a.canvas; jj += blockDim.x) s_H[jj] = INFINITY;   // committed: excluded
+    __syncthreads();
+    for (int it = 0; it < n_iter && it < 4; ++it)
+      if (my_unc[it]) s_H[threadIdx.x + it * blockDim.x] = my_H[it];
+    __syncthreads();
+  }
+  for (int it = 0; it < n_iter && it < 4; ++it) {
+    if (!my_unc[it]) continue;
+    const int jj = threadIdx.x + it * blockDim.x;
+    bool commits;
+    if (a.commit_rule == 1) {
+      const float hi = my_H[it];
+      float run = 0.f;
+      for (int k = 0; k < a.canvas; ++k) {
+        const float hk = s_H[k];
+        if (hk < hi || (hk == hi && k <= jj)) run += hk;
+      }
+      commits = run <= a.entropy_bound;
+    } else {
+      commits = my_H[it] <= a.entropy_bound;
+    }
+    if (commits) {
+      my_id[it] = my_y[it];
       my_c[it] = 1;
     } else {
-      my_id[it] = H > a.rerand_entropy ? rr : bidx;
+      my_id[it] = my_H[it] > a.rerand_entropy ? my_rr[it] : my_y[it];
       my_c[it] = 0;
       all_part = 0;
     }
-    Hsum_part += H;
   }
   // canvas-mean entropy and the all-committed test
   float hs = warp_sum(Hsum_part);

@@ -105,6 +105,7 @@ DG_API dg_status dg_sample_noalloc(const float* d_logits, int n_seq, int vocab, 
   a.entropy_bound = p->entropy_bound;
   a.stop_mean_entropy = p->stop_mean_entropy;
   a.rerand_entropy = p->rerand_entropy;
+  a.commit_rule = p->commit_rule;
   const cudaError_t le = dg::sampler_run(a, static_cast<cudaStream_t>(stream));
   if (le != cudaSuccess) {
     char msg[160];

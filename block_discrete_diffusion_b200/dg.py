@@ -60,16 +60,17 @@ class dg_weights(ctypes.Structure):
 class dg_sampler_params(ctypes.Structure):
     _fields_ = [("canvas_len", c_int), ("max_steps", c_int), ("fixed_steps", c_int), ("t_start", c_float),
                 ("t_end", c_float), ("entropy_bound", c_float), ("stop_mean_entropy", c_float),
-                ("rerand_entropy", c_float), ("seed", c_uint64), ("eos_id", c_int), ("commit_mode", c_int)]
+                ("rerand_entropy", c_float), ("seed", c_uint64), ("eos_id", c_int), ("commit_mode", c_int),
+                ("commit_rule", c_int)]
 
 
 def sampler_params(vocab, seed=0, canvas_len=256, max_steps=48, fixed_steps=0, t_start=0.8, t_end=0.4,
                    entropy_bound=0.1, stop_mean_entropy=0.005, rerand_entropy=None, eos_id=-1,
-                   commit_mode=0) -> dg_sampler_params:
+                   commit_mode=0, commit_rule=0) -> dg_sampler_params:
     if rerand_entropy is None:
         rerand_entropy = 0.5 * math.log(vocab)
     return dg_sampler_params(canvas_len, max_steps, fixed_steps, t_start, t_end, entropy_bound, stop_mean_entropy,
-                             rerand_entropy, seed, eos_id, commit_mode)
+                             rerand_entropy, seed, eos_id, commit_mode, commit_rule)
 
 
 _LIB = None

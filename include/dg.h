@@ -108,6 +108,9 @@ typedef struct {
   int eos_id;              /* -1: no EOS */
   int commit_mode;         /* dg_decode's block commit: 0 dg_block_commit (recompute, default),
                               1 dg_block_commit_last_kv (keep the last step's K/V) */
+  int commit_rule;         /* 0: an uncommitted position commits iff H <= entropy_bound (default);
+                              1: cumulative: the uncommitted positions in ascending (H, position)
+                              order commit while their running entropy sum stays <= entropy_bound */
 } dg_sampler_params;
 
 /* Message for the last non-OK status returned on this thread ("" if none). */

@@ -61,7 +61,7 @@ def lib():
             getattr(L, name).argtypes = [c_int, c_int, c_void_p, c_void_p, c_void_p, c_float, c_uint64, c_int,
                                          c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_step_rule.argtypes = [c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_double, c_double,
-                                    c_double, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
+                                    c_double, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_step_rule.restype = c_int
         L.orc_canvas_init.argtypes = [c_int, c_int, c_uint64, c_int, c_void_p, c_void_p]
         _LIB = L
@@ -324,7 +324,10 @@ def sample_rows(logits, skip, pos, T, seed, step):
 
 
 def step_rule(commit, ids, H, y, rr, s, entropy_bound=0.1, rerand_entropy=None, stop_mean_entropy=0.005,
-              max_steps=48, fixed_steps=0, vocab=None):
+              max_steps=48, fixed_steps=0, vocab=None, cumulative=False):
+    """One step's decisions.  cumulative: the entropy-bound reading that commits the lowest-entropy
+    positions while their entropy sum stays within the bound; the result then also holds "cum",
+    each uncommitted position's running sum in ascending (H, position) order."""
     n = len(ids)
     if rerand_entropy is None:
         rerand_entropy = 0.5 * np.log(vocab)
@@ -336,9 +339,15 @@ def step_rule(commit, ids, H, y, rr, s, entropy_bound=0.1, rerand_entropy=None, 
     ids_out = np.empty(n, np.int32)
     commit_out = np.empty(n, np.uint8)
     mean = np.zeros(1)
+    cum = np.zeros(n)
     stop = lib().orc_step_rule(n, _p(commit), _p(ids), _p(H), _p(y), _p(rr), entropy_bound, rerand_entropy,
-                               stop_mean_entropy, s, max_steps, fixed_steps, _p(ids_out), _p(commit_out), _p(mean))
-    return {"ids": ids_out, "commit": commit_out, "stop": int(stop), "mean_H": float(mean[0])}
+                               stop_mean_entropy, s, max_steps, fixed_steps, int(bool(cumulative)), _p(ids_out),
+                               _p(commit_out), _p(mean), _p(cum))
+    assert stop >= 0
+    out = {"ids": ids_out, "commit": commit_out, "stop": int(stop), "mean_H": float(mean[0])}
+    if cumulative:
+        out["cum"] = cum
+    return out
 
 
 def canvas_init(n, P, seed, vocab):
@@ -354,8 +363,10 @@ def canvas_init(n, P, seed, vocab):
 
 class SamplerParams:
     def __init__(self, vocab, canvas_len=256, max_steps=48, fixed_steps=0, t_start=0.8, t_end=0.4,
-                 entropy_bound=0.1, stop_mean_entropy=0.005, rerand_entropy=None, seed=0, eos_id=-1):
+                 entropy_bound=0.1, stop_mean_entropy=0.005, rerand_entropy=None, seed=0, eos_id=-1,
+                 commit_rule=0):
         self.canvas_len, self.max_steps, self.fixed_steps = canvas_len, max_steps, fixed_steps
+        self.commit_rule = commit_rule
         self.t_start, self.t_end = t_start, t_end
         self.entropy_bound, self.stop_mean_entropy = entropy_bound, stop_mean_entropy
         self.rerand_entropy = 0.5 * np.log(vocab) if rerand_entropy is None else rerand_entropy
@@ -400,7 +411,8 @@ class Sequence:
         T = temperature(self.step, prm.max_steps, prm.t_start, prm.t_end)
         smp = sample_rows(fw["logits"], commit, pos, T, prm.seed, self.step)
         rule = step_rule(commit, ids, smp["H"], smp["y"], smp["rr"], self.step, prm.entropy_bound,
-                         prm.rerand_entropy, prm.stop_mean_entropy, prm.max_steps, prm.fixed_steps)
+                         prm.rerand_entropy, prm.stop_mean_entropy, prm.max_steps, prm.fixed_steps,
+                         cumulative=prm.commit_rule == 1)
         out = dict(smp)
         out.update(rule)
         out.update({"T": T, "step": self.step, "logits": fw["logits"], "hidden": fw["hidden"],

@@ -540,10 +540,23 @@ void orc_sample_rows_f64(int n, int V, const double *logits, const uint8_t *skip
     }
 }
 
+/* Sort key of the cumulative rule: entropy, then position. */
+static const double *g_sort_H;
+static int cmp_entropy_then_index(const void *a, const void *b)
+{
+    int i = *(const int *)a, j = *(const int *)b;
+    if (g_sort_H[i] < g_sort_H[j]) return -1;
+    if (g_sort_H[i] > g_sort_H[j]) return 1;
+    return (i > j) - (i < j);
+}
+
 /* Decision rule of one step [reading of the entropy-bound sampler, self-correction and adaptive
  * stop]:
  *   - a committed position keeps its id (committed positions are anchors and never change);
- *   - an uncommitted position with H <= entropy_bound commits with id y;
+ *   - cumulative == 0: an uncommitted position with H <= entropy_bound commits with id y;
+ *     cumulative == 1: the uncommitted positions in ascending (H, position) order commit with id y
+ *     while the running sum of their entropies stays <= entropy_bound (the longest such prefix);
+ *     cum (nullable) receives each uncommitted position's running sum in that order;
  *   - otherwise it is re-randomised (id rr) when H > rerand_entropy, else takes y;
  *   - stop after this step when every position is committed, or mean(H over all n positions,
  *     committed ones counting 0) <= stop_mean_entropy, or s + 1 == max_steps; with
@@ -552,19 +565,41 @@ void orc_sample_rows_f64(int n, int V, const double *logits, const uint8_t *skip
  * Returns the stop flag; *mean_H receives the canvas-mean entropy. */
 int orc_step_rule(int n, const uint8_t *commit_in, const int32_t *ids_in, const double *H,
                   const int32_t *y, const int32_t *rr, double entropy_bound, double rerand_entropy,
-                  double stop_mean_entropy, int s, int max_steps, int fixed_steps,
-                  int32_t *ids_out, uint8_t *commit_out, double *mean_H)
+                  double stop_mean_entropy, int s, int max_steps, int fixed_steps, int cumulative,
+                  int32_t *ids_out, uint8_t *commit_out, double *mean_H, double *cum)
 {
+    uint8_t *commits_now = (uint8_t *)calloc((size_t)n, 1);
+    if (!commits_now) return -1;
+    if (cumulative) {
+        int *order = (int *)malloc(sizeof(int) * (size_t)n);
+        if (!order) { free(commits_now); return -1; }
+        int m = 0;
+        for (int i = 0; i < n; ++i)
+            if (!commit_in[i]) order[m++] = i;
+        g_sort_H = H;
+        qsort(order, (size_t)m, sizeof(int), cmp_entropy_then_index);
+        double run = 0.0;
+        for (int k = 0; k < m; ++k) {
+            run += H[order[k]];
+            if (cum) cum[order[k]] = run;
+            if (run <= entropy_bound) commits_now[order[k]] = 1;
+        }
+        free(order);
+    } else {
+        for (int i = 0; i < n; ++i)
+            commits_now[i] = !commit_in[i] && H[i] <= entropy_bound;
+    }
     double sumH = 0.0;
     int all = 1;
     for (int i = 0; i < n; ++i) {
         if (commit_in[i]) {
             ids_out[i] = ids_in[i];
             commit_out[i] = 1;
+            if (cum) cum[i] = 0.0;
             continue;
         }
         sumH += H[i];
-        if (H[i] <= entropy_bound) {
+        if (commits_now[i]) {
             ids_out[i] = y[i];
             commit_out[i] = 1;
         } else {
@@ -573,6 +608,7 @@ int orc_step_rule(int n, const uint8_t *commit_in, const int32_t *ids_in, const 
             all = 0;
         }
     }
+    free(commits_now);
     double mean = sumH / n;
     *mean_H = mean;
     int stop;

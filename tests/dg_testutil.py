@@ -123,7 +123,8 @@ def judge_step(gpu, orc, prm, commit_before, exclude=None, margin_tol=None, h_to
     for i in bad[:5]:
         fails.append(f"entropy row {i}: gpu {H_g[i]} oracle {H_o[i]} tol {h_tol[i]}")
     band = np.maximum(DECISION_BAND, h_tol)
-    near_bound = np.abs(H_o - prm.entropy_bound) <= band
+    # per-position rule: H against the bound; cumulative rule: the running entropy sum ("cum")
+    near_bound = np.abs((orc["cum"] if "cum" in orc else H_o) - prm.entropy_bound) <= band
     near_rr = np.abs(H_o - prm.rerand_entropy) <= band
     # The stop flag is judged when no admissible difference can move it: a fixed budget, or a canvas
     # mean far from the threshold even if every excluded row's entropy moved by its whole range

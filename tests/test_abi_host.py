@@ -88,7 +88,7 @@ def test_sampler_params_defaults(dg):
     assert math.isclose(p.entropy_bound, 0.1, rel_tol=1e-7)
     assert math.isclose(p.stop_mean_entropy, 0.005, rel_tol=1e-6)
     assert math.isclose(p.rerand_entropy, 0.5 * math.log(262144), rel_tol=1e-6)
-    assert ctypes.sizeof(dg.dg_sampler_params) == 48
+    assert ctypes.sizeof(dg.dg_sampler_params) == 56
 
 
 def test_product_path_does_not_import_the_oracle():

@@ -97,6 +97,40 @@ def test_sampler_matches_oracle(dg, vocab, spike, step, rows_checked):
         assert g["commit"][spiked].all()       # near-one-hot rows commit
 
 
+def test_sampler_cumulative_commit_rule_matches_oracle(dg):
+    """commit_rule 1: the lowest-entropy uncommitted positions commit while their entropy sum stays
+    within the bound.  Every third row gets a spike of height 11-14 above N(0,1) logits, so the
+    spiked rows have entropies between ~0.002 and ~0.1 and the running sum crosses the bound part
+    of the way through them."""
+    vocab, canvas, step = 4096, 256, 0
+    rng = np.random.default_rng(21)
+    lg = rng.normal(size=(canvas, vocab)).astype(np.float32)
+    for r in range(0, canvas, 3):
+        lg[r, rng.integers(vocab)] += rng.uniform(11.0, 14.0)
+    commit0 = (rng.random(canvas) < 0.1).astype(np.uint8)
+    ids0 = rng.integers(0, vocab, canvas).astype(np.int32)
+    prm_o = oracle.SamplerParams(vocab, seed=3, commit_rule=1)
+    prm = dg.sampler_params(vocab, seed=3, commit_rule=1)
+    ids = torch.from_numpy(ids0).cuda()
+    commit = torch.from_numpy(commit0).cuda()
+    H = torch.empty(canvas, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device="cuda")
+    dg.dg_sample(torch.from_numpy(lg).cuda(), 1, vocab, prm, step, None, ids, commit, H, stop, ws)
+    torch.cuda.synchronize()
+    g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(), "stop": int(stop.item())}
+    T = oracle.temperature(step)
+    smp = oracle.sample_rows(lg, commit0, np.arange(canvas), T, 3, step)
+    o = dict(smp)
+    o.update(oracle.step_rule(commit0, ids0, smp["H"], smp["y"], smp["rr"], step, vocab=vocab, cumulative=True))
+    fails, judged = judge_step(g, o, prm_o, commit0)
+    assert not fails, fails[:10]
+    new_commits = int(o["commit"].sum() - commit0.sum())
+    per_position = int(((smp["H"] <= 0.1) & (commit0 == 0)).sum())
+    assert 0 < new_commits < per_position            # the cumulative rule cut in, but not at zero
+    assert judged > canvas // 2
+
+
 def test_sampler_is_deterministic(dg):
     vocab, canvas = 262144, 256
     logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=3)

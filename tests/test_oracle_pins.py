@@ -528,3 +528,29 @@ def test_fp8_layer_equals_bf16_layer_holding_q_times_s():
     b = oracle.layer_forward(Mb, 0, x, pos, P, kc, vc)
     for u, v in zip(a, b):
         np.testing.assert_array_equal(u, v)
+
+
+def test_cumulative_entropy_bound_commits_the_lowest_entropy_prefix():
+    """The cumulative reading of the entropy bound: uncommitted positions in ascending (H, position)
+    order commit while the running entropy sum stays within the bound.  Hand-built case: with bound
+    0.1 the per-position rule commits every H <= 0.1, the cumulative one only the prefix 0.015, 0.02,
+    0.03, 0.03 (equal entropies by position) -> sums 0.015, 0.035, 0.065, 0.095; the next (0.04)
+    would exceed."""
+    V = 4096
+    H = np.array([0.04, 0.03, 0.5, 0.02, 0.03, 0.015, 3.0, 0.09])
+    commit = np.array([0, 0, 0, 0, 0, 0, 0, 1], np.uint8)          # position 7 already committed
+    ids = np.arange(8, dtype=np.int32) + 100
+    y = np.arange(8, dtype=np.int32) + 200
+    rr = np.arange(8, dtype=np.int32) + 300
+    per = oracle.step_rule(commit, ids, H, y, rr, s=0, rerand_entropy=1.0, vocab=V)
+    np.testing.assert_array_equal(per["commit"], [1, 1, 0, 1, 1, 1, 0, 1])
+    cu = oracle.step_rule(commit, ids, H, y, rr, s=0, rerand_entropy=1.0, vocab=V, cumulative=True)
+    np.testing.assert_array_equal(cu["commit"], [0, 1, 0, 1, 1, 1, 0, 1])
+    np.testing.assert_array_equal(cu["ids"], [200, 201, 202, 203, 204, 205, 306, 107])   # 6 re-randomised
+    np.testing.assert_allclose(cu["cum"][[5, 3, 1, 4, 0]], [0.015, 0.035, 0.065, 0.095, 0.135], rtol=1e-12)
+    assert cu["cum"][7] == 0.0
+    # a bound below every entropy commits nothing; a huge bound commits every uncommitted position
+    assert oracle.step_rule(commit, ids, H, y, rr, s=0, entropy_bound=0.01, rerand_entropy=1.0, vocab=V,
+                            cumulative=True)["commit"].sum() == 1
+    assert oracle.step_rule(commit, ids, H, y, rr, s=0, entropy_bound=10.0, rerand_entropy=1.0, vocab=V,
+                            cumulative=True)["commit"].all()
