@@ -293,6 +293,14 @@ def forward(model: Model, ids, pos, P, k_caches, v_caches, causal=False, write_c
     return {"hidden": hid, "router": rtr, "logits": logits}
 
 
+def embed(model: Model, ids):
+    """Embedding rows of ids (bf16 upcast exactly) as fp64 [n, d]."""
+    ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
+    x = np.empty((ids.shape[0], model.cfg.d_model))
+    lib().orc_embed(ctypes.byref(model.c_cfg), model.c_model.emb, ids.shape[0], _p(ids), _p(x))
+    return x
+
+
 def head(model: Model, x):
     x = _f64(x)
     n = x.shape[0]

@@ -1,0 +1,77 @@
+"""The 30-layer benchmark model (d 2816, 128 experts top-8, vocabulary 262144, bf16, residual-scaled
+random init) against the oracle, layer by layer.
+
+Each layer runs on the GPU (dg_layer_forward, canvas mode, behind a 2048-position synthetic prefix)
+from the oracle's input to that layer, so a router near-tie in one layer does not carry into the
+next; every layer's attention-block output, router logits, layer output and canvas K/V are judged
+with the spec tolerance, tokens with a router near-tie in that layer excluded.  Marked gpu.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from dg_testutil import HIDDEN_TOL, kv_views, rel_err, router_tie_tokens
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg(cuda_ok):
+    from block_discrete_diffusion_b200 import build, dg as dgmod
+    build.build()
+    return dgmod
+
+
+def _host(t):
+    return {k: v.cpu() for k, v in t.items()} if isinstance(t, dict) else t.cpu()
+
+
+def test_full_stack_every_layer_matches_oracle(dg):
+    cfg = synthetic.FULL
+    P = 2048
+    w = synthetic.make_model_weights(cfg, 2, device="cuda", **synthetic.full_stack_init(cfg))
+    model = dg.dg_model_create(cfg, w)
+    max_ctx = P + 256
+    seqs = dg.dg_seqs_create(model, 1, max_ctx)
+    ks, vs = synthetic.make_prefix_kv(cfg.n_layers, P, cfg.n_kv, cfg.d_head, 5, device="cuda")
+    dg.dg_load_prefix(seqs, 0, P, ks, vs)
+    prm = dg.sampler_params(cfg.vocab, seed=2)
+    ids = torch.empty(256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    torch.cuda.synchronize()
+    ids_h = ids.cpu().numpy()
+    Me = oracle.Model(cfg, {"emb": w["emb"].cpu()}, layers=[])
+    x = oracle.embed(Me, ids_h)
+    del Me
+    pos = np.arange(P, P + 256)
+    c1 = dataclasses.replace(cfg, n_layers=1)
+    judged_min = 256
+    for l in range(cfg.n_layers):
+        L = {k: _host(v) for k, v in w["layers"][l].items()}
+        M = oracle.Model(c1, {"layers": [L]}, layers=[L])
+        kc, vc = ks[l].double().cpu().numpy(), vs[l].double().cpu().numpy()
+        xo, kn, vn, rlo, mido = oracle.layer_forward(M, 0, x, pos, P, kc, vc, want_mid=True)
+        xd = torch.from_numpy(x).float().cuda()
+        mid = torch.zeros_like(xd)
+        rl = torch.zeros(256, cfg.n_exp, device="cuda")
+        dg.dg_layer_forward(seqs, l, xd, mid, rl)
+        torch.cuda.synchronize()
+        e_mid = rel_err(mid.cpu().numpy(), mido)
+        e_rl = rel_err(rl.cpu().numpy(), rlo)
+        keep = ~router_tie_tokens(rlo, cfg.top_k)
+        e_out = rel_err(xd.cpu().numpy()[keep], xo[keep])
+        K, Vt = kv_views(seqs.kv, cfg, 1, max_ctx)
+        kg = K[l, 0, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
+        vg = Vt[l, 0, :, :, P:P + 256].permute(2, 0, 1).float().cpu().numpy()
+        assert e_mid <= HIDDEN_TOL and e_rl <= HIDDEN_TOL, (l, e_mid, e_rl)
+        assert e_out <= HIDDEN_TOL, (l, e_out, int(keep.sum()))
+        assert rel_err(kg, kn) <= HIDDEN_TOL and rel_err(vg, vn) <= HIDDEN_TOL, l
+        judged_min = min(judged_min, int(keep.sum()))
+        x = xo
+    assert judged_min >= 128
+    assert dg.dg_device_error(seqs) == 0
