@@ -311,6 +311,7 @@ struct dg_seqs {
   int step;
   bool block_open;
   int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
+  int pre_bytes;    // bytes per weight row the gate|up GEMM brings into L2 before its wait (DG_EXPERT_PREFETCH)
   // statistics: launches per kernel class; optional event timing
   long long launches[DG_K_COUNT];
   double ms[DG_K_COUNT];
@@ -516,6 +517,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->next_pair = 0;
   s->max_splits = kMaxSplits;
   if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
+  s->pre_bytes = 4096;
+  if (const char* v = getenv("DG_EXPERT_PREFETCH")) s->pre_bytes = std::max(0, atoi(v));
 
   const uint64_t d = c.d_model, R = L.R, A = L.A;
   const uint64_t zdim = (uint64_t)c.n_layers * n_seq * c.n_kv;
@@ -694,6 +697,10 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   const int wide = rows * c.top_k >= 128 * c.n_exp ? 1 : 0;
   const LayerMaps& ME = s->m->maps[l];   // expert weight descriptors: bf16, or e4m3 bytes in the FP8 form
   ExpertParams xu = xp, xd = xp;
+  if (!fp8 && !wide && s->pre_bytes > 0) {
+    xu.w_base = W.w_gate_up;
+    xu.pre_bytes = std::min(s->pre_bytes, d * 2) & ~15;
+  }
   if (fp8) {
     xu.w_scale = W.s_gate_up;
     xu.w_scale_cols = (d + 127) / 128;
