@@ -517,7 +517,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->next_pair = 0;
   s->max_splits = kMaxSplits;
   if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
-  s->pre_bytes = 4096;
+  s->pre_bytes = 1 << 20;   // capped at the row length: the whole first tile
   if (const char* v = getenv("DG_EXPERT_PREFETCH")) s->pre_bytes = std::max(0, atoi(v));
 
   const uint64_t d = c.d_model, R = L.R, A = L.A;

@@ -89,8 +89,8 @@ struct ExpertParams {
   int d, F;
   const float* w_scale;  // FP8 weights: fp32 scale per 128 x 128 tile of the weight matrix viewed as
   int w_scale_cols;      // 2-D, w_scale_cols tiles per row; nullptr for bf16 weights
-  const void* w_base;    // bf16 MODE 1: the weight matrix, and the bytes of each row of the CTA's first
-  int pre_bytes;         // tile to bring into L2 before the grid-dependency wait (0: none; % 16 == 0)
+  const void* w_base;    // bf16 weights [rows][K], and the bytes of each row of the CTA's first tile to
+  int pre_bytes;         // bring into L2 before the grid-dependency wait (0: none; % 16 == 0)
 };
 
 struct AttnParams {

@@ -411,16 +411,16 @@ __global__ void __launch_bounds__(FP8 ? kExpThreadsFp8 : kExpThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
-  if (!FP8 && MODE == 1 && p.pre_bytes > 0 && (int)blockIdx.x < n_items) {
+  if (!FP8 && p.pre_bytes > 0 && (int)blockIdx.x < n_items) {
     // While the preceding (light) kernels still run, the HBM is idle: bring the first columns of
     // this CTA's first weight tile into L2 (weights are never written by this step).  One range
     // per weight row (rows are K-contiguous); TMA reads them after the wait.
     const int e = blockIdx.x / MT, mt = blockIdx.x % MT;
-    const int r0 = e * 2 * p.F + mt * 64;
     const uint8_t* wbase = static_cast<const uint8_t*>(p.w_base);
     for (int i = threadIdx.x; i < 128; i += blockDim.x) {
-      const int row = i < 64 ? r0 + i : r0 + p.F + (i - 64);
-      l2_prefetch_bulk(wbase + (size_t)row * p.d * 2, (uint32_t)p.pre_bytes);
+      const int row = MODE == 1 ? (i < 64 ? e * 2 * p.F + mt * 64 + i : e * 2 * p.F + p.F + mt * 64 + (i - 64))
+                                : e * p.d + mt * 128 + i;
+      l2_prefetch_bulk(wbase + (size_t)row * K * 2, (uint32_t)p.pre_bytes);
     }
   }
   pdl_wait();   // the routing (offsets) and the activation rows come from the preceding kernels
