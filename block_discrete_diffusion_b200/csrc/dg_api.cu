@@ -149,7 +149,7 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
-      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, total;
+      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, total;
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
 
@@ -227,6 +227,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.splitk = take(4 * (size_t)kSplitKSlots * 128 * 128);
   L.head_off = take(8);
   L.cursor = take(4 * 256);
+  L.topk_done = take(64);
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
@@ -306,6 +307,7 @@ struct dg_seqs {
   CUtensorMap xn32_map;         // xn in 32-row boxes (token operand of the persistent head GEMM)
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
+  int32_t* topk_done;           // launch counter of the top-k kernel that also buckets
   __nv_bfloat16* wq[5];         // FP8 form: the scratch matrices (qkv, o, router, gate_up, down)
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
@@ -504,6 +506,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->splitk = reinterpret_cast<float*>(b + L.splitk);
   s->head_off = reinterpret_cast<int32_t*>(b + L.head_off);
   s->cursor = reinterpret_cast<int32_t*>(b + L.cursor);
+  s->topk_done = reinterpret_cast<int32_t*>(b + L.topk_done);
   for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 && i < 3 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
@@ -546,6 +549,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   // clear the cache and the buffers whose stale contents a masked lane may read, build the table
   cudaError_t e = cudaMemsetAsync(kv, 0, need_kv, s->st);
   if (e == cudaSuccess) e = cudaMemsetAsync(s->ws, 0, L.rope, s->st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(s->topk_done, 0, 64, s->st);   // launch counter starts at 0
 
   if (e == cudaSuccess) e = rope_table(s->rope, max_ctx, c.d_head, c.rope_theta, s->st);
   if (e == cudaSuccess) {
@@ -677,13 +681,19 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   er.part_slots = kSplitKSlots;
   er.k_splits = std::min(kRouterSplits, dense_splits((rows + 127) / 128, d / 64));
   LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
-  LAUNCH(s, DG_K_TOPK, 1, router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, st));
+  // one canvas: the last CTA of the top-k launch also does the bucketing (one launch fewer)
+  const bool fuse_assign = rows * c.top_k <= 8192 && c.n_exp <= 256;
+  FusedAssignArgs fa{s->topk_done, s->offsets, s->perm_gate, s->perm_tok, s->slot};
+  LAUNCH(s, DG_K_TOPK, 1,
+         router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, fuse_assign ? &fa : nullptr, st));
   if (rlog_out)
     CK(cudaMemcpyAsync(rlog_out, s->rlog, sizeof(float) * (size_t)rows * c.n_exp, cudaMemcpyDeviceToDevice, st));
-  int n_assign_k = 1;
-  LAUNCH(s, DG_K_BUCKET, n_assign_k,
-         assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->perm_gate,
-                     s->perm_tok, s->slot, &n_assign_k, st));
+  if (!fuse_assign) {
+    int n_assign_k = 1;
+    LAUNCH(s, DG_K_BUCKET, n_assign_k,
+           assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->perm_gate,
+                       s->perm_tok, s->slot, &n_assign_k, st));
+  }
   LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
   ExpertParams xp{};
   xp.offsets = s->offsets;

@@ -126,8 +126,16 @@ cudaError_t rmsnorm_rows(const float* x, const float* g, int n_rows, int d, floa
                          cudaStream_t st);
 cudaError_t dequant_fp8(const DequantArgs& a, int n_sms, cudaStream_t st);
 cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStream_t st);
+// Bucketing done by the last CTA of the top-k launch (one canvas: n_rows * top_k <= 8192).
+struct FusedAssignArgs {
+  int32_t* done;         // zero-initialised launch counter (reset by that CTA)
+  int32_t* offsets;
+  float* perm_gate;
+  int32_t* perm_tok;
+  int32_t* slot;
+};
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
-                        int32_t* sel, float* gate, int32_t* counts, cudaStream_t st);
+                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused, cudaStream_t st);
 // expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
                         int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,

@@ -106,14 +106,51 @@ __global__ void rope_table_kernel(float2* table, int dh, double theta) {
 // The router logits arrive as n_parts split-K partial planes (part_stride apart), summed here in
 // plane order.  Lane l owns experts [l*V, l*V + V), V = ceil(E/32) <= 8.
 template <int V>
+__device__ __forceinline__ void router_topk_row(const float* __restrict__ logits, int n_parts, size_t part_stride,
+                                                int row, int n_exp, int top_k, int32_t* __restrict__ sel,
+                                                float* __restrict__ gate, int32_t* __restrict__ counts,
+                                                int lane);
+__device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t* counts, int n_assign, int top_k,
+                                  int n_exp, int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
+                                  int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot);
+
+struct FusedAssign {   // the last CTA of the top-k launch also buckets the assignments (done != nullptr)
+  int32_t* done;       // launch counter, reset to 0 by that CTA
+  int32_t* offsets;
+  float* perm_gate;
+  int32_t* perm_tok;
+  int32_t* slot;
+};
+
+template <int V>
 __global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts, size_t part_stride, int n_rows,
                                    int n_exp, int top_k, int32_t* __restrict__ sel, float* __restrict__ gate,
-                                   int32_t* __restrict__ counts) {
+                                   int32_t* __restrict__ counts, FusedAssign fa) {
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= n_rows) return;
+  if (row < n_rows) router_topk_row<V>(logits, n_parts, part_stride, row, n_exp, top_k, sel, gate, counts, lane);
+  if (fa.done) {
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(fa.done, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      assign_rows_block(sel, gate, counts, n_rows * top_k, top_k, n_exp, fa.offsets, fa.perm_gate, fa.perm_tok,
+                        fa.slot);
+      if (threadIdx.x == 0) *fa.done = 0;
+    }
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void router_topk_row(const float* __restrict__ logits, int n_parts, size_t part_stride,
+                                                int row, int n_exp, int top_k, int32_t* __restrict__ sel,
+                                                float* __restrict__ gate, int32_t* __restrict__ counts,
+                                                int lane) {
   float v[V];
   const float* lr = logits + (size_t)row * n_exp + lane * V;
 #pragma unroll
@@ -179,19 +216,18 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts
 // every (token, rank) assignment.  Rows inside an expert are handed out with shared-memory atomics,
 // so their order varies between runs; no result depends on it (each expert-GEMM column reads only
 // its own row, and the combine sums a token's rows in rank order).
-__global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate,
-                                   const int32_t* __restrict__ counts, int n_assign, int top_k, int n_exp,
-                                   int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
-                                   int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
-  pdl_trigger();
-  pdl_wait();
+// Offsets (exclusive prefix sum of the counts, by the first 256 threads) and the bucketed row of
+// every assignment; counts cleared for the next layer.  Needs blockDim.x >= 256.  Loads bypass L1
+// (sel, gate and counts may come from other CTAs of the same launch).
+__device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t* counts, int n_assign, int top_k,
+                                  int n_exp, int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
+                                  int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
   __shared__ int s_off[257];
   __shared__ int s_cur[256];
   __shared__ int s_wsum[8];
-  // exclusive prefix sum of the counts by the first 256 threads (warp scans, then the warp totals)
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   if (threadIdx.x < 256) {
-    const int c = threadIdx.x < n_exp ? counts[threadIdx.x] : 0;
+    const int c = threadIdx.x < n_exp ? __ldcg(counts + threadIdx.x) : 0;
     int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -204,7 +240,7 @@ __global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float*
   }
   __syncthreads();
   // the counts are consumed: clear them for the next layer's router (no separate memset)
-  if (threadIdx.x < n_exp) const_cast<int32_t*>(counts)[threadIdx.x] = 0;
+  if (threadIdx.x < n_exp) counts[threadIdx.x] = 0;
   if (threadIdx.x < 256) {
     int base = 0;
     for (int i = 0; i < w; ++i) base += s_wsum[i];
@@ -219,12 +255,21 @@ __global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float*
   __syncthreads();
   for (int e = threadIdx.x; e <= n_exp; e += blockDim.x) offsets[e] = s_off[e];
   for (int a = threadIdx.x; a < n_assign; a += blockDim.x) {
-    const int e = sel[a];
+    const int e = __ldcg(sel + a);
     const int row = s_off[e] + atomicAdd(&s_cur[e], 1);
-    perm_gate[row] = gate[a];
+    perm_gate[row] = __ldcg(gate + a);
     perm_tok[row] = a / top_k;
     slot[a] = row;
   }
+}
+
+__global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate,
+                                   int32_t* __restrict__ counts, int n_assign, int top_k, int n_exp,
+                                   int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
+                                   int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+  pdl_trigger();
+  pdl_wait();
+  assign_rows_block(sel, gate, counts, n_assign, top_k, n_exp, offsets, perm_gate, perm_tok, slot);
 }
 
 // Many assignments (several canvases): the offsets come from one small CTA (prefix sum; per-expert
@@ -397,19 +442,20 @@ cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStre
   return launch_k(rope_table_kernel, dim3(max_ctx), dim3(dh / 2), 0, st, 1, table, dh, (double)theta);
 }
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
-                        int32_t* sel, float* gate, int32_t* counts, cudaStream_t st) {
+                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
   const int V = (n_exp + 31) / 32;
   const dim3 grid((n_rows + 7) / 8);
+  FusedAssign fa{};
+  if (fused) fa = FusedAssign{fused->done, fused->offsets, fused->perm_gate, fused->perm_tok, fused->slot};
 #define DG_TOPK_CASE(V_) \
-  if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts);
+  if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts, fa);
   DG_TOPK_CASE(1)
   DG_TOPK_CASE(2)
   DG_TOPK_CASE(4)
   DG_TOPK_CASE(8)
 #undef DG_TOPK_CASE
-  return launch_k(router_topk_kernel<8>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k,
-                  sel, gate, counts);
+  return cudaErrorInvalidValue;
 }
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
                         int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,
