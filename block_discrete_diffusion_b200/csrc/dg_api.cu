@@ -148,7 +148,7 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 // ---------------------------------------------------------------------------------------------
 struct WsLayout {
   int R, A, split_cap, chunks;
-  size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, perm_gate, perm_tok, slot, xp, hb,
+  size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, slot, xp, hb,
       y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, total;
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
@@ -211,8 +211,6 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.gate = take(4 * A);
   L.counts = take(4 * (size_t)c.n_exp);
   L.offsets = take(4 * (size_t)(c.n_exp + 1));
-  L.perm_gate = take(4 * A);
-  L.perm_tok = take(4 * A);
   L.slot = take(4 * A);
   L.xp = take(2 * A * d);
   L.hb = take(2 * A * (size_t)c.d_ff);
@@ -295,9 +293,9 @@ struct dg_seqs {
   uint8_t* ws;
   // typed workspace views
   int *err, *seqP;
-  float *x, *opart, *ml, *rlog, *gate, *perm_gate, *y, *logits, *samp, *splitk;
+  float *x, *opart, *ml, *rlog, *gate, *y, *logits, *samp, *splitk;
   __nv_bfloat16 *xn, *q, *attn, *xp, *hb;
-  int32_t *sel, *counts, *offsets, *perm_tok, *slot, *cids, *cstop;
+  int32_t *sel, *counts, *offsets, *slot, *cids, *cstop;
   uint8_t* ccommit;
   float* cH;
 
@@ -490,8 +488,6 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->gate = reinterpret_cast<float*>(b + L.gate);
   s->counts = reinterpret_cast<int32_t*>(b + L.counts);
   s->offsets = reinterpret_cast<int32_t*>(b + L.offsets);
-  s->perm_gate = reinterpret_cast<float*>(b + L.perm_gate);
-  s->perm_tok = reinterpret_cast<int32_t*>(b + L.perm_tok);
   s->slot = reinterpret_cast<int32_t*>(b + L.slot);
   s->xp = reinterpret_cast<__nv_bfloat16*>(b + L.xp);
   s->hb = reinterpret_cast<__nv_bfloat16*>(b + L.hb);
@@ -683,7 +679,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
   // one canvas: the last CTA of the top-k launch also does the bucketing (one launch fewer)
   const bool fuse_assign = rows * c.top_k <= 8192 && c.n_exp <= 256;
-  FusedAssignArgs fa{s->topk_done, s->offsets, s->perm_gate, s->perm_tok, s->slot};
+  FusedAssignArgs fa{s->topk_done, s->offsets, s->slot};
   LAUNCH(s, DG_K_TOPK, 1,
          router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, fuse_assign ? &fa : nullptr, st));
   if (rlog_out)
@@ -691,14 +687,12 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   if (!fuse_assign) {
     int n_assign_k = 1;
     LAUNCH(s, DG_K_BUCKET, n_assign_k,
-           assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->perm_gate,
-                       s->perm_tok, s->slot, &n_assign_k, st));
+           assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->slot,
+                       &n_assign_k, st));
   }
   LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
   ExpertParams xp{};
   xp.offsets = s->offsets;
-  xp.perm_gate = s->perm_gate;
-  xp.perm_tok = s->perm_tok;
   xp.h_out = s->hb;
   xp.y_out = s->y;
   xp.d = d;

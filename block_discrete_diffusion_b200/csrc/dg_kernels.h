@@ -82,8 +82,6 @@ struct DequantArgs {
 
 struct ExpertParams {
   const int* offsets;    // [E+1] first bucketed row of each expert (expert e owns rows [off[e], off[e+1]))
-  const float* perm_gate;  // [A] gate weight of each bucketed row
-  const int* perm_tok;   // [A] token (row of the normed activations) of each bucketed row
   __nv_bfloat16* h_out;  // MODE 1: SwiGLU rows [A][F]
   float* y_out;          // MODE 2: expert outputs [A][d] (the combine applies the gates)
   int d, F;
@@ -130,16 +128,13 @@ cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStre
 struct FusedAssignArgs {
   int32_t* done;         // zero-initialised launch counter (reset by that CTA)
   int32_t* offsets;
-  float* perm_gate;
-  int32_t* perm_tok;
   int32_t* slot;
 };
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
                         int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused, cudaStream_t st);
 // expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
-                        int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,
-                        int* n_launched, cudaStream_t st);
+                        int32_t* offsets, int32_t* cursor, int32_t* slot, int* n_launched, cudaStream_t st);
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st);
 // g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g

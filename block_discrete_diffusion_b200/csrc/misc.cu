@@ -111,14 +111,11 @@ __device__ __forceinline__ void router_topk_row(const float* __restrict__ logits
                                                 float* __restrict__ gate, int32_t* __restrict__ counts,
                                                 int lane);
 __device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t* counts, int n_assign, int top_k,
-                                  int n_exp, int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
-                                  int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot);
+                                  int n_exp, int32_t* __restrict__ offsets, int32_t* __restrict__ slot);
 
 struct FusedAssign {   // the last CTA of the top-k launch also buckets the assignments (done != nullptr)
   int32_t* done;       // launch counter, reset to 0 by that CTA
   int32_t* offsets;
-  float* perm_gate;
-  int32_t* perm_tok;
   int32_t* slot;
 };
 
@@ -139,8 +136,7 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts
     __syncthreads();
     if (s_last) {
       __threadfence();
-      assign_rows_block(sel, gate, counts, n_rows * top_k, top_k, n_exp, fa.offsets, fa.perm_gate, fa.perm_tok,
-                        fa.slot);
+      assign_rows_block(sel, gate, counts, n_rows * top_k, top_k, n_exp, fa.offsets, fa.slot);
       if (threadIdx.x == 0) *fa.done = 0;
     }
   }
@@ -220,8 +216,7 @@ __device__ __forceinline__ void router_topk_row(const float* __restrict__ logits
 // every assignment; counts cleared for the next layer.  Needs blockDim.x >= 256.  Loads bypass L1
 // (sel, gate and counts may come from other CTAs of the same launch).
 __device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t* counts, int n_assign, int top_k,
-                                  int n_exp, int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
-                                  int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+                                  int n_exp, int32_t* __restrict__ offsets, int32_t* __restrict__ slot) {
   __shared__ int s_off[257];
   __shared__ int s_cur[256];
   __shared__ int s_wsum[8];
@@ -256,20 +251,16 @@ __device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t
   for (int e = threadIdx.x; e <= n_exp; e += blockDim.x) offsets[e] = s_off[e];
   for (int a = threadIdx.x; a < n_assign; a += blockDim.x) {
     const int e = __ldcg(sel + a);
-    const int row = s_off[e] + atomicAdd(&s_cur[e], 1);
-    perm_gate[row] = __ldcg(gate + a);
-    perm_tok[row] = a / top_k;
-    slot[a] = row;
+    slot[a] = s_off[e] + atomicAdd(&s_cur[e], 1);
   }
 }
 
 __global__ void assign_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate,
                                    int32_t* __restrict__ counts, int n_assign, int top_k, int n_exp,
-                                   int32_t* __restrict__ offsets, float* __restrict__ perm_gate,
-                                   int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+                                   int32_t* __restrict__ offsets, int32_t* __restrict__ slot) {
   pdl_trigger();
   pdl_wait();
-  assign_rows_block(sel, gate, counts, n_assign, top_k, n_exp, offsets, perm_gate, perm_tok, slot);
+  assign_rows_block(sel, gate, counts, n_assign, top_k, n_exp, offsets, slot);
 }
 
 // Many assignments (several canvases): the offsets come from one small CTA (prefix sum; per-expert
@@ -300,17 +291,13 @@ __global__ void expert_offsets_kernel(int32_t* __restrict__ counts, int n_exp, i
   if (threadIdx.x == n_exp - 1) offsets[n_exp] = base + incl;
 }
 
-__global__ void scatter_rows_kernel(const int32_t* __restrict__ sel, const float* __restrict__ gate, int n_assign,
-                                    int top_k, int32_t* __restrict__ cursor, float* __restrict__ perm_gate,
-                                    int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot) {
+__global__ void scatter_rows_kernel(const int32_t* __restrict__ sel, int n_assign, int32_t* __restrict__ cursor,
+                                    int32_t* __restrict__ slot) {
   pdl_trigger();
   pdl_wait();
   const int a = blockIdx.x * blockDim.x + threadIdx.x;
   if (a >= n_assign) return;
-  const int row = atomicAdd(&cursor[sel[a]], 1);
-  perm_gate[row] = gate[a];
-  perm_tok[row] = a / top_k;
-  slot[a] = row;
+  slot[a] = atomicAdd(&cursor[sel[a]], 1);
 }
 
 // xp[slot[t*k + r]] = xn[t] for every rank r: one warp per token reads the row once.
@@ -447,7 +434,7 @@ cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, in
   const int V = (n_exp + 31) / 32;
   const dim3 grid((n_rows + 7) / 8);
   FusedAssign fa{};
-  if (fused) fa = FusedAssign{fused->done, fused->offsets, fused->perm_gate, fused->perm_tok, fused->slot};
+  if (fused) fa = FusedAssign{fused->done, fused->offsets, fused->slot};
 #define DG_TOPK_CASE(V_) \
   if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts, fa);
   DG_TOPK_CASE(1)
@@ -458,20 +445,18 @@ cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, in
   return cudaErrorInvalidValue;
 }
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
-                        int32_t* offsets, int32_t* cursor, float* perm_gate, int32_t* perm_tok, int32_t* slot,
-                        int* n_launched, cudaStream_t st) {
+                        int32_t* offsets, int32_t* cursor, int32_t* slot, int* n_launched, cudaStream_t st) {
   if (n_exp > 256) return cudaErrorInvalidValue;
   const int n_assign = n_rows * top_k;
   if (n_assign <= 8192) {   // one canvas: a single CTA does both (one launch)
     *n_launched = 1;
     return launch_k(assign_rows_kernel, dim3(1), dim3(1024), 0, st, 1, sel, gate, counts, n_assign, top_k, n_exp,
-                    offsets, perm_gate, perm_tok, slot);
+                    offsets, slot);
   }
   *n_launched = 2;
   cudaError_t e = launch_k(expert_offsets_kernel, dim3(1), dim3(256), 0, st, 1, counts, n_exp, offsets, cursor);
   if (e != cudaSuccess) return e;
-  return launch_k(scatter_rows_kernel, dim3((n_assign + 255) / 256), dim3(256), 0, st, 1, sel, gate, n_assign, top_k,
-                  cursor, perm_gate, perm_tok, slot);
+  return launch_k(scatter_rows_kernel, dim3((n_assign + 255) / 256), dim3(256), 0, st, 1, sel, n_assign, cursor, slot);
 }
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st) {
