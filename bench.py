@@ -213,8 +213,8 @@ def run_steps(dg, seqs, prm, st, k, state):
 
 # DRAM bytes (read + write) of one bf16 gate|up launch at batch 1 (256 rows x top-8, all 128 experts
 # routed), from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of this kernel:
-# 1,026,681,344 + 3,599,616.  Set to None when the kernel changes until it is captured again.
-EXPERT_UP_TRAFFIC_BF16 = 1_026_681_344 + 3_599_616
+# 1,028,473,600 + 3,732,224.  Set to None when the kernel changes until it is captured again.
+EXPERT_UP_TRAFFIC_BF16 = 1_028_473_600 + 3_732_224
 
 
 def expert_up_bytes(cfg):
@@ -411,14 +411,15 @@ def cpu_baseline_sample(cfg, w, sample_rows_layer, head_rows, samp_rows, rounds=
         t0 = time.perf_counter()
         oracle.sample_rows(lg, None, np.arange(samp_rows), 0.8, 7, 0)
         t_samp += time.perf_counter() - t0
+    t_total = t_layer + t_head + t_samp
     t_layer, t_head, t_samp = t_layer / rounds, t_head / rounds, t_samp / rounds
     step_s = (cfg.n_layers * t_layer * CANVAS / sample_rows_layer + t_head * CANVAS / head_rows
               + t_samp * CANVAS / samp_rows)
     return {"value": round(1.0 / step_s, 6), "unit": "steps/s", "cores": _host_threads(), "kind": "oracle",
-            "sample": (f"1 of {cfg.n_layers} layers on {sample_rows_layer} of 256 canvas rows "
+            "sample": (f"{rounds} round(s) of: 1 of {cfg.n_layers} layers on {sample_rows_layer} of 256 canvas rows "
                        f"({t_layer:.2f} s), LM head on {head_rows} rows ({t_head:.2f} s), sampler on {samp_rows} rows "
                        f"({t_samp:.2f} s); extrapolated to one full step ({step_s:.1f} s)"),
-            "seconds_measured": round(t_layer + t_head + t_samp, 2)}
+            "seconds_measured": round(t_total, 2)}
 
 
 def main_reference(args):
