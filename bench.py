@@ -624,7 +624,7 @@ def main_fp8_b32(args):
             "decode": {"blocks": 1, "steps_per_block": steps_per_block, "tokens": sum(n_out),
                        "seconds": round(td, 3)},
             "gpu_launches": launches,
-            "roofline": {"kernel": "attn_partial (canvas attention)", "bound": "tensor",
+            "roofline": {"kernel": "attn_fwd (canvas attention)", "bound": "tensor",
                          "achieved": round(fl / attn_s / 1e12, 1), "peak": tflops, "unit": "TFLOP/s",
                          "frac": round(fl / attn_s / 1e12 / tflops, 4), "traffic": None,
                          "algorithmic_flops_per_launch": fl, "launch_ms": round(attn_s * 1e3, 3),

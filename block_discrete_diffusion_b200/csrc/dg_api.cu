@@ -654,7 +654,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   ap.seq_P = s->seqP;
   ap.opart = s->opart;
   ap.ml = s->ml;
-  LAUNCH(s, DG_K_ATTN, 1, attention_partial(s->q_map, s->k_map, s->v_map, ap, n_local, s->attn, s->err, st));
+  LAUNCH(s, DG_K_ATTN, 1, attention_fwd(s->q_map, s->k_map, s->v_map, ap, n_local, s->attn, s->err, st));
   if (ap.n_splits > 1) LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
 
   EpiParams eo{};

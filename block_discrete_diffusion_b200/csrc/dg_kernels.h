@@ -112,7 +112,7 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
 // 256-token (else 64-token) accumulator chunks
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                         int n_ctas, int wide, int* err, cudaStream_t st);
-cudaError_t attention_partial(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+cudaError_t attention_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st);
 cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st);
 

@@ -3,20 +3,24 @@
 // All products are D = A * B^T with A [M][K] and B [N][K] bf16, K-major (row-major with K
 // contiguous), fp32 accumulation in tensor memory.  Operand tiles are TMA-loaded with 128-byte
 // swizzle into a ring of shared-memory stages; one thread issues the loads, one thread issues the
-// MMAs, and the four warps of the CTA drain TMEM in the epilogue.
+// MMAs, and the epilogue warps drain TMEM.
 //
-//   dense_gemm_kernel<BN, EPI>   one 128 x BN tile per CTA (A = activations, B = weights):
-//     EPI_QKV    the fused Q|K|V projection; rotary embedding (NeoX half split, positions P+j)
-//                applied in registers; Q to the head-major query buffer, K to the cache rows,
-//                V to the transposed value cache (decoder layer "attention block": pre-norm
-//                Gemma-style layer, read from "same architecture as Gemma 4 26B A4B").
+//   dense_gemm_kernel<BN, EPI, Z>  one 128 x BN tile per cluster of Z CTAs (split-K over the
+//                cluster when there are few tiles; A = activations, B = weights), epilogue from
+//                shared memory with coalesced stores:
+//     EPI_QKV    the fused Q|K|V projection; rotary embedding (NeoX half split, positions P+j);
+//                Q to the head-major query buffer, K to the cache rows, V to the transposed value
+//                cache (decoder layer "attention block": pre-norm Gemma-style layer, read from
+//                "same architecture as Gemma 4 26B A4B").
 //     EPI_RESID  x += D (attention output projection + residual).
-//     EPI_F32    out = D (router logits, vocabulary logits).
-//   expert_gemm_kernel<MODE, BN> grouped, swap-AB (weights are the 128-row M side, the few tokens
-//                routed to one expert are the N side):
+//     EPI_F32    out = D (router logits; vocabulary logits of several canvases).
+//   expert_gemm_kernel<MODE, BN, FP8>  persistent, warp-specialised, swap-AB (weights are the
+//                128-row M side, the tokens routed to one expert the N side, BN tokens per chunk):
 //     MODE 1     [gate | up] rows of expert e times its gathered tokens; SwiGLU in the epilogue.
 //     MODE 2     down-projection rows of expert e times its SwiGLU rows (the combine applies the
-//                gate weights; top-k routed MoE of the 26B-A4B model, 3.8B active).
+//                gate weights; top-k routed MoE of the 26B-A4B model, 3.8B active); also the
+//                vocabulary head of one canvas (one "expert" holding all 256 rows).
+//     FP8        weights as e4m3 bytes, expanded to bf16(q * s) in shared memory by converter warps.
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 

@@ -1,5 +1,6 @@
 // misc.cu -- bandwidth/latency kernels around the GEMMs: embedding gather, RMSNorm, the rotary
-// table, the top-k router, expert bucketing with the activation gather, the MoE combine, canvas
+// table, the top-k router (with the expert bucketing in its last CTA for one canvas), the
+// multi-CTA bucketing for many canvases, the activation gather, the MoE combine, canvas
 // initialisation and cache loading.
 #include <math.h>
 

@@ -128,8 +128,8 @@ void dg_model_destroy(dg_model *m);
  *   K[l][seq][h][pos][c]   keys after rotary embedding, head-major
  *   Vt[l][seq][h][c][pos]  values, transposed (positions contiguous) */
 size_t dg_kv_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
-/* With DG_WDTYPE_FP8_BLOCK128 the workspace also holds one layer's matrices in bf16 (each layer is
- * expanded there just before it runs). */
+/* With DG_WDTYPE_FP8_BLOCK128 the workspace also holds one layer's QKV, O and router matrices in
+ * bf16 (expanded there just before the layer runs; the expert GEMMs read the e4m3 bytes directly). */
 size_t dg_workspace_bytes(const dg_model_config *cfg, int n_seq, int max_ctx);
 
 /* Sequence set: n_seq independent sequences (1 = batch 1) with max_ctx positions each.  kv and ws
