@@ -7,6 +7,8 @@
 #pragma once
 #include <stdint.h>
 
+#include "dg_device.cuh"
+
 namespace dg {
 
 enum : uint32_t { RNG_TAG_GUMBEL = 0, RNG_TAG_RERAND = 1, RNG_TAG_INIT = 2 };
@@ -28,9 +30,11 @@ __device__ __forceinline__ uint4 rng_block(uint64_t seed, uint32_t c0, uint32_t 
   return philox4x32_10(make_uint4(c0, pos, step, tag), (uint32_t)seed, (uint32_t)(seed >> 32));
 }
 
-// Open-interval uniform (2*(x>>9)+1) * 2^-24, exact in fp32.
+// Open-interval uniform (2*(x>>9)+1) * 2^-24, exact in fp32: the float 1 + (x>>9) * 2^-23 built
+// from its bits, minus 1 - 2^-24 (the two operands are within a factor of two, so the difference is
+// exact).
 __device__ __forceinline__ float u01_open(uint32_t x) {
-  return __uint2float_rn(((x >> 9) << 1) | 1u) * 5.9604644775390625e-08f;
+  return __fsub_rn(__uint_as_float(0x3F800000u | (x >> 9)), __uint_as_float(0x3F7FFFFFu));
 }
 
 // Standard Gumbel draw -log(-log u) with full-precision logf (u is within 2^-24 of 1 at the top).
@@ -38,14 +42,23 @@ __device__ __forceinline__ float gumbel_from_word(uint32_t x) {
   return -logf(-logf(u01_open(x)));
 }
 
-// Prefilter for the Gumbel-max: -__logf(-__logf(u)) with the hardware logarithm.  Below u = 0.999
-// the documented __logf error bounds (absolute 2^-21.41 on [0.5, 2], 3 ulp elsewhere) keep it within
-// 4e-4 of gumbel_from_word; kGumbelFastSlack covers that, so an element whose prefiltered score is
-// more than the slack below the running best cannot reach it.  From u = 0.999 upwards (the largest
-// draws) the accurate value is always taken.
+// Screen for the Gumbel-max.  -ln(-ln u) = -ln(ln 2) - ln 2 * log2(-log2 u); with both base-2
+// logarithms from lg2.approx (documented error: absolute 2^-22 on [0.5, 2], relative 2^-22
+// elsewhere) and u < 0.999, the inner value is at least 1.44e-3, so it carries a relative error
+// below 1.7e-4 and the screened draw is within 1.7e-4 + 2e-6 of gumbel_from_word.  Scores of
+// tempered logits up to kScreenMaxZ in magnitude add at most three roundings of 6.2e-5 each, so
+// the screened score plus kGumbelFastSlack is above the accurate score and less than two slacks
+// below it.  Draws with u >= kGumbelFastMaxU and larger logits always take the accurate value.
 constexpr float kGumbelFastSlack = 1e-3f;
 constexpr float kGumbelFastMaxU = 0.999f;
-__device__ __forceinline__ float gumbel_fast_from_u(float u) { return -__logf(-__logf(u)); }
+constexpr float kScreenMaxZ = 1024.f;
+constexpr float kNegLnLn2 = 0.36651292058166435f;   // -ln(ln 2)
+
+// Screened score z + g + kGumbelFastSlack of an element with tempered logit l * inv_temp.
+__device__ __forceinline__ float gumbel_screen_score(float l, float inv_temp, float u) {
+  const float L = fast_log2(-fast_log2(u));
+  return __fmaf_rn(-0.6931471805599453f, L, __fmaf_rn(l, inv_temp, kNegLnLn2 + kGumbelFastSlack));
+}
 
 // Largest Gumbel value any word can give, rounded up: -log(-log(1 - 2^-24)) = 16.6355...
 constexpr float kGumbelMax = 16.6400f;

@@ -15,11 +15,15 @@
 //   step budget is reached (fixed_steps > 0: exactly fixed_steps steps); on stop the remaining
 //   positions take y and commit.
 //
-// sampler_partial_kernel: grid (vocab chunk, row).  One pass over the chunk with 16-byte loads;
-// each thread keeps (m, S, A) of the tempered softmax in the exp2 domain with one rescale per 16
-// elements, and the best perturbed score.  A group of four logits whose largest tempered value
-// cannot beat the running best even with the largest possible Gumbel draw skips the Philox call
-// and the two logarithms (exact pruning).
+// sampler_partial_kernel: grid (vocab chunk, row).  One pass over the chunk with 16-byte loads, 16
+// logits per thread per batch; each thread keeps (m, S, A) of the tempered softmax in the exp2
+// domain (packed fp32 pairs, one rescale per batch) and its best perturbed score.  Gumbel-max with a
+// warp-wide lower bound `lim` on the chunk's best score: a group of four logits whose largest
+// tempered value cannot reach it even with the largest possible Gumbel draw skips the Philox call;
+// the other draws get a screened score from hardware logarithms, the warp's largest screened score
+// (minus the screen's error) raises the bound, and only draws whose screened score still reaches it
+// take the accurate logarithms.  Both tests only drop elements whose accurate score is below a
+// score that some element reaches, so the result is the exact Gumbel-max of the accurate scores.
 // sampler_finalize_kernel: one CTA per sequence, one thread per canvas position.
 #include <math.h>
 
@@ -75,61 +79,99 @@ __global__ void __launch_bounds__(kSampThreads)
   const float4* lr = reinterpret_cast<const float4*>(logits + (size_t)row * vocab);
   const float s2 = inv_temp * kLog2e;
 
-  SoftStats st = {-INFINITY, 0.f, 0.f};
-  float best = -INFINITY;
+  // softmax statistics: running max m (exp2 domain) and (S, A) as two packed lanes each
+  float m = -INFINITY;
+  uint64_t S2 = 0, A2 = 0;
+  float best = -INFINITY;   // this thread's best accurate score and its element
   int bidx = 0x7fffffff;
+  float lim = -INFINITY;    // a score some element of the chunk reaches or exceeds (pruning bound)
+  const float kSkip = __int_as_float(0x7fffffff);   // NaN: compares false, marks draws not taken
 
-  for (int gb = g0 + threadIdx.x; gb < g1; gb += 4 * kSampThreads) {
+  // the trip count is the same for every thread (the warp-wide maximum below needs all lanes)
+  for (int base = g0; base < g1; base += 4 * kSampThreads) {
+    const int gb = base + threadIdx.x;
+    // the next batch's 16 KB move into L2 while this one is processed
+    const int nb = base + 4 * kSampThreads;
+    if (threadIdx.x == 0 && nb < g1) l2_prefetch_bulk(lr + nb, (uint32_t)min(4 * kSampThreads, g1 - nb) * 16u);
     float4 q[4];
     bool have[4];
+    float gmax[4], gabs[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int g = gb + u * kSampThreads;
       have[u] = g < g1;
       q[u] = have[u] ? __ldcs(lr + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      gmax[u] = fmaxf(fmaxf(q[u].x, q[u].y), fmaxf(q[u].z, q[u].w));
+      gabs[u] = fmaxf(fmaxf(fabsf(q[u].x), fabsf(q[u].y)), fmaxf(fabsf(q[u].z), fabsf(q[u].w)));
     }
     // batch max in the exp2 domain, then one rescale of (S, A)
-    float bm = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) bm = fmaxf(bm, fmaxf(fmaxf(q[u].x, q[u].y), fmaxf(q[u].z, q[u].w)));
-    bm *= s2;
-    if (bm > st.m) {
-      if (st.m != -INFINITY) {
-        const float f = fast_exp2(st.m - bm);
-        st.A = f * (st.A + st.S * (st.m - bm));
-        st.S *= f;
+    const float bm = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3])) * s2;
+    if (bm > m) {
+      if (m != -INFINITY) {
+        const float f = fast_exp2(m - bm);
+        A2 = fmul_f32x2(ffma_f32x2(S2, pack_f32x2(m - bm, m - bm), A2), pack_f32x2(f, f));
+        S2 = fmul_f32x2(S2, pack_f32x2(f, f));
       }
-      st.m = bm;
+      m = bm;
     }
+    const uint64_t s2p = pack_f32x2(s2, s2), negm = pack_f32x2(-m, -m);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       if (!have[u]) continue;
-      const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-      float zmax = -INFINITY;
+      const uint64_t t01 = ffma_f32x2(pack_f32x2(q[u].x, q[u].y), s2p, negm);
+      const uint64_t t23 = ffma_f32x2(pack_f32x2(q[u].z, q[u].w), s2p, negm);
+      const uint64_t e01 = pack_f32x2(fast_exp2(lo_f32(t01)), fast_exp2(hi_f32(t01)));
+      const uint64_t e23 = pack_f32x2(fast_exp2(lo_f32(t23)), fast_exp2(hi_f32(t23)));
+      S2 = fadd_f32x2(S2, fadd_f32x2(e01, e23));
+      A2 = ffma_f32x2(e23, t23, ffma_f32x2(e01, t01, A2));
+    }
+
+    // Gumbel draws of the groups that can reach the bound, screened with hardware logarithms
+    uint32_t wd[4][4];
+    float fs[4][4];
+    float fmax_ = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float t2 = zz[i] * s2 - st.m;
-        const float e = fast_exp2(t2);
-        st.S += e;
-        st.A += e * t2;
-        zmax = fmaxf(zmax, zz[i]);
-      }
-      // Gumbel-max over the 4 elements of this group, unless none can beat the running best
-      if (zmax * inv_temp + kGumbelMax >= best) {
-        const int g = gb + u * kSampThreads;
-        const uint4 w = philox4x32_10(make_uint4((uint32_t)g, pos, (uint32_t)step, RNG_TAG_GUMBEL), k0, k1);
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) fs[u][i] = kSkip;
+      if (have[u] && __fmaf_rn(gmax[u], inv_temp, kGumbelMax) >= lim) {
+        const uint4 w = philox4x32_10(make_uint4((uint32_t)(gb + u * kSampThreads), pos, (uint32_t)step,
+                                                 RNG_TAG_GUMBEL), k0, k1);
+        const bool screen = gabs[u] * inv_temp <= kScreenMaxZ;
+        const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float sc = zz[i] * inv_temp + gumbel_from_word(ww[i]);
+          wd[u][i] = ww[i];
+          const float uu = u01_open(ww[i]);
+          const float f = gumbel_screen_score(zz[i], inv_temp, uu);
+          const bool exact_only = !screen || uu >= kGumbelFastMaxU;
+          fs[u][i] = exact_only ? INFINITY : f;
+          fmax_ = fmaxf(fmax_, exact_only ? -INFINITY : f);
+        }
+      }
+    }
+    // every screened score minus two slacks is below that element's accurate score
+    lim = fmaxf(lim, warp_max(fmax_) - 2.f * kGumbelFastSlack);
+    // accurate scores only where the screened score reaches the bound (elements in increasing
+    // index order, so the strict comparison keeps the lowest index among equal scores)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (fs[u][i] >= lim) {
+          const float sc = __fmaf_rn(zz[i], inv_temp, gumbel_from_word(wd[u][i]));
           if (sc > best) {
             best = sc;
-            bidx = 4 * g + i;
+            bidx = 4 * (gb + u * kSampThreads) + i;
           }
         }
       }
     }
+    lim = fmaxf(lim, best);
   }
+  SoftStats st = {m, lo_f32(S2) + hi_f32(S2), lo_f32(A2) + hi_f32(A2)};
 
   // block reduction: warp shuffles, then the 8 warp results through shared memory
 #pragma unroll

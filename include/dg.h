@@ -200,7 +200,7 @@ dg_status dg_decode(dg_seqs *s, const dg_sampler_params *p, int max_blocks, int3
 dg_status dg_layer_forward(dg_seqs *s, int layer, int n_rows, int causal, float *d_x, float *d_x_mid,
                            float *d_router_logits);
 
-/* Sampler alone over caller logits (fp32 [n_seq*canvas_len][vocab]): the entropy / Gumbel-argmax /
+/* Sampler alone over caller logits (finite fp32 [n_seq*canvas_len][vocab]): the entropy / Gumbel-argmax /
  * commit / re-randomise / stop rule of one step.  d_seq_P (nullable, int32 [n_seq]): absolute
  * position of each sequence's first canvas row (0 if NULL).  d_ids, d_commit in/out as in
  * dg_canvas_step.  ws: device scratch of dg_sample_workspace_bytes(n_seq*canvas_len, vocab). */
