@@ -39,16 +39,18 @@ def _oracle_sample(logits_cpu, commit, ids, pos, prm, step, vocab):
 # sampler alone
 # ------------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("vocab,spike,step,rows_checked", [
-    (4096, 12.0, 0, None),
-    (4096, 40.0, 47, None),
-    (262144, 12.0, 12, None),          # the full-size sampler workload, every row
-    (262144, 40.0, 0, 48),             # spike +40 rows commit; sampled rows
-    (262144, 12.0, 47, 48),
+@pytest.mark.parametrize("vocab,spike,step,rows_checked,std", [
+    (4096, 12.0, 0, None, 3.0),
+    (4096, 40.0, 47, None, 3.0),
+    (5120, 12.0, 5, None, 3.0),        # 1280 float4 groups: a full batch of 1024 and a ragged one
+    (4096, 12.0, 30, None, 1000.0),    # tempered logits beyond the screen's range: accurate draws only
+    (262144, 12.0, 12, None, 3.0),     # the full-size sampler workload, every row
+    (262144, 40.0, 0, 48, 3.0),        # spike +40 rows commit; sampled rows
+    (262144, 12.0, 47, 48, 3.0),
 ])
-def test_sampler_matches_oracle(dg, vocab, spike, step, rows_checked):
+def test_sampler_matches_oracle(dg, vocab, spike, step, rows_checked, std):
     n_seq, canvas = 1, 256
-    logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, spike=spike)
+    logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, std=std, spike=spike)
     prm_o = oracle.SamplerParams(vocab, seed=7)
     prm = dg.sampler_params(vocab, seed=7)
     rng = np.random.default_rng(step)
