@@ -486,3 +486,44 @@ def test_capacity_and_argument_errors(dg):
     dg.dg_canvas_step(seqs2, prm, ids_bad, commit, H, stop)
     assert dg.dg_device_error(seqs2) != 0
     assert dg.dg_device_error(seqs2) == 0         # the record is cleared by reading it
+
+
+def test_block_replays_bit_identically_from_a_cuda_graph(dg):
+    """The library issues only stream-ordered work on the sequence set's stream (no host reads,
+    allocations or synchronisation inside a step), so a whole block -- canvas init and its fixed
+    steps -- can be captured into a CUDA graph (the programmatic dependent launches become
+    programmatic edges) and replayed with the same results as the direct calls."""
+    cfg, w, model, M = _tiny_model_pair(dg, 50.0, seed=4, top_k=2)
+    s = torch.cuda.Stream()
+    seqs = dg.dg_seqs_create(model, 1, 512, stream=s)
+    prm = dg.sampler_params(cfg.vocab, seed=11, fixed_steps=6)
+    prompt = synthetic.make_ids(128, cfg.vocab, seed=5, device="cuda")
+    ids = torch.empty(256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(256, dtype=torch.uint8, device="cuda")
+    H = torch.empty(256, device="cuda")
+    stop = torch.empty(1, dtype=torch.int32, device="cuda")
+
+    def block():
+        dg.dg_canvas_init(seqs, prm, ids, commit)
+        for _ in range(6):
+            dg.dg_canvas_step(seqs, prm, ids, commit, H, stop)
+
+    with torch.cuda.stream(s):
+        dg.dg_prefill(seqs, prompt, [128])
+        block()
+    torch.cuda.synchronize()
+    direct = (ids.clone(), commit.clone(), H.clone(), stop.clone())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        block()
+    for t in (ids, commit, H, stop):
+        t.zero_()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        with torch.cuda.stream(s):
+            g.replay()
+        torch.cuda.synchronize()
+        for a, b in zip((ids, commit, H, stop), direct):
+            assert torch.equal(a, b)
+    assert dg.dg_device_error(seqs) == 0
+    del g
