@@ -456,7 +456,7 @@ static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, con
 // n_splits == 1: the attention output is written directly to `out`; otherwise the partials are
 // left for attention_merge.
 cudaError_t attention_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
+                          const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
   if (p.dh == 128) return launch_attn<128>(tq, tk, tv, p, n_seq, out, err, st);
   if (p.dh == 64) return launch_attn<64>(tq, tk, tv, p, n_seq, out, err, st);
   return cudaErrorInvalidValue;
