@@ -127,7 +127,6 @@ __global__ void __launch_bounds__(kSampThreads)
     }
 
     // Gumbel draws of the groups that can reach the bound, screened with hardware logarithms
-    uint32_t wd[4][4];
     float fs[4][4];
     float fmax_ = -INFINITY;
 #pragma unroll
@@ -142,7 +141,6 @@ __global__ void __launch_bounds__(kSampThreads)
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          wd[u][i] = ww[i];
           const float uu = u01_open(ww[i]);
           const float f = gumbel_screen_score(zz[i], inv_temp, uu);
           const bool exact_only = !screen || uu >= kGumbelFastMaxU;
@@ -154,17 +152,23 @@ __global__ void __launch_bounds__(kSampThreads)
     // every screened score minus two slacks is below that element's accurate score
     lim = fmaxf(lim, warp_max(fmax_) - 2.f * kGumbelFastSlack);
     // accurate scores only where the screened score reaches the bound (elements in increasing
-    // index order, so the strict comparison keeps the lowest index among equal scores)
+    // index order, so the strict comparison keeps the lowest index among equal scores); the few
+    // groups holding such a draw generate their Philox block again rather than keep 16 words live
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+      if (fs[u][0] >= lim || fs[u][1] >= lim || fs[u][2] >= lim || fs[u][3] >= lim) {
+        const int g = gb + u * kSampThreads;
+        const uint4 w = philox4x32_10(make_uint4((uint32_t)g, pos, (uint32_t)step, RNG_TAG_GUMBEL), k0, k1);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        const float zz[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (fs[u][i] >= lim) {
-          const float sc = __fmaf_rn(zz[i], inv_temp, gumbel_from_word(wd[u][i]));
-          if (sc > best) {
-            best = sc;
-            bidx = 4 * (gb + u * kSampThreads) + i;
+        for (int i = 0; i < 4; ++i) {
+          if (fs[u][i] >= lim) {
+            const float sc = __fmaf_rn(zz[i], inv_temp, gumbel_from_word(ww[i]));
+            if (sc > best) {
+              best = sc;
+              bidx = 4 * g + i;
+            }
           }
         }
       }
