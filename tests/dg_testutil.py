@@ -2,7 +2,7 @@
 cache layout of include/dg.h, and the judging rules for comparing the CUDA path with the oracle.
 
 Judging rules.
-  Spec tolerances (used as stated wherever the compared quantities come from identical inputs, and
+  Base tolerances (used as stated wherever the compared quantities come from identical inputs, and
   for end-to-end steps whose logits are small):
     - hidden states: max|gpu - oracle| / max|oracle| <= 2e-2 per (layer, tensor);
     - entropies: |gpu - oracle| <= 1e-3 absolute;
@@ -18,9 +18,9 @@ Judging rules.
   products; with 2L+1 sequential roundings the rms relative error of z is about
   sqrt(2L+1) * 2^-9 / sqrt(3).  Judging at 4 sigma gives c_z = 4 sqrt(2L+1) 2^-9 / sqrt(3)
   (1.0e-2 for L = 2; FP8 weights add 5L roundings, see c_z).  Where c_z * std(z_row) exceeds
-  the spec margin, ids are judged where the oracle margin exceeds c_z * std(z_row), and
+  the base margin, ids are judged where the oracle margin exceeds c_z * std(z_row), and
   entropies within c_z * (std(z) std_p(z) + Var_p(z)) (the first-order change of the entropy under a perturbation of that size: random part
-  std(dz) std_p(z), scale part Var_p(z) c_z).  These derived bounds reduce to the spec's at small
+  std(dz) std_p(z), scale part Var_p(z) c_z).  These derived bounds reduce to the base ones at small
   logits and are only used by the tests that say so.
 """
 import math
@@ -87,7 +87,7 @@ def c_z(n_layers, fp8=False):
 
 def derived_tolerances(logits, T, n_layers, fp8=False):
     """Per-row (margin, entropy) judging tolerances for end-to-end steps at large logits (see the
-    module docstring); never below the spec's 1e-2 / 1e-3."""
+    module docstring); never below the base 1e-2 / 1e-3."""
     z = np.asarray(logits, np.float64) / T
     cz = c_z(n_layers, fp8)
     std_z = z.std(axis=1)
@@ -110,7 +110,7 @@ def prm_vocab(orc):
 def judge_step(gpu, orc, prm, commit_before, exclude=None, margin_tol=None, h_tol=None):
     """Compare one sampler step.  gpu/orc: dicts with ids, commit, H (numpy), stop; orc also y, margin,
     rr, mean_H.  exclude: rows not judged (router near-ties).  margin_tol / h_tol: per-row tolerances
-    (default: the spec's).  Returns (failures, number of ids judged)."""
+    (default: the base tolerances).  Returns (failures, number of ids judged)."""
     n = len(orc["H"])
     exclude = np.zeros(n, bool) if exclude is None else np.asarray(exclude, bool)
     margin_tol = np.full(n, MARGIN) if margin_tol is None else np.asarray(margin_tol)

@@ -37,7 +37,7 @@ def test_batched_sequences_match_their_oracles(dg, wdtype, head_scale):
     """Three sequences (prompts of 128, 300 and 0 tokens) prefilled, initialised and stepped in one
     batch; each sequence's hidden states, logits and sampler decisions match its own oracle run
     (resynchronised every step), then one block commit per sequence.  Head x50: rows commit, ids and
-    entropies judged with the derived large-logit tolerances; head x1: the spec's tolerances."""
+    entropies judged with the derived large-logit tolerances; head x1: the base tolerances."""
     cfg, w = _tiny(wdtype, head_scale)
     tol = HIDDEN_TOL if wdtype == 0 else HIDDEN_TOL_FP8
     model = dg.dg_model_create(cfg, to_device(w))

@@ -4,7 +4,7 @@ random init) against the oracle, layer by layer.
 Each layer runs on the GPU (dg_layer_forward, canvas mode, behind a 2048-position synthetic prefix)
 from the oracle's input to that layer, so a router near-tie in one layer does not carry into the
 next; every layer's attention-block output, router logits, layer output and canvas K/V are judged
-with the spec tolerance, tokens with a router near-tie in that layer excluded.  Marked gpu.
+with the base tolerance, tokens with a router near-tie in that layer excluded.  Marked gpu.
 """
 import dataclasses
 

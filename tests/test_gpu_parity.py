@@ -238,7 +238,7 @@ def _cache_rows(seqs, cfg, max_ctx, l, a, b):
 
 
 # top_k = E (8 of 8 experts): the step has no routing decision, so every step and token is judged
-# with the spec tolerances (small head) or the derived large-logit tolerances (head x50, where rows
+# with the base tolerances (small head) or the derived large-logit tolerances (head x50, where rows
 # commit).  top_k = 2: tokens with router near-ties are excluded, and steps with a near-tie before
 # the last layer are not judged (see the loop).
 @pytest.mark.parametrize("top_k,head_scale,prompt_len,n_steps", [
@@ -303,7 +303,7 @@ def test_canvas_steps_match_oracle(dg, top_k, head_scale, prompt_len, n_steps):
             g = {"ids": ids.cpu().numpy(), "commit": commit.cpu().numpy(), "H": H.cpu().numpy(),
                  "stop": int(stop.item())}
             if head_scale == 1.0:
-                mt, ht = None, None                                   # the spec's tolerances
+                mt, ht = None, None                                   # the base tolerances
             else:
                 mt, ht = derived_tolerances(r["logits"], r["T"], cfg.n_layers)
             fails, judged = judge_step(g, r, prm_o, ocommit, exclude=tie, margin_tol=mt, h_tol=ht)
