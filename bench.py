@@ -216,6 +216,11 @@ def run_steps(dg, seqs, prm, st, k, state):
 # 1,028,473,600 + 3,732,224.  Set to None when the kernel changes until it is captured again.
 EXPERT_UP_TRAFFIC_BF16 = 1_028_473_600 + 3_732_224
 
+# DRAM bytes (read + write) of one sampler_partial_kernel launch on the 256 x 262144 sampler workload,
+# from an ncu capture of this kernel: 268,503,552 + 3,422,720.  None when the kernel changes until it is
+# captured again.
+SAMPLER_PARTIAL_TRAFFIC = 268_503_552 + 3_422_720
+
 
 def expert_up_bytes(cfg):
     """Algorithmic bytes of one grouped gate|up launch at batch 1: every expert's [2F x d] weights
@@ -530,8 +535,11 @@ def main_aux(args):
         line = {"metric": "sampler steps/s (256 x 262144 fp32 logits)", "value": round(1 / t, 2), "unit": "steps/s",
                 "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
                 "config": {"workload": "sampler: logits N(0, 3^2), 10% of rows +12 spike, step 12 of 48, seed 7"},
-                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                             "frac": round(gbs / hbm, 4), "note": "includes the commit-mask reset (256 B)"}}
+                "roofline": {"kernel": "sampler_partial + sampler_finalize (one dg_sample call)", "bound": "hbm",
+                             "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                             "traffic": SAMPLER_PARTIAL_TRAFFIC,
+                             "note": "includes the commit-mask reset (256 B); the kernel is instruction-bound "
+                                     "(one Philox word, an exp2 and two hardware logarithms per logit)"}}
     print(json.dumps(line), flush=True)
 
 
