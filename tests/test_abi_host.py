@@ -98,3 +98,34 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt and "dg_oracle" not in txt, f
+
+
+@pytest.mark.parametrize("case,expected", [
+    ("null_logits", "DG_ERR_INVALID_ARG"), ("vocab_not_multiple_of_1024", "DG_ERR_INVALID_ARG"),
+    ("canvas_128", "DG_ERR_UNSUPPORTED"), ("negative_step", "DG_ERR_INVALID_ARG"),
+    ("workspace_too_small", "DG_ERR_CAPACITY"), ("no_rows", "DG_ERR_INVALID_ARG"),
+])
+def test_sampler_argument_checks_happen_on_the_host(dg, case, expected):
+    """dg_sample rejects bad arguments before it touches the device (fake, never dereferenced
+    pointers stand in for device buffers)."""
+    vocab, n_seq, step = 4096, 1, 0
+    prm = dg.sampler_params(vocab, seed=1)
+    fake = ctypes.c_void_p(4096)
+    logits = fake
+    ws_bytes = dg.dg_sample_workspace_bytes(256, vocab)
+    if case == "null_logits":
+        logits = None
+    elif case == "vocab_not_multiple_of_1024":
+        vocab = 4000
+    elif case == "canvas_128":
+        prm.canvas_len = 128
+    elif case == "negative_step":
+        step = -1
+    elif case == "workspace_too_small":
+        ws_bytes -= 1
+    elif case == "no_rows":
+        n_seq = 0
+    st = dg.lib().dg_sample(logits, n_seq, vocab, ctypes.byref(prm), step, None, fake, fake, fake, fake, fake,
+                            ws_bytes, None)
+    assert st == getattr(dg, expected)
+    assert dg.lib().dg_last_error().decode()
