@@ -129,3 +129,32 @@ def test_sampler_argument_checks_happen_on_the_host(dg, case, expected):
                             ws_bytes, None)
     assert st == getattr(dg, expected)
     assert dg.lib().dg_last_error().decode()
+
+
+def test_binding_structs_match_the_header_layout(dg, tmp_path):
+    """Every ctypes structure of the binding has the size and field offsets the C compiler gives the
+    structure of include/dg.h (a small C program built with the host compiler prints them)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = [dg.dg_model_config, dg.dg_layer_weights, dg.dg_weights, dg.dg_sampler_params]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "dg.h"', "int main(void) {"]
+    for S in structs:
+        lines.append(f'  printf("{S.__name__} size %zu\\n", sizeof({S.__name__}));')
+        for name, _ in S._fields_:
+            lines.append(f'  printf("{S.__name__} {name} %zu\\n", offsetof({S.__name__}, {name}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for S in structs:
+        assert got[(S.__name__, "size")] == ctypes.sizeof(S), S.__name__
+        for name, _ in S._fields_:
+            assert got[(S.__name__, name)] == getattr(S, name).offset, (S.__name__, name)
