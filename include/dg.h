@@ -24,6 +24,8 @@
  *    device.  A kernel that sees a bad index or whose pipeline wait runs out records a code that
  *    dg_device_error returns (DG_ERR_DEVICE).  dg_last_error() gives a message for the last non-OK
  *    status of the calling thread.
+ *  - Devices: one process drives one GPU (launched one process per GPU).  The kernels' shared-memory
+ *    attributes are set once per process, on the device current at the first launch.
  *  - Determinism: outputs depend only on (weights, inputs, params, seed).
  *  - Layouts are row-major; bf16 is IEEE bfloat16, fp32 is IEEE binary32.
  */
