@@ -48,13 +48,18 @@ def lib():
         L.orc_attention.argtypes = [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p]
         L.orc_router_topk.argtypes = [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
+        L.orc_router_topk_flip.argtypes = [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_moe.argtypes = [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_layer_forward.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p,
                                         c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
         L.orc_layer_forward.restype = c_int
+        L.orc_layer_forward_flip.argtypes = L.orc_layer_forward.argtypes + [c_void_p]
+        L.orc_layer_forward_flip.restype = c_int
         L.orc_forward.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
                                   c_int, c_int, c_void_p, c_void_p, c_void_p]
         L.orc_forward.restype = c_int
+        L.orc_forward_flip.argtypes = L.orc_forward.argtypes + [c_void_p]
+        L.orc_forward_flip.restype = c_int
         L.orc_head.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p]
         L.orc_embed.argtypes = [c_void_p, c_void_p, c_int, c_void_p, c_void_p]
         for name in ("orc_sample_rows_f32", "orc_sample_rows_f64"):
@@ -142,12 +147,18 @@ def attention(q, k, v, mask) -> np.ndarray:
     return out
 
 
-def router_topk(logits, k):
+def router_topk(logits, k, flip=None):
+    """Top-k selection and gates; flip (optional bool [n]): those tokens take their (k+1)-th expert in
+    place of their k-th (the other choice at a near-tie)."""
     logits = _f64(logits)
     n, E = logits.shape
     sel = np.empty((n, k), dtype=np.int32)
     gate = np.empty((n, k))
-    lib().orc_router_topk(n, E, k, _p(logits), _p(sel), _p(gate))
+    if flip is None:
+        lib().orc_router_topk(n, E, k, _p(logits), _p(sel), _p(gate))
+    else:
+        fl = np.ascontiguousarray(np.asarray(flip, dtype=np.uint8))
+        lib().orc_router_topk_flip(n, E, k, _p(logits), _p(fl), _p(sel), _p(gate))
     return sel, gate
 
 
@@ -238,10 +249,12 @@ class Model:
                       self._mat(L["w_down"], c.n_exp * c.d_model, c.d_ff))
 
 
-def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=None, causal=False, want_mid=False):
+def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=None, causal=False, want_mid=False,
+                  flip=None):
     """One decoder layer on rows x [n, d] (fp64, updated copy returned) at positions pos, keys =
     cache[0:P] + the rows.  Returns (x_out, k_new, v_new, router_logits) and, with want_mid, x after
-    the attention residual as a fifth item."""
+    the attention residual as a fifth item.  flip (optional bool [n]): tokens routed to their
+    (k+1)-th expert in place of their k-th."""
     c = model.cfg
     x = _f64(x).copy()
     n = x.shape[0]
@@ -252,9 +265,10 @@ def layer_forward(model: Model, layer: int, x, pos, P=0, k_cache=None, v_cache=N
     vn = np.empty((n, c.n_kv, c.d_head))
     rl = np.empty((n, c.n_exp))
     mid = np.empty_like(x) if want_mid else None
-    rc = lib().orc_layer_forward(ctypes.byref(model.c_cfg), ctypes.byref(model.c_layers[layer]), n, _p(pos),
-                                 _p(x), P, _p(kc), _p(vc), int(causal), _p(kn), _p(vn), _p(rl),
-                                 None if mid is None else _p(mid))
+    fl = None if flip is None else np.ascontiguousarray(np.asarray(flip, dtype=np.uint8))
+    rc = lib().orc_layer_forward_flip(ctypes.byref(model.c_cfg), ctypes.byref(model.c_layers[layer]), n, _p(pos),
+                                      _p(x), P, _p(kc), _p(vc), int(causal), _p(kn), _p(vn), _p(rl),
+                                      None if mid is None else _p(mid), None if fl is None else _p(fl))
     assert rc == 0
     return (x, kn, vn, rl, mid) if want_mid else (x, kn, vn, rl)
 
@@ -271,9 +285,10 @@ def moe(model: Model, layer: int, h, sel, gate):
 
 
 def forward(model: Model, ids, pos, P, k_caches, v_caches, causal=False, write_cache=False,
-            want_hidden=False, want_router=False, want_logits=True):
+            want_hidden=False, want_router=False, want_logits=True, flip=None):
     """Full stack on rows ids at positions pos; caches are per-layer fp64 arrays [ctx, Hkv, dh]
-    (rows [0:P) read; with write_cache rows [P:P+n) receive the rows' K/V)."""
+    (rows [0:P) read; with write_cache rows [P:P+n) receive the rows' K/V).  flip (optional bool
+    [L, n]): per layer, tokens routed to their (k+1)-th expert in place of their k-th."""
     c = model.cfg
     ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
     pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int32))
@@ -285,10 +300,11 @@ def forward(model: Model, ids, pos, P, k_caches, v_caches, causal=False, write_c
     hid = np.empty((c.n_layers + 1, n, c.d_model)) if want_hidden else None
     rtr = np.empty((c.n_layers, n, c.n_exp)) if want_router else None
     logits = np.empty((n, c.vocab)) if want_logits else None
-    rc = lib().orc_forward(ctypes.byref(model.c_cfg), ctypes.byref(model.c_model), n, _p(ids), _p(pos), P,
-                           kp, vp, int(causal), int(write_cache),
-                           None if hid is None else _p(hid), None if rtr is None else _p(rtr),
-                           None if logits is None else _p(logits))
+    fl = None if flip is None else np.ascontiguousarray(np.asarray(flip, dtype=np.uint8).reshape(c.n_layers, n))
+    rc = lib().orc_forward_flip(ctypes.byref(model.c_cfg), ctypes.byref(model.c_model), n, _p(ids), _p(pos), P,
+                                kp, vp, int(causal), int(write_cache),
+                                None if hid is None else _p(hid), None if rtr is None else _p(rtr),
+                                None if logits is None else _p(logits), None if fl is None else _p(fl))
     assert rc == 0
     return {"hidden": hid, "router": rtr, "logits": logits}
 
@@ -411,11 +427,15 @@ class Sequence:
         self.step = 0
         return canvas_init(prm.canvas_len, self.P, prm.seed, self.model.cfg.vocab)
 
-    def canvas_step(self, prm: SamplerParams, ids, commit, want_hidden=False, want_router=False):
+    def canvas_step(self, prm: SamplerParams, ids, commit, want_hidden=False, want_router=False, flip=None,
+                    advance=True):
+        """One denoising step.  flip (optional bool [L, n]): the routing alternative for the flagged
+        (layer, token) pairs (see forward).  advance=False leaves the step counter as it is (a second
+        evaluation of the same step)."""
         n = len(ids)
         pos = np.arange(self.P, self.P + n)
         fw = forward(self.model, ids, pos, self.P, self.k, self.v, causal=False, write_cache=False,
-                     want_hidden=want_hidden, want_router=want_router, want_logits=True)
+                     want_hidden=want_hidden, want_router=want_router, want_logits=True, flip=flip)
         T = temperature(self.step, prm.max_steps, prm.t_start, prm.t_end)
         smp = sample_rows(fw["logits"], commit, pos, T, prm.seed, self.step)
         rule = step_rule(commit, ids, smp["H"], smp["y"], smp["rr"], self.step, prm.entropy_bound,
@@ -425,7 +445,8 @@ class Sequence:
         out.update(rule)
         out.update({"T": T, "step": self.step, "logits": fw["logits"], "hidden": fw["hidden"],
                     "router": fw["router"]})
-        self.step += 1
+        if advance:
+            self.step += 1
         return out
 
     def block_commit(self, ids, want_router=False):

@@ -264,26 +264,43 @@ void orc_attention(int n_rows, int n_keys, int n_q, int n_kv, int dh, const doub
 }
 
 /* Router [reading]: logits = h . W_r^T; the top_k experts by logit (ties -> lower expert id);
- * gates = softmax over the selected logits only.  sel/gate are [n][top_k] in rank order. */
-void orc_router_topk(int n, int n_exp, int top_k, const double *logits, int32_t *sel, double *gate)
+ * gates = softmax over the selected logits only.  sel/gate are [n][top_k] in rank order.
+ * flip (nullable, [n]): a token with flip[t] != 0 takes its (top_k+1)-th expert in place of its
+ * top_k-th one (the other choice of a token whose k-th and (k+1)-th logits are a near-tie); the
+ * gates are the softmax over the logits it then selects.  Used by the tests to measure how much
+ * such a choice moves the other tokens; flip = NULL is the router of the model. */
+void orc_router_topk_flip(int n, int n_exp, int top_k, const double *logits, const uint8_t *flip, int32_t *sel,
+                          double *gate)
 {
+    int32_t ranked[257];
     for (int t = 0; t < n; ++t) {
         const double *l = logits + (size_t)t * n_exp;
-        int32_t *s = sel + (size_t)t * top_k;
-        for (int r = 0; r < top_k; ++r) {
+        const int alt = flip && flip[t] && top_k < n_exp;
+        const int n_rank = top_k + alt;
+        for (int r = 0; r < n_rank; ++r) {
             int best = -1;
             for (int e = 0; e < n_exp; ++e) {
                 int taken = 0;
-                for (int q = 0; q < r; ++q) taken |= (s[q] == e);
+                for (int q = 0; q < r; ++q) taken |= (ranked[q] == e);
                 if (taken) continue;
                 if (best < 0 || l[e] > l[best]) best = e;   /* strict '>' keeps the lower id on ties */
             }
-            s[r] = best;
+            ranked[r] = best;
         }
-        double mx = l[s[0]], den = 0.0;
+        if (alt) ranked[top_k - 1] = ranked[top_k];
+        int32_t *s = sel + (size_t)t * top_k;
+        for (int r = 0; r < top_k; ++r) s[r] = ranked[r];
+        double mx = l[s[0]];
+        for (int r = 1; r < top_k; ++r) if (l[s[r]] > mx) mx = l[s[r]];
+        double den = 0.0;
         for (int r = 0; r < top_k; ++r) den += exp(l[s[r]] - mx);
         for (int r = 0; r < top_k; ++r) gate[(size_t)t * top_k + r] = exp(l[s[r]] - mx) / den;
     }
+}
+
+void orc_router_topk(int n, int n_exp, int top_k, const double *logits, int32_t *sel, double *gate)
+{
+    orc_router_topk_flip(n, n_exp, top_k, logits, NULL, sel, gate);
 }
 
 static double silu(double a) { return a / (1.0 + exp(-a)); }
@@ -364,10 +381,11 @@ void orc_moe(const orc_config *c, const orc_layer_weights *w, int n, int k, cons
  * guide "Dual attention of prefill and denoising", report "Composition", training recipe);
  * causal = 1: row i sees cache and rows j <= i (prompt prefill).
  * k_new/v_new receive the rows' post-RoPE K and V ([n][n_kv][dh]); router_logits is [n][E];
- * x_mid (nullable) receives x after the attention residual. */
-int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, const int32_t *pos,
-                      double *x, int P, const double *k_cache, const double *v_cache, int causal,
-                      double *k_new, double *v_new, double *router_logits, double *x_mid)
+ * x_mid (nullable) receives x after the attention residual.  flip (nullable, [n]): the routing
+ * alternative of orc_router_topk_flip for the flagged tokens (test use; NULL is the model). */
+int orc_layer_forward_flip(const orc_config *c, const orc_layer_weights *w, int n, const int32_t *pos,
+                           double *x, int P, const double *k_cache, const double *v_cache, int causal,
+                           double *k_new, double *v_new, double *router_logits, double *x_mid, const uint8_t *flip)
 {
     int d = c->d_model, nq = c->n_q, nkv = c->n_kv, dh = c->d_head, E = c->n_exp;
     int nqkv = (nq + 2 * nkv) * dh, nkeys = P + n;
@@ -413,7 +431,7 @@ int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, co
     /* MoE block */
     orc_rmsnorm(n, d, x, w->ffn_norm, c->rms_eps, h);
     mat_apply(&w->w_router, n, h, rl, E);
-    orc_router_topk(n, E, c->top_k, rl, sel, gate);
+    orc_router_topk_flip(n, E, c->top_k, rl, flip, sel, gate);
     moe_apply(c, w, n, c->top_k, h, sel, gate, o);
     for (size_t i = 0; i < (size_t)n * d; ++i) x[i] += o[i];
     if (router_logits) memcpy(router_logits, rl, sizeof(double) * (size_t)n * E);
@@ -421,6 +439,14 @@ int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, co
     free(h); free(qkv); free(q); free(keys); free(vals); free(mask); free(att); free(o);
     free(rl); free(sel); free(gate);
     return 0;
+}
+
+int orc_layer_forward(const orc_config *c, const orc_layer_weights *w, int n, const int32_t *pos,
+                      double *x, int P, const double *k_cache, const double *v_cache, int causal,
+                      double *k_new, double *v_new, double *router_logits, double *x_mid)
+{
+    return orc_layer_forward_flip(c, w, n, pos, x, P, k_cache, v_cache, causal, k_new, v_new, router_logits, x_mid,
+                                  NULL);
 }
 
 /* Embedding lookup: rows of the bf16 embedding table (no scaling; reading). */
@@ -445,10 +471,11 @@ void orc_head(const orc_config *c, const orc_model_weights *m, int n, const doub
 /* Full forward of n rows at positions pos, against caches [layer][P][n_kv][dh].
  * write_cache: also store each layer's post-RoPE K and V of the rows into cache rows [P, P+n).
  * hidden_dbg (nullable): [L+1][n][d] residual stream before layer 0 .. after the last layer.
- * logits (nullable): [n][V]. */
-int orc_forward(const orc_config *c, const orc_model_weights *m, int n, const int32_t *ids,
-                const int32_t *pos, int P, double *const *k_cache, double *const *v_cache, int causal,
-                int write_cache, double *hidden_dbg, double *router_dbg, double *logits)
+ * logits (nullable): [n][V].  flip (nullable, [L][n]): per layer, the tokens that take the routing
+ * alternative of orc_router_topk_flip (test use; NULL is the model). */
+int orc_forward_flip(const orc_config *c, const orc_model_weights *m, int n, const int32_t *ids,
+                     const int32_t *pos, int P, double *const *k_cache, double *const *v_cache, int causal,
+                     int write_cache, double *hidden_dbg, double *router_dbg, double *logits, const uint8_t *flip)
 {
     int d = c->d_model, kvw = c->n_kv * c->d_head;
     double *x = (double *)malloc(sizeof(double) * (size_t)n * d);
@@ -459,7 +486,8 @@ int orc_forward(const orc_config *c, const orc_model_weights *m, int n, const in
     if (hidden_dbg) memcpy(hidden_dbg, x, sizeof(double) * (size_t)n * d);
     for (int l = 0; l < c->n_layers; ++l) {
         double *rl = router_dbg ? router_dbg + (size_t)l * n * c->n_exp : NULL;
-        if (orc_layer_forward(c, &m->layers[l], n, pos, x, P, k_cache[l], v_cache[l], causal, kn, vn, rl, NULL))
+        if (orc_layer_forward_flip(c, &m->layers[l], n, pos, x, P, k_cache[l], v_cache[l], causal, kn, vn, rl, NULL,
+                                   flip ? flip + (size_t)l * n : NULL))
             return -1;
         if (write_cache) {
             memcpy(k_cache[l] + (size_t)P * kvw, kn, sizeof(double) * (size_t)n * kvw);
@@ -470,6 +498,14 @@ int orc_forward(const orc_config *c, const orc_model_weights *m, int n, const in
     if (logits) orc_head(c, m, n, x, logits);
     free(x); free(kn); free(vn);
     return 0;
+}
+
+int orc_forward(const orc_config *c, const orc_model_weights *m, int n, const int32_t *ids,
+                const int32_t *pos, int P, double *const *k_cache, double *const *v_cache, int causal,
+                int write_cache, double *hidden_dbg, double *router_dbg, double *logits)
+{
+    return orc_forward_flip(c, m, n, ids, pos, P, k_cache, v_cache, causal, write_cache, hidden_dbg, router_dbg,
+                            logits, NULL);
 }
 
 /* ------------------------------------------------------------------------------------------ */

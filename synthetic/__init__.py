@@ -144,11 +144,37 @@ def dequantize_fp8_block128(m: dict) -> torch.Tensor:
     return (v * s).reshape(shape)
 
 
+GAIN_SEED_OFFSET = 7919
+
+
+def draw_gains(w: dict, d: int, seed: int, gain_std: float, device="cpu") -> dict:
+    """Replace every RMSNorm gain of a weight set (each layer's attn_norm and ffn_norm, then
+    final_norm) by an independent draw 1 + N(0, gain_std^2) in fp32, from a generator of its own
+    (seed + GAIN_SEED_OFFSET) so that the matrices drawn before stay the same."""
+    gen = _gen(seed + GAIN_SEED_OFFSET, device)
+
+    def one():
+        return torch.randn(d, generator=gen, device=device, dtype=torch.float32).mul_(gain_std).add_(1.0)
+
+    for L in w["layers"]:
+        L["attn_norm"] = one()
+        L["ffn_norm"] = one()
+    if "final_norm" in w:
+        w["final_norm"] = one()
+    return w
+
+
 def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, router_std=None,
-                       head_scale=1.0, emb_std=None, out_std=None) -> dict:
-    """Random-init weights N(0, w_std^2) rounded to bf16 (round-to-nearest-even), norm gains 1.
+                       head_scale=1.0, emb_std=None, out_std=None, gain_std=0.0, emb_levels=None,
+                       copy_head=0.0) -> dict:
+    """Random-init weights N(0, w_std^2) rounded to bf16 (round-to-nearest-even).  Norm gains are 1,
+    or with gain_std > 0 independent draws 1 + N(0, gain_std^2) (see draw_gains).
     ``head_scale`` multiplies the LM head's std (a larger head gives confident rows that commit);
-    ``emb_std`` / ``out_std`` override the embedding std and the residual-output std."""
+    ``emb_std`` / ``out_std`` override the embedding std and the residual-output std.
+    ``emb_levels`` (a sequence of stds): every embedding row is rescaled to one of these stds, drawn
+    uniformly per row; ``copy_head`` = s adds s * emb to the head (a head that scores each position's
+    own token: rows of a loud token are confident, rows of a quiet one are not).  Both are applied
+    after every other draw, so the other weights do not change."""
     gen = _gen(seed, device)
     w = {
         "emb": _normal_bf16((cfg.vocab, cfg.d_model), w_std if emb_std is None else emb_std, gen, device),
@@ -156,6 +182,14 @@ def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, ro
         "final_norm": torch.ones(cfg.d_model, dtype=torch.float32, device=device),
     }
     w["head"] = _normal_bf16((cfg.vocab, cfg.d_model), w_std * head_scale, gen, device)
+    if emb_levels is not None:
+        lv = torch.tensor(list(emb_levels), dtype=torch.float32, device=device)
+        pick = torch.randint(0, lv.numel(), (cfg.vocab,), generator=gen, device=device)
+        w["emb"] = (w["emb"].float() * lv[pick][:, None]).to(torch.bfloat16)
+    if copy_head:
+        w["head"] = (w["head"].float() + copy_head * w["emb"].float()).to(torch.bfloat16)
+    if gain_std > 0:
+        draw_gains(w, cfg.d_model, seed, gain_std, device)
     return w
 
 

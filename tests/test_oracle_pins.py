@@ -354,11 +354,16 @@ def test_moe_sparse_selection_equals_dense_masked_mixture():
 # layer / model invariants
 # ------------------------------------------------------------------------------------------------
 
-def test_layer_forward_composition_matches_pieces():
+@pytest.mark.parametrize("gain_std", [0.0, 0.1])
+def test_layer_forward_composition_matches_pieces(gain_std):
     """The layer equals its pieces strung together: norm -> QKV -> RoPE -> masked attention -> O ->
-    residual -> norm -> router -> top-k -> experts -> residual (each piece pinned above)."""
-    cfg, w, M = _tiny_model(6)
+    residual -> norm -> router -> top-k -> experts -> residual (each piece pinned above).  With
+    gain_std > 0 the attention and MoE norms have distinct random gains, so a layer that applied one
+    in place of the other, or left a gain out, would not match."""
+    cfg, w, M = _tiny_model(6, gain_std=gain_std)
     L = w["layers"][0]
+    if gain_std:
+        assert not torch.equal(L["attn_norm"], L["ffn_norm"])
     rng = np.random.default_rng(6)
     n, P = 9, 5
     x = rng.normal(size=(n, cfg.d_model))
@@ -384,6 +389,68 @@ def test_layer_forward_composition_matches_pieces():
     np.testing.assert_allclose(kn, k, rtol=1e-12)
     np.testing.assert_allclose(vn, v, rtol=1e-12)
     np.testing.assert_allclose(rl, r, rtol=1e-10, atol=1e-14)
+
+
+def test_routing_flip_takes_the_next_expert():
+    """The tests' routing alternative: a flagged token takes its (k+1)-th expert in place of its k-th,
+    gates renormalised over the new selection; unflagged tokens keep the model's routing.  Pinned
+    against hand-picked logits and against the layer built from its pieces with that selection."""
+    l = np.array([[0.1, 3.0, -1.0, 2.5, 2.0, 0.0, 5.0, 1.0], [0.0, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0]])
+    sel, gate = oracle.router_topk(l, 3, flip=[1, 0])
+    np.testing.assert_array_equal(sel, [[6, 1, 4], [7, 6, 5]])
+    e = np.exp(np.array([5.0, 3.0, 2.0]) - 5.0)
+    np.testing.assert_allclose(gate[0], e / e.sum(), rtol=1e-14)
+    s0, g0 = oracle.router_topk(l, 3)
+    np.testing.assert_array_equal(s0[1], sel[1])
+    np.testing.assert_array_equal(g0[1], gate[1])
+    # a layer with flagged tokens equals its pieces with the flipped selection
+    cfg, w, M = _tiny_model(14, gain_std=0.1)
+    L = w["layers"][0]
+    rng = np.random.default_rng(14)
+    n = 6
+    x = rng.normal(size=(n, cfg.d_model))
+    pos = np.arange(n)
+    flip = np.array([1, 0, 0, 1, 1, 0], np.uint8)
+    out, _, _, r, mid = oracle.layer_forward(M, 0, x, pos, want_mid=True, flip=flip)
+    h2 = oracle.rmsnorm(mid, L["ffn_norm"].numpy())
+    sel, gate = oracle.router_topk(r, cfg.top_k, flip=flip)
+    np.testing.assert_allclose(out, mid + oracle.moe(M, 0, h2, sel, gate), rtol=1e-12, atol=1e-13)
+    plain = oracle.layer_forward(M, 0, x, pos)[0]
+    np.testing.assert_array_equal(out[flip == 0], plain[flip == 0])   # no attention after the MoE
+    assert np.abs(out[flip == 1] - plain[flip == 1]).max() > 1e-4
+
+
+def test_head_is_final_norm_then_vocabulary_projection():
+    """The vocabulary head is the final RMSNorm (with its own gain) followed by x W_head^T, built here
+    from the pinned RMSNorm and a torch matmul; a head that skipped the norm or used another gain
+    would not match."""
+    cfg, w, M = _tiny_model(12, gain_std=0.1)
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(5, cfg.d_model)) * 3.0
+    want = oracle.rmsnorm(x, w["final_norm"].numpy()) @ w["head"].to(torch.float64).numpy().T
+    np.testing.assert_allclose(oracle.head(M, x), want, rtol=1e-10, atol=1e-12)
+    plain = oracle.rmsnorm(x, np.ones(cfg.d_model, np.float32)) @ w["head"].to(torch.float64).numpy().T
+    assert np.abs(oracle.head(M, x) - plain).max() > 1e-3
+
+
+def test_forward_chains_layers_in_order_with_their_own_gains():
+    """The full forward is embedding -> layer 0 -> layer 1 -> head, each layer with its own weights and
+    gains (distinct random gains per layer): hidden[l + 1] = layer_forward(l, hidden[l]) and the
+    logits are the head of the last hidden state."""
+    cfg, w, M = _tiny_model(13, gain_std=0.1)
+    ids = synthetic.make_ids(20, cfg.vocab, 13).numpy()
+    P = 7
+    rng = np.random.default_rng(13)
+    kc = [rng.normal(size=(64, cfg.n_kv, cfg.d_head)) for _ in range(cfg.n_layers)]
+    vc = [rng.normal(size=(64, cfg.n_kv, cfg.d_head)) for _ in range(cfg.n_layers)]
+    pos = np.arange(P, P + 20)
+    fw = oracle.forward(M, ids, pos, P, kc, vc, want_hidden=True)
+    x = fw["hidden"][0]
+    np.testing.assert_array_equal(x, w["emb"][torch.from_numpy(ids).long()].to(torch.float64).numpy())
+    for l in range(cfg.n_layers):
+        x = oracle.layer_forward(M, l, x, pos, P, kc[l][:P], vc[l][:P])[0]
+        np.testing.assert_allclose(fw["hidden"][l + 1], x, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(fw["logits"], oracle.head(M, x), rtol=1e-12, atol=1e-13)
 
 
 def test_canvas_layer_is_permutation_equivariant():
