@@ -265,6 +265,24 @@ dg_status dg::record_error(dg_status st, const char* msg) {
   return st;
 }
 
+// The sampler settings every entry point shares.  The temperature schedule is only defined on
+// steps 0 .. max_steps - 1 (it reaches t_end at the last one and would extrapolate past it), so a
+// fixed budget above max_steps and a step outside the schedule are rejected.
+dg_status dg::check_sampler_params(const dg_sampler_params* p, int step, const char* fn) {
+  if (!p) return fail(DG_ERR_INVALID_ARG, "%ssampler params are null", fn);
+  if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "%scanvas_len must be 256", fn);
+  if (p->max_steps <= 0 || p->fixed_steps < 0) return fail(DG_ERR_INVALID_ARG, "%sbad step budget", fn);
+  if (p->fixed_steps > p->max_steps)
+    return fail(DG_ERR_INVALID_ARG, "%sfixed_steps %d exceeds max_steps %d (the temperature schedule's length)", fn,
+                p->fixed_steps, p->max_steps);
+  if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "%stemperatures must be > 0", fn);
+  if (p->commit_mode != 0 && p->commit_mode != 1) return fail(DG_ERR_INVALID_ARG, "%scommit_mode must be 0 or 1", fn);
+  if (p->commit_rule != 0 && p->commit_rule != 1) return fail(DG_ERR_INVALID_ARG, "%scommit_rule must be 0 or 1", fn);
+  if (step >= p->max_steps)
+    return fail(DG_ERR_INVALID_ARG, "%sstep %d is outside the %d-step temperature schedule", fn, step, p->max_steps);
+  return DG_OK;
+}
+
 // ---------------------------------------------------------------------------------------------
 // handles
 // ---------------------------------------------------------------------------------------------
@@ -739,14 +757,8 @@ dg_status run_canvas_stack(dg_seqs* s, const int32_t* d_ids, float* hidden) {
 }
 
 dg_status check_params(const dg_seqs* s, const dg_sampler_params* p) {
-  if (!p) return fail(DG_ERR_INVALID_ARG, "sampler params are null");
-  if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "canvas_len must be 256");
-  if (p->max_steps <= 0 || p->fixed_steps < 0) return fail(DG_ERR_INVALID_ARG, "bad step budget");
-  if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
-  if (p->commit_mode != 0 && p->commit_mode != 1) return fail(DG_ERR_INVALID_ARG, "commit_mode must be 0 or 1");
-  if (p->commit_rule != 0 && p->commit_rule != 1) return fail(DG_ERR_INVALID_ARG, "commit_rule must be 0 or 1");
   (void)s;
-  return DG_OK;
+  return check_sampler_params(p, -1, "");
 }
 
 }  // namespace
@@ -984,9 +996,11 @@ DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg
   NvtxRange nvtx_range("dg_sample");
   if (!d_logits || !p || !d_ids || !d_commit || !d_entropy || !d_stop || !ws)
     return fail(DG_ERR_INVALID_ARG, "null argument");
-  if (n_seq <= 0 || vocab <= 0 || vocab % 1024) return fail(DG_ERR_INVALID_ARG, "bad n_seq / vocab");
-  if (p->canvas_len != kCanvas) return fail(DG_ERR_UNSUPPORTED, "canvas_len must be 256");
-  if (step < 0 || p->max_steps <= 0) return fail(DG_ERR_INVALID_ARG, "bad step");
+  if (n_seq <= 0 || vocab <= 0 || vocab % 1024 || n_seq > (1 << 20))
+    return fail(DG_ERR_INVALID_ARG, "bad n_seq / vocab");
+  if (step < 0) return fail(DG_ERR_INVALID_ARG, "bad step");
+  const dg_status ps = check_sampler_params(p, step, "dg_sample: ");
+  if (ps != DG_OK) return ps;
   const int rows = n_seq * kCanvas;
   if (ws_bytes < dg_sample_workspace_bytes(rows, vocab)) return fail(DG_ERR_CAPACITY, "sampler workspace too small");
   SamplerArgs a{};

@@ -14,6 +14,10 @@ namespace dg {
 // Set the calling thread's dg_last_error() message; returns st.
 dg_status record_error(dg_status st, const char* msg);
 
+// Host-side checks of the sampler settings shared by every entry point (fn prefixes the message).
+// step >= 0: also that the step lies inside the max_steps-step temperature schedule.
+dg_status check_sampler_params(const dg_sampler_params* p, int step, const char* fn);
+
 // Programmatic dependent launch on/off for every kernel of the library (on unless DG_PDL=0).
 bool pdl_enabled();
 

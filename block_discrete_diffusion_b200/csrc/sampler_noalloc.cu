@@ -10,7 +10,9 @@
 // that loads libdg.so holds its own copy until the process exits.  Host code cannot use the
 // array's name as a device address (on the host it names a host-side stand-in), so the first call
 // on each device looks the device address up with cudaGetSymbolAddress, with that device current,
-// and caches it; that first call should therefore happen before any stream capture.  All calls on
+// and caches it for the life of the process; that first call should therefore happen before any
+// stream capture, and a cudaDeviceReset after it is not supported (the reset unloads the module, so
+// the cached address would point at freed memory).  All calls on
 // a device share the one array and it keeps the last call's contents; nothing in it has to start
 // at zero (every record is written by the partial kernel before the finalize kernel reads it).
 // Calls that overlap on the GPU (different streams, or different threads without ordering) race
@@ -55,7 +57,7 @@ cudaError_t scratch_address(float** out) {
 }  // namespace
 
 DG_API size_t dg_sample_noalloc_max_rows(int vocab) {
-  if (vocab <= 0) return 0;
+  if (vocab <= 0 || vocab % 1024) return 0;   // vocabularies the sampler rejects
   return (size_t)kNoAllocSlots / (size_t)dg::sampler_chunks(vocab);
 }
 
@@ -66,14 +68,16 @@ DG_API dg_status dg_sample_noalloc(const float* d_logits, int n_seq, int vocab, 
     return dg::record_error(DG_ERR_INVALID_ARG, "dg_sample_noalloc: null argument");
   if (n_seq <= 0 || vocab <= 0 || vocab % 1024)
     return dg::record_error(DG_ERR_INVALID_ARG, "dg_sample_noalloc: bad n_seq / vocab");
-  if (p->canvas_len != 256) return dg::record_error(DG_ERR_UNSUPPORTED, "dg_sample_noalloc: canvas_len must be 256");
-  if (step < 0 || p->max_steps <= 0) return dg::record_error(DG_ERR_INVALID_ARG, "dg_sample_noalloc: bad step");
-  const int rows = n_seq * 256;
+  if (step < 0) return dg::record_error(DG_ERR_INVALID_ARG, "dg_sample_noalloc: bad step");
+  const dg_status ps = dg::check_sampler_params(p, step, "dg_sample_noalloc: ");
+  if (ps != DG_OK) return ps;
   const int chunks = dg::sampler_chunks(vocab);
-  if ((size_t)rows * chunks > (size_t)kNoAllocSlots) {
-    char msg[160];
-    snprintf(msg, sizeof msg, "dg_sample_noalloc: %d rows x %d vocabulary chunks exceed the static scratch of %d records",
-             rows, chunks, kNoAllocSlots);
+  // compare in size_t before forming n_seq * 256 (no int overflow for any n_seq)
+  if ((size_t)n_seq * 256u * (size_t)chunks > (size_t)kNoAllocSlots) {
+    char msg[192];
+    snprintf(msg, sizeof msg,
+             "dg_sample_noalloc: %d canvases x 256 rows x %d vocabulary chunks exceed the static scratch of %d records",
+             n_seq, chunks, kNoAllocSlots);
     return dg::record_error(DG_ERR_CAPACITY, msg);
   }
   float* scratch = nullptr;

@@ -101,7 +101,8 @@ typedef struct {
 typedef struct {
   int canvas_len;          /* must be 256 */
   int max_steps;           /* step budget of the temperature schedule (48) */
-  int fixed_steps;         /* > 0: exactly this many steps per block, adaptive stop off; 0: adaptive */
+  int fixed_steps;         /* > 0: exactly this many steps per block (<= max_steps), adaptive stop
+                              off; 0: adaptive */
   float t_start, t_end;    /* 0.8, 0.4 */
   float entropy_bound;     /* 0.1 */
   float stop_mean_entropy; /* 0.005 */
@@ -203,7 +204,8 @@ dg_status dg_layer_forward(dg_seqs *s, int layer, int n_rows, int causal, float 
                            float *d_router_logits);
 
 /* Sampler alone over caller logits (finite fp32 [n_seq*canvas_len][vocab]): the entropy / Gumbel-argmax /
- * commit / re-randomise / stop rule of one step.  d_seq_P (nullable, int32 [n_seq]): absolute
+ * commit / re-randomise / stop rule of step `step` (0 <= step < max_steps, the temperature
+ * schedule's range; DG_ERR_INVALID_ARG otherwise).  d_seq_P (nullable, int32 [n_seq]): absolute
  * position of each sequence's first canvas row (0 if NULL).  d_ids, d_commit in/out as in
  * dg_canvas_step.  ws: device scratch of dg_sample_workspace_bytes(n_seq*canvas_len, vocab). */
 size_t dg_sample_workspace_bytes(int n_rows, int vocab);
@@ -216,16 +218,19 @@ dg_status dg_sample(const float *d_logits, int n_seq, int vocab, const dg_sample
  * free HBM, a real-time loop that must not allocate, a C component with no CUDA allocator -- the
  * sampler's per-(row, vocabulary chunk) partial results live in a static device array of the
  * library (1 MiB, held on every GPU that loads the library until the process exits).  Limit:
- * n_seq * 256 * chunks <= 32768 records, chunks = max(1, vocab / 32768) (16 canvases at vocab
- * 262144); larger requests return DG_ERR_CAPACITY.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress, with that device current): make it before any
- * stream capture.  It allocates nothing (no cudaMalloc / cudaFree).  All calls on a device share
+ * n_seq * 256 * chunks <= 32768 records, where chunks is the sampler's split of the vocabulary:
+ * the largest c <= max(1, vocab / 32768) with vocab % (4 c) == 0 (8 chunks, so 16 canvases, at
+ * vocab 262144); larger requests return DG_ERR_CAPACITY.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current) and keeps it for the
+ * life of the process: make that call before any stream capture, and do not call cudaDeviceReset
+ * after it.  It allocates nothing (no cudaMalloc / cudaFree).  All calls on a device share
  * the array and it keeps the last call's contents (nothing in it needs to start at zero); calls
  * that may overlap on the GPU race and must not be issued.  Arguments and outputs as dg_sample. */
 dg_status dg_sample_noalloc(const float *d_logits, int n_seq, int vocab, const dg_sampler_params *p, int step,
                             const int32_t *d_seq_P, int32_t *d_ids, uint8_t *d_commit, float *d_entropy,
                             int32_t *d_stop, void *stream);
-/* Largest n_seq * 256 that dg_sample_noalloc accepts for this vocabulary size. */
+/* Largest n_seq * 256 that dg_sample_noalloc accepts for this vocabulary size (0 for a vocabulary
+ * the sampler rejects: vocab <= 0 or vocab % 1024 != 0). */
 size_t dg_sample_noalloc_max_rows(int vocab);
 
 /* Synchronise the handle's stream and return the first device-side error code recorded since the

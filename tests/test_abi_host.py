@@ -104,6 +104,8 @@ def test_product_path_does_not_import_the_oracle():
     ("null_logits", "DG_ERR_INVALID_ARG"), ("vocab_not_multiple_of_1024", "DG_ERR_INVALID_ARG"),
     ("canvas_128", "DG_ERR_UNSUPPORTED"), ("negative_step", "DG_ERR_INVALID_ARG"),
     ("workspace_too_small", "DG_ERR_CAPACITY"), ("no_rows", "DG_ERR_INVALID_ARG"),
+    ("step_past_schedule", "DG_ERR_INVALID_ARG"), ("fixed_steps_past_schedule", "DG_ERR_INVALID_ARG"),
+    ("zero_temperature", "DG_ERR_INVALID_ARG"),
 ])
 def test_sampler_argument_checks_happen_on_the_host(dg, case, expected):
     """dg_sample rejects bad arguments before it touches the device (fake, never dereferenced
@@ -125,6 +127,12 @@ def test_sampler_argument_checks_happen_on_the_host(dg, case, expected):
         ws_bytes -= 1
     elif case == "no_rows":
         n_seq = 0
+    elif case == "step_past_schedule":
+        step = prm.max_steps                      # the schedule has steps 0 .. max_steps - 1
+    elif case == "fixed_steps_past_schedule":
+        prm.fixed_steps = prm.max_steps + 1
+    elif case == "zero_temperature":
+        prm.t_end = 0.0
     st = dg.lib().dg_sample(logits, n_seq, vocab, ctypes.byref(prm), step, None, fake, fake, fake, fake, fake,
                             ws_bytes, None)
     assert st == getattr(dg, expected)
@@ -158,3 +166,26 @@ def test_binding_structs_match_the_header_layout(dg, tmp_path):
         assert got[(S.__name__, "size")] == ctypes.sizeof(S), S.__name__
         for name, _ in S._fields_:
             assert got[(S.__name__, name)] == getattr(S, name).offset, (S.__name__, name)
+
+
+@pytest.mark.parametrize("case", ["step_past_schedule", "fixed_steps_past_schedule", "bad_vocab", "huge_n_seq"])
+def test_noalloc_argument_checks_happen_on_the_host(dg, case):
+    """dg_sample_noalloc checks its arguments like dg_sample, and compares its capacity without an
+    integer overflow for any canvas count; its limit query answers 0 for vocabularies it rejects."""
+    vocab, n_seq, step = 262144, 1, 0
+    prm = dg.sampler_params(vocab, seed=1)
+    fake = ctypes.c_void_p(4096)
+    expected = dg.DG_ERR_INVALID_ARG
+    if case == "step_past_schedule":
+        step = prm.max_steps
+    elif case == "fixed_steps_past_schedule":
+        prm.fixed_steps = prm.max_steps + 1
+    elif case == "bad_vocab":
+        vocab = 99000
+        assert dg.dg_sample_noalloc_max_rows(vocab) == 0
+    elif case == "huge_n_seq":
+        n_seq = 2 ** 31 - 1                          # n_seq * 256 would overflow an int
+        expected = dg.DG_ERR_CAPACITY
+    st = dg.lib().dg_sample_noalloc(fake, n_seq, vocab, ctypes.byref(prm), step, None, fake, fake, fake, fake, None)
+    assert st == expected, (st, dg.lib().dg_last_error().decode())
+    assert dg.dg_sample_noalloc_max_rows(99328) == 32768 // 2      # 99328 = 97 * 1024: two chunks
