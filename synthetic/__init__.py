@@ -165,16 +165,18 @@ def draw_gains(w: dict, d: int, seed: int, gain_std: float, device="cpu") -> dic
 
 
 def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, router_std=None,
-                       head_scale=1.0, emb_std=None, out_std=None, gain_std=0.0, emb_levels=None,
+                       head_scale=1.0, emb_std=None, out_std=None, gain_std=0.0, emb_split=None,
                        copy_head=0.0) -> dict:
     """Random-init weights N(0, w_std^2) rounded to bf16 (round-to-nearest-even).  Norm gains are 1,
     or with gain_std > 0 independent draws 1 + N(0, gain_std^2) (see draw_gains).
     ``head_scale`` multiplies the LM head's std (a larger head gives confident rows that commit);
     ``emb_std`` / ``out_std`` override the embedding std and the residual-output std.
-    ``emb_levels`` (a sequence of stds): every embedding row is rescaled to one of these stds, drawn
-    uniformly per row; ``copy_head`` = s adds s * emb to the head (a head that scores each position's
-    own token: rows of a loud token are confident, rows of a quiet one are not).  Both are applied
-    after every other draw, so the other weights do not change."""
+    ``emb_split`` = (k, loud_std, quiet_std, loud_frac): a fraction loud_frac of the tokens ("loud")
+    get embedding rows N(0, loud_std^2) in the first k channels and 0 elsewhere, the others
+    ("quiet") N(0, quiet_std^2) in the remaining channels and 0 in the first k; ``copy_head`` = s adds
+    s * emb to the head, so each position scores its own token: a loud token's row is confident, a
+    quiet token's row sees only small logits (the two kinds live in orthogonal channels).  Both are
+    applied after every other draw, so the other weights do not change."""
     gen = _gen(seed, device)
     w = {
         "emb": _normal_bf16((cfg.vocab, cfg.d_model), w_std if emb_std is None else emb_std, gen, device),
@@ -182,10 +184,13 @@ def make_model_weights(cfg: ModelConfig, seed: int, device="cpu", w_std=0.02, ro
         "final_norm": torch.ones(cfg.d_model, dtype=torch.float32, device=device),
     }
     w["head"] = _normal_bf16((cfg.vocab, cfg.d_model), w_std * head_scale, gen, device)
-    if emb_levels is not None:
-        lv = torch.tensor(list(emb_levels), dtype=torch.float32, device=device)
-        pick = torch.randint(0, lv.numel(), (cfg.vocab,), generator=gen, device=device)
-        w["emb"] = (w["emb"].float() * lv[pick][:, None]).to(torch.bfloat16)
+    if emb_split is not None:
+        k, loud_std, quiet_std, loud_frac = emb_split
+        loud = torch.rand(cfg.vocab, generator=gen, device=device) < loud_frac
+        e = torch.randn((cfg.vocab, cfg.d_model), generator=gen, device=device)
+        e[:, :k].mul_(loud_std).mul_(loud[:, None])
+        e[:, k:].mul_(quiet_std).mul_(~loud[:, None])
+        w["emb"] = e.to(torch.bfloat16)
     if copy_head:
         w["head"] = (w["head"].float() + copy_head * w["emb"].float()).to(torch.bfloat16)
     if gain_std > 0:

@@ -16,12 +16,13 @@ Judging rules.
   Large logits: the tempered scores z = l/T of an end-to-end step carry the bf16 rounding of the
   step's sequential GEMM inputs.  Each rounding adds a relative error of rms 2^-9/sqrt(3) to its
   products; with 2L+1 sequential roundings the rms relative error of z is about
-  sqrt(2L+1) * 2^-9 / sqrt(3).  Judging at 4 sigma gives c_z = 4 sqrt(2L+1) 2^-9 / sqrt(3)
-  (1.0e-2 for L = 2; FP8 weights add 5L roundings, see c_z).  Where c_z * std(z_row) exceeds
-  the base margin, ids are judged where the oracle margin exceeds c_z * std(z_row), and
-  entropies within c_z * (std(z) std_p(z) + Var_p(z)) (the first-order change of the entropy under a perturbation of that size: random part
-  std(dz) std_p(z), scale part Var_p(z) c_z).  These derived bounds reduce to the base ones at small
-  logits and are only used by the tests that say so.
+  sigma_z = sqrt(2L+1) * 2^-9 / sqrt(3) (FP8 weights add 5L roundings, see c_z).  A test judges
+  thousands of decisions, so the bounds sit at 6 sigma: c_z = 6 sigma_z (1.5e-2 for L = 2).  Where
+  c_z * std(z_row) exceeds the base margin, ids are judged where the oracle margin -- a difference of
+  two scores, whose error is sqrt(2) times that of one -- exceeds sqrt(2) c_z std(z_row), and
+  entropies within c_z * (std(z) std_p(z) + Var_p(z)) (the first-order change of the entropy under a
+  perturbation of that size: random part std(dz) std_p(z), scale part Var_p(z) c_z).  These derived
+  bounds are only used by the tests that say so (the head x50 cases).
 """
 import math
 
@@ -63,8 +64,18 @@ def kv_views(kv: torch.Tensor, cfg, n_seq, max_ctx):
     return K, Vt
 
 
-def router_tie_tokens(router_logits, top_k, margin=MARGIN):
-    """Tokens whose k-th and (k+1)-th router logits are closer than `margin` in any layer."""
+# Router near-ties in end-to-end steps.  A token's router logits in an end-to-end step carry, besides
+# the bf16 rounding of the layer's normed input, the hidden-state error carried from the layers before,
+# so the gap between its k-th and (k+1)-th logits is known only to a fraction of a percent of the
+# logits' spread: on unit-spread logits the GPU routed tokens the other way at gaps of 1.1e-2 to
+# 1.9e-2 (a few among ~1e5 decisions).  End-to-end comparisons therefore treat gaps below 5% of the
+# layer's router-logit standard deviation, and never below the base 1e-2, as near-ties.
+ROUTER_TIE_REL_E2E = 0.05
+
+
+def router_tie_tokens(router_logits, top_k, margin=MARGIN, rel=0.0):
+    """Tokens whose k-th and (k+1)-th router logits are closer than max(margin, rel * std of that
+    layer's router logits) in any layer."""
     r = np.asarray(router_logits)
     if r.ndim == 2:
         r = r[None]
@@ -72,17 +83,18 @@ def router_tie_tokens(router_logits, top_k, margin=MARGIN):
     if r.shape[2] <= top_k:
         return bad
     s = -np.sort(-r, axis=2)
-    bad |= ((s[:, :, top_k - 1] - s[:, :, top_k]) < margin).any(0)
+    tol = np.maximum(margin, rel * r.reshape(r.shape[0], -1).std(axis=1))[:, None]
+    bad |= ((s[:, :, top_k - 1] - s[:, :, top_k]) < tol).any(0)
     return bad
 
 
 def c_z(n_layers, fp8=False):
-    """4-sigma relative error of the tempered scores after n_r sequential bf16 roundings:
+    """6-sigma relative error of the tempered scores after n_r sequential bf16 roundings:
     n_r = 2L+1 activation roundings; with FP8 weights each of the five per-layer matrices is also
     rounded once (the kernels multiply bf16(q*s), the oracle q*s), 5L more roundings of the same
     size, independent of the others."""
     n_r = 2 * n_layers + 1 + (5 * n_layers if fp8 else 0)
-    return 4.0 * math.sqrt(n_r) * 2.0 ** -9 / math.sqrt(3.0)
+    return 6.0 * math.sqrt(n_r) * 2.0 ** -9 / math.sqrt(3.0)
 
 
 def derived_tolerances(logits, T, n_layers, fp8=False):
@@ -96,7 +108,7 @@ def derived_tolerances(logits, T, n_layers, fp8=False):
     p /= p.sum(axis=1, keepdims=True)
     mean_p = (p * z).sum(axis=1, keepdims=True)
     var_p = (p * (z - mean_p) ** 2).sum(axis=1)
-    margin = np.maximum(MARGIN, cz * std_z)
+    margin = np.maximum(MARGIN, math.sqrt(2.0) * cz * std_z)
     htol = np.maximum(ENTROPY_TOL, cz * (std_z * np.sqrt(var_p) + var_p))
     return margin, htol
 
@@ -137,13 +149,30 @@ def judge_step(gpu, orc, prm, commit_before, exclude=None, margin_tol=None, h_to
         abs(orc["mean_H"] - prm.stop_mean_entropy) > mean_band and (not exclude.any() or open_row))
     if stop_judged and int(gpu["stop"]) != int(orc["stop"]):
         fails.append(f"stop flag gpu {gpu['stop']} oracle {orc['stop']} (mean H {orc['mean_H']})")
+    # a row that commits in this step, or takes its Gumbel-argmax y without committing (entropy below
+    # the re-randomisation threshold), ends with id y whether the block stops or not: its id (and, if it
+    # commits, its commit bit) is judged even when the stop flag is not
+    crit = orc["cum"] if "cum" in orc else H_o
+    commits_anyway = crit <= prm.entropy_bound
     judged = 0
     for i in range(n):
         if was[i]:
             if gpu["ids"][i] != orc["ids"][i] or not gpu["commit"][i]:
                 fails.append(f"committed row {i} changed")
             continue
-        if exclude[i] or near_bound[i] or not stop_judged:
+        if exclude[i] or near_bound[i]:
+            continue
+        if not stop_judged:
+            if near_rr[i] or not (commits_anyway[i] or H_o[i] <= prm.rerand_entropy):
+                continue                      # re-randomised unless the block stops: open
+            if commits_anyway[i] and not gpu["commit"][i]:
+                fails.append(f"commit row {i}: gpu 0 oracle 1 H {H_o[i]}")
+                continue
+            if orc["margin"][i] > margin_tol[i]:
+                judged += 1
+                if gpu["ids"][i] != orc["y"][i]:
+                    fails.append(f"sampled id row {i}: gpu {gpu['ids'][i]} oracle {orc['y'][i]} "
+                                 f"margin {orc['margin'][i]} tol {margin_tol[i]}")
             continue
         if gpu["commit"][i] != orc["commit"][i]:
             fails.append(f"commit row {i}: gpu {gpu['commit'][i]} oracle {orc['commit'][i]} H {H_o[i]}")

@@ -28,7 +28,7 @@ def dg(cuda_ok):
 
 def _tiny(wdtype, head_scale=50.0, seed=0):
     cfg = dataclasses.replace(synthetic.TINY, top_k=8, wdtype=wdtype)    # top_k = E: no routing decision
-    w = synthetic.make_model_weights(cfg, seed, head_scale=head_scale)
+    w = synthetic.make_model_weights(cfg, seed, head_scale=head_scale, gain_std=0.1)
     return cfg, w
 
 
@@ -130,7 +130,7 @@ def test_batched_sequences_match_their_oracles(dg, wdtype, head_scale):
 def _layer_sequences(dg, cfg, n_seq, prefix_lens, seed, check):
     """One full-width FP8 layer on n_seq canvases with prefixes of the given lengths; the
     sequences in `check` are compared with the oracle."""
-    w = synthetic.make_model_weights(cfg, seed, device="cuda", router_std=cfg.d_model ** -0.5)
+    w = synthetic.make_model_weights(cfg, seed, device="cuda", router_std=cfg.d_model ** -0.5, gain_std=0.1)
     model = dg.dg_model_create(cfg, w)
     max_ctx = ((max(prefix_lens) + 256 + 255) // 256) * 256
     seqs = dg.dg_seqs_create(model, n_seq, max_ctx)
@@ -181,3 +181,85 @@ def test_fp8_layer_32_sequences_of_32k_prefix(dg):
     full-width layer); the first and the last sequence are compared with the oracle."""
     cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024, wdtype=1)
     _layer_sequences(dg, cfg, 32, [32768] * 32, 31, check=[0, 31])
+
+
+def test_fp8_full_stack_32_sequences_sampled(dg):
+    """The 32-sequence configuration end to end: the 30-layer stack with FP8 per-layer matrices and
+    random RMSNorm gains, 32 canvases each behind its own 32768-position prefix, one dg_canvas_step
+    with the residual stream and the logits copied out.  Two sequences (the first and the last) are
+    judged against the oracle from the GPU's own inputs: layers 0, 15 and 29 (the oracle's layer on
+    the GPU's hidden state before it and on that sequence's cache, 6e-2), the final RMSNorm + head on
+    four rows each, and the sampler on that sequence's logits (its own stream, seed + index)."""
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()                  # the earlier tests' blocks: this case needs ~180 GB
+    cfg = dataclasses.replace(synthetic.FULL, wdtype=1)
+    n_seq, P = 32, 32768
+    w = synthetic.make_model_weights(cfg, 3, device="cuda", gain_std=0.1, **synthetic.full_stack_init(cfg))
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    model = dg.dg_model_create(cfg, w)
+    max_ctx = P + 256
+    seqs = dg.dg_seqs_create(model, n_seq, max_ctx)
+    for i in range(n_seq):
+        ks, vs = synthetic.make_prefix_kv(cfg.n_layers, P, cfg.n_kv, cfg.d_head, 3 + i, device="cuda")
+        dg.dg_load_prefix(seqs, i, P, ks, vs)
+        del ks, vs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    prm = dg.sampler_params(cfg.vocab, seed=3, fixed_steps=12, rerand_entropy=1e9)
+    ids = torch.empty(n_seq, 256, dtype=torch.int32, device="cuda")
+    commit = torch.empty(n_seq, 256, dtype=torch.uint8, device="cuda")
+    H = torch.empty(n_seq, 256, device="cuda")
+    stop = torch.empty(n_seq, dtype=torch.int32, device="cuda")
+    hidden = torch.empty(cfg.n_layers + 1, n_seq * 256, cfg.d_model, device="cuda")
+    logits = torch.empty(n_seq * 256, cfg.vocab, device="cuda")
+    dg.dg_canvas_init(seqs, prm, ids, commit)
+    ids0 = ids.cpu().numpy().copy()
+    dg.dg_canvas_step(seqs, prm, ids, commit, H, stop, hidden, logits)
+    torch.cuda.synchronize()
+    assert dg.dg_device_error(seqs) == 0
+    check_layers = (0, 15, 29)
+    check_seqs = (0, n_seq - 1)
+    planes = sorted({l for l in check_layers} | {l + 1 for l in check_layers} | {cfg.n_layers})
+    hg = {(s, l): hidden[l, 256 * s: 256 * (s + 1)].double().cpu().numpy() for s in check_seqs for l in planes}
+    lg = {s: logits[256 * s: 256 * (s + 1)].cpu().numpy() for s in check_seqs}
+    del hidden, logits
+    K, Vt = kv_views(seqs.kv, cfg, n_seq, max_ctx)
+    pos = np.arange(P, P + 256)
+    c1 = dataclasses.replace(cfg, n_layers=1)
+    for l in check_layers:
+        L = {k: ({a: b.cpu() for a, b in v.items()} if isinstance(v, dict) else v.cpu())
+             for k, v in w["layers"][l].items()}
+        M = oracle.Model(c1, {"layers": [L]}, layers=[L])
+        for s in check_seqs:
+            kc = K[l, s, :, :P].permute(1, 0, 2).double().cpu().numpy()
+            vc = Vt[l, s, :, :, :P].permute(2, 0, 1).double().cpu().numpy()
+            xo, kn, vn, rlo = oracle.layer_forward(M, 0, hg[(s, l)], pos, P, kc, vc)
+            del kc, vc
+            keep = ~router_tie_tokens(rlo, cfg.top_k)
+            e = rel_err(hg[(s, l + 1)][keep], xo[keep])
+            assert e <= HIDDEN_TOL_FP8, ("layer output", l, s, e, int(keep.sum()))
+            assert keep.sum() >= 128
+            kg = K[l, s, :, P:P + 256].permute(1, 0, 2).float().cpu().numpy()
+            assert rel_err(kg, kn) <= HIDDEN_TOL_FP8, ("canvas K", l, s)
+    Mh = oracle.Model(cfg, {"layers": [], "head": w["head"].cpu(), "final_norm": w["final_norm"].cpu()}, layers=[])
+    rows = np.array([0, 99, 180, 255])
+    T = oracle.temperature(0)
+    for s in check_seqs:
+        e_head = rel_err(lg[s][rows], oracle.head(Mh, hg[(s, cfg.n_layers)][rows]))
+        assert e_head <= HIDDEN_TOL, ("head logits (bf16 head, same input)", s, e_head)
+        prm_o = oracle.SamplerParams(cfg.vocab, seed=3 + s, fixed_steps=12, rerand_entropy=1e9)
+        smp = oracle.sample_rows(lg[s], np.zeros(256, np.uint8), pos, T, 3 + s, 0)
+        rule = oracle.step_rule(np.zeros(256, np.uint8), ids0[s], smp["H"], smp["y"], smp["rr"], 0,
+                                prm_o.entropy_bound, prm_o.rerand_entropy, prm_o.stop_mean_entropy, prm_o.max_steps,
+                                prm_o.fixed_steps)
+        orc = dict(smp)
+        orc.update(rule)
+        orc["step"] = 0
+        orc["logits"] = lg[s]
+        g = {"ids": ids[s].cpu().numpy(), "commit": commit[s].cpu().numpy(), "H": H[s].cpu().numpy(),
+             "stop": int(stop[s].item())}
+        fails, judged = judge_step(g, orc, prm_o, np.zeros(256, np.uint8))
+        assert not fails, (s, fails[:10])
+        assert judged >= 240, (s, judged)
