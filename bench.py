@@ -51,13 +51,17 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="full_b1", choices=["full_b1", "one_layer", "sampler", "fp8_b32"],
+    ap.add_argument("--no-aux", action="store_true", help="full_b1: leave out the one-layer and sampler sub-records")
+    ap.add_argument("--workload", default="full_b1",
+                    choices=["full_b1", "one_layer", "sampler", "head_sampler", "fp8_b32"],
                     help="full_b1: the benchmark line; one_layer / sampler: the single-layer and "
                          "sampler-alone configurations (their own lines, used for per-kernel profiles); "
                          "fp8_b32: the 30-layer FP8 stack on 32 sequences behind 32768-token prefixes")
     ap.add_argument("--seqs", type=int, default=32, help="fp8_b32: number of sequences")
     ap.add_argument("--prefix", type=int, default=32768, help="fp8_b32: prefix length of every sequence")
     ap.add_argument("--fp8", action="store_true", help="full_b1 / one_layer: FP8 block-scaled per-layer weights")
+    ap.add_argument("--nv", type=int, default=128, choices=[2, 128, 256],
+                    help="head_sampler: vocabulary rows per tile of the fused head (2: pairs of SMs)")
     a = ap.parse_args()
     a.seqs_given = seqs_given
     return a
@@ -328,11 +332,17 @@ def main_dg(args):
            "d2h_bytes_per_step": CANVAS * 4 + CANVAS + CANVAS * 4 + 4}
 
     # ---- committed tokens/s: dg_decode of 4 blocks x 12 fixed steps with a commit pass per block ----
-    seqs2 = dg.dg_seqs_create(model, 1, PROMPT + BLOCKS * CANVAS)
+    # (a first dg_decode of one block builds the handle's device-resident step-loop graph, a one-time
+    # set-up that later calls reuse; it is timed separately)
+    seqs2 = dg.dg_seqs_create(model, 1, PROMPT + (BLOCKS + 1) * CANVAS)
     import synthetic
     prompt = synthetic.make_ids(PROMPT, cfg.vocab, seed=replica_seed(rank), device=device)
     dg.dg_prefill(seqs2, prompt, [PROMPT])
     out = torch.empty(1, BLOCKS * CANVAS, dtype=torch.int32, device=device)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    dg.dg_decode(seqs2, prm, 1, out)
+    first_block_s = time.perf_counter() - w0
     torch.cuda.synchronize()
     g0 = time.perf_counter()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -344,6 +354,13 @@ def main_dg(args):
     committed_tok_s = whole_job_rate(world, sum(n_out), td)
     code = dg.dg_device_error(seqs)
     assert code == 0, f"device error {code}"
+
+    # the one-layer and sampler-alone configurations, on this GPU, with their own clocks (one GPU only)
+    aux = {}
+    if world == 1 and not args.no_aux:
+        aux["one_layer"] = measure_one_layer(20, 5, gpu_index=local)
+        aux["sampler"] = measure_sampler(20, 5, gpu_index=local)
+        aux["head_sampler"] = measure_head_sampler(20, 5, gpu_index=local)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
@@ -360,9 +377,12 @@ def main_dg(args):
                                  + " of weights streamed per step"},
                 "committed_tok_s": round(committed_tok_s, 1),
                 "decode": {"blocks": BLOCKS, "steps_per_block": steps_per_block, "tokens": sum(n_out),
-                           "seconds": round(td, 4), "includes": "canvas init, 12 steps and a commit pass per block"},
+                           "seconds": round(td, 4), "includes": "canvas init, 12 steps and a commit pass per block",
+                           "step_loop": "on the device (CUDA graph while-node; no host read per step)",
+                           "first_call_one_block_s": round(first_block_s, 4)},
                 "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "kernel_ms_per_step": kernel_ms,
                 "clocks": clk.summary(), "cpu_baseline": cpu}
+        line.update(aux)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -478,68 +498,143 @@ def _timed(fn, k, warmup):
     return e0.elapsed_time(e1) / 1e3 / k
 
 
-def main_aux(args):
+def measure_one_layer(steps, warmup, n_seq=1, fp8=False, gpu_index=0):
+    """The one-layer configuration: one decoder layer at full width (a2-a9) on n_seq canvases of 256
+    rows x ~ N(0,1), each behind a 4096-token prefix of N(0,1) K/V.  Returns its record."""
     import dataclasses
 
     import torch
 
     import synthetic
-    from block_discrete_diffusion_b200 import build, dg
+    from block_discrete_diffusion_b200 import dg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024, wdtype=1 if fp8 else 0)
+    w = synthetic.make_model_weights(cfg, 1, device=dev, router_std=cfg.d_model ** -0.5)
+    model = dg.dg_model_create(cfg, w)
+    P = 4096
+    seqs = dg.dg_seqs_create(model, n_seq, P + CANVAS)
+    for i in range(n_seq):
+        ks, vs = synthetic.make_prefix_kv(1, P, cfg.n_kv, cfg.d_head, 1 + i, device=dev)
+        dg.dg_load_prefix(seqs, i, P, ks, vs)
+    x0 = synthetic.make_hidden(n_seq * CANVAS, cfg.d_model, 1, device=dev)
+    x = x0.clone()
+
+    def step():
+        x.copy_(x0)
+        dg.dg_layer_forward(seqs, 0, x)
+    with ClockSampler(gpu_index) as clk:
+        torch.cuda.synchronize()
+        clk.mark_start()
+        t = _timed(step, steps, warmup)
+        clk.mark_end()
+    dg.dg_stats_reset(seqs, timing=True)
+    for _ in range(steps):
+        step()
+    stats = dg.dg_stats_read(seqs)
+    assert dg.dg_device_error(seqs) == 0
+    return {"metric": "decoder-layer steps/s (a2-a9, one full-width layer)", "value": round(1 / t, 2),
+            "unit": "steps/s", "ms_per_step": round(t * 1e3, 4), "steps": steps, "warmup": warmup,
+            "config": {"workload": f"one_layer: d 2816, 16/8 heads x 128, 128 experts top-8 FFN 704, "
+                                   f"{n_seq} canvas(es) of 256 each behind a 4096-token prefix, "
+                                   f"{'fp8 e4m3 block-scaled' if fp8 else 'bf16'} weights"},
+            "kernel_ms_per_step": {k: round(v[1] / steps, 4) for k, v in stats.items() if v[0]},
+            "kernel_ms_note": "CUDA events around every launch (a second pass; serialises the dependent launches)",
+            "clocks": clk.summary()}
+
+
+def measure_sampler(steps, warmup, gpu_index=0):
+    """The sampler-alone configuration: 256 x 262144 fp32 logits N(0, 3^2) with a +12 spike in every
+    tenth row, step 12 of the 48-step schedule, seed 7.  Returns its record."""
+    import torch
+
+    import synthetic
+    from block_discrete_diffusion_b200 import dg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    vocab, canvas = 262144, 256
+    logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, device=dev)
+    prm = dg.sampler_params(vocab, seed=7)
+    ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device=dev)
+    ids = torch.zeros(canvas, dtype=torch.int32, device=dev)
+    commit = torch.zeros(canvas, dtype=torch.uint8, device=dev)
+    H = torch.empty(canvas, device=dev)
+    stop = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def step():
+        commit.zero_()
+        dg.dg_sample(logits, 1, vocab, prm, 12, None, ids, commit, H, stop, ws)
+    with ClockSampler(gpu_index) as clk:
+        torch.cuda.synchronize()
+        clk.mark_start()
+        t = _timed(step, steps, warmup)
+        clk.mark_end()
+    hbm, _, kind = peaks()
+    gbs = canvas * vocab * 4 / t / 1e9
+    return {"metric": "sampler steps/s (256 x 262144 fp32 logits)", "value": round(1 / t, 2), "unit": "steps/s",
+            "ms_per_step": round(t * 1e3, 4), "steps": steps, "warmup": warmup,
+            "config": {"workload": "sampler: logits N(0, 3^2), 10% of rows +12 spike, step 12 of 48, seed 7",
+                       "l2": "inputs larger than L2: 268 MB of logits per call"},
+            "roofline": {"kernel": "sampler_partial + sampler_finalize (one dg_sample call)", "bound": "hbm",
+                         "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                         "traffic": SAMPLER_PARTIAL_TRAFFIC, "peak_source": kind,
+                         "note": "includes the commit-mask reset (256 B); the kernel is instruction-bound "
+                                 "(one Philox word, an exp2 and two hardware logarithms per logit)"},
+            "clocks": clk.summary()}
+
+
+def measure_head_sampler(steps, warmup, nv=128, gpu_index=0):
+    """The fused vocabulary head + sampler of one canvas alone (dg_head_sample): normed rows
+    xn ~ N(0, 1) [256, 2816] bf16, head rows N(0, (3/sqrt(2816))^2) [262144, 2816] bf16 so the logits
+    are ~N(0, 3^2) like the sampler workload, step 12, seed 7.  Roofline: the head's weight stream."""
+    import torch
+
+    from block_discrete_diffusion_b200 import dg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d, vocab = 2816, 262144
+    g = torch.Generator(device=dev).manual_seed(7)
+    xn = torch.randn(256, d, generator=g, device=dev).to(torch.bfloat16)
+    head = torch.randn(vocab, d, generator=g, device=dev).mul_(3.0 / d ** 0.5).to(torch.bfloat16)
+    prm = dg.sampler_params(vocab, seed=7)
+    ws = torch.empty(dg.dg_head_sample_workspace_bytes(vocab), dtype=torch.uint8, device=dev)
+    ids = torch.zeros(256, dtype=torch.int32, device=dev)
+    commit = torch.zeros(256, dtype=torch.uint8, device=dev)
+    H = torch.empty(256, device=dev)
+    stop = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def step():
+        dg.dg_head_sample(xn, head, prm, 12, None, ids, commit, H, stop, ws, nv=nv)
+    with ClockSampler(gpu_index) as clk:
+        torch.cuda.synchronize()
+        clk.mark_start()
+        t = _timed(step, steps, warmup)
+        clk.mark_end()
+    assert dg.dg_head_sample_error(ws) == 0
+    hbm, _, kind = peaks()
+    nbytes = vocab * d * 2 + 256 * d * 2
+    gbs = nbytes / t / 1e9
+    return {"metric": "fused head + sampler calls/s (256 x 2816 x 262144)", "value": round(1 / t, 2),
+            "unit": "calls/s", "ms_per_step": round(t * 1e3, 4), "steps": steps, "warmup": warmup,
+            "config": {"workload": "head_sampler: one canvas, normed rows N(0,1), head N(0, (3/sqrt(2816))^2), "
+                                   f"logits ~N(0, 3^2), step 12 of 48, seed 7, "
+                                   + ("CTA pairs, 256 vocabulary rows per pair tile" if nv == 2 else f"{nv} vocabulary rows per tile"),
+                       "l2": "inputs larger than L2: 1.48 GB of head weights per call"},
+            "roofline": {"kernel": "head_sampler_kernel + sampler_finalize (one dg_head_sample call)", "bound": "hbm",
+                         "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                         "algorithmic_bytes_per_launch": nbytes, "traffic": None, "peak_source": kind},
+            "clocks": clk.summary()}
+
+
+def main_aux(args):
+    import torch
+
+    from block_discrete_diffusion_b200 import build
     build.build()
-    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
     if args.workload == "one_layer":
-        # one decoder layer at full width: x ~ N(0,1) [256, 2816], prefix K/V ~ N(0,1) of 4096 tokens
-        # --seqs n (default 1) canvases each behind a 4096-token prefix; --fp8: FP8 block-scaled weights
-        cfg = dataclasses.replace(synthetic.ONE_LAYER, vocab=1024, wdtype=1 if args.fp8 else 0)
-        n_seq = args.seqs if args.seqs_given else 1
-        w = synthetic.make_model_weights(cfg, 1, device=dev, router_std=cfg.d_model ** -0.5)
-        model = dg.dg_model_create(cfg, w)
-        P = 4096
-        seqs = dg.dg_seqs_create(model, n_seq, P + CANVAS)
-        for i in range(n_seq):
-            ks, vs = synthetic.make_prefix_kv(1, P, cfg.n_kv, cfg.d_head, 1 + i, device=dev)
-            dg.dg_load_prefix(seqs, i, P, ks, vs)
-        x0 = synthetic.make_hidden(n_seq * CANVAS, cfg.d_model, 1, device=dev)
-        x = x0.clone()
-
-        def step():
-            x.copy_(x0)
-            dg.dg_layer_forward(seqs, 0, x)
-        t = _timed(step, args.steps, args.warmup)
-        dg.dg_stats_reset(seqs, timing=True)
-        for _ in range(args.steps):
-            step()
-        stats = dg.dg_stats_read(seqs)
-        line = {"metric": "decoder-layer steps/s (a2-a9, one full-width layer)", "value": round(1 / t, 2),
-                "unit": "steps/s", "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
-                "config": {"workload": f"one_layer: d 2816, 16/8 heads x 128, 128 experts top-8 FFN 704, "
-                                       f"{n_seq} canvas(es) of 256 each behind a 4096-token prefix, "
-                                       f"{'fp8 e4m3 block-scaled' if args.fp8 else 'bf16'} weights"},
-                "kernel_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in stats.items() if v[0]}}
+        line = measure_one_layer(args.steps, args.warmup, args.seqs if args.seqs_given else 1, args.fp8)
+    elif args.workload == "head_sampler":
+        line = measure_head_sampler(args.steps, args.warmup, args.nv)
     else:
-        vocab, canvas = 262144, 256
-        logits, _ = synthetic.make_sampler_logits(canvas, vocab, seed=7, device=dev)
-        prm = dg.sampler_params(vocab, seed=7)
-        ws = torch.empty(dg.dg_sample_workspace_bytes(canvas, vocab), dtype=torch.uint8, device=dev)
-        ids = torch.zeros(canvas, dtype=torch.int32, device=dev)
-        commit = torch.zeros(canvas, dtype=torch.uint8, device=dev)
-        H = torch.empty(canvas, device=dev)
-        stop = torch.empty(1, dtype=torch.int32, device=dev)
-
-        def step():
-            commit.zero_()
-            dg.dg_sample(logits, 1, vocab, prm, 12, None, ids, commit, H, stop, ws)
-        t = _timed(step, args.steps, args.warmup)
-        hbm, _, kind = peaks()
-        gbs = canvas * vocab * 4 / t / 1e9
-        line = {"metric": "sampler steps/s (256 x 262144 fp32 logits)", "value": round(1 / t, 2), "unit": "steps/s",
-                "ms_per_step": round(t * 1e3, 4), "steps": args.steps, "warmup": args.warmup,
-                "config": {"workload": "sampler: logits N(0, 3^2), 10% of rows +12 spike, step 12 of 48, seed 7"},
-                "roofline": {"kernel": "sampler_partial + sampler_finalize (one dg_sample call)", "bound": "hbm",
-                             "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
-                             "traffic": SAMPLER_PARTIAL_TRAFFIC,
-                             "note": "includes the commit-mask reset (256 B); the kernel is instruction-bound "
-                                     "(one Philox word, an exp2 and two hardware logarithms per logit)"}}
+        line = measure_sampler(args.steps, args.warmup)
     print(json.dumps(line), flush=True)
 
 

@@ -15,7 +15,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdg.so")
-SOURCES = ["dg_api.cu", "gemm.cu", "attention.cu", "misc.cu", "sampler.cu", "sampler_noalloc.cu", "dequant.cu"]
+SOURCES = ["dg_api.cu", "gemm.cu", "attention.cu", "misc.cu", "sampler.cu", "sampler_noalloc.cu", "dequant.cu",
+           "head_sampler.cu", "expert_fp8.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -61,6 +61,7 @@ constexpr int kMaxSplits = 16;
 constexpr int kRouterSplits = 8;        // cluster size of the router GEMM's split-K
 constexpr int kGemmTargetCtas = 296;    // two CTAs per SM for the 128-wide dense GEMM tiles
 constexpr int kSplitKSlots = kGemmTargetCtas;   // split-K partial tiles: tiles x splits <= this (dense_splits)
+constexpr int kHeadSamplerMaxCtas = 256;        // CTAs of the fused head + sampler (one per SM)
 
 // Cluster size (power of two, <= 8) of the split-K dense GEMMs for `tiles` output tiles over nk
 // 64-deep k-blocks: enough CTAs for about two per SM, at least 4 k-blocks per CTA.
@@ -128,6 +129,26 @@ dg_status map_2d_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t col
   return DG_OK;
 }
 
+// 2-D bytes [rows][cols] (e4m3 operands of the tensor cores), box box_rows x 128 bytes, 128-byte swizzle
+// (the K-major layout kind::f8f6f4 reads: 128 K elements per 128-byte row).
+dg_status map_2d_u8_sw128(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || cols % 16)
+    return fail(DG_ERR_INVALID_ARG, "FP8 TMA operand not 16-byte aligned (ptr %p, row bytes %llu)", ptr,
+                (unsigned long long)cols);
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (2d u8 sw128, %llux%llu box %u) failed: %d",
+                                     (unsigned long long)rows, (unsigned long long)cols, box_rows, (int)r);
+  return DG_OK;
+}
+
 // 3-D bf16 [d2][d1][d0] (d0 contiguous), box {64, box1, 1}, 128-byte swizzle.
 dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
   EncodeTiledFn f = encode_fn();
@@ -149,7 +170,9 @@ dg_status map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
 struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, slot, xp, hb,
-      y, logits, samp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, total;
+      y, logits, samp, hsamp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, dstep, bsteps,
+      xq, xs, hq, hs, total;
+  bool f8mma;     // FP8 form with few tokens per expert: e4m3 activations for the e4m3 x e4m3 expert GEMMs
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
 
@@ -185,6 +208,17 @@ int attn_split_cap(const dg_model_config& c, int n_seq) {
   return best;
 }
 
+// Many tokens per expert on average (several canvases): 256-token accumulator chunks.  DG_EXPERT_WIDE
+// = 0 / 1 forces the narrow (32 or 64-token) / wide chunks for every row count (read once).
+bool expert_chunks_wide(const dg_model_config& c, int rows) {
+  static const int force = [] {
+    const char* v = getenv("DG_EXPERT_WIDE");
+    return v ? (atoi(v) != 0 ? 1 : 0) : -1;
+  }();
+  if (force >= 0) return force == 1;
+  return rows * c.top_k >= 128 * c.n_exp;
+}
+
 WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   WsLayout L{};
   L.R = n_seq * kCanvas;
@@ -217,6 +251,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.y = take(4 * A * d);
   L.logits = take(4 * R * (size_t)c.vocab);
   L.samp = take(4 * 8 * R * (size_t)L.chunks);
+  L.hsamp = take(4 * 8 * (size_t)kCanvas * kHeadSamplerMaxCtas);   // one canvas: the fused head's records
   L.rope = take(8 * (size_t)max_ctx * (dh / 2));
   L.cids = take(4 * R);
   L.ccommit = take(R);
@@ -226,10 +261,20 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.head_off = take(8);
   L.cursor = take(4 * 256);
   L.topk_done = take(64);
+  L.dstep = take(64);
+  L.bsteps = take(4 * ((size_t)max_ctx / kCanvas + 1));
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
     for (int i = 0; i < 3; ++i) L.wq[i] = take(2 * rows[i] * cols[i]);   // the expert GEMMs read e4m3 directly
+    // few tokens per expert: the expert GEMMs multiply e4m3 by e4m3 (quantized activations + scales)
+    L.f8mma = !expert_chunks_wide(c, L.R) && c.d_model % 128 == 0 && c.d_ff % 64 == 0;
+    if (L.f8mma) {
+      L.xq = take(A * d);
+      L.xs = take(4 * A * (d / 128));
+      L.hq = take(A * (size_t)c.d_ff);
+      L.hs = take(4 * A * (size_t)(c.d_ff / 64));
+    }
   }
 
   L.total = off + 1024;   // slack for base alignment
@@ -288,6 +333,7 @@ dg_status dg::check_sampler_params(const dg_sampler_params* p, int step, const c
 // ---------------------------------------------------------------------------------------------
 struct LayerMaps {
   CUtensorMap wqkv, wo, wrouter, wgu, wdown;
+  CUtensorMap wgu8, wdown8;   // FP8 form: the expert matrices with 128-byte swizzled boxes (e4m3 MMA)
 };
 
 struct dg_model {
@@ -311,7 +357,7 @@ struct dg_seqs {
   uint8_t* ws;
   // typed workspace views
   int *err, *seqP;
-  float *x, *opart, *ml, *rlog, *gate, *y, *logits, *samp, *splitk;
+  float *x, *opart, *ml, *rlog, *gate, *y, *logits, *samp, *hsamp, *splitk;
   __nv_bfloat16 *xn, *q, *attn, *xp, *hb;
   int32_t *sel, *counts, *offsets, *slot, *cids, *cstop;
   uint8_t* ccommit;
@@ -321,15 +367,30 @@ struct dg_seqs {
   CUtensorMap xn_map, xp_map, attn_map, hb_map, q_map, k_map, v_map;
   LayerMaps wmaps;              // FP8 form: descriptors of the bf16 scratch matrices
   CUtensorMap xn32_map;         // xn in 32-row boxes (token operand of the persistent head GEMM)
+  CUtensorMap xq_map, hq_map;   // FP8 form, few tokens per expert: e4m3 token operands (32-row boxes)
+  uint8_t *xq, *hq;             // ... the gathered rows and the SwiGLU rows in e4m3
+  float *xs, *hs;               // ... and their scales
+  bool fp8_native;              // use the e4m3 x e4m3 expert GEMMs where available (DG_FP8_NATIVE, default on)
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
   int32_t* topk_done;           // launch counter of the top-k kernel that also buckets
+  int* dstep;                   // the device-resident block loop: step index of the current block
+  int* bsteps;                  // ... and the step count of each block of a dg_decode call
+  int attn_plan_P;              // >= 0: plan the attention key splits for this committed length (a captured
+                                // step body serves every block of a decode call); -1: the current lengths
+  cudaStream_t cap_stream;      // private stream the decode loop's step body is captured on (lazily created)
+  int decode_graph;             // dg_decode runs each block's steps as a CUDA graph while-loop (DG_DECODE_GRAPH)
+  cudaGraphExec_t loop_exec;    // that graph, kept for later dg_decode calls with the same sampler settings
+  dg_sampler_params loop_prm;   // (its attention splits are planned for the largest committed length,
+                                // max_ctx - 256, so it serves every block of every call)
   __nv_bfloat16* wq[5];         // FP8 form: the scratch matrices (qkv, o, router, gate_up, down)
   std::vector<int> P;   // host mirror of the committed lengths
   int step;
   bool block_open;
   int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
   int pre_bytes;    // bytes per weight row the gate|up GEMM brings into L2 before its wait (DG_EXPERT_PREFETCH)
+  int head_nv;      // one canvas: vocabulary rows per item of the fused head + sampler (128 or 256; 0: the
+                    // head GEMM writes the logits and the standalone sampler reads them; DG_HEAD_SAMPLER)
   // statistics: launches per kernel class; optional event timing
   long long launches[DG_K_COUNT];
   double ms[DG_K_COUNT];
@@ -339,6 +400,11 @@ struct dg_seqs {
   int next_pair;
   ~dg_seqs() {
     for (cudaEvent_t e : events) cudaEventDestroy(e);
+    if (loop_exec) {
+      cudaStreamSynchronize(st);
+      cudaGraphExecDestroy(loop_exec);
+    }
+    if (cap_stream) cudaStreamDestroy(cap_stream);
   }
 };
 
@@ -431,6 +497,8 @@ DG_API dg_status dg_model_create(const dg_model_config* cfg, const dg_weights* w
     LayerMaps& M = m->maps[l];
     if ((st = map_2d_u8(&M.wgu, L.w_gate_up, (uint64_t)c.n_exp * 2 * c.d_ff, d, 64)) != DG_OK) break;
     if ((st = map_2d_u8(&M.wdown, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
+    if ((st = map_2d_u8_sw128(&M.wgu8, L.w_gate_up, (uint64_t)c.n_exp * 2 * c.d_ff, d, 64)) != DG_OK) break;
+    if ((st = map_2d_u8_sw128(&M.wdown8, L.w_down, (uint64_t)c.n_exp * d, c.d_ff, 128)) != DG_OK) break;
   }
   for (int l = 0; l < c.n_layers && st == DG_OK && !fp8; ++l) {
     const dg_layer_weights& L = m->layers[l];
@@ -512,6 +580,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->y = reinterpret_cast<float*>(b + L.y);
   s->logits = reinterpret_cast<float*>(b + L.logits);
   s->samp = reinterpret_cast<float*>(b + L.samp);
+  s->hsamp = reinterpret_cast<float*>(b + L.hsamp);
   s->rope = reinterpret_cast<float2*>(b + L.rope);
   s->cids = reinterpret_cast<int32_t*>(b + L.cids);
   s->ccommit = b + L.ccommit;
@@ -521,6 +590,20 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->head_off = reinterpret_cast<int32_t*>(b + L.head_off);
   s->cursor = reinterpret_cast<int32_t*>(b + L.cursor);
   s->topk_done = reinterpret_cast<int32_t*>(b + L.topk_done);
+  s->xq = L.f8mma ? b + L.xq : nullptr;
+  s->hq = L.f8mma ? b + L.hq : nullptr;
+  s->xs = L.f8mma ? reinterpret_cast<float*>(b + L.xs) : nullptr;
+  s->hs = L.f8mma ? reinterpret_cast<float*>(b + L.hs) : nullptr;
+  s->fp8_native = true;
+  if (const char* v = getenv("DG_FP8_NATIVE")) s->fp8_native = atoi(v) != 0;
+  s->dstep = reinterpret_cast<int*>(b + L.dstep);
+  s->bsteps = reinterpret_cast<int*>(b + L.bsteps);
+  s->attn_plan_P = -1;
+  s->cap_stream = nullptr;
+  s->loop_exec = nullptr;
+  memset(&s->loop_prm, 0, sizeof s->loop_prm);
+  s->decode_graph = 1;
+  if (const char* v = getenv("DG_DECODE_GRAPH")) s->decode_graph = atoi(v) != 0;
   for (int i = 0; i < 5; ++i) s->wq[i] = m->fp8 && i < 3 ? reinterpret_cast<__nv_bfloat16*>(b + L.wq[i]) : nullptr;
 
   s->P.assign(n_seq, 0);
@@ -535,6 +618,13 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->max_splits = kMaxSplits;
   if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
   s->pre_bytes = 1 << 20;   // capped at the row length: the whole first tile
+  s->head_nv = 128;
+  if (const char* v = getenv("DG_HEAD_SAMPLER")) {
+    const int nv = atoi(v);
+    s->head_nv = (nv == 0 || nv == 128 || nv == 256 || nv == kHeadSamplerPair) ? nv : 128;
+  }
+  if (c.vocab % 256 || (s->head_nv && head_sampler_ctas(c.vocab, s->head_nv, m->n_sms) > kHeadSamplerMaxCtas))
+    s->head_nv = 0;
   if (const char* v = getenv("DG_EXPERT_PREFETCH")) s->pre_bytes = std::max(0, atoi(v));
 
   const uint64_t d = c.d_model, R = L.R, A = L.A;
@@ -548,6 +638,10 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (st == DG_OK) st = map_2d(&s->q_map, s->q, (uint64_t)n_seq * c.n_q * kCanvas, c.d_head, 128);
   if (st == DG_OK) st = map_3d(&s->k_map, s->kc, c.d_head, max_ctx, zdim, 128);
   if (st == DG_OK) st = map_3d(&s->v_map, s->vt, max_ctx, c.d_head, zdim, c.d_head);
+  if (st == DG_OK && L.f8mma) {
+    st = map_2d_u8_sw128(&s->xq_map, s->xq, A, d, 32);
+    if (st == DG_OK) st = map_2d_u8_sw128(&s->hq_map, s->hq, A, c.d_ff, 32);
+  }
   if (st == DG_OK && m->fp8) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
@@ -591,8 +685,7 @@ DG_API dg_status dg_seqs_get_state(const dg_seqs* s, int* h_P, int* h_step) {
 
 DG_API float dg_temperature(const dg_sampler_params* p, int step) {
   if (!p) return 0.f;
-  const double frac = p->max_steps > 1 ? (double)step / (double)(p->max_steps - 1) : 0.0;
-  return (float)((double)p->t_start - ((double)p->t_start - (double)p->t_end) * frac);
+  return schedule_temperature(p->t_start, p->t_end, p->max_steps, step);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -654,6 +747,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   // attention over cache [0, P) + the Tq new rows
   int Pmax = 0;
   for (int i = 0; i < n_local; ++i) Pmax = std::max(Pmax, s->P[seq_base + i]);
+  if (s->attn_plan_P >= 0) Pmax = std::max(Pmax, s->attn_plan_P);   // splits beyond the keys stay empty
   const int ntiles = (Pmax + Tq + 127) / 128;
   AttnParams ap{};
   ap.n_q = c.n_q;
@@ -708,6 +802,33 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
            assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->slot,
                        &n_assign_k, st));
   }
+  const bool f8mma = fp8 && s->L.f8mma && s->fp8_native && !expert_chunks_wide(c, rows);
+  if (f8mma) {
+    // e4m3 x e4m3: the gathered rows quantized per 128 channels, the SwiGLU rows per 64 features
+    LAUNCH(s, DG_K_BUCKET, 1, gather_rows_q8(s->xn, s->slot, rows, c.top_k, d, s->xq, s->xs, st));
+    ExpertParams q{};
+    q.offsets = s->offsets;
+    q.d = d;
+    q.F = c.d_ff;
+    const LayerMaps& ME = s->m->maps[l];
+    ExpertParams qu = q, qd = q;
+    qu.w_scale = W.s_gate_up;
+    qu.w_scale_cols = (d + 127) / 128;
+    qu.a_scale = s->xs;
+    qu.a_scale_cols = d / 128;
+    qu.hq_out = s->hq;
+    qu.hs_out = s->hs;
+    qd.w_scale = W.s_down;
+    qd.w_scale_cols = (c.d_ff + 127) / 128;
+    qd.a_scale = s->hs;
+    qd.a_scale_cols = c.d_ff / 64;
+    qd.y_out = s->y;
+    LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert_f8(1, ME.wgu8, s->xq_map, qu, c.n_exp, s->m->n_sms, s->err, st));
+    LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert_f8(2, ME.wdown8, s->hq_map, qd, c.n_exp, s->m->n_sms, s->err, st));
+    LAUNCH(s, DG_K_COMBINE, 1,
+           moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
+    return DG_OK;
+  }
   LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
   ExpertParams xp{};
   xp.offsets = s->offsets;
@@ -716,7 +837,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   xp.d = d;
   xp.F = c.d_ff;
   // many tokens per expert on average (several canvases): 256-token accumulator chunks
-  const int wide = rows * c.top_k >= 128 * c.n_exp ? 1 : 0;
+  const int wide = expert_chunks_wide(c, rows) ? 1 : 0;
   const LayerMaps& ME = s->m->maps[l];   // expert weight descriptors: bf16, or e4m3 bytes in the FP8 form
   ExpertParams xu = xp, xd = xp;
   if (!fp8 && !wide && s->pre_bytes > 0) {
@@ -827,38 +948,16 @@ DG_API dg_status dg_canvas_init(dg_seqs* s, const dg_sampler_params* p, int32_t*
   return DG_OK;
 }
 
-DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit,
-                                float* d_entropy, int32_t* d_stop, float* d_hidden, float* d_logits_out) {
-  NvtxRange nvtx_range("dg_canvas_step");
-  if (!s || !d_ids || !d_commit || !d_entropy || !d_stop) return fail(DG_ERR_INVALID_ARG, "null argument");
-  dg_status r = check_params(s, p);
-  if (r != DG_OK) return r;
-  if (!s->block_open) return fail(DG_ERR_STATE, "no open canvas: call dg_canvas_init first");
-  const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
-  if (s->step >= budget) return fail(DG_ERR_STATE, "step budget of %d already used", budget);
+namespace {
+
+// The launches of one canvas step (layer stack, head, sampler).  d_step == nullptr: the step index and
+// temperature are host values (s->step); otherwise the kernels read the step index from *d_step (the
+// body of the device-resident block loop, which advances it on the device).
+dg_status issue_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit, float* d_entropy,
+                     int32_t* d_stop, float* d_hidden, float* d_logits_out, const int* d_step) {
   const dg_model_config& c = s->m->cfg;
-  r = run_canvas_stack(s, d_ids, d_hidden);   // leaves RMSNorm_final(x) in xn
+  dg_status r = run_canvas_stack(s, d_ids, d_hidden);   // leaves RMSNorm_final(x) in xn
   if (r != DG_OK) return r;
-  if (s->L.R <= kCanvas) {
-    // one canvas: the head as a persistent swap-AB GEMM (vocabulary rows are the 128-row side, the
-    // 256 canvas rows one 256-wide chunk), one CTA per SM, epilogues overlapping the weight stream
-    ExpertParams hp{};
-    hp.offsets = s->head_off;
-    hp.y_out = s->logits;
-    hp.d = c.vocab;        // output rows of the weight (logit columns)
-    hp.F = c.d_model;      // reduction length
-    LAUNCH(s, DG_K_HEAD, 1,
-           gemm_expert(2, s->m->head_map128, s->xn32_map, hp, 1, s->m->n_sms, 1, s->err, s->st));
-  } else {
-    EpiParams eh{};
-    eh.out = s->logits;
-    eh.ldo = c.vocab;
-    LAUNCH(s, DG_K_HEAD, 1,
-           gemm_dense(256, EPI_F32, s->xn_map, s->m->head_map, s->L.R, c.vocab, c.d_model, eh, s->err, s->st));
-  }
-  if (d_logits_out)
-    CK(cudaMemcpyAsync(d_logits_out, s->logits, sizeof(float) * (size_t)s->L.R * c.vocab, cudaMemcpyDeviceToDevice,
-                       s->st));
   SamplerArgs a{};
   a.logits = s->logits;
   a.n_seq = s->n_seq;
@@ -882,7 +981,71 @@ DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t*
   a.stop_mean_entropy = p->stop_mean_entropy;
   a.rerand_entropy = p->rerand_entropy;
   a.commit_rule = p->commit_rule;
+  a.d_step = d_step;
+  a.t_start = p->t_start;
+  a.t_end = p->t_end;
+  if (s->L.R == kCanvas && s->head_nv > 0) {
+    // one canvas: the head's logits folded into the sampler's per-row reductions tile by tile in
+    // TMEM (the logits reach HBM only as the optional debug copy), then the step rule
+    HeadSamplerArgs hs{};
+    hs.d = c.d_model;
+    hs.vocab = c.vocab;
+    hs.seq_P = s->seqP;
+    hs.commit_in = d_commit;
+    hs.inv_temp = a.inv_temp;
+    hs.seed = p->seed;
+    hs.step = s->step;
+    hs.partial = s->hsamp;
+    hs.logits_out = d_logits_out;
+    hs.d_step = d_step;
+    hs.t_start = p->t_start;
+    hs.t_end = p->t_end;
+    hs.max_steps = p->max_steps;
+    const int n_ctas = head_sampler_ctas(c.vocab, s->head_nv, s->m->n_sms);
+    a.partial = s->hsamp;
+    a.n_chunks = n_ctas;
+    LAUNCH(s, DG_K_HEAD, 2,
+           head_sampler_run(s->xn_map, s->head_nv == 256 ? s->m->head_map : s->m->head_map128, s->head_nv, hs, n_ctas,
+                            a, s->err, s->st));
+    return DG_OK;
+  }
+  if (s->L.R <= kCanvas) {
+    // one canvas: the head as a persistent swap-AB GEMM (vocabulary rows are the 128-row side, the
+    // 256 canvas rows one 256-wide chunk), one CTA per SM, epilogues overlapping the weight stream
+    ExpertParams hp{};
+    hp.offsets = s->head_off;
+    hp.y_out = s->logits;
+    hp.d = c.vocab;        // output rows of the weight (logit columns)
+    hp.F = c.d_model;      // reduction length
+    LAUNCH(s, DG_K_HEAD, 1,
+           gemm_expert(2, s->m->head_map128, s->xn32_map, hp, 1, s->m->n_sms, 1, s->err, s->st));
+  } else {
+    EpiParams eh{};
+    eh.out = s->logits;
+    eh.ldo = c.vocab;
+    LAUNCH(s, DG_K_HEAD, 1,
+           gemm_dense(256, EPI_F32, s->xn_map, s->m->head_map, s->L.R, c.vocab, c.d_model, eh, s->err, s->st));
+  }
+  if (d_logits_out)
+    CK(cudaMemcpyAsync(d_logits_out, s->logits, sizeof(float) * (size_t)s->L.R * c.vocab, cudaMemcpyDeviceToDevice,
+                       s->st));
   LAUNCH(s, DG_K_SAMPLER, 2, sampler_run(a, s->st));
+  return DG_OK;
+}
+
+}  // namespace
+
+DG_API dg_status dg_canvas_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uint8_t* d_commit,
+                                float* d_entropy, int32_t* d_stop, float* d_hidden, float* d_logits_out) {
+  NvtxRange nvtx_range("dg_canvas_step");
+  if (!s || !d_ids || !d_commit || !d_entropy || !d_stop) return fail(DG_ERR_INVALID_ARG, "null argument");
+  dg_status r = check_params(s, p);
+  if (r != DG_OK) return r;
+  if (!s->block_open) return fail(DG_ERR_STATE, "no open canvas: call dg_canvas_init first");
+  const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
+  if (s->step >= budget) return fail(DG_ERR_STATE, "step budget of %d already used", budget);
+  r = issue_step(s, p, d_ids, d_commit, d_entropy, d_stop, d_hidden, d_logits_out, nullptr);
+  if (r != DG_OK) return r;
   s->step += 1;
   return DG_OK;
 }
@@ -926,6 +1089,81 @@ DG_API dg_status dg_layer_forward(dg_seqs* s, int layer, int n_rows, int causal,
   return run_layer(s, layer, d_x, n_rows, 1, 0, n_rows, causal != 0, d_x_mid, d_router_logits);
 }
 
+namespace {
+
+// One block's step loop as a CUDA graph: a while-node whose body is one canvas step (every kernel reads
+// the step index from s->dstep) followed by the loop control, which advances the index and sets the
+// node's condition from the stop flags.  The graph runs the loop without the host: no read of the
+// stop flags and no launch per step.  The body is captured on a private stream (capture needs a
+// stream other than the legacy default) with the attention splits planned for plan_P, the largest
+// committed length the loop will see, so one graph serves every block of a decode call.
+dg_status build_step_loop(dg_seqs* s, const dg_sampler_params* p, int plan_P, cudaGraphExec_t* out) {
+  *out = nullptr;
+  const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
+  if (!s->cap_stream) CK(cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking));
+  cudaGraph_t g = nullptr;
+  CK(cudaGraphCreate(&g, 0));
+  cudaGraphConditionalHandle h;
+  cudaError_t e = cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault);   // the body runs once
+  cudaGraphNodeParams np = {};
+  cudaGraphNode_t node;
+  if (e == cudaSuccess) {
+    np.type = cudaGraphNodeTypeConditional;
+    np.conditional.handle = h;
+    np.conditional.type = cudaGraphCondTypeWhile;
+    np.conditional.size = 1;
+    e = cudaGraphAddNode(&node, g, nullptr, 0, &np);
+  }
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return fail(DG_ERR_CUDA, "decode loop graph: %s", cudaGetErrorString(e));
+  }
+  cudaGraph_t body = np.conditional.phGraph_out[0];
+  // capture the body: the launches go to the private stream, uncounted and untimed
+  cudaStream_t saved_st = s->st;
+  const bool saved_timing = s->timing;
+  long long saved_launches[DG_K_COUNT];
+  for (int k = 0; k < DG_K_COUNT; ++k) saved_launches[k] = s->launches[k];
+  s->st = s->cap_stream;
+  s->timing = false;
+  s->attn_plan_P = plan_P;
+  dg_status r = DG_OK;
+  e = cudaStreamBeginCaptureToGraph(s->st, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+  if (e == cudaSuccess) {
+    r = issue_step(s, p, s->cids, s->ccommit, s->cH, s->cstop, nullptr, nullptr, s->dstep);
+    if (r == DG_OK) {
+      const cudaError_t le = decode_loop_control(s->cstop, s->n_seq, s->dstep, budget, h, s->st);
+      if (le != cudaSuccess) r = fail(DG_ERR_CUDA, "decode loop control: %s", cudaGetErrorString(le));
+    }
+    cudaGraph_t captured = nullptr;
+    const cudaError_t ee = cudaStreamEndCapture(s->st, &captured);
+    if (r == DG_OK && ee != cudaSuccess) r = fail(DG_ERR_CUDA, "decode loop capture: %s", cudaGetErrorString(ee));
+  } else {
+    r = fail(DG_ERR_CUDA, "decode loop capture: %s", cudaGetErrorString(e));
+  }
+  s->st = saved_st;
+  s->timing = saved_timing;
+  s->attn_plan_P = -1;
+  for (int k = 0; k < DG_K_COUNT; ++k) s->launches[k] = saved_launches[k];
+  if (r == DG_OK) {
+    e = cudaGraphInstantiate(out, g, 0);
+    if (e != cudaSuccess) r = fail(DG_ERR_CUDA, "decode loop instantiate: %s", cudaGetErrorString(e));
+  }
+  cudaGraphDestroy(g);
+  return r;
+}
+
+// Conditional nodes need a driver of CUDA 12.4 or later.
+bool graph_loop_supported() {
+  static const int ok = [] {
+    int v = 0;
+    return cudaDriverGetVersion(&v) == cudaSuccess && v >= 12040 ? 1 : 0;
+  }();
+  return ok != 0;
+}
+
+}  // namespace
+
 DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_blocks, int32_t* d_out, int32_t* h_n_out,
                            int32_t* h_steps) {
   NvtxRange nvtx_range("dg_decode");
@@ -935,37 +1173,80 @@ DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_block
   const int n = s->n_seq;
   const int budget = p->fixed_steps > 0 ? p->fixed_steps : p->max_steps;
   const size_t out_stride = (size_t)max_blocks * kCanvas;
-  for (int i = 0; i < n; ++i)
+  int Pmax = 0;
+  for (int i = 0; i < n; ++i) {
     if (s->P[i] + max_blocks * kCanvas > s->max_ctx)
       return fail(DG_ERR_CAPACITY, "sequence %d: %d blocks do not fit (P=%d, max_ctx=%d)", i, max_blocks, s->P[i],
                   s->max_ctx);
+    Pmax = std::max(Pmax, s->P[i]);
+  }
+  (void)Pmax;
+  // device-resident step loop: one graph per sequence set and sampler settings, kept across calls
+  cudaGraphExec_t loop = nullptr;
+  if (s->decode_graph && graph_loop_supported()) {
+    if (s->loop_exec && memcmp(&s->loop_prm, p, sizeof *p) != 0) {
+      CK(cudaStreamSynchronize(s->st));
+      cudaGraphExecDestroy(s->loop_exec);
+      s->loop_exec = nullptr;
+    }
+    if (!s->loop_exec) {
+      r = build_step_loop(s, p, s->max_ctx - kCanvas, &s->loop_exec);
+      if (r != DG_OK) return r;
+      s->loop_prm = *p;
+    }
+    loop = s->loop_exec;
+  }
   std::vector<int32_t> h_stop(n), h_ids((size_t)n * kCanvas);
   std::vector<int> done(n, 0);
   for (int i = 0; i < n; ++i) h_n_out[i] = 0;
+  int blocks_run = 0;
   for (int b = 0; b < max_blocks; ++b) {
     r = dg_canvas_init(s, p, s->cids, s->ccommit);
-    if (r != DG_OK) return r;
+    if (r != DG_OK) break;
     int steps = 0;
-    for (;;) {
-      r = dg_canvas_step(s, p, s->cids, s->ccommit, s->cH, s->cstop, nullptr, nullptr);
-      if (r != DG_OK) return r;
-      ++steps;
-      CK(cudaMemcpyAsync(h_stop.data(), s->cstop, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s->st));
-      CK(cudaStreamSynchronize(s->st));
-      bool all = true;
-      for (int i = 0; i < n; ++i) all = all && h_stop[i] != 0;
-      if (all || steps >= budget) break;
+    if (loop) {
+      cudaError_t e = cudaMemsetAsync(s->dstep, 0, sizeof(int), s->st);
+      if (e == cudaSuccess) e = cudaGraphLaunch(loop, s->st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(s->bsteps + b, s->dstep, sizeof(int), cudaMemcpyDeviceToDevice, s->st);
+      if (e != cudaSuccess) {
+        r = fail(DG_ERR_CUDA, "decode loop launch: %s", cudaGetErrorString(e));
+        break;
+      }
+    } else {
+      for (;;) {
+        r = dg_canvas_step(s, p, s->cids, s->ccommit, s->cH, s->cstop, nullptr, nullptr);
+        if (r != DG_OK) break;
+        ++steps;
+        cudaError_t e = cudaMemcpyAsync(h_stop.data(), s->cstop, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s->st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s->st);
+        if (e != cudaSuccess) {
+          r = fail(DG_ERR_CUDA, "stop flags: %s", cudaGetErrorString(e));
+          break;
+        }
+        bool all = true;
+        for (int i = 0; i < n; ++i) all = all && h_stop[i] != 0;
+        if (all || steps >= budget) break;
+      }
+      if (r != DG_OK) break;
+      if (h_steps) h_steps[b] = steps;
     }
-    if (h_steps) h_steps[b] = steps;
+    ++blocks_run;
+    if (loop) s->step = budget;   // the graph ran the block's steps (their count is on the device)
     r = p->commit_mode == 1 ? dg_block_commit_last_kv(s) : dg_block_commit(s, s->cids);
-    if (r != DG_OK) return r;
-    CK(cudaMemcpy2DAsync(d_out + (size_t)b * kCanvas, out_stride * sizeof(int32_t), s->cids,
-                         kCanvas * sizeof(int32_t), kCanvas * sizeof(int32_t), n, cudaMemcpyDeviceToDevice, s->st));
-    bool all_done = true;
-    if (p->eos_id >= 0) {
-      CK(cudaMemcpyAsync(h_ids.data(), s->cids, sizeof(int32_t) * h_ids.size(), cudaMemcpyDeviceToHost, s->st));
-      CK(cudaStreamSynchronize(s->st));
+    if (r != DG_OK) break;
+    cudaError_t e = cudaMemcpy2DAsync(d_out + (size_t)b * kCanvas, out_stride * sizeof(int32_t), s->cids,
+                                      kCanvas * sizeof(int32_t), kCanvas * sizeof(int32_t), n, cudaMemcpyDeviceToDevice,
+                                      s->st);
+    if (e == cudaSuccess && p->eos_id >= 0) {
+      e = cudaMemcpyAsync(h_ids.data(), s->cids, sizeof(int32_t) * h_ids.size(), cudaMemcpyDeviceToHost, s->st);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(s->st);
     }
+    if (e != cudaSuccess) {
+      r = fail(DG_ERR_CUDA, "decode output: %s", cudaGetErrorString(e));
+      break;
+    }
+    bool all_done = true;
     for (int i = 0; i < n; ++i) {
       if (done[i]) continue;
       int take = kCanvas;
@@ -981,6 +1262,17 @@ DG_API dg_status dg_decode(dg_seqs* s, const dg_sampler_params* p, int max_block
     }
     if (all_done) break;
   }
+  if (loop) {
+    if (r == DG_OK && h_steps && blocks_run > 0) {
+      const cudaError_t e = cudaMemcpyAsync(h_steps, s->bsteps, sizeof(int32_t) * blocks_run, cudaMemcpyDeviceToHost,
+                                            s->st);
+      if (e != cudaSuccess) r = fail(DG_ERR_CUDA, "block step counts: %s", cudaGetErrorString(e));
+    }
+    const cudaError_t e = cudaStreamSynchronize(s->st);
+    if (r == DG_OK && e != cudaSuccess) r = fail(DG_ERR_CUDA, "decode: %s", cudaGetErrorString(e));
+    return r;
+  }
+  if (r != DG_OK) return r;
   CK(cudaStreamSynchronize(s->st));
   return DG_OK;
 }
@@ -1027,6 +1319,85 @@ DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg
   a.rerand_entropy = p->rerand_entropy;
   a.commit_rule = p->commit_rule;
   CK(sampler_run(a, static_cast<cudaStream_t>(stream)));
+  return DG_OK;
+}
+
+DG_API size_t dg_head_sample_workspace_bytes(int vocab) {
+  if (vocab <= 0 || vocab % 1024) return 0;
+  return (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas + 4 + 1024;   // partial records + error word
+}
+
+DG_API dg_status dg_head_sample(const void* d_xn, const void* d_head, int d_model, int vocab, int nv,
+                                const dg_sampler_params* p, int step, const int32_t* d_seq_P, int32_t* d_ids,
+                                uint8_t* d_commit, float* d_entropy, int32_t* d_stop, float* d_logits_out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dg_head_sample");
+  if (!d_xn || !d_head || !d_ids || !d_commit || !d_entropy || !d_stop || !ws)
+    return fail(DG_ERR_INVALID_ARG, "dg_head_sample: null argument");
+  if (d_model <= 0 || d_model % 64 || vocab <= 0 || vocab % 1024)
+    return fail(DG_ERR_INVALID_ARG, "dg_head_sample: d_model %% 64 == 0 and vocab %% 1024 == 0 needed");
+  if (nv != 128 && nv != 256 && nv != kHeadSamplerPair)
+    return fail(DG_ERR_INVALID_ARG, "dg_head_sample: nv must be 128, 256 or 2 (CTA pairs)");
+  if (step < 0) return fail(DG_ERR_INVALID_ARG, "dg_head_sample: bad step");
+  const dg_status ps = check_sampler_params(p, step, "dg_head_sample: ");
+  if (ps != DG_OK) return ps;
+  if (ws_bytes < dg_head_sample_workspace_bytes(vocab)) return fail(DG_ERR_CAPACITY, "dg_head_sample: workspace too small");
+  int dev = 0, n_sms = 148;
+  CK(cudaGetDevice(&dev));
+  CK(cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev));
+  CUtensorMap xn_map, head_map;
+  dg_status st = map_2d(&xn_map, d_xn, kCanvas, d_model, 128);
+  if (st == DG_OK) st = map_2d(&head_map, d_head, vocab, d_model, nv == kHeadSamplerPair ? 128 : nv);
+  if (st != DG_OK) return st;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  float* partial = reinterpret_cast<float*>(base);
+  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  CK(cudaMemsetAsync(err, 0, sizeof(int), cs));
+  const int n_ctas = std::min(head_sampler_ctas(vocab, nv, n_sms), kHeadSamplerMaxCtas);
+  HeadSamplerArgs hs{};
+  hs.d = d_model;
+  hs.vocab = vocab;
+  hs.seq_P = d_seq_P;
+  hs.commit_in = d_commit;
+  hs.inv_temp = 1.0f / dg_temperature(p, step);
+  hs.seed = p->seed;
+  hs.step = step;
+  hs.partial = partial;
+  hs.logits_out = d_logits_out;
+  SamplerArgs a{};
+  a.n_seq = 1;
+  a.canvas = kCanvas;
+  a.vocab = vocab;
+  a.n_chunks = n_ctas;
+  a.seq_P = d_seq_P;
+  a.ids_in = d_ids;
+  a.commit_in = d_commit;
+  a.ids_out = d_ids;
+  a.commit_out = d_commit;
+  a.entropy = d_entropy;
+  a.stop = d_stop;
+  a.partial = partial;
+  a.inv_temp = hs.inv_temp;
+  a.seed = p->seed;
+  a.step = step;
+  a.max_steps = p->max_steps;
+  a.fixed_steps = p->fixed_steps;
+  a.entropy_bound = p->entropy_bound;
+  a.stop_mean_entropy = p->stop_mean_entropy;
+  a.rerand_entropy = p->rerand_entropy;
+  a.commit_rule = p->commit_rule;
+  CK(head_sampler_run(xn_map, head_map, nv, hs, n_ctas, a, err, cs));
+  return DG_OK;
+}
+
+DG_API dg_status dg_head_sample_error(void* ws, void* stream, int* h_code) {
+  if (!ws || !h_code) return fail(DG_ERR_INVALID_ARG, "null argument");
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas);
+  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  CK(cudaMemcpy(h_code, err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (*h_code) return fail(DG_ERR_DEVICE, "device-side error code %d", *h_code);
   return DG_OK;
 }
 

@@ -93,6 +93,13 @@ struct ExpertParams {
   int w_scale_cols;      // 2-D, w_scale_cols tiles per row; nullptr for bf16 weights
   const void* w_base;    // bf16 weights [rows][K], and the bytes of each row of the CTA's first tile to
   int pre_bytes;         // bring into L2 before the grid-dependency wait (0: none; % 16 == 0)
+  // e4m3 activations (gemm_expert_f8): the token operand's scales [A][a_scale_cols] (MODE 1: per 128
+  // channels of the gathered rows; MODE 2: per 64 features of the SwiGLU rows), and MODE 1's output:
+  // SwiGLU rows in e4m3 [A][F] with one scale per (row, 64 features) [A][F/64]
+  const float* a_scale;
+  int a_scale_cols;
+  uint8_t* hq_out;
+  float* hs_out;
 };
 
 struct AttnParams {
@@ -116,6 +123,14 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
 // 256-token (else 64-token) accumulator chunks
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                         int n_ctas, int wide, int* err, cudaStream_t st);
+// e4m3 x e4m3 grouped expert GEMMs (expert_fp8.cu): chunks of 32 tokens, per-slice scale promotion;
+// w: e4m3 weights with 128-byte boxes (64 rows for MODE 1, 128 for MODE 2), x: e4m3 token rows, 32-row
+// boxes of 128 bytes, both 128-byte swizzled
+cudaError_t gemm_expert_f8(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
+                           int n_ctas, int* err, cudaStream_t st);
+// gather the normed rows into the bucketed order as e4m3 with one scale per (row, 128 channels)
+cudaError_t gather_rows_q8(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, uint8_t* xq,
+                           float* xs, cudaStream_t st);
 cudaError_t attention_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st);
 cudaError_t attention_merge(const AttnParams& p, int n_seq, __nv_bfloat16* out, cudaStream_t st);
@@ -150,6 +165,10 @@ cudaError_t load_prefix(const __nv_bfloat16* k_in, const __nv_bfloat16* v_in, in
                         __nv_bfloat16* kc, __nv_bfloat16* vt, cudaStream_t st);
 cudaError_t canvas_init_ids(const int* seq_P, int n_seq, int canvas, uint64_t seed, int vocab, int32_t* ids,
                             uint8_t* commit, cudaStream_t st);
+// body end of the device-resident block loop: *step += 1; the while-node condition = not all stopped and
+// *step < budget
+cudaError_t decode_loop_control(const int32_t* stop, int n_seq, int* step, int budget,
+                                cudaGraphConditionalHandle handle, cudaStream_t st);
 
 // sampler (sampler.cu)
 struct SamplerArgs {
@@ -168,8 +187,43 @@ struct SamplerArgs {
   int step, max_steps, fixed_steps;
   float entropy_bound, stop_mean_entropy, rerand_entropy;
   int commit_rule;       // 0 per-position entropy bound, 1 cumulative entropy bound
+  const int* d_step;     // nullable: the step index lives on the device (a step loop that runs without the
+  float t_start, t_end;  // host); step and inv_temp are then derived from *d_step on the schedule
 };
 cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st);
+// the finalize kernel alone (a.partial holds a.n_chunks records per row)
+cudaError_t sampler_finalize_run(const SamplerArgs& a, cudaStream_t st);
 int sampler_chunks(int vocab);
+
+// vocabulary head fused with the sampler's reductions, one canvas (head_sampler.cu)
+struct HeadSamplerArgs {
+  int d, vocab;
+  const int* seq_P;        // committed length of the sequence (device; nullptr -> 0)
+  const uint8_t* commit_in;
+  float inv_temp;
+  uint64_t seed;
+  int step;
+  float* partial;          // [256][n_ctas][8] per-row partial records (one per CTA)
+  float* logits_out;       // nullable: [256][vocab] fp32 copy of the logits
+  const int* d_step;       // nullable: step index on the device (see SamplerArgs)
+  float t_start, t_end;
+  int max_steps;
+};
+
+// Temperature of step s on the linear schedule, computed as the host's dg_temperature does (double
+// arithmetic, one rounding to fp32), and the sampler's 1 / T.
+__host__ __device__ inline float schedule_temperature(float t_start, float t_end, int max_steps, int s) {
+  const double frac = max_steps > 1 ? (double)s / (double)(max_steps - 1) : 0.0;
+  return (float)((double)t_start - ((double)t_start - (double)t_end) * frac);
+}
+// nv value selecting the CTA-pair form (tcgen05 cta_group::2, 256 vocabulary rows per pair item)
+constexpr int kHeadSamplerPair = 2;
+// CTAs of the fused head for nv vocabulary rows per item (one per SM, at most one per item; the pair
+// form: an even count, one pair per two SMs)
+int head_sampler_ctas(int vocab, int nv, int n_sms);
+// the fused head (xn_map: 128-row boxes of the normed rows; head_map: nv-row boxes of the head),
+// then the sampler's finalize with fin.partial = p.partial and fin.n_chunks = n_ctas
+cudaError_t head_sampler_run(const CUtensorMap& xn_map, const CUtensorMap& head_map, int nv, const HeadSamplerArgs& p,
+                             int n_ctas, const SamplerArgs& fin, int* err, cudaStream_t st);
 
 }  // namespace dg

@@ -487,4 +487,24 @@ cudaError_t canvas_init_ids(const int* seq_P, int n_seq, int canvas, uint64_t se
   return launch_k(canvas_init_kernel, dim3(n_seq), dim3(256), 0, st, 1, seq_P, canvas, seed, vocab, ids, commit);
 }
 
+// The adaptive-stop test of the block loop ("Composition of DiffusionGemma" flowchart: refine, check
+// the stop condition, refine again) on the device: after a step, advance the step index and let the
+// graph's while-node run the body again unless every sequence has stopped or the budget is spent.
+__global__ void decode_loop_control_kernel(const int32_t* __restrict__ stop, int n_seq, int* step, int budget,
+                                           cudaGraphConditionalHandle handle) {
+  pdl_trigger();
+  pdl_wait();
+  if (threadIdx.x != 0) return;
+  int all = 1;
+  for (int i = 0; i < n_seq; ++i) all &= stop[i] != 0;
+  const int s = *step + 1;
+  *step = s;
+  cudaGraphSetConditional(handle, (!all && s < budget) ? 1u : 0u);
+}
+
+cudaError_t decode_loop_control(const int32_t* stop, int n_seq, int* step, int budget,
+                                cudaGraphConditionalHandle handle, cudaStream_t st) {
+  return launch_k(decode_loop_control_kernel, dim3(1), dim3(32), 0, st, 1, stop, n_seq, step, budget, handle);
+}
+
 }  // namespace dg

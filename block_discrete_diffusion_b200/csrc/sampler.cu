@@ -65,9 +65,14 @@ __device__ __forceinline__ void best_merge(float& bs, int& bi, float os, int oi)
 __global__ void __launch_bounds__(kSampThreads)
     sampler_partial_kernel(const float* __restrict__ logits, int canvas, int vocab, int n_chunks,
                            const int* __restrict__ seq_P, const uint8_t* __restrict__ commit_in, float inv_temp,
-                           uint64_t seed, int step, float* __restrict__ partial) {
+                           uint64_t seed, int step, float* __restrict__ partial, const int* __restrict__ d_step,
+                           float t_start, float t_end, int max_steps) {
   pdl_trigger();
   pdl_wait();
+  if (d_step) {   // step index kept on the device: this step's index and temperature
+    step = *d_step;
+    inv_temp = __fdiv_rn(1.0f, schedule_temperature(t_start, t_end, max_steps, step));
+  }
   const int row = blockIdx.y, chunk = blockIdx.x;
   if (commit_in[row]) return;
   const int seq = row / canvas, j = row % canvas;
@@ -215,6 +220,7 @@ __global__ void __launch_bounds__(kSampThreads)
 __global__ void sampler_finalize_kernel(SamplerArgs a) {
   pdl_trigger();
   pdl_wait();
+  if (a.d_step) a.step = *a.d_step;
   __shared__ float red_h[32];
   __shared__ int red_c[32];
   const int seq = blockIdx.x;
@@ -340,8 +346,14 @@ cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st) {
   if (a.canvas > 4 * 256 || a.vocab % (4 * a.n_chunks) != 0) return cudaErrorInvalidValue;
   dim3 grid(a.n_chunks, a.n_seq * a.canvas);
   cudaError_t e = launch_k(sampler_partial_kernel, grid, dim3(kSampThreads), 0, st, 1, a.logits, a.canvas, a.vocab,
-                           a.n_chunks, a.seq_P, a.commit_in, a.inv_temp, a.seed, a.step, a.partial);
+                           a.n_chunks, a.seq_P, a.commit_in, a.inv_temp, a.seed, a.step, a.partial, a.d_step,
+                           a.t_start, a.t_end, a.max_steps);
   if (e != cudaSuccess) return e;
+  return sampler_finalize_run(a, st);
+}
+
+cudaError_t sampler_finalize_run(const SamplerArgs& a, cudaStream_t st) {
+  if (a.canvas > 4 * 256 || a.n_chunks <= 0) return cudaErrorInvalidValue;
   return launch_k(sampler_finalize_kernel, dim3(a.n_seq), dim3(256), 0, st, 1, a);
 }
 

@@ -24,7 +24,7 @@ ENTRY_POINTS = (
     "dg_seqs_destroy", "dg_seqs_get_state", "dg_load_prefix", "dg_prefill", "dg_canvas_init", "dg_canvas_step",
     "dg_block_commit", "dg_decode", "dg_layer_forward", "dg_sample_workspace_bytes", "dg_sample", "dg_device_error",
     "dg_temperature", "dg_stats_reset", "dg_stats_read", "dg_sample_noalloc", "dg_sample_noalloc_max_rows",
-    "dg_block_commit_last_kv",
+    "dg_block_commit_last_kv", "dg_head_sample_workspace_bytes", "dg_head_sample", "dg_head_sample_error",
 )
 
 # dg_kernel_class, in order
@@ -114,6 +114,11 @@ def lib():
                                         c_void_p, c_void_p, c_void_p, c_void_p]
         L.dg_sample_noalloc_max_rows.argtypes = [c_int]
         L.dg_sample_noalloc_max_rows.restype = c_size_t
+        L.dg_head_sample_workspace_bytes.argtypes = [c_int]
+        L.dg_head_sample_workspace_bytes.restype = c_size_t
+        L.dg_head_sample.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, P(dg_sampler_params), c_int, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+        L.dg_head_sample_error.argtypes = [c_void_p, c_void_p, P(c_int)]
         L.dg_device_error.argtypes = [c_void_p, P(c_int)]
         L.dg_stats_reset.argtypes = [c_void_p, c_int]
         L.dg_stats_read.argtypes = [c_void_p, c_void_p, c_void_p]
@@ -285,6 +290,26 @@ def dg_sample_noalloc(logits, n_seq, vocab, params, step, seq_P, ids, commit, en
 
 def dg_sample_noalloc_max_rows(vocab) -> int:
     return int(lib().dg_sample_noalloc_max_rows(vocab))
+
+
+def dg_head_sample_workspace_bytes(vocab) -> int:
+    return int(lib().dg_head_sample_workspace_bytes(vocab))
+
+
+def dg_head_sample(xn, head, params, step, seq_P, ids, commit, entropy, stop, ws, nv=128, logits=None, stream=None):
+    """The fused vocabulary head + sampler on caller inputs (xn bf16 [256, d], head bf16 [V, d])."""
+    _check("dg_head_sample", lib().dg_head_sample(_ptr(xn), _ptr(head), xn.shape[1], head.shape[0], nv,
+                                                  ctypes.byref(params), step, _ptr(seq_P), _ptr(ids), _ptr(commit),
+                                                  _ptr(entropy), _ptr(stop), _ptr(logits), _ptr(ws), ws.numel(),
+                                                  _stream_handle(stream)))
+
+
+def dg_head_sample_error(ws, stream=None) -> int:
+    code = c_int()
+    st = lib().dg_head_sample_error(_ptr(ws), _stream_handle(stream), ctypes.byref(code))
+    if st not in (DG_OK, DG_ERR_DEVICE):
+        _check("dg_head_sample_error", st)
+    return code.value
 
 
 def dg_device_error(seqs: Seqs) -> int:

@@ -18,8 +18,8 @@
  *    outputs), typically allocated through PyTorch.  The library allocates no device memory; its
  *    handles are small host structures.  Every pointer named d_* is device memory; h_* is host.
  *  - Asynchrony: every call is enqueued on the stream given to dg_seqs_create and returns without
- *    waiting, except dg_decode (one 4-byte-per-sequence read of the stop flags per step) and
- *    dg_device_error (synchronises the stream).
+ *    waiting, except dg_decode (synchronises once at the end, and once per block to find an EOS)
+ *    and dg_device_error (synchronises the stream).
  *  - Errors: arguments and state are checked on the host before any launch; nothing traps on the
  *    device.  A kernel that sees a bad index or whose pipeline wait runs out records a code that
  *    dg_device_error returns (DG_ERR_DEVICE).  dg_last_error() gives a message for the last non-OK
@@ -189,7 +189,13 @@ dg_status dg_block_commit_last_kv(dg_seqs *s);
  * dg_canvas_step until every sequence's stop flag is set (sequences that stopped keep their ids),
  * dg_block_commit; a sequence ends after the block that contains eos_id (its output cut after the
  * first EOS).  d_out int32 [n_seq][max_blocks*256] receives the committed tokens, h_n_out[n_seq]
- * their counts.  h_steps (nullable) [max_blocks] receives the step count of each block. */
+ * their counts.  h_steps (nullable) [max_blocks] receives the step count of each block.
+ * The steps of a block run on the device without the host: a CUDA graph whose while-node repeats
+ * one canvas step (step index and temperature kept on the device) until every stop flag is set or
+ * the budget is spent (the adaptive-stop test of the flowchart).  The graph is built on the first
+ * call (driver 12.4+; captured on a private stream) and kept in the handle for later calls with
+ * the same sampler settings.  The host reads the ids once per block only when eos_id >= 0, and
+ * synchronises once at the end. */
 dg_status dg_decode(dg_seqs *s, const dg_sampler_params *p, int max_blocks, int32_t *d_out, int32_t *h_n_out,
                     int32_t *h_steps);
 
@@ -232,6 +238,26 @@ dg_status dg_sample_noalloc(const float *d_logits, int n_seq, int vocab, const d
 /* Largest n_seq * 256 that dg_sample_noalloc accepts for this vocabulary size (0 for a vocabulary
  * the sampler rejects: vocab <= 0 or vocab % 1024 != 0). */
 size_t dg_sample_noalloc_max_rows(int vocab);
+
+/* The vocabulary head fused with the sampler, on caller inputs, for one canvas: logits
+ * l = xn head^T (d_xn bf16 [256][d_model], the final-normed canvas rows; d_head bf16
+ * [vocab][d_model]) computed tile by tile in tensor memory and folded into the sampler's per-row
+ * reductions without being written to memory, then the step rule of `step` as in dg_sample
+ * (d_seq_P nullable: the sequence's committed length, 0 if NULL; ids / commit in/out, entropy and
+ * stop out).  This is the head + sampler of dg_canvas_step at one canvas ([guide] "Serving with
+ * vLLM": the entropy_bound sampler runs on the head's output every step).  nv: the tiling -- 128 or
+ * 256 vocabulary rows per tile on one SM, or 2: pairs of SMs (256 vocabulary rows per pair tile, the
+ * pair's tensor cores multiplying all 256 canvas rows at once).  d_logits_out (nullable): fp32
+ * [256][vocab] copy of the logits.  ws: device
+ * scratch of dg_head_sample_workspace_bytes(vocab) bytes; a device-side error (a pipeline wait
+ * that ran out) is recorded there and returned by dg_head_sample_error, which synchronises the
+ * stream.  Buffers 16-byte aligned; d_model % 64 == 0, vocab % 1024 == 0. */
+size_t dg_head_sample_workspace_bytes(int vocab);
+dg_status dg_head_sample(const void *d_xn, const void *d_head, int d_model, int vocab, int nv,
+                         const dg_sampler_params *p, int step, const int32_t *d_seq_P, int32_t *d_ids,
+                         uint8_t *d_commit, float *d_entropy, int32_t *d_stop, float *d_logits_out, void *ws,
+                         size_t ws_bytes, void *stream);
+dg_status dg_head_sample_error(void *ws, void *stream, int *h_code);
 
 /* Synchronise the handle's stream and return the first device-side error code recorded since the
  * last call (0 = none) in *h_code; the record is cleared.  Returns DG_ERR_DEVICE if non-zero. */
