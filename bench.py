@@ -219,6 +219,9 @@ def run_steps(dg, seqs, prm, st, k, state):
 # routed), from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of this kernel:
 # 1,028,473,600 + 3,732,224.  Set to None when the kernel changes until it is captured again.
 EXPERT_UP_TRAFFIC_BF16 = 1_028_473_600 + 3_732_224
+# DRAM bytes (read + write) of one merged gate|up -> down launch at batch 1 (bf16), from an ncu capture of
+# that kernel on the one-layer workload; None until captured.
+EXPERT_UPDOWN_TRAFFIC_BF16 = None
 
 # DRAM bytes (read + write) of one sampler_partial_kernel launch on the 256 x 262144 sampler workload,
 # from an ncu capture of this kernel: 268,503,552 + 3,422,720.  None when the kernel changes until it is
@@ -230,11 +233,24 @@ def expert_up_bytes(cfg):
     """Algorithmic bytes of one grouped gate|up launch at batch 1: every expert's [2F x d] weights
     (bf16, or e4m3 bytes plus one fp32 scale per 128x128 tile; all 128 experts are routed to with
     probability 1 - 128*(120/128)^256 > 0.99999), the gathered activations read once, the SwiGLU
-    rows written once."""
+    rows written once (bf16; e4m3 with a scale per 64 features in the FP8 form)."""
     A = CANVAS * cfg.top_k
     n_w = cfg.n_exp * 2 * cfg.d_ff * cfg.d_model
-    w_bytes = n_w + 4 * (n_w // (128 * 128)) if getattr(cfg, "wdtype", 0) == 1 else 2 * n_w
-    return w_bytes + A * cfg.d_model * 2 + A * cfg.d_ff * 2
+    if getattr(cfg, "wdtype", 0) == 1:
+        return n_w + 4 * (n_w // (128 * 128)) + A * cfg.d_model + 4 * A * (cfg.d_model // 128) + A * cfg.d_ff \
+            + 4 * A * (cfg.d_ff // 64)
+    return 2 * n_w + A * cfg.d_model * 2 + A * cfg.d_ff * 2
+
+
+def expert_down_bytes(cfg):
+    """Algorithmic bytes of the grouped down projection at batch 1: every expert's [d x F] weights, the
+    SwiGLU rows read once, the fp32 expert outputs written once."""
+    A = CANVAS * cfg.top_k
+    n_w = cfg.n_exp * cfg.d_model * cfg.d_ff
+    if getattr(cfg, "wdtype", 0) == 1:
+        return n_w + 4 * (-(-cfg.n_exp * cfg.d_model // 128) * -(-cfg.d_ff // 128)) + A * cfg.d_ff \
+            + 4 * A * (cfg.d_ff // 64) + 4 * A * cfg.d_model
+    return 2 * n_w + 2 * A * cfg.d_ff + 4 * A * cfg.d_model
 
 
 def main_dg(args):
@@ -292,11 +308,13 @@ def main_dg(args):
     dominant = max(stats, key=lambda k: stats[k][1])
     hbm, tflops, peak_kind = peaks()
     up_launch_s = stats["expert_up"][1] / 1e3 / max(stats["expert_up"][0], 1)
-    up_bytes = expert_up_bytes(cfg)
-    roofline = {"kernel": "expert_up (grouped gate|up GEMM + SwiGLU)", "bound": "hbm",
+    merged = stats["expert_down"][0] == 0           # gate|up and down in one launch (bf16, batch 1)
+    up_bytes = expert_up_bytes(cfg) + (expert_down_bytes(cfg) if merged else 0)
+    roofline = {"kernel": ("expert_updown (grouped gate|up + SwiGLU, then down, one persistent launch)" if merged
+                           else "expert_up (grouped gate|up GEMM + SwiGLU)"), "bound": "hbm",
                 "achieved": round(up_bytes / up_launch_s / 1e9, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(up_bytes / up_launch_s / 1e9 / hbm, 4),
-                "traffic": None if args.fp8 else EXPERT_UP_TRAFFIC_BF16,
+                "traffic": (EXPERT_UPDOWN_TRAFFIC_BF16 if merged else None) if not args.fp8 else None,
                 "algorithmic_bytes_per_launch": up_bytes, "launch_ms": round(up_launch_s * 1e3, 4),
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind,
                 "dominant_by_time": dominant}

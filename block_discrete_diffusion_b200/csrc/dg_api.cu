@@ -171,7 +171,7 @@ struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, slot, xp, hb,
       y, logits, samp, hsamp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, dstep, bsteps,
-      xq, xs, hq, hs, total;
+      xq, xs, hq, hs, xdone, total;
   bool f8mma;     // FP8 form with few tokens per expert: e4m3 activations for the e4m3 x e4m3 expert GEMMs
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
@@ -251,7 +251,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.y = take(4 * A * d);
   L.logits = take(4 * R * (size_t)c.vocab);
   L.samp = take(4 * 8 * R * (size_t)L.chunks);
-  L.hsamp = take(4 * 8 * (size_t)kCanvas * kHeadSamplerMaxCtas);   // one canvas: the fused head's records
+  L.hsamp = take(4 * 8 * (size_t)kCanvas * (kHeadSamplerMaxCtas + 1));   // one canvas: the fused head's records
   L.rope = take(8 * (size_t)max_ctx * (dh / 2));
   L.cids = take(4 * R);
   L.ccommit = take(R);
@@ -262,6 +262,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.cursor = take(4 * 256);
   L.topk_done = take(64);
   L.dstep = take(64);
+  L.xdone = take(4 * (size_t)c.n_exp);
   L.bsteps = take(4 * ((size_t)max_ctx / kCanvas + 1));
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
@@ -371,6 +372,8 @@ struct dg_seqs {
   uint8_t *xq, *hq;             // ... the gathered rows and the SwiGLU rows in e4m3
   float *xs, *hs;               // ... and their scales
   bool fp8_native;              // use the e4m3 x e4m3 expert GEMMs where available (DG_FP8_NATIVE, default on)
+  int32_t* xdone;               // per-expert count of finished gate|up tiles (merged expert launch)
+  bool expert_merged;           // bf16, narrow chunks: gate|up and down in one launch (DG_EXPERT_MERGED, default on)
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
   int32_t* topk_done;           // launch counter of the top-k kernel that also buckets
@@ -389,8 +392,9 @@ struct dg_seqs {
   bool block_open;
   int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
   int pre_bytes;    // bytes per weight row the gate|up GEMM brings into L2 before its wait (DG_EXPERT_PREFETCH)
-  int head_nv;      // one canvas: vocabulary rows per item of the fused head + sampler (128 or 256; 0: the
-                    // head GEMM writes the logits and the standalone sampler reads them; DG_HEAD_SAMPLER)
+  int head_nv;      // one canvas: tiling of the fused head + sampler (kHeadSamplerPair: CTA pairs; 128 or 256
+                    // vocabulary rows per single-SM tile; 0: the head GEMM writes the logits and the
+                    // standalone sampler reads them; DG_HEAD_SAMPLER)
   // statistics: launches per kernel class; optional event timing
   long long launches[DG_K_COUNT];
   double ms[DG_K_COUNT];
@@ -596,6 +600,9 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->hs = L.f8mma ? reinterpret_cast<float*>(b + L.hs) : nullptr;
   s->fp8_native = true;
   if (const char* v = getenv("DG_FP8_NATIVE")) s->fp8_native = atoi(v) != 0;
+  s->xdone = reinterpret_cast<int32_t*>(b + L.xdone);
+  s->expert_merged = true;
+  if (const char* v = getenv("DG_EXPERT_MERGED")) s->expert_merged = atoi(v) != 0;
   s->dstep = reinterpret_cast<int*>(b + L.dstep);
   s->bsteps = reinterpret_cast<int*>(b + L.bsteps);
   s->attn_plan_P = -1;
@@ -618,10 +625,10 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->max_splits = kMaxSplits;
   if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
   s->pre_bytes = 1 << 20;   // capped at the row length: the whole first tile
-  s->head_nv = 128;
+  s->head_nv = kHeadSamplerPair;   // CTA pairs: the fastest form measured on B200 (0.44 vs 0.47 ms at V 262144)
   if (const char* v = getenv("DG_HEAD_SAMPLER")) {
     const int nv = atoi(v);
-    s->head_nv = (nv == 0 || nv == 128 || nv == 256 || nv == kHeadSamplerPair) ? nv : 128;
+    s->head_nv = (nv == 0 || nv == 128 || nv == 256 || nv == kHeadSamplerPair) ? nv : kHeadSamplerPair;
   }
   if (c.vocab % 256 || (s->head_nv && head_sampler_ctas(c.vocab, s->head_nv, m->n_sms) > kHeadSamplerMaxCtas))
     s->head_nv = 0;
@@ -829,15 +836,17 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
            moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
     return DG_OK;
   }
-  LAUNCH(s, DG_K_BUCKET, 1, gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st));
+  // many tokens per expert on average (several canvases): 256-token accumulator chunks
+  const int wide = expert_chunks_wide(c, rows) ? 1 : 0;
+  const bool merged = !fp8 && !wide && s->expert_merged;
+  LAUNCH(s, DG_K_BUCKET, 1,
+         gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st, merged ? s->xdone : nullptr, c.n_exp));
   ExpertParams xp{};
   xp.offsets = s->offsets;
   xp.h_out = s->hb;
   xp.y_out = s->y;
   xp.d = d;
   xp.F = c.d_ff;
-  // many tokens per expert on average (several canvases): 256-token accumulator chunks
-  const int wide = expert_chunks_wide(c, rows) ? 1 : 0;
   const LayerMaps& ME = s->m->maps[l];   // expert weight descriptors: bf16, or e4m3 bytes in the FP8 form
   ExpertParams xu = xp, xd = xp;
   if (!fp8 && !wide && s->pre_bytes > 0) {
@@ -850,8 +859,17 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
     xd.w_scale = W.s_down;
     xd.w_scale_cols = (c.d_ff + 127) / 128;
   }
-  LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, ME.wgu, s->xp_map, xu, c.n_exp, s->m->n_sms, wide, s->err, st));
-  LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, ME.wdown, s->hb_map, xd, c.n_exp, s->m->n_sms, wide, s->err, st));
+  if (merged) {
+    // gate|up, then down, in one persistent launch (counted as the gate|up class)
+    ExpertParams xm = xp;
+    xm.w_base = xu.w_base;
+    xm.pre_bytes = xu.pre_bytes;
+    LAUNCH(s, DG_K_EXPERT_UP, 1,
+           gemm_expert_updown(ME.wgu, s->xp_map, ME.wdown, s->hb_map, xm, c.n_exp, s->m->n_sms, s->xdone, s->err, st));
+  } else {
+    LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert(1, ME.wgu, s->xp_map, xu, c.n_exp, s->m->n_sms, wide, s->err, st));
+    LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert(2, ME.wdown, s->hb_map, xd, c.n_exp, s->m->n_sms, wide, s->err, st));
+  }
   LAUNCH(s, DG_K_COMBINE, 1, moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
   return DG_OK;
 }
@@ -1004,7 +1022,7 @@ dg_status issue_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uin
     const int n_ctas = head_sampler_ctas(c.vocab, s->head_nv, s->m->n_sms);
     a.partial = s->hsamp;
     a.n_chunks = n_ctas;
-    LAUNCH(s, DG_K_HEAD, 2,
+    LAUNCH(s, DG_K_HEAD, 3,
            head_sampler_run(s->xn_map, s->head_nv == 256 ? s->m->head_map : s->m->head_map128, s->head_nv, hs, n_ctas,
                             a, s->err, s->st));
     return DG_OK;
@@ -1324,7 +1342,7 @@ DG_API dg_status dg_sample(const float* d_logits, int n_seq, int vocab, const dg
 
 DG_API size_t dg_head_sample_workspace_bytes(int vocab) {
   if (vocab <= 0 || vocab % 1024) return 0;
-  return (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas + 4 + 1024;   // partial records + error word
+  return (size_t)4 * 8 * kCanvas * (kHeadSamplerMaxCtas + 1) + 4 + 1024;   // partial + merged records, error word
 }
 
 DG_API dg_status dg_head_sample(const void* d_xn, const void* d_head, int d_model, int vocab, int nv,
@@ -1351,7 +1369,7 @@ DG_API dg_status dg_head_sample(const void* d_xn, const void* d_head, int d_mode
   if (st != DG_OK) return st;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   float* partial = reinterpret_cast<float*>(base);
-  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas);
+  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * (kHeadSamplerMaxCtas + 1));
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   CK(cudaMemsetAsync(err, 0, sizeof(int), cs));
   const int n_ctas = std::min(head_sampler_ctas(vocab, nv, n_sms), kHeadSamplerMaxCtas);
@@ -1394,7 +1412,7 @@ DG_API dg_status dg_head_sample(const void* d_xn, const void* d_head, int d_mode
 DG_API dg_status dg_head_sample_error(void* ws, void* stream, int* h_code) {
   if (!ws || !h_code) return fail(DG_ERR_INVALID_ARG, "null argument");
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
-  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * kHeadSamplerMaxCtas);
+  int* err = reinterpret_cast<int*>(base + (size_t)4 * 8 * kCanvas * (kHeadSamplerMaxCtas + 1));
   CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   CK(cudaMemcpy(h_code, err, sizeof(int), cudaMemcpyDeviceToHost));
   if (*h_code) return fail(DG_ERR_DEVICE, "device-side error code %d", *h_code);

@@ -123,6 +123,11 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
 // 256-token (else 64-token) accumulator chunks
 cudaError_t gemm_expert(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                         int n_ctas, int wide, int* err, cudaStream_t st);
+// gate|up (MODE 1 items, then) down (MODE 2 items) in one persistent launch, bf16 weights, 64-token
+// chunks: wu/x as gemm_expert mode 1, wd/h as mode 2; done[n_exp] zeroed before the launch (a down item
+// of expert e waits until done[e] counts e's F/64 gate|up tiles); one CTA per SM, all resident
+cudaError_t gemm_expert_updown(const CUtensorMap& wu, const CUtensorMap& x, const CUtensorMap& wd, const CUtensorMap& h,
+                               const ExpertParams& p, int n_exp, int n_ctas, int* done, int* err, cudaStream_t st);
 // e4m3 x e4m3 grouped expert GEMMs (expert_fp8.cu): chunks of 32 tokens, per-slice scale promotion;
 // w: e4m3 weights with 128-byte boxes (64 rows for MODE 1, 128 for MODE 2), x: e4m3 token rows, 32-row
 // boxes of 128 bytes, both 128-byte swizzled
@@ -154,8 +159,9 @@ cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, in
 // expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
                         int32_t* offsets, int32_t* cursor, int32_t* slot, int* n_launched, cudaStream_t st);
+// zero (nullable): n_zero ints set to 0 by the launch (the expert kernels' per-launch counters)
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
-                        cudaStream_t st);
+                        cudaStream_t st, int32_t* zero = nullptr, int n_zero = 0);
 // g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g
 cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x, const float* g,
                         float eps, __nv_bfloat16* xn, cudaStream_t st);
@@ -193,6 +199,9 @@ struct SamplerArgs {
 cudaError_t sampler_run(const SamplerArgs& a, cudaStream_t st);
 // the finalize kernel alone (a.partial holds a.n_chunks records per row)
 cudaError_t sampler_finalize_run(const SamplerArgs& a, cudaStream_t st);
+// many records per row: one warp per row merges a.partial's a.n_chunks records into merged [rows][8], then
+// the finalize runs on the merged records
+cudaError_t sampler_premerge_finalize_run(const SamplerArgs& a, float* merged, cudaStream_t st);
 int sampler_chunks(int vocab);
 
 // vocabulary head fused with the sampler's reductions, one canvas (head_sampler.cu)
@@ -203,7 +212,7 @@ struct HeadSamplerArgs {
   float inv_temp;
   uint64_t seed;
   int step;
-  float* partial;          // [256][n_ctas][8] per-row partial records (one per CTA)
+  float* partial;          // [256][n_ctas][8] per-row partial records (one per CTA), then [256][8] merged ones
   float* logits_out;       // nullable: [256][vocab] fp32 copy of the logits
   const int* d_step;       // nullable: step index on the device (see SamplerArgs)
   float t_start, t_end;

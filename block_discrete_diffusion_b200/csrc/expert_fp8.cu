@@ -11,9 +11,10 @@
 // while the next slices run.  Against the bf16 path this halves the weight bytes streamed from HBM
 // (the bound at these token counts) and needs no expansion of the weights to bf16.
 //
-// Roles (192 threads): warp 0 TMA producer (e4m3 weight tile 128 rows x 128 bytes and the chunk's
-// 32 token rows x 128 bytes per stage, 128-byte swizzle), warp 1 MMA issuer, warps 2-5 promotion and
-// epilogue.  MODE 1: gate|up rows of one expert (64 + 64 rows) times its tokens, SwiGLU in the
+// Roles (320 threads): warp 0 TMA producer (e4m3 weight tile 128 rows x 128 bytes and the chunk's
+// 32 token rows x 128 bytes per stage, 128-byte swizzle), warp 1 MMA issuer, warps 2-9 promotion and
+// epilogue (two warps per TMEM lane quadrant, 16 token columns each; per chunk one table of the
+// combined scales s_w * s_a, so a slice costs a TMEM load and one FMA per column).  MODE 1: gate|up rows of one expert (64 + 64 rows) times its tokens, SwiGLU in the
 // epilogue, the result quantized per (token, 64 features) to e4m3 for the down GEMM; MODE 2: down
 // rows (128) times the tokens' SwiGLU rows, fp32 outputs for the combine.
 //
@@ -30,7 +31,8 @@ namespace dg {
 
 namespace {
 
-constexpr int kF8Threads = 192;
+constexpr int kF8Threads = 320;                    // warps 0 (TMA), 1 (MMA), 2-9 (promotion + epilogue)
+constexpr int kF8EpiThreads = 256;
 constexpr int kF8BN = 32;                          // token columns per chunk
 constexpr uint32_t kF8WTile = 128 * 128;           // 128 weight rows x 128 bytes of K
 constexpr uint32_t kF8XTile = kF8BN * 128;         // 32 token rows x 128 bytes of K
@@ -41,7 +43,7 @@ constexpr int kF8Slices = 16;                      // TMEM slice buffers of 32 c
 constexpr int kF8MaxSl = 64;                       // scale blocks per token row (d / 128 or F / 64)
 constexpr int kF8EpiStride = kF8BN + 1;
 constexpr size_t kF8Smem = 1024 + (size_t)kF8Stages * kF8Stage + 128 * kF8EpiStride * 4 +
-                           (size_t)kF8BN * kF8MaxSl * 4 + 2 * 32 * 4 + 512;
+                           2 * (size_t)kF8BN * kF8MaxSl * 4 + 512;
 static_assert(kF8Smem <= 232448, "shared memory budget");
 
 struct F8Barriers {
@@ -68,7 +70,22 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-__device__ __forceinline__ void f8_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void f8_epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive fp32 columns of TMEM (thread `lane` of warp w: lane 32 (w % 4) + lane).
+__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 // Two floats to two e4m3 bytes (round to nearest even, saturating to +-448).
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
@@ -83,9 +100,9 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   pdl_trigger();
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kF8Stages * kF8Stage);
-  float* sa_s = stage_out + 128 * kF8EpiStride;                 // [32 tokens][kF8MaxSl] activation scales
-  float* sw_s = sa_s + kF8BN * kF8MaxSl;                        // [2][32] the item's weight scales per K block
-  F8Barriers* bars = reinterpret_cast<F8Barriers*>(sw_s + 2 * 32);
+  // [2][kF8MaxSl][32 tokens] combined scales s_w * s_a per (weight-row half, slice, token) of a chunk
+  float* cs_s = stage_out + 128 * kF8EpiStride;
+  F8Barriers* bars = reinterpret_cast<F8Barriers*>(cs_s + 2 * kF8BN * kF8MaxSl);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = MODE == 1 ? p.d : p.F;
   const int nkb = (K + 127) / 128;                              // 128-byte K stages
@@ -100,7 +117,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     }
     for (int s = 0; s < kF8Slices; ++s) {
       mbar_init(&bars->sfull[s], 1);
-      mbar_init(&bars->sempty[s], 4);
+      mbar_init(&bars->sempty[s], 8);
     }
     fence_mbar_init();
   }
@@ -188,83 +205,91 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       }
     }
   } else {
-    // ------------------------------ promotion + epilogue (warps 2-5) ------------------------------
+    // ------------------------------ promotion + epilogue (warps 2-9) ------------------------------
+    // Warps w and w + 4 read the same TMEM lanes (weight rows 32 (w % 4) ..) and split the chunk's 32
+    // token columns: columns 16 ch .. 16 ch + 15 with ch = (w - 2) / 4.
     const int quarter = warp & 3;                 // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int ch = (warp - 2) >> 2;               // token-column half
     const int r = quarter * 32 + lane;            // weight row of the tile
-    const int et = threadIdx.x - 64;              // 0..127 among the epilogue threads
+    const int et = threadIdx.x - 64;              // 0..255 among the epilogue threads
+    const int half_row = MODE == 1 && r >= 64 ? 1 : 0;   // gate (0) or up (1) rows in MODE 1
     uint32_t g = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const int e = item / MT, mt = item % MT;
       const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
-      // weight scales of the item per K block (MODE 1: the gate half [0] and the up half [1] sit in
-      // different 128-row tiles) and the chunk's activation scales go to shared memory once, off the
-      // per-slice path
       const int nwb = p.w_scale_cols;
       for (int c0 = 0; c0 < n_e; c0 += kF8BN) {
         const int nc = min(kF8BN, n_e - c0);
-        f8_epi_sync();                            // the previous chunk is done with sa_s, sw_s and stage_out
-        for (int i = et; i < kF8BN * nsl; i += 128) {
-          const int n = i / nsl, b = i % nsl;
-          sa_s[n * kF8MaxSl + b] = n < nc ? __ldg(p.a_scale + (size_t)(off + c0 + n) * p.a_scale_cols + b) : 0.f;
-        }
-        if (et < 2 * 32) {
-          const int half = et >> 5, b = et & 31;
-          const int srow = MODE == 1 ? (e * 2 * p.F + half * p.F + mt * 64) / 128 : (e * p.d + mt * 128) / 128;
-          sw_s[et] = b < nwb ? __ldg(p.w_scale + (size_t)srow * nwb + b) : 0.f;
+        f8_epi_sync();                            // the previous chunk is done with cs_s and stage_out
+        // combined scale s_w(half, K block of the slice) * s_a(token, slice), once per chunk, off the
+        // per-slice path
+        const int halves = MODE == 1 ? 2 : 1;
+        for (int i = et; i < halves * nsl * kF8BN; i += kF8EpiThreads) {
+          const int n = i % kF8BN, sl = (i / kF8BN) % nsl, hf = i / (kF8BN * nsl);
+          const int srow = MODE == 1 ? (e * 2 * p.F + hf * p.F + mt * 64) / 128 : (e * p.d + mt * 128) / 128;
+          const int kb = MODE == 1 ? sl : sl >> 1;
+          const float sw = kb < nwb ? __ldg(p.w_scale + (size_t)srow * nwb + kb) : 0.f;
+          const float sa = n < nc ? __ldg(p.a_scale + (size_t)(off + c0 + n) * p.a_scale_cols + sl) : 0.f;
+          cs_s[(hf * kF8MaxSl + sl) * kF8BN + n] = sw * sa;
         }
         f8_epi_sync();
-        const float* sw_row = sw_s + (MODE == 1 && r >= 64 ? 32 : 0);
-        float acc[kF8BN];
+        const float* cs_row = cs_s + (size_t)half_row * kF8MaxSl * kF8BN + ch * 16;
+        float acc[16];
 #pragma unroll
-        for (int n = 0; n < kF8BN; ++n) acc[n] = 0.f;
+        for (int n = 0; n < 16; ++n) acc[n] = 0.f;
         for (int sl = 0; sl < nsl; ++sl, ++g) {
           const uint32_t b = g % kF8Slices;
           ok = ok && mbar_wait(&bars->sfull[b], (g / kF8Slices) & 1, err, DEV_ERR_TIMEOUT_EPILOGUE);
           tc_fence_after();
-          float v[32];
-          tmem_ld_32cols(tmem + ((uint32_t)(quarter * 32) << 16) + b * kF8BN, v);
+          float v[16];
+          tmem_ld_16cols(tmem + ((uint32_t)(quarter * 32) << 16) + b * kF8BN + ch * 16, v);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->sempty[b]);
-          const float sw = sw_row[MODE == 1 ? sl : sl >> 1];
+          const float4* c4 = reinterpret_cast<const float4*>(cs_row + sl * kF8BN);
 #pragma unroll
-          for (int n = 0; n < kF8BN; ++n) acc[n] = __fmaf_rn(v[n], sw * sa_s[n * kF8MaxSl + sl], acc[n]);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 c = c4[q4];
+            acc[4 * q4 + 0] = __fmaf_rn(v[4 * q4 + 0], c.x, acc[4 * q4 + 0]);
+            acc[4 * q4 + 1] = __fmaf_rn(v[4 * q4 + 1], c.y, acc[4 * q4 + 1]);
+            acc[4 * q4 + 2] = __fmaf_rn(v[4 * q4 + 2], c.z, acc[4 * q4 + 2]);
+            acc[4 * q4 + 3] = __fmaf_rn(v[4 * q4 + 3], c.w, acc[4 * q4 + 3]);
+          }
         }
         if (MODE == 2) {
           if (ok) {
             const int m = mt * 128 + r;           // output feature of the down projection
 #pragma unroll
-            for (int n = 0; n < kF8BN; ++n)
-              if (n < nc) p.y_out[(size_t)(off + c0 + n) * p.d + m] = acc[n];
+            for (int n = 0; n < 16; ++n)
+              if (ch * 16 + n < nc) p.y_out[(size_t)(off + c0 + ch * 16 + n) * p.d + m] = acc[n];
           }
         } else {
           // gate rows 0-63, up rows 64-127: SwiGLU of (row f, row 64 + f) through shared memory
 #pragma unroll
-          for (int n = 0; n < kF8BN; ++n) stage_out[r * kF8EpiStride + n] = acc[n];
+          for (int n = 0; n < 16; ++n) stage_out[r * kF8EpiStride + ch * 16 + n] = acc[n];
           f8_epi_sync();
-          // thread -> token n = et / 4, features fq .. fq + 15 with fq = 16 (et % 4); the 4 threads of a
+          // thread -> token n = et / 8, features fq .. fq + 7 with fq = 8 (et % 8); the 8 threads of a
           // token (adjacent lanes) share the amax of its 64 features
-          const int n = et >> 2, fq = (et & 3) * 16;
-          float h[16];
+          const int n = et >> 3, fq = (et & 7) * 8;
+          float h[8];
           float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const float gg = stage_out[(fq + i) * kF8EpiStride + n], uu = stage_out[(64 + fq + i) * kF8EpiStride + n];
             h[i] = gg / (1.f + __expf(-gg)) * uu;
             amax = fmaxf(amax, fabsf(h[i]));
           }
           amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
           amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
           const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
           if (ok && n < nc) {
-            uint32_t q[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              q[i] = e4m3x2(h[4 * i] * inv, h[4 * i + 1] * inv) | (e4m3x2(h[4 * i + 2] * inv, h[4 * i + 3] * inv) << 16);
+            const uint32_t q0 = e4m3x2(h[0] * inv, h[1] * inv) | (e4m3x2(h[2] * inv, h[3] * inv) << 16);
+            const uint32_t q1 = e4m3x2(h[4] * inv, h[5] * inv) | (e4m3x2(h[6] * inv, h[7] * inv) << 16);
             const size_t row = (size_t)(off + c0 + n);
-            *reinterpret_cast<uint4*>(p.hq_out + row * p.F + mt * 64 + fq) = make_uint4(q[0], q[1], q[2], q[3]);
-            if ((et & 3) == 0) p.hs_out[row * (p.F / 64) + mt] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+            *reinterpret_cast<uint2*>(p.hq_out + row * p.F + mt * 64 + fq) = make_uint2(q0, q1);
+            if ((et & 7) == 0) p.hs_out[row * (p.F / 64) + mt] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
           }
         }
       }

@@ -651,6 +651,263 @@ __global__ void __launch_bounds__(FP8 ? kExpThreadsFp8 : kExpThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
+// gate|up and down in one persistent launch (bf16 weights, 64-token chunks)
+// ---------------------------------------------------------------------------------------------
+// The work list is every (expert, 64 gate + 64 up rows) item, then every (expert, 128 down rows)
+// item, dealt round-robin to one CTA per SM.  A CTA's down items come after its own gate|up items
+// in its order, and a down item of expert e reads the SwiGLU rows of all of e's gate|up items: its
+// producer waits (bounded) until done[e] counts them, after which the TMA reads rows other CTAs
+// wrote.  Against two launches this fills the half-empty last round of the gate|up items with down
+// items and removes the launch in between.  done[] is zeroed by the gather that precedes the launch.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// generic-proxy writes of other threads (already acquired) -> this thread's later async-proxy (TMA) reads
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+template <int BN>
+__global__ void __launch_bounds__(kExpThreads, 1)
+    expert_updown_kernel(const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmX,
+                         const __grid_constant__ CUtensorMap tmWd, const __grid_constant__ CUtensorMap tmH,
+                         ExpertParams p, int n_exp, int* done, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  pdl_trigger();
+  uint8_t* tiles = align1024(smem_raw);
+  using C = ExpCfg<BN, false>;
+  constexpr int kStages = C::kStages;
+  constexpr uint32_t kStageBytes = C::kStageBytes;
+  float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kStages * kStageBytes);
+  constexpr int kEpiCols = C::kEpiCols, kEpiStride = C::kEpiStride;
+  ExpBarriers* bars = reinterpret_cast<ExpBarriers*>(stage_out + 128 * kEpiStride);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int MTu = p.F / 64, MTd = p.d / 128;             // weight tiles per expert: gate|up, down
+  const int n_up = n_exp * MTu, n_items = n_up + n_exp * MTd;
+  // item -> (gate|up?, expert, tile)
+  auto decode = [&](int item, bool& up, int& e, int& mt) {
+    up = item < n_up;
+    const int j = up ? item : item - n_up;
+    const int MT = up ? MTu : MTd;
+    e = j / MT;
+    mt = j % MT;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->acc_full[b], 1);
+      mbar_init(&bars->acc_empty[b], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&bars->tmem_slot, 2 * BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+  if (p.pre_bytes > 0 && (int)blockIdx.x < n_up) {
+    // the first gate|up tile into L2 while the preceding (light) kernels still run
+    const int e = blockIdx.x / MTu, mt = blockIdx.x % MTu;
+    const uint8_t* wbase = static_cast<const uint8_t*>(p.w_base);
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+      const int row = i < 64 ? e * 2 * p.F + mt * 64 + i : e * 2 * p.F + p.F + mt * 64 + (i - 64);
+      l2_prefetch_bulk(wbase + (size_t)row * p.d * 2, (uint32_t)p.pre_bytes);
+    }
+  }
+  pdl_wait();   // routing, the gathered rows and done[] (zeroed) come from the preceding kernels
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        bool up;
+        int e, mt;
+        decode(item, up, e, mt);
+        const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
+        if (!up && n_e > 0) {
+          // every gate|up tile of expert e has written its SwiGLU rows (bounded wait)
+          if (ld_acquire_gpu(done + e) < MTu) {
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t i = 1; ld_acquire_gpu(done + e) < MTu; ++i) {
+              if ((i & 63) == 0) {
+                if (*reinterpret_cast<volatile int*>(err) != 0) { ok = false; break; }
+                if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                  report_error(err, DEV_ERR_TIMEOUT_PRODUCER);
+                  ok = false;
+                  break;
+                }
+              }
+            }
+            if (!ok) break;
+          }
+          fence_proxy_async_global();
+        }
+        const int K = up ? p.d : p.F;
+        const int nk = K / 64;
+        for (int c0 = 0; c0 < n_e && ok; c0 += BN) {
+          const int nb = (min(BN, n_e - c0) + 31) >> 5;
+          const uint32_t tx = kATileBytes + (uint32_t)nb * 4096u;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a = tiles + (size_t)s * kStageBytes;
+            mbar_arrive_expect_tx(&bars->full[s], tx);
+            if (up) {
+              const int r0 = e * 2 * p.F + mt * 64;
+              tma_load_2d_hint(&tmWu, &bars->full[s], a, kb * 64, r0, pol_w);               // gate rows
+              tma_load_2d_hint(&tmWu, &bars->full[s], a + 8192, kb * 64, r0 + p.F, pol_w);  // up rows
+              for (int b = 0; b < nb; ++b)
+                tma_load_2d(&tmX, &bars->full[s], a + C::kAOff + b * 4096, kb * 64, off + c0 + 32 * b);
+            } else {
+              tma_load_2d_hint(&tmWd, &bars->full[s], a, kb * 64, e * p.d + mt * 128, pol_w);
+              for (int b = 0; b < nb; ++b)
+                tma_load_2d(&tmH, &bars->full[s], a + C::kAOff + b * 4096, kb * 64, off + c0 + 32 * b);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      uint32_t it = 0, j = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        bool up;
+        int e, mt;
+        decode(item, up, e, mt);
+        const int n_e = p.offsets[e + 1] - p.offsets[e];
+        const int nk = (up ? p.d : p.F) / 64;
+        for (int c0 = 0; c0 < n_e && ok; c0 += BN, ++j) {
+          const int nmma = (min(BN, n_e - c0) + 15) & ~15;
+          const uint32_t idesc = idesc_bf16_f32(128, nmma);
+          const uint32_t b = j & 1;
+          if (!mbar_wait(&bars->acc_empty[b], ((j >> 1) & 1) ^ 1, err, DEV_ERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t acc = tmem + b * BN;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&bars->full[s], (it / kStages) & 1, err, DEV_ERR_TIMEOUT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t* a = tiles + (size_t)s * kStageBytes;
+            const uint64_t ad = smem_desc_sw128(smem_u32(a));
+            const uint64_t bd = smem_desc_sw128(smem_u32(a + C::kAOff));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(acc, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0);
+            umma_commit(&bars->empty[s]);
+          }
+          umma_commit(&bars->acc_full[b]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------ epilogue (warps 2-5) ------------------------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;
+    uint32_t j = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      bool up;
+      int e, mt;
+      decode(item, up, e, mt);
+      const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
+      bool item_ok = true;
+      for (int c0 = 0; c0 < n_e; c0 += BN, ++j) {
+        const int nc = min(BN, n_e - c0);
+        const int nmma = (nc + 15) & ~15;
+        const uint32_t b = j & 1;
+        const bool ok = mbar_wait(&bars->acc_full[b], (j >> 1) & 1, err, DEV_ERR_TIMEOUT_EPILOGUE);
+        item_ok = item_ok && ok;
+        tc_fence_after();
+        const uint32_t acc = tmem + ((uint32_t)(quarter * 32) << 16) + b * BN;
+        if (up) {
+          for (int cs = 0; cs < nmma; cs += kEpiCols) {
+            const int ncs = min(kEpiCols, nmma - cs);
+            for (int cb = 0; cb < ncs; cb += 32) {
+              float v[32];
+              tmem_ld_32cols(acc + cs + cb, v);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) stage_out[r * kEpiStride + cb + i] = v[i];
+            }
+            if (cs + kEpiCols >= nmma) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+            }
+            epi_bar_sync();
+            if (ok) {
+              const int fq = (et & 3) * 16;
+              const int ncv = min(ncs, nc - cs);
+              for (int n = et >> 2; n < ncv; n += 32) {
+                uint32_t packed[8];
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                  const float g0 = stage_out[(fq + i) * kEpiStride + n], u0 = stage_out[(64 + fq + i) * kEpiStride + n];
+                  const float g1 = stage_out[(fq + i + 1) * kEpiStride + n],
+                              u1 = stage_out[(64 + fq + i + 1) * kEpiStride + n];
+                  packed[i / 2] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(off + c0 + cs + n) * p.F + mt * 64 + fq);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              }
+            }
+            epi_bar_sync();
+          }
+        } else {
+          const int m = mt * 128 + r;
+          for (int cb = 0; cb < nmma; cb += 32) {
+            float v[32];
+            tmem_ld_32cols(acc + cb, v);
+            if (cb + 32 >= nmma) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+            }
+            if (!ok) continue;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int n = cb + i;
+              if (n < nc) p.y_out[(size_t)(off + c0 + n) * p.d + m] = v[i];
+            }
+          }
+        }
+      }
+      if (up) {
+        // this tile's SwiGLU rows of expert e are written: count them for e's down items
+        __threadfence();
+        epi_bar_sync();
+        if (et == 0 && item_ok) red_release_gpu_add(done + e, 1);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+}
+
+// ---------------------------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------------------------
 template <int BN, int EPI, int Z>
@@ -714,6 +971,24 @@ static cudaError_t launch_expert(const CUtensorMap& w, const CUtensorMap& x, con
   const int items = n_exp * (MODE == 1 ? p.F / 64 : p.d / 128);
   return launch_k(expert_gemm_kernel<MODE, BN, FP8>, dim3(n_ctas < items ? n_ctas : items),
                   dim3(FP8 ? kExpThreadsFp8 : kExpThreads), C::kSmemBytes, st, 1, w, x, p, n_exp, err);
+}
+
+cudaError_t gemm_expert_updown(const CUtensorMap& wu, const CUtensorMap& x, const CUtensorMap& wd, const CUtensorMap& h,
+                               const ExpertParams& p, int n_exp, int n_ctas, int* done, int* err, cudaStream_t st) {
+  if (p.w_scale || !done || p.d % 128 || p.F % 64) return cudaErrorInvalidValue;
+  using C = ExpCfg<64, false>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(expert_updown_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(expert_updown_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int items = n_exp * (p.F / 64 + p.d / 128);
+  return launch_k(expert_updown_kernel<64>, dim3(n_ctas < items ? n_ctas : items), dim3(kExpThreads), C::kSmemBytes,
+                  st, 1, wu, x, wd, h, p, n_exp, done, err);
 }
 
 // wide = 1: 256-token accumulator chunks (many tokens per expert); 0: 64-token chunks.  p.w_scale

@@ -97,26 +97,28 @@ __device__ __forceinline__ void absorb16(RowState& st, const float* v, int v0, f
     st.S2 = fadd_f32x2(st.S2, fadd_f32x2(e01, e23));
     st.A2 = ffma_f32x2(e23, t23, ffma_f32x2(e01, t01, st.A2));
   }
-  // Gumbel draws of the groups that can reach the bound, screened with hardware logarithms
+  // Gumbel draws screened with hardware logarithms.  The four Philox blocks are computed without a
+  // branch (straight-line code, so their rounds overlap: one thread per row leaves little else to hide
+  // their latency); a group that cannot reach the bound even with the largest draw is masked out after.
   const float kSkip = __int_as_float(0x7fffffff);   // NaN: compares false, marks draws not taken
+  uint4 w4[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    w4[g] = philox4x32_10(make_uint4((uint32_t)((v0 >> 2) + g), pos, step, RNG_TAG_GUMBEL), k0, k1);
   float fs[4][4];
   float fmax_ = -INFINITY;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
+    const bool take = __fmaf_rn(gmax[g], inv_temp, kGumbelMax) >= st.lim;
+    const bool screen = gabs[g] * inv_temp <= kScreenMaxZ;
+    const uint32_t ww[4] = {w4[g].x, w4[g].y, w4[g].z, w4[g].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) fs[g][i] = kSkip;
-    if (__fmaf_rn(gmax[g], inv_temp, kGumbelMax) >= st.lim) {
-      const uint4 w = philox4x32_10(make_uint4((uint32_t)((v0 >> 2) + g), pos, step, RNG_TAG_GUMBEL), k0, k1);
-      const bool screen = gabs[g] * inv_temp <= kScreenMaxZ;
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float uu = u01_open(ww[i]);
-        const float f = gumbel_screen_score(v[4 * g + i], inv_temp, uu);
-        const bool exact_only = !screen || uu >= kGumbelFastMaxU;
-        fs[g][i] = exact_only ? INFINITY : f;
-        fmax_ = fmaxf(fmax_, exact_only ? -INFINITY : f);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const float uu = u01_open(ww[i]);
+      const float f = gumbel_screen_score(v[4 * g + i], inv_temp, uu);
+      const bool exact_only = !screen || uu >= kGumbelFastMaxU;
+      fs[g][i] = !take ? kSkip : (exact_only ? INFINITY : f);
+      fmax_ = fmaxf(fmax_, (take && !exact_only) ? f : -INFINITY);
     }
   }
   // every screened score minus two slacks is below that element's accurate score
@@ -126,8 +128,7 @@ __device__ __forceinline__ void absorb16(RowState& st, const float* v, int v0, f
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     if (fs[g][0] >= st.lim || fs[g][1] >= st.lim || fs[g][2] >= st.lim || fs[g][3] >= st.lim) {
-      const uint4 w = philox4x32_10(make_uint4((uint32_t)((v0 >> 2) + g), pos, step, RNG_TAG_GUMBEL), k0, k1);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t ww[4] = {w4[g].x, w4[g].y, w4[g].z, w4[g].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (fs[g][i] >= st.lim) {
@@ -595,7 +596,8 @@ cudaError_t head_sampler_run(const CUtensorMap& xn_map, const CUtensorMap& head_
                   : launch_head_sampler<256>(xn_map, head_map, p, n_ctas, err, st);
   }
   if (e != cudaSuccess) return e;
-  return sampler_finalize_run(fin, st);
+  // one record per row and CTA: merged one warp per row, then the step rule
+  return sampler_premerge_finalize_run(fin, p.partial + (size_t)256 * n_ctas * 8, st);
 }
 
 }  // namespace dg

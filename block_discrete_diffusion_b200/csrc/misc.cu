@@ -303,9 +303,12 @@ __global__ void scatter_rows_kernel(const int32_t* __restrict__ sel, int n_assig
 
 // xp[slot[t*k + r]] = xn[t] for every rank r: one warp per token reads the row once.
 __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const int32_t* __restrict__ slot, int n_rows,
-                                   int top_k, int d, __nv_bfloat16* __restrict__ xp) {
+                                   int top_k, int d, __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ zero,
+                                   int n_zero) {
   pdl_trigger();
   pdl_wait();
+  if (zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= n_rows) return;
   const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
@@ -460,10 +463,11 @@ cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, 
   return launch_k(scatter_rows_kernel, dim3((n_assign + 255) / 256), dim3(256), 0, st, 1, sel, n_assign, cursor, slot);
 }
 cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
-                        cudaStream_t st) {
+                        cudaStream_t st, int32_t* zero, int n_zero) {
   if (n_rows <= 0) return cudaSuccess;
   // two tokens (warps) per CTA: the copy of 256 tokens spreads over 128 SMs
-  return launch_k(gather_rows_kernel, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, xn, slot, n_rows, top_k, d, xp);
+  return launch_k(gather_rows_kernel, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, xn, slot, n_rows, top_k, d, xp, zero,
+                  n_zero);
 }
 cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x,
                         const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st) {

@@ -335,6 +335,52 @@ __global__ void sampler_finalize_kernel(SamplerArgs a) {
   if (threadIdx.x == 0) a.stop[seq] = stop;
 }
 
+// Many partial records per row (one per CTA of the fused head): one warp per row merges them -- lane
+// l takes records l, l + 32, ... in order, then the lanes combine by shuffles -- into a single record
+// per row (the same (m, S, A, best, index) merge as the finalize; ties of the best score go to the
+// lower index in both).  Rows committed before the step are skipped, as the finalize skips them.
+__global__ void sampler_premerge_kernel(const float* __restrict__ partial, int n_rows, int n_chunks,
+                                        const uint8_t* __restrict__ commit_in, float* __restrict__ merged) {
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= n_rows || commit_in[row]) return;
+  SoftStats st = {-INFINITY, 0.f, 0.f};
+  float best = -INFINITY;
+  int bidx = 0x7fffffff;
+  for (int c = lane; c < n_chunks; c += 32) {
+    const float* pr = partial + ((size_t)row * n_chunks + c) * 8;
+    const float4 a = *reinterpret_cast<const float4*>(pr);
+    const float b = pr[4];
+    st = stats_merge(st, SoftStats{a.x, a.y, a.z});
+    best_merge(best, bidx, a.w, __float_as_int(b));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    SoftStats other = {__shfl_xor_sync(0xffffffffu, st.m, o), __shfl_xor_sync(0xffffffffu, st.S, o),
+                       __shfl_xor_sync(0xffffffffu, st.A, o)};
+    st = stats_merge(st, other);
+    best_merge(best, bidx, __shfl_xor_sync(0xffffffffu, best, o), __shfl_xor_sync(0xffffffffu, bidx, o));
+  }
+  if (lane == 0) {
+    float* out = merged + (size_t)row * 8;
+    *reinterpret_cast<float4*>(out) = make_float4(st.m, st.S, st.A, best);
+    out[4] = __int_as_float(bidx);
+  }
+}
+
+cudaError_t sampler_premerge_finalize_run(const SamplerArgs& a, float* merged, cudaStream_t st) {
+  if (a.canvas > 4 * 256 || a.n_chunks <= 0) return cudaErrorInvalidValue;
+  const int rows = a.n_seq * a.canvas;
+  cudaError_t e = launch_k(sampler_premerge_kernel, dim3((rows + 7) / 8), dim3(256), 0, st, 1, a.partial, rows,
+                           a.n_chunks, a.commit_in, merged);
+  if (e != cudaSuccess) return e;
+  SamplerArgs f = a;
+  f.partial = merged;
+  f.n_chunks = 1;
+  return sampler_finalize_run(f, st);
+}
+
 int sampler_chunks(int vocab) {
   int c = vocab / 32768;
   if (c < 1) c = 1;
