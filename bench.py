@@ -206,12 +206,18 @@ def setup_full(rank, device, fp8=False):
     return cfg, w, model, seqs, prm, st
 
 
-def run_steps(dg, seqs, prm, st, k, state):
-    """k canvas steps; a new canvas every FIXED_STEPS steps (the block's step budget)."""
+def run_steps(dg, seqs, prm, st, k, state, nvtx=False):
+    """k canvas steps; a new canvas every FIXED_STEPS steps (the block's step budget).  nvtx: mark every
+    step as an NVTX range "dg_canvas_step" (the warm-up steps, so that a launch list can select them)."""
+    import torch
     for _ in range(k):
         if state["step"] % FIXED_STEPS == 0:
             dg.dg_canvas_init(seqs, prm, st["ids"], st["commit"])
+        if nvtx:
+            torch.cuda.nvtx.range_push("dg_canvas_step")
         dg.dg_canvas_step(seqs, prm, st["ids"], st["commit"], st["H"], st["stop"])
+        if nvtx:
+            torch.cuda.nvtx.range_pop()
         state["step"] += 1
 
 
@@ -273,7 +279,7 @@ def main_dg(args):
         dist.barrier()
     cfg, w, model, seqs, prm, st = setup_full(rank, device, fp8=args.fp8)
     state = {"step": 0}
-    run_steps(dg, seqs, prm, st, args.warmup, state)
+    run_steps(dg, seqs, prm, st, args.warmup, state, nvtx=True)
     torch.cuda.synchronize()
     code = dg.dg_device_error(seqs)
     assert code == 0, f"device error {code} during warm-up"
