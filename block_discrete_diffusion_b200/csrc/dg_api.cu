@@ -62,6 +62,7 @@ constexpr int kRouterSplits = 8;        // cluster size of the router GEMM's spl
 constexpr int kGemmTargetCtas = 296;    // two CTAs per SM for the 128-wide dense GEMM tiles
 constexpr int kSplitKSlots = kGemmTargetCtas;   // split-K partial tiles: tiles x splits <= this (dense_splits)
 constexpr int kHeadSamplerMaxCtas = 256;        // CTAs of the fused head + sampler (one per SM)
+constexpr int kRouteRows = 1024;                // rows up to which the router folds into the O epilogue
 
 // Cluster size (power of two, <= 8) of the split-K dense GEMMs for `tiles` output tiles over nk
 // 64-deep k-blocks: enough CTAs for about two per SM, at least 4 k-blocks per CTA.
@@ -171,7 +172,8 @@ struct WsLayout {
   int R, A, split_cap, chunks;
   size_t err, seqP, x, xn, q, opart, ml, attn, rlog, sel, gate, counts, offsets, slot, xp, hb,
       y, logits, samp, hsamp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, dstep, bsteps,
-      xq, xs, hq, hs, xdone, total;
+      xq, xs, hq, hs, xdone, rpart, ssq, rr, total;
+  int route_rows;   // rows up to which the FFN RMSNorm and router fold into the O epilogue (0: never)
   bool f8mma;     // FP8 form with few tokens per expert: e4m3 activations for the e4m3 x e4m3 expert GEMMs
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
@@ -263,6 +265,14 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.topk_done = take(64);
   L.dstep = take(64);
   L.xdone = take(4 * (size_t)c.n_exp);
+  // the FFN RMSNorm + router folded into the O-projection epilogue (up to kRouteRows rows: the
+  // per-tile partial planes stay small): router partials [d/128][rows][E], sums of squares, 1/rms
+  L.route_rows = (c.n_exp % 8 == 0 && c.n_exp <= 128) ? std::min(L.R, kRouteRows) : 0;
+  if (L.route_rows) {
+    L.rpart = take(4 * (d / 128) * (size_t)L.route_rows * c.n_exp);
+    L.ssq = take(4 * (d / 128) * (size_t)L.route_rows);
+    L.rr = take(4 * (size_t)L.route_rows);
+  }
   L.bsteps = take(4 * ((size_t)max_ctx / kCanvas + 1));
   if (c.wdtype == DG_WDTYPE_FP8_BLOCK128) {
     uint64_t rows[5], cols[5];
@@ -373,6 +383,10 @@ struct dg_seqs {
   float *xs, *hs;               // ... and their scales
   bool fp8_native;              // use the e4m3 x e4m3 expert GEMMs where available (DG_FP8_NATIVE, default on)
   int32_t* xdone;               // per-expert count of finished gate|up tiles (merged expert launch)
+  float* rpart;                 // folded router: per-tile router partials, sums of squares, 1/rms per row
+  float* ssq;
+  float* rr;
+  bool route_fused;             // fold the FFN RMSNorm + router into the O epilogue (DG_ROUTE_FUSED, default on)
   bool expert_merged;           // bf16, narrow chunks: gate|up and down in one launch (DG_EXPERT_MERGED, default on)
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
@@ -392,6 +406,7 @@ struct dg_seqs {
   bool block_open;
   int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
   int pre_bytes;    // bytes per weight row the gate|up GEMM brings into L2 before its wait (DG_EXPERT_PREFETCH)
+  bool prefetch_early;   // merged expert launch: the top-k launch issues that prefetch too (DG_PREFETCH_EARLY=1)
   int head_nv;      // one canvas: tiling of the fused head + sampler (kHeadSamplerPair: CTA pairs; 128 or 256
                     // vocabulary rows per single-SM tile; 0: the head GEMM writes the logits and the
                     // standalone sampler reads them; DG_HEAD_SAMPLER)
@@ -601,6 +616,11 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->fp8_native = true;
   if (const char* v = getenv("DG_FP8_NATIVE")) s->fp8_native = atoi(v) != 0;
   s->xdone = reinterpret_cast<int32_t*>(b + L.xdone);
+  s->rpart = L.route_rows ? reinterpret_cast<float*>(b + L.rpart) : nullptr;
+  s->ssq = L.route_rows ? reinterpret_cast<float*>(b + L.ssq) : nullptr;
+  s->rr = L.route_rows ? reinterpret_cast<float*>(b + L.rr) : nullptr;
+  s->route_fused = true;
+  if (const char* v = getenv("DG_ROUTE_FUSED")) s->route_fused = atoi(v) != 0;
   s->expert_merged = true;
   if (const char* v = getenv("DG_EXPERT_MERGED")) s->expert_merged = atoi(v) != 0;
   s->dstep = reinterpret_cast<int*>(b + L.dstep);
@@ -633,6 +653,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (c.vocab % 256 || (s->head_nv && head_sampler_ctas(c.vocab, s->head_nv, m->n_sms) > kHeadSamplerMaxCtas))
     s->head_nv = 0;
   if (const char* v = getenv("DG_EXPERT_PREFETCH")) s->pre_bytes = std::max(0, atoi(v));
+  s->prefetch_early = false;
+  if (const char* v = getenv("DG_PREFETCH_EARLY")) s->prefetch_early = atoi(v) != 0;
 
   const uint64_t d = c.d_model, R = L.R, A = L.A;
   const uint64_t zdim = (uint64_t)c.n_layers * n_seq * c.n_kv;
@@ -776,6 +798,11 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   LAUNCH(s, DG_K_ATTN, 1, attention_fwd(s->q_map, s->k_map, s->v_map, ap, n_local, s->attn, s->err, st));
   if (ap.n_splits > 1) LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
 
+  // Few rows: the FFN RMSNorm and the router fold into the O epilogue (the router is linear and the
+  // RMSNorm scales a row by one factor: logits = (x' g) W^T / rms(x')), and the gather forms the
+  // normed rows; no RMSNorm or router launch.
+  const float* ffn_g = static_cast<const float*>(W.ffn_norm);
+  const bool route = s->route_fused && rows <= s->L.route_rows;
   EpiParams eo{};
   eo.x = x;
   eo.ldo = d;
@@ -783,24 +810,47 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   eo.part = s->splitk;
   eo.part_slots = kSplitKSlots;
   eo.k_splits = dense_splits(((rows + 127) / 128) * (d / 128), c.n_q * dh / 64);
+  if (route) {
+    eo.rw = fp8 ? s->wq[2] : static_cast<const __nv_bfloat16*>(W.w_router);
+    eo.rg = ffn_g;
+    eo.rpart = s->rpart;
+    eo.ssq = s->ssq;
+    eo.n_exp = c.n_exp;
+  }
   LAUNCH(s, DG_K_OPROJ, 1, gemm_dense(128, EPI_RESID, s->attn_map, M.wo, rows, d, c.n_q * dh, eo, s->err, st));
   if (x_mid) CK(cudaMemcpyAsync(x_mid, x, sizeof(float) * (size_t)rows * d, cudaMemcpyDeviceToDevice, st));
 
   // mixture of experts
-  LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, static_cast<const float*>(W.ffn_norm), rows, d, c.rms_eps, s->xn, st));
-  EpiParams er{};
-  er.out = s->rlog;
-  er.ldo = c.n_exp;
-  er.late_weights = fp8;
-  er.part = s->splitk;
-  er.part_slots = kSplitKSlots;
-  er.k_splits = std::min(kRouterSplits, dense_splits((rows + 127) / 128, d / 64));
-  LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
+  if (!route) {
+    LAUNCH(s, DG_K_RMSNORM, 1, rmsnorm_rows(x, ffn_g, rows, d, c.rms_eps, s->xn, st));
+    EpiParams er{};
+    er.out = s->rlog;
+    er.ldo = c.n_exp;
+    er.late_weights = fp8;
+    er.part = s->splitk;
+    er.part_slots = kSplitKSlots;
+    er.k_splits = std::min(kRouterSplits, dense_splits((rows + 127) / 128, d / 64));
+    LAUNCH(s, DG_K_ROUTER, 1, gemm_dense(128, EPI_F32, s->xn_map, M.wrouter, rows, c.n_exp, d, er, s->err, st));
+  }
   // one canvas: the last CTA of the top-k launch also does the bucketing (one launch fewer)
   const bool fuse_assign = rows * c.top_k <= 8192 && c.n_exp <= 256;
   FusedAssignArgs fa{s->topk_done, s->offsets, s->slot};
-  LAUNCH(s, DG_K_TOPK, 1,
-         router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, fuse_assign ? &fa : nullptr, st));
+  const RouterNormArgs rn{s->ssq, d / 128, d, c.rms_eps, s->rr, s->rlog};
+  const GatherSrc gsrc = route ? GatherSrc{nullptr, x, s->rr, ffn_g} : GatherSrc{s->xn, nullptr, nullptr, nullptr};
+  // the merged bf16 expert launch's first weight tiles go into L2 from the top-k launch (two kernels early)
+  const int wide = expert_chunks_wide(c, rows) ? 1 : 0;
+  const bool merged = !fp8 && !wide && s->expert_merged;
+  const bool early = merged && s->pre_bytes > 0 && s->prefetch_early;
+  const int n_exp_ctas = std::min(s->m->n_sms, c.n_exp * (c.d_ff / 64));
+  const ExpertPrefetchArgs pfa{W.w_gate_up, n_exp_ctas, c.d_ff, d, std::min(s->pre_bytes, d * 2) & ~15};
+  if (route)
+    LAUNCH(s, DG_K_TOPK, 1,
+           router_topk(s->rpart, d / 128, (size_t)rows * c.n_exp, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts,
+                       fuse_assign ? &fa : nullptr, &rn, early ? &pfa : nullptr, st));
+  else
+    LAUNCH(s, DG_K_TOPK, 1,
+           router_topk(s->rlog, 1, 0, rows, c.n_exp, c.top_k, s->sel, s->gate, s->counts, fuse_assign ? &fa : nullptr,
+                       nullptr, early ? &pfa : nullptr, st));
   if (rlog_out)
     CK(cudaMemcpyAsync(rlog_out, s->rlog, sizeof(float) * (size_t)rows * c.n_exp, cudaMemcpyDeviceToDevice, st));
   if (!fuse_assign) {
@@ -812,7 +862,7 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   const bool f8mma = fp8 && s->L.f8mma && s->fp8_native && !expert_chunks_wide(c, rows);
   if (f8mma) {
     // e4m3 x e4m3: the gathered rows quantized per 128 channels, the SwiGLU rows per 64 features
-    LAUNCH(s, DG_K_BUCKET, 1, gather_rows_q8(s->xn, s->slot, rows, c.top_k, d, s->xq, s->xs, st));
+    LAUNCH(s, DG_K_BUCKET, 1, gather_rows_q8(gsrc, s->slot, rows, c.top_k, d, s->xq, s->xs, st));
     ExpertParams q{};
     q.offsets = s->offsets;
     q.d = d;
@@ -836,11 +886,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
            moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
     return DG_OK;
   }
-  // many tokens per expert on average (several canvases): 256-token accumulator chunks
-  const int wide = expert_chunks_wide(c, rows) ? 1 : 0;
-  const bool merged = !fp8 && !wide && s->expert_merged;
+  // many tokens per expert on average (several canvases): 256-token accumulator chunks (wide)
   LAUNCH(s, DG_K_BUCKET, 1,
-         gather_rows(s->xn, s->slot, rows, c.top_k, d, s->xp, st, merged ? s->xdone : nullptr, c.n_exp));
+         gather_rows(gsrc, s->slot, rows, c.top_k, d, s->xp, st, merged ? s->xdone : nullptr, c.n_exp));
   ExpertParams xp{};
   xp.offsets = s->offsets;
   xp.h_out = s->hb;

@@ -69,6 +69,17 @@ struct EpiParams {
                          // only after the grid-dependency wait
   float* part;           // k_splits > 1: fp32 scratch of part_slots [128][BN] partial tiles
   int part_slots;
+  // EPI_RESID with rw != nullptr (BN = 128, ldo % 128 == 0, n_exp % 8 == 0, n_exp <= 128): the FFN
+  // RMSNorm and the router folded into the residual epilogue.  For the updated rows x' and the
+  // tile's 128 columns (tile t = n0 / 128): ssq[t][row] = sum of x'^2, and rpart[t][row][e] = sum over
+  // the columns c of bf16(x'[c] rg[c]) * rw[e][c] (fp32 sums).  The router logit of a row is
+  // (sum over t of rpart[t][row][e]) / sqrt(sum over t of ssq[t][row] / ldo + eps), formed by the
+  // top-k kernel, because RMSNorm scales a whole row by one factor and the router is linear.
+  const __nv_bfloat16* rw;   // router weights [n_exp][ldo]
+  const float* rg;           // FFN RMSNorm gain [ldo]
+  float* rpart;              // [ldo / 128][M][n_exp]
+  float* ssq;                // [ldo / 128][M]
+  int n_exp;
 };
 
 // One FP8 block-scaled matrix to expand: e4m3 q [rows][cols], scales s [ceil(rows/128)][ceil(cols/128)].
@@ -133,8 +144,16 @@ cudaError_t gemm_expert_updown(const CUtensorMap& wu, const CUtensorMap& x, cons
 // boxes of 128 bytes, both 128-byte swizzled
 cudaError_t gemm_expert_f8(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                            int n_ctas, int* err, cudaStream_t st);
+// The rows a gather copies: bf16 normed rows xn, or (xn == nullptr) formed from the residual stream,
+// bf16(x[t] * r[t] * g) with r[t] = 1/rms of row t (the FFN RMSNorm folded into the gather).
+struct GatherSrc {
+  const __nv_bfloat16* xn;
+  const float* x;
+  const float* r;
+  const float* g;
+};
 // gather the normed rows into the bucketed order as e4m3 with one scale per (row, 128 channels)
-cudaError_t gather_rows_q8(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, uint8_t* xq,
+cudaError_t gather_rows_q8(const GatherSrc& src, const int32_t* slot, int n_rows, int top_k, int d, uint8_t* xq,
                            float* xs, cudaStream_t st);
 cudaError_t attention_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st);
@@ -154,13 +173,33 @@ struct FusedAssignArgs {
   int32_t* offsets;
   int32_t* slot;
 };
+// The FFN RMSNorm folded into the router (EpiParams::rw): the top-k kernel scales the summed logit
+// planes of each row by r = 1/sqrt(sum of the n_ssq partial sums of squares / d + eps), writes r and
+// the scaled logits.
+struct RouterNormArgs {
+  const float* ssq;      // [n_ssq][n_rows]
+  int n_ssq, d;
+  float eps;
+  float* r_out;          // [n_rows]
+  float* logits_out;     // [n_rows][n_exp]
+};
+// The first gate|up weight tile of each of n_ctas persistent expert CTAs (CTA c starts with item c:
+// expert c / (F/64), 64 gate rows and 64 up rows at tile c % (F/64)), brought into L2 by the top-k
+// launch, so that the weight stream of the expert launch two kernels later starts in L2.
+struct ExpertPrefetchArgs {
+  const void* w_gate_up;   // bf16 [n_exp][2F][d]
+  int n_ctas, F, d;
+  int row_bytes;           // bytes of each weight row to prefetch (multiple of 16, <= 2 d)
+};
+// norm, prefetch: nullable (the logits are final; no prefetch)
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
-                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused, cudaStream_t st);
+                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused,
+                        const RouterNormArgs* norm, const ExpertPrefetchArgs* prefetch, cudaStream_t st);
 // expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
                         int32_t* offsets, int32_t* cursor, int32_t* slot, int* n_launched, cudaStream_t st);
 // zero (nullable): n_zero ints set to 0 by the launch (the expert kernels' per-launch counters)
-cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
+cudaError_t gather_rows(const GatherSrc& src, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st, int32_t* zero = nullptr, int n_zero = 0);
 // g != nullptr: also the RMSNorm of each updated row into xn (bf16), gain g
 cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x, const float* g,

@@ -304,8 +304,13 @@ __global__ void __launch_bounds__(kF8Threads, 1)
 // xq[slot[t*k + r]] = e4m3(xn[t] / s), xs[slot[t*k + r]][b] = s = amax / 448 of channel block b (128
 // channels) of the row: one warp per (token, block) -- many independent warps, so the loads of all
 // blocks are in flight at once -- writes the block's k copies.
-__global__ void gather_rows_q8_kernel(const __nv_bfloat16* __restrict__ xn, const int32_t* __restrict__ slot,
-                                      int n_rows, int top_k, int d, uint8_t* __restrict__ xq, float* __restrict__ xs) {
+// The normed row's 4 values at column c of row t: read from xn, or formed as bf16(x * r * g) (the
+// FFN RMSNorm folded into the gather, the product order of the RMSNorm kernel).
+template <bool FROM_X>
+__global__ void gather_rows_q8_kernel(const __nv_bfloat16* __restrict__ xn, const float* __restrict__ x,
+                                      const float* __restrict__ rr, const float* __restrict__ g,
+                                      const int32_t* __restrict__ slot, int n_rows, int top_k, int d,
+                                      uint8_t* __restrict__ xq, float* __restrict__ xs) {
   pdl_trigger();
   pdl_wait();
   const int nblk = d / 128;
@@ -313,10 +318,22 @@ __global__ void gather_rows_q8_kernel(const __nv_bfloat16* __restrict__ xn, cons
   if (wid >= n_rows * nblk) return;
   const int t = wid / nblk, b = wid % nblk;
   const int my_slot = lane < top_k ? slot[(size_t)t * top_k + lane] : 0;
-  const uint2 raw = *reinterpret_cast<const uint2*>(xn + (size_t)t * d + b * 128 + lane * 4);
-  const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-  const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-  const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1), v3 = __high2float(p1);
+  const int c = b * 128 + lane * 4;
+  float v0, v1, v2, v3;
+  if constexpr (FROM_X) {
+    const float r = rr[t];
+    const float4 xv = *reinterpret_cast<const float4*>(x + (size_t)t * d + c);
+    const float4 gv = __ldg(reinterpret_cast<const float4*>(g + c));
+    v0 = __bfloat162float(__float2bfloat16_rn(xv.x * r * gv.x));
+    v1 = __bfloat162float(__float2bfloat16_rn(xv.y * r * gv.y));
+    v2 = __bfloat162float(__float2bfloat16_rn(xv.z * r * gv.z));
+    v3 = __bfloat162float(__float2bfloat16_rn(xv.w * r * gv.w));
+  } else {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xn + (size_t)t * d + c);
+    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    v0 = __low2float(p0); v1 = __high2float(p0); v2 = __low2float(p1); v3 = __high2float(p1);
+  }
   const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
   const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
   const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
@@ -347,12 +364,15 @@ cudaError_t launch_f8(const CUtensorMap& w, const CUtensorMap& x, const ExpertPa
 
 }  // namespace
 
-cudaError_t gather_rows_q8(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, uint8_t* xq,
+cudaError_t gather_rows_q8(const GatherSrc& src, const int32_t* slot, int n_rows, int top_k, int d, uint8_t* xq,
                            float* xs, cudaStream_t st) {
-  if (d % 128 || top_k > 32) return cudaErrorInvalidValue;
+  if (d % 128 || top_k > 32 || (!src.xn && (!src.x || !src.r || !src.g))) return cudaErrorInvalidValue;
   const int warps = n_rows * (d / 128);
-  return launch_k(gather_rows_q8_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, 1, xn, slot, n_rows, top_k, d, xq,
-                  xs);
+  if (src.xn)
+    return launch_k(gather_rows_q8_kernel<false>, dim3((warps + 7) / 8), dim3(256), 0, st, 1, src.xn, src.x, src.r,
+                    src.g, slot, n_rows, top_k, d, xq, xs);
+  return launch_k(gather_rows_q8_kernel<true>, dim3((warps + 7) / 8), dim3(256), 0, st, 1, src.xn, src.x, src.r, src.g,
+                  slot, n_rows, top_k, d, xq, xs);
 }
 
 cudaError_t gemm_expert_f8(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,

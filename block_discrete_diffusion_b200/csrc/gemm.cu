@@ -62,8 +62,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // columns); Q and K heads rotated pairwise by one warp per row (lane = rotary pair), stored
 // head-major; V heads by one warp per channel (lane = row, positions contiguous in the
 // transposed value cache).
+// With ep.rw (EPI_RESID, BN = 128): the updated rows x' also go back into the shared tile, and the
+// tile's per-row sums of squares to ep.ssq (the FFN RMSNorm's statistics, folded in here).
 template <int BN, int EPI, int RPC>
-__device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const float* t, int rs, int row0, int n0,
+__device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, float* t, int rs, int row0, int n0,
                                                    int M, int N) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kGemmThreads / 32;
@@ -144,7 +146,8 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
         const int r = warp + NW * (kb + k);
         if (kb + k >= RPW || r >= RPC || row0 + r >= M) break;
         float* dst = (EPI == EPI_RESID ? ep.x : ep.out) + (size_t)(row0 + r) * ep.ldo + n0;
-        const float* tr = t + r * rs;
+        float* tr = t + r * rs;
+        float ss = 0.f;
 #pragma unroll
         for (int g = 0; g < CG; ++g) {
           const int c = g * 128 + lane * 4;
@@ -152,6 +155,10 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
             float4 v = *reinterpret_cast<const float4*>(tr + c);
             if (EPI == EPI_RESID) {
               v.x += xv[k][g].x; v.y += xv[k][g].y; v.z += xv[k][g].z; v.w += xv[k][g].w;
+              if (ep.rw) {
+                *reinterpret_cast<float4*>(tr + c) = v;
+                ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+              }
             }
             *reinterpret_cast<float4*>(dst + c) = v;
           } else {
@@ -159,6 +166,94 @@ __device__ __forceinline__ void epilogue_from_smem(const EpiParams& ep, const fl
               dst[c + q] = (EPI == EPI_RESID ? dst[c + q] : 0.f) + tr[c + q];
           }
         }
+        if (EPI == EPI_RESID && ep.rw) {
+          ss = warp_sum(ss);
+          if (lane == 0) ep.ssq[(size_t)(n0 / 128) * M + row0 + r] = ss;
+        }
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void mma_bf16_m16n8k16(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The folded router's operands of a 128-column tile: the router weights W[e][n0 + c] of this warp's
+// 8-expert groups (w, w + 4, w + 8, w + 12) as mma.sync B fragments, and the gains g[n0 + c] of this
+// lane's columns.  Loaded once the accumulator is complete, so that their latency hides under the
+// drain, the split-K reduction and the residual epilogue.
+struct RouterFrags {
+  uint32_t b[4][8][2];
+  float2 g[8][2];
+};
+__device__ __forceinline__ void router_frags_load(const EpiParams& ep, int n0, RouterFrags& f) {
+  constexpr int NW = kGemmThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;   // fragment row group / column pair
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    f.g[ks][0] = __ldg(reinterpret_cast<const float2*>(ep.rg + n0 + 16 * ks + 2 * tig));
+    f.g[ks][1] = __ldg(reinterpret_cast<const float2*>(ep.rg + n0 + 16 * ks + 8 + 2 * tig));
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int nt = warp + NW * j;
+    if (nt < ep.n_exp / 8) {
+      const __nv_bfloat16* wr = ep.rw + (size_t)(nt * 8 + gid) * ep.ldo + n0 + 2 * tig;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        f.b[j][ks][0] = __ldg(reinterpret_cast<const unsigned int*>(wr + 16 * ks));
+        f.b[j][ks][1] = __ldg(reinterpret_cast<const unsigned int*>(wr + 16 * ks + 8));
+      }
+    }
+  }
+}
+
+// The router's share of the tile (ep.rw): rpart[n0/128][row][e] = sum over the tile's 128 columns c of
+// bf16(x'[row][c] g[c]) * W[e][c], for the RPC updated rows held in shared memory.  A small product
+// (RPC x n_exp x 128), so it runs on warp-level mma.sync (16 rows x 8 experts x 16 columns per
+// instruction, fp32 accumulation) inside the epilogue; warp w takes the 8-expert groups w, w + 4, ...
+template <int RPC>
+__device__ __forceinline__ void router_partial_from_smem(const EpiParams& ep, const RouterFrags& f, const float* t,
+                                                         int rs, int row0, int n0, int M) {
+  static_assert(RPC % 16 == 0, "16-row blocks");
+  constexpr int NW = kGemmThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  float* out = ep.rpart + (size_t)(n0 / 128) * M * ep.n_exp;
+#pragma unroll 1
+  for (int mt = 0; mt < RPC / 16; ++mt) {
+    // A fragments of this 16-row block (bf16(x' g)), shared by the warp's expert groups
+    uint32_t a[8][4];
+    const float* r0 = t + (mt * 16 + gid) * rs + 2 * tig;
+    const float* r1 = r0 + 8 * rs;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const float2 x00 = *reinterpret_cast<const float2*>(r0 + 16 * ks);
+      const float2 x10 = *reinterpret_cast<const float2*>(r1 + 16 * ks);
+      const float2 x01 = *reinterpret_cast<const float2*>(r0 + 16 * ks + 8);
+      const float2 x11 = *reinterpret_cast<const float2*>(r1 + 16 * ks + 8);
+      a[ks][0] = pack_bf16x2(x00.x * f.g[ks][0].x, x00.y * f.g[ks][0].y);
+      a[ks][1] = pack_bf16x2(x10.x * f.g[ks][0].x, x10.y * f.g[ks][0].y);
+      a[ks][2] = pack_bf16x2(x01.x * f.g[ks][1].x, x01.y * f.g[ks][1].y);
+      a[ks][3] = pack_bf16x2(x11.x * f.g[ks][1].x, x11.y * f.g[ks][1].y);
+    }
+    const int ra = row0 + mt * 16 + gid;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int nt = warp + NW * j;
+      if (nt < ep.n_exp / 8) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_bf16_m16n8k16(c, a[ks], f.b[j][ks][0], f.b[j][ks][1]);
+        const int e = nt * 8 + 2 * tig;
+        if (ra < M) *reinterpret_cast<float2*>(out + (size_t)ra * ep.n_exp + e) = make_float2(c[0], c[1]);
+        if (ra + 8 < M) *reinterpret_cast<float2*>(out + (size_t)(ra + 8) * ep.n_exp + e) = make_float2(c[2], c[3]);
       }
     }
   }
@@ -252,6 +347,10 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
 
   const bool ok = mbar_wait(&bars->accum, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
   tc_fence_after();
+  RouterFrags rf;
+  if constexpr (EPI == EPI_RESID && BN == 128) {
+    if (ep.rw) router_frags_load(ep, n0, rf);
+  }
   const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
 
   if constexpr (Z == 1) {
@@ -268,8 +367,15 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
           *reinterpret_cast<float4*>(red + r * RS + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
-    __syncthreads();
-    if (ok) epilogue_from_smem<BN, EPI, 128>(ep, red, RS, m0, n0, M, N);
+    if (__syncthreads_and(ok)) {
+      epilogue_from_smem<BN, EPI, 128>(ep, red, RS, m0, n0, M, N);
+      if constexpr (EPI == EPI_RESID && BN == 128) {
+        if (ep.rw) {
+          __syncthreads();
+          router_partial_from_smem<128>(ep, rf, red, RS, m0, n0, M);
+        }
+      }
+    }
   } else {
     // ---------------- split-K: partials through an L2-resident scratch, summed in rank order ----------------
     constexpr int RS = BN + 4;                 // padded row stride of the shared-memory tiles
@@ -294,20 +400,43 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       for (int i = threadIdx.x; i < 128 * F4; i += kGemmThreads)
         __stcg(dst + i, *reinterpret_cast<const float4*>(red + (i / F4) * RS + 4 * (i % F4)));
     }
-    __threadfence();
-    cluster_sync();   // every slot of the tile is written (and this CTA's shared tile is free again)
-    for (int i = threadIdx.x; i < RPC * F4; i += kGemmThreads) {
-      const size_t off = (size_t)(zz * RPC + i / F4) * BN + 4 * (i % F4);
-      float4 acc = __ldcg(reinterpret_cast<const float4*>(slots + off));
+    // every slot of the tile is written (the barrier's release / acquire at cluster scope makes the
+    // peers' global stores visible), and this CTA's shared tile is free again
+    cluster_sync();
+    {
+      constexpr int IT = RPC * F4 / kGemmThreads;           // float4 per thread
+      constexpr int B = IT < 16 / Z ? IT : 16 / Z;          // iterations whose Z loads are in flight together
+      static_assert((RPC * F4) % kGemmThreads == 0 && IT % B == 0, "reduction split");
+      for (int i0 = 0; i0 < IT; i0 += B) {
+        float4 v[B][Z];
 #pragma unroll
-      for (int z = 1; z < Z; ++z) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(slots + (size_t)z * 128 * BN + off));
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        for (int b = 0; b < B; ++b) {
+          const int i = threadIdx.x + (i0 + b) * kGemmThreads;
+          const size_t off = (size_t)(zz * RPC + i / F4) * BN + 4 * (i % F4);
+#pragma unroll
+          for (int z = 0; z < Z; ++z) v[b][z] = __ldcg(reinterpret_cast<const float4*>(slots + (size_t)z * 128 * BN + off));
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int i = threadIdx.x + (i0 + b) * kGemmThreads;
+          float4 acc = v[b][0];
+#pragma unroll
+          for (int z = 1; z < Z; ++z) {
+            acc.x += v[b][z].x; acc.y += v[b][z].y; acc.z += v[b][z].z; acc.w += v[b][z].w;
+          }
+          *reinterpret_cast<float4*>(red + (i / F4) * RS + 4 * (i % F4)) = acc;
+        }
       }
-      *reinterpret_cast<float4*>(red + (i / F4) * RS + 4 * (i % F4)) = acc;
     }
-    __syncthreads();
-    if (ok) epilogue_from_smem<BN, EPI, RPC>(ep, red, RS, m0 + zz * RPC, n0, M, N);
+    if (__syncthreads_and(ok)) {
+      epilogue_from_smem<BN, EPI, RPC>(ep, red, RS, m0 + zz * RPC, n0, M, N);
+      if constexpr (EPI == EPI_RESID && BN == 128) {
+        if (ep.rw) {
+          __syncthreads();
+          router_partial_from_smem<RPC>(ep, rf, red, RS, m0 + zz * RPC, n0, M);
+        }
+      }
+    }
   }
 
   tc_fence_before();
@@ -936,6 +1065,9 @@ cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap&
   if (z > K / 64) return cudaErrorInvalidValue;
   if (z > 1 && (!ep.part || (long long)((M + 127) / 128) * ((N + bn - 1) / bn) * z > ep.part_slots || bn != 128))
     return cudaErrorInvalidValue;   // the split-K scratch holds part_slots [128][128] tiles
+  if (ep.rw && (epi != EPI_RESID || bn != 128 || N % 128 || ep.ldo != N || ep.n_exp <= 0 || ep.n_exp % 8 ||
+                ep.n_exp > 128 || !ep.rg || !ep.rpart || !ep.ssq))
+    return cudaErrorInvalidValue;   // the folded router: whole 128-column tiles, 8-expert groups
 #define DG_DENSE_CASE(BN_, EPI_, Z_) \
   if (bn == BN_ && epi == EPI_ && z == Z_) return launch_dense<BN_, EPI_, Z_>(a, b, M, N, K, ep, err, st);
   DG_DENSE_CASE(128, EPI_QKV, 1)

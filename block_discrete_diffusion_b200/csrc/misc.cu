@@ -106,11 +106,19 @@ __global__ void rope_table_kernel(float2* table, int dh, double theta) {
 // the selected logits; per-expert counts accumulate with integer atomics (order-free, exact).
 // The router logits arrive as n_parts split-K partial planes (part_stride apart), summed here in
 // plane order.  Lane l owns experts [l*V, l*V + V), V = ceil(E/32) <= 8.
+struct RouterNorm {    // the FFN RMSNorm folded into the router (ssq == nullptr: the logits are final)
+  const float* ssq;
+  int n_ssq, d;
+  float eps;
+  float* r_out;
+  float* logits_out;
+};
+
 template <int V>
 __device__ __forceinline__ void router_topk_row(const float* __restrict__ logits, int n_parts, size_t part_stride,
-                                                int row, int n_exp, int top_k, int32_t* __restrict__ sel,
+                                                int row, int n_rows, int n_exp, int top_k, int32_t* __restrict__ sel,
                                                 float* __restrict__ gate, int32_t* __restrict__ counts,
-                                                int lane);
+                                                const RouterNorm& rn, int lane);
 __device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t* counts, int n_assign, int top_k,
                                   int n_exp, int32_t* __restrict__ offsets, int32_t* __restrict__ slot);
 
@@ -120,15 +128,34 @@ struct FusedAssign {   // the last CTA of the top-k launch also buckets the assi
   int32_t* slot;
 };
 
+struct ExpertPrefetch {   // w == nullptr: none
+  const uint8_t* w;
+  int n_ctas, F, d, row_bytes;
+};
+
 template <int V>
 __global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts, size_t part_stride, int n_rows,
                                    int n_exp, int top_k, int32_t* __restrict__ sel, float* __restrict__ gate,
-                                   int32_t* __restrict__ counts, FusedAssign fa) {
+                                   int32_t* __restrict__ counts, FusedAssign fa, RouterNorm rn, ExpertPrefetch pf) {
   pdl_trigger();
   pdl_wait();
+  if (pf.w) {
+    // the expert launch's first weight tiles into L2 (HBM is otherwise idle until that launch): whole
+    // rows as one request per 64-row block (gate or up half of a tile, contiguous), else per row
+    const int MTu = pf.F / 64;
+    const bool blocks = pf.row_bytes == 2 * pf.d;
+    const int n = pf.n_ctas * (blocks ? 2 : 128);
+    for (int i = threadIdx.x * gridDim.x + blockIdx.x; i < n; i += gridDim.x * blockDim.x) {   // spread over CTAs
+      const int c = blocks ? i >> 1 : i >> 7, k = blocks ? (i & 1) * 64 : i & 127;
+      const int e = c / MTu, mt = c % MTu;
+      const int row = e * 2 * pf.F + (k < 64 ? mt * 64 + k : pf.F + mt * 64 + (k - 64));
+      l2_prefetch_bulk(pf.w + (size_t)row * pf.d * 2, (uint32_t)(blocks ? 64 * pf.row_bytes : pf.row_bytes));
+    }
+  }
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row < n_rows) router_topk_row<V>(logits, n_parts, part_stride, row, n_exp, top_k, sel, gate, counts, lane);
+  if (row < n_rows)
+    router_topk_row<V>(logits, n_parts, part_stride, row, n_rows, n_exp, top_k, sel, gate, counts, rn, lane);
   if (fa.done) {
     __shared__ int s_last;
     __threadfence();
@@ -145,28 +172,61 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int n_parts
 
 template <int V>
 __device__ __forceinline__ void router_topk_row(const float* __restrict__ logits, int n_parts, size_t part_stride,
-                                                int row, int n_exp, int top_k, int32_t* __restrict__ sel,
+                                                int row, int n_rows, int n_exp, int top_k, int32_t* __restrict__ sel,
                                                 float* __restrict__ gate, int32_t* __restrict__ counts,
-                                                int lane) {
+                                                const RouterNorm& rn, int lane) {
   float v[V];
   const float* lr = logits + (size_t)row * n_exp + lane * V;
 #pragma unroll
   for (int i = 0; i < V; ++i) v[i] = 0.f;
   bool done = false;
+  // the row's sums of squares are loaded first, so that their latency overlaps the planes'
+  float ss = 0.f;
+  if (rn.ssq)
+    for (int t = lane; t < rn.n_ssq; t += 32) ss += __ldcg(rn.ssq + (size_t)t * n_rows + row);
+  // planes in batches (24 with float4 lanes, 8 otherwise) whose loads are all in flight together,
+  // summed in plane order (a missing plane adds an exact 0)
   if constexpr (V == 4) {
     if ((n_exp % 4) == 0 && lane * V < n_exp) {
-      for (int z = 0; z < n_parts; ++z) {
-        const float4 q = __ldcg(reinterpret_cast<const float4*>(lr + z * part_stride));
-        v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
+      for (int z0 = 0; z0 < n_parts; z0 += 24) {
+        float4 q[24];
+#pragma unroll
+        for (int u = 0; u < 24; ++u)
+          q[u] = z0 + u < n_parts ? __ldcg(reinterpret_cast<const float4*>(lr + (z0 + u) * part_stride))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 24; ++u) {
+          v[0] += q[u].x; v[1] += q[u].y; v[2] += q[u].z; v[3] += q[u].w;
+        }
       }
       done = true;
     }
   }
   if (!done) {
-    for (int z = 0; z < n_parts; ++z)
+    for (int z0 = 0; z0 < n_parts; z0 += 8) {
+      float q[8][V];
 #pragma unroll
-      for (int i = 0; i < V; ++i)
-        if (lane * V + i < n_exp) v[i] += lr[z * part_stride + i];
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+          q[u][i] = (z0 + u < n_parts && lane * V + i < n_exp) ? __ldcg(lr + (z0 + u) * part_stride + i) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int i = 0; i < V; ++i) v[i] += q[u][i];
+    }
+  }
+  if (rn.ssq) {
+    // 1/rms of the row from the residual epilogue's per-tile sums of squares (fixed summation order)
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)rn.d + rn.eps);
+    if (lane == 0) rn.r_out[row] = r;
+    float* lo = rn.logits_out + (size_t)row * n_exp + lane * V;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      v[i] *= r;
+      if (lane * V + i < n_exp) lo[i] = v[i];
+    }
   }
 #pragma unroll
   for (int i = 0; i < V; ++i)
@@ -250,9 +310,17 @@ __device__ void assign_rows_block(const int32_t* sel, const float* gate, int32_t
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= n_exp; e += blockDim.x) offsets[e] = s_off[e];
-  for (int a = threadIdx.x; a < n_assign; a += blockDim.x) {
-    const int e = __ldcg(sel + a);
-    slot[a] = s_off[e] + atomicAdd(&s_cur[e], 1);
+  // 8 assignments per thread per pass, their expert ids loaded together
+  for (int a0 = threadIdx.x; a0 < n_assign; a0 += 8 * blockDim.x) {
+    int e[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int a = a0 + u * blockDim.x;
+      e[u] = a < n_assign ? __ldcg(sel + a) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (e[u] >= 0) slot[a0 + u * blockDim.x] = s_off[e[u]] + atomicAdd(&s_cur[e[u]], 1);
   }
 }
 
@@ -301,10 +369,20 @@ __global__ void scatter_rows_kernel(const int32_t* __restrict__ sel, int n_assig
   slot[a] = atomicAdd(&cursor[sel[a]], 1);
 }
 
-// xp[slot[t*k + r]] = xn[t] for every rank r: one warp per token reads the row once.
-__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const int32_t* __restrict__ slot, int n_rows,
-                                   int top_k, int d, __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ zero,
-                                   int n_zero) {
+// 8 elements of a normed row: bf16(x * r * g), the product order of rmsnorm_kernel.
+__device__ __forceinline__ uint4 norm8(const float4 (&x)[2], const float4 (&g)[2], float r) {
+  const float4 a = x[0], b = x[1], ga = g[0], gb = g[1];
+  return make_uint4(pack_bf16x2(a.x * r * ga.x, a.y * r * ga.y), pack_bf16x2(a.z * r * ga.z, a.w * r * ga.w),
+                    pack_bf16x2(b.x * r * gb.x, b.y * r * gb.y), pack_bf16x2(b.z * r * gb.z, b.w * r * gb.w));
+}
+
+// xp[slot[t*k + r]] = row t for every rank r: one warp per token reads the row once.  The row is
+// xn[t] (bf16), or with FROM_X the FFN RMSNorm formed here, bf16(x[t] * rr[t] * g).
+template <bool FROM_X>
+__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const float* __restrict__ x,
+                                   const float* __restrict__ rr, const float* __restrict__ g,
+                                   const int32_t* __restrict__ slot, int n_rows, int top_k, int d,
+                                   __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ zero, int n_zero) {
   pdl_trigger();
   pdl_wait();
   if (zero && blockIdx.x == 0)
@@ -312,16 +390,36 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const i
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= n_rows) return;
   const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
-  const int n16 = d / 8;   // 16-byte chunks per row
+  const float* xr = x + (size_t)t * d;
+  const float r = FROM_X ? rr[t] : 0.f;
+  const int my_slot = lane < top_k ? slot[(size_t)t * top_k + lane] : 0;   // rank `lane`'s row, loaded once
+  const int n16 = d / 8;   // 16-byte chunks (8 elements) per bf16 row
   for (int c0 = 0; c0 < n16; c0 += 32 * 4) {
     uint4 v[4];
+    if constexpr (FROM_X) {
+      // all 16 loads of the 4 chunks in flight before any product
+      float4 xa[4][2], ga[4][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * 32 + lane;
-      if (c < n16) v[u] = src[c];
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n16) {
+          xa[u][0] = *reinterpret_cast<const float4*>(xr + 8 * c);
+          xa[u][1] = *reinterpret_cast<const float4*>(xr + 8 * c + 4);
+          ga[u][0] = __ldg(reinterpret_cast<const float4*>(g + 8 * c));
+          ga[u][1] = __ldg(reinterpret_cast<const float4*>(g + 8 * c + 4));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = norm8(xa[u], ga[u], r);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n16) v[u] = src[c];
+      }
     }
     for (int r = 0; r < top_k; ++r) {
-      uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)slot[(size_t)t * top_k + r] * d);
+      uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)__shfl_sync(0xffffffffu, my_slot, r) * d);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = c0 + u * 32 + lane;
@@ -349,14 +447,24 @@ __global__ void moe_combine_kernel(const float* __restrict__ y, const int32_t* _
   __syncthreads();
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
   float ss = 0.f;
+#pragma unroll 1
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int r = 0; r < top_k; ++r) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(y + (size_t)rows[r] * d) + c);
-      const float w = gw[r];
-      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+    const float4 xo = xr[c];
+    // ranks in batches of 8: the batch's loads are all in flight before its products are summed (rank order)
+    for (int r0 = 0; r0 < top_k; r0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (r0 + u < top_k) v[u] = __ldcs(reinterpret_cast<const float4*>(y + (size_t)rows[r0 + u] * d) + c);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (r0 + u < top_k) {
+          const float w = gw[r0 + u];
+          acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+        }
     }
-    float4 o = xr[c];
+    float4 o = xo;
     o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
     xr[c] = o;
     ss += o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
@@ -433,14 +541,28 @@ cudaError_t rope_table(float2* table, int max_ctx, int dh, float theta, cudaStre
   return launch_k(rope_table_kernel, dim3(max_ctx), dim3(dh / 2), 0, st, 1, table, dh, (double)theta);
 }
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
-                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused, cudaStream_t st) {
+                        int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused,
+                        const RouterNormArgs* norm, const ExpertPrefetchArgs* prefetch, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
   const int V = (n_exp + 31) / 32;
   const dim3 grid((n_rows + 7) / 8);
   FusedAssign fa{};
   if (fused) fa = FusedAssign{fused->done, fused->offsets, fused->slot};
+  RouterNorm rn{};
+  if (norm) {
+    if (!norm->ssq || !norm->r_out || !norm->logits_out || norm->n_ssq <= 0 || norm->d <= 0) return cudaErrorInvalidValue;
+    rn = RouterNorm{norm->ssq, norm->n_ssq, norm->d, norm->eps, norm->r_out, norm->logits_out};
+  }
+  ExpertPrefetch pf{};
+  if (prefetch && prefetch->w_gate_up) {
+    if (prefetch->F % 64 || prefetch->row_bytes <= 0 || prefetch->row_bytes % 16 || prefetch->row_bytes > 2 * prefetch->d ||
+        prefetch->n_ctas > n_exp * (prefetch->F / 64))
+      return cudaErrorInvalidValue;
+    pf = ExpertPrefetch{static_cast<const uint8_t*>(prefetch->w_gate_up), prefetch->n_ctas, prefetch->F, prefetch->d,
+                        prefetch->row_bytes};
+  }
 #define DG_TOPK_CASE(V_) \
-  if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts, fa);
+  if (V == V_) return launch_k(router_topk_kernel<V_>, grid, dim3(256), 0, st, 1, logits, n_parts, part_stride, n_rows, n_exp, top_k, sel, gate, counts, fa, rn, pf);
   DG_TOPK_CASE(1)
   DG_TOPK_CASE(2)
   DG_TOPK_CASE(4)
@@ -462,12 +584,16 @@ cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, 
   if (e != cudaSuccess) return e;
   return launch_k(scatter_rows_kernel, dim3((n_assign + 255) / 256), dim3(256), 0, st, 1, sel, n_assign, cursor, slot);
 }
-cudaError_t gather_rows(const __nv_bfloat16* xn, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
+cudaError_t gather_rows(const GatherSrc& src, const int32_t* slot, int n_rows, int top_k, int d, __nv_bfloat16* xp,
                         cudaStream_t st, int32_t* zero, int n_zero) {
   if (n_rows <= 0) return cudaSuccess;
+  if (d % 8 || (!src.xn && (!src.x || !src.r || !src.g))) return cudaErrorInvalidValue;
   // two tokens (warps) per CTA: the copy of 256 tokens spreads over 128 SMs
-  return launch_k(gather_rows_kernel, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, xn, slot, n_rows, top_k, d, xp, zero,
-                  n_zero);
+  if (src.xn)
+    return launch_k(gather_rows_kernel<false>, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, src.xn, src.x, src.r, src.g,
+                    slot, n_rows, top_k, d, xp, zero, n_zero);
+  return launch_k(gather_rows_kernel<true>, dim3((n_rows + 1) / 2), dim3(64), 0, st, 1, src.xn, src.x, src.r, src.g,
+                  slot, n_rows, top_k, d, xp, zero, n_zero);
 }
 cudaError_t moe_combine(const float* y, const int32_t* slot, const float* gate, int n_rows, int top_k, int d, float* x,
                         const float* g, float eps, __nv_bfloat16* xn, cudaStream_t st) {

@@ -171,14 +171,19 @@ def _layer_case(dg, cfg, P, seed, router_std=None):
     return w, model, seqs, ks, vs, x
 
 
-@pytest.mark.parametrize("cfg_name,P,n_rows,causal", [
-    ("tiny", 0, 256, False), ("tiny", 128, 256, False), ("tiny", 300, 256, False),
-    ("tiny", 0, 44, True), ("tiny", 256, 128, True), ("tiny", 200, 56, True), ("tiny", 384, 256, True),
-    ("one_layer", 4096, 256, False), ("one_layer", 2048, 200, True),
+@pytest.mark.parametrize("cfg_name,P,n_rows,causal,route", [
+    ("tiny", 0, 256, False, "folded"), ("tiny", 128, 256, False, "folded"), ("tiny", 300, 256, False, "folded"),
+    ("tiny", 0, 44, True, "folded"), ("tiny", 256, 128, True, "folded"), ("tiny", 200, 56, True, "folded"),
+    ("tiny", 384, 256, True, "folded"), ("tiny", 128, 256, False, "separate"), ("tiny", 200, 56, True, "separate"),
+    ("one_layer", 4096, 256, False, "folded"), ("one_layer", 2048, 200, True, "folded"),
+    ("one_layer", 4096, 256, False, "separate"),
 ])
-def test_layer_matches_oracle(dg, cfg_name, P, n_rows, causal):
+def test_layer_matches_oracle(dg, monkeypatch, cfg_name, P, n_rows, causal, route):
     """One layer (attention block, then MoE block) on canvas rows (bidirectional) or on a prefill
-    chunk (causal, ragged row counts), against a committed prefix of P positions."""
+    chunk (causal, ragged row counts), against a committed prefix of P positions.  route "folded":
+    the FFN RMSNorm and the router folded into the O-projection epilogue (the default for up to 1024
+    rows); "separate": DG_ROUTE_FUSED=0, an RMSNorm launch and a router GEMM."""
+    monkeypatch.setenv("DG_ROUTE_FUSED", "1" if route == "folded" else "0")
     if cfg_name == "tiny":
         cfg, router_std = synthetic.TINY, None
     else:
