@@ -741,6 +741,23 @@ def main_fp8_b32(args):
     hbm, tflops, kind = peaks(sustained=True)   # the attention launches are timed inside a long step
     attn_s = stats["attn"][1] / 1e3 / max(stats["attn"][0], 1)
     fl = attention_flops(cfg, n_seq, P)
+    # the expert GEMMs: e4m3 x e4m3 on CTA pairs (peak: the measured bf16 rate x the nominal 2:1 fp8 ratio),
+    # or with DG_FP8_PAIR=0 weights expanded to bf16 (bf16 peak)
+    n_assign = n_seq * CANVAS * cfg.top_k
+    e4m3 = os.environ.get("DG_FP8_PAIR", "1") != "0"
+    x_peak = 2 * tflops if e4m3 else tflops
+    expert_roof = {"kernels": ("expert_f8_pair_kernel<1> (gate|up + SwiGLU), <2> (down): tcgen05 kind::f8f6f4, "
+                               "CTA pairs" if e4m3 else "expert_gemm_kernel<MODE, 256, FP8> (e4m3 expanded to bf16, "
+                               "kind::f16)"),
+                   "bound": "tensor", "unit": "TFLOP/s", "peak": x_peak,
+                   "peak_source": (f"{kind}: 2 x bf16_tflops_sustained (nominal fp8 : bf16 = 4.5 : 2.25)" if e4m3
+                                   else f"{kind} bf16_tflops_sustained")}
+    for key, flops in (("expert_up", 2.0 * n_assign * 2 * cfg.d_ff * cfg.d_model),
+                       ("expert_down", 2.0 * n_assign * cfg.d_model * cfg.d_ff)):
+        if stats.get(key, (0, 0.0))[0]:
+            sec = stats[key][1] / 1e3 / stats[key][0]
+            expert_roof[key] = {"achieved": round(flops / sec / 1e12, 1), "frac": round(flops / sec / 1e12 / x_peak, 4),
+                                "algorithmic_flops_per_launch": flops, "launch_ms": round(sec * 1e3, 3)}
     line = {"metric": "canvas denoise steps/s", "value": round(k / t, 4), "unit": "steps/s",
             "ms_per_step": round(1e3 * t / k, 2), "steps": k, "warmup": args.warmup, "higher_is_better": True,
             "dtype": "bf16 arithmetic, fp8 e4m3 weights", "data": "synthetic",
@@ -758,6 +775,7 @@ def main_fp8_b32(args):
                          "algorithmic_flops_per_launch": fl, "launch_ms": round(attn_s * 1e3, 3),
                          "peak_source": f"{kind} bf16_tflops_sustained (kernel timed inside a long step)",
                          "frac_of_burst_peak": round(fl / attn_s / 1e12 / peaks()[1], 4)},
+            "expert_roofline": expert_roof,
             "kernel_ms_per_step": {kk: round(v[1] / k, 3) for kk, v in stats.items() if v[0]},
             "clocks": clk.summary(), "setup_seconds": round(t_setup, 1),
             "device_memory_gb": round(torch.cuda.max_memory_allocated() / 1e9, 1)}

@@ -174,7 +174,7 @@ struct WsLayout {
       y, logits, samp, hsamp, rope, cids, ccommit, cH, cstop, splitk, head_off, cursor, topk_done, dstep, bsteps,
       xq, xs, hq, hs, xdone, rpart, ssq, rr, total;
   int route_rows;   // rows up to which the FFN RMSNorm and router fold into the O epilogue (0: never)
-  bool f8mma;     // FP8 form with few tokens per expert: e4m3 activations for the e4m3 x e4m3 expert GEMMs
+  bool f8mma;     // FP8 form: e4m3 activations for the e4m3 x e4m3 expert GEMMs
   size_t wq[5];   // FP8 form only: one layer's matrices in bf16 (qkv, o, router, gate_up, down)
 };
 
@@ -278,8 +278,9 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
     uint64_t rows[5], cols[5];
     layer_matrix_shapes(c, rows, cols);
     for (int i = 0; i < 3; ++i) L.wq[i] = take(2 * rows[i] * cols[i]);   // the expert GEMMs read e4m3 directly
-    // few tokens per expert: the expert GEMMs multiply e4m3 by e4m3 (quantized activations + scales)
-    L.f8mma = !expert_chunks_wide(c, L.R) && c.d_model % 128 == 0 && c.d_ff % 64 == 0;
+    // the expert GEMMs multiply e4m3 by e4m3 (quantized activations + scales): few tokens per expert
+    // on single CTAs, many on CTA pairs
+    L.f8mma = c.d_model % 128 == 0 && c.d_ff % 64 == 0;
     if (L.f8mma) {
       L.xq = take(A * d);
       L.xs = take(4 * A * (d / 128));
@@ -382,6 +383,8 @@ struct dg_seqs {
   uint8_t *xq, *hq;             // ... the gathered rows and the SwiGLU rows in e4m3
   float *xs, *hs;               // ... and their scales
   bool fp8_native;              // use the e4m3 x e4m3 expert GEMMs where available (DG_FP8_NATIVE, default on)
+  bool fp8_pair;                // many tokens per expert: the CTA-pair e4m3 kernels (DG_FP8_PAIR=1; off by
+                                // default), else the kernels that expand e4m3 weights to bf16
   int32_t* xdone;               // per-expert count of finished gate|up tiles (merged expert launch)
   float* rpart;                 // folded router: per-tile router partials, sums of squares, 1/rms per row
   float* ssq;
@@ -615,6 +618,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->hs = L.f8mma ? reinterpret_cast<float*>(b + L.hs) : nullptr;
   s->fp8_native = true;
   if (const char* v = getenv("DG_FP8_NATIVE")) s->fp8_native = atoi(v) != 0;
+  s->fp8_pair = false;
+  if (const char* v = getenv("DG_FP8_PAIR")) s->fp8_pair = atoi(v) != 0;
   s->xdone = reinterpret_cast<int32_t*>(b + L.xdone);
   s->rpart = L.route_rows ? reinterpret_cast<float*>(b + L.rpart) : nullptr;
   s->ssq = L.route_rows ? reinterpret_cast<float*>(b + L.ssq) : nullptr;
@@ -859,7 +864,9 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
            assign_rows(s->sel, s->gate, s->counts, rows, c.top_k, c.n_exp, s->offsets, s->cursor, s->slot,
                        &n_assign_k, st));
   }
-  const bool f8mma = fp8 && s->L.f8mma && s->fp8_native && !expert_chunks_wide(c, rows);
+  const bool wide_rows = expert_chunks_wide(c, rows);
+  const bool f8pair = wide_rows && s->fp8_pair && d % 256 == 0;
+  const bool f8mma = fp8 && s->L.f8mma && s->fp8_native && (!wide_rows || f8pair);
   if (f8mma) {
     // e4m3 x e4m3: the gathered rows quantized per 128 channels, the SwiGLU rows per 64 features
     LAUNCH(s, DG_K_BUCKET, 1, gather_rows_q8(gsrc, s->slot, rows, c.top_k, d, s->xq, s->xs, st));
@@ -880,8 +887,13 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
     qd.a_scale = s->hs;
     qd.a_scale_cols = c.d_ff / 64;
     qd.y_out = s->y;
-    LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert_f8(1, ME.wgu8, s->xq_map, qu, c.n_exp, s->m->n_sms, s->err, st));
-    LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert_f8(2, ME.wdown8, s->hq_map, qd, c.n_exp, s->m->n_sms, s->err, st));
+    if (f8pair) {
+      LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert_f8_pair(1, ME.wgu8, s->xq_map, qu, c.n_exp, s->m->n_sms, s->err, st));
+      LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert_f8_pair(2, ME.wdown8, s->hq_map, qd, c.n_exp, s->m->n_sms, s->err, st));
+    } else {
+      LAUNCH(s, DG_K_EXPERT_UP, 1, gemm_expert_f8(1, ME.wgu8, s->xq_map, qu, c.n_exp, s->m->n_sms, s->err, st));
+      LAUNCH(s, DG_K_EXPERT_DOWN, 1, gemm_expert_f8(2, ME.wdown8, s->hq_map, qd, c.n_exp, s->m->n_sms, s->err, st));
+    }
     LAUNCH(s, DG_K_COMBINE, 1,
            moe_combine(s->y, s->slot, s->gate, rows, c.top_k, d, x, next_gain, c.rms_eps, s->xn, st));
     return DG_OK;

@@ -144,6 +144,11 @@ cudaError_t gemm_expert_updown(const CUtensorMap& wu, const CUtensorMap& x, cons
 // boxes of 128 bytes, both 128-byte swizzled
 cudaError_t gemm_expert_f8(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
                            int n_ctas, int* err, cudaStream_t st);
+// e4m3 x e4m3 grouped expert GEMMs on CTA pairs for many tokens per expert (256-token chunks, 256
+// weight rows per tile): w as gemm_expert_f8 (64-row boxes for MODE 1, 128-row for MODE 2), x 32-row
+// boxes; n_ctas even (pairs)
+cudaError_t gemm_expert_f8_pair(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p,
+                                int n_exp, int n_ctas, int* err, cudaStream_t st);
 // The rows a gather copies: bf16 normed rows xn, or (xn == nullptr) formed from the residual stream,
 // bf16(x[t] * r[t] * g) with r[t] = 1/rms of row t (the FFN RMSNorm folded into the gather).
 struct GatherSrc {

@@ -1,5 +1,6 @@
 // expert_fp8.cu -- grouped expert GEMMs with both operands in e4m3 on the tensor cores
-// (tcgen05.mma kind::f8f6f4), for chunks of up to 32 tokens per expert (one or a few canvases).
+// (tcgen05.mma kind::f8f6f4): expert_f8_kernel for chunks of up to 32 tokens per expert (one or a few
+// canvases), expert_f8_pair_kernel on CTA pairs for 256-token chunks (many canvases; further below).
 //
 // The FP8 form of the per-layer matrices stores e4m3 bytes q with one fp32 scale s_w per 128 x 128
 // tile (w = q * s_w).  Here the activations are e4m3 too, with one fp32 scale per token and per
@@ -23,6 +24,7 @@
 // per-tile scales are fp32 (not the power-of-two block scales the hardware's block-scaled MMA takes),
 // so the scales are applied in the epilogue per slice.
 #include <cuda_fp8.h>
+#include <stdio.h>
 
 #include "dg_device.cuh"
 #include "dg_kernels.h"
@@ -86,6 +88,18 @@ __device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// 32 lanes x 16 columns of TMEM into registers without waiting (tmem_wait_ld16 completes the loads).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld16() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Two floats to two e4m3 bytes (round to nearest even, saturating to +-448).
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
@@ -345,6 +359,353 @@ __global__ void gather_rows_q8_kernel(const __nv_bfloat16* __restrict__ xn, cons
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Many tokens per expert (several canvases): CTA pairs
+// ---------------------------------------------------------------------------------------------
+// With hundreds of tokens per expert the product is bound by the tensor cores, so the tile grows to
+// 256 tokens x 256 weight rows on a CTA pair (tcgen05 cta_group::2, M = 256): the tokens are the M
+// side (128 rows in each CTA), the weight rows the N side, half in each CTA -- MODE 1: the gate rows of
+// 128 features in the leader and the up rows of the same features in the peer, so that one
+// accumulator row holds both halves of every SwiGLU feature; MODE 2: 128 output features in each.
+// Thread = token row, so a slice's activation scale is one number per thread and its weight scale one
+// number per block of columns: the promotion is one FMA per accumulator element, and the
+// accumulators (128 per thread) stay in registers.  Two TMEM slice buffers of 256 columns: the MMAs
+// of one slice overlap the promotion of the other.  Work items are (expert, weight tile, 256-token
+// chunk), chunks innermost, so that the chunks of one weight tile run at the same time on
+// neighbouring pairs and share its HBM read through L2.
+constexpr int kFpThreads = 320;                // warp 0 TMA (both CTAs), warp 1 MMA (leader), warps 2-9 promotion
+constexpr int kFpStages = 6;
+constexpr uint32_t kFpATile = 128 * 128;       // 128 token rows x 128 bytes of K
+constexpr uint32_t kFpBTile = 128 * 128;       // up to 128 weight rows x 128 bytes of K
+constexpr uint32_t kFpStage = kFpATile + kFpBTile;
+constexpr int kFpMaxExp = 256;
+constexpr int kFpCumInts = (kFpMaxExp + 1 + 3) / 4 * 4;   // the barriers after them stay 16-byte aligned
+constexpr size_t kFpSmem = 1024 + (size_t)kFpStages * kFpStage + 2 * 128 * 4 + kFpCumInts * 4 + 256;
+static_assert(kFpSmem <= 232448, "shared memory budget");
+
+struct FpBarriers {
+  uint64_t full[kFpStages];
+  uint64_t empty[kFpStages];
+  uint64_t sfull[2];
+  uint64_t sempty[2];
+  uint32_t tmem_slot;
+};
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFpThreads, 1)
+    expert_f8_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                          ExpertParams p, int n_exp, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  pdl_trigger();
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* amx = reinterpret_cast<float*>(tiles + (size_t)kFpStages * kFpStage);   // [2][128]: half-block amax
+  int* s_cum = reinterpret_cast<int*>(amx + 256);                                // first item of each expert
+  FpBarriers* bars = reinterpret_cast<FpBarriers*>(s_cum + kFpCumInts);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();       // 0: leader, 1: peer
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int K = MODE == 1 ? p.d : p.F;
+  const int nkb = (K + 127) / 128;                              // 128-byte K stages
+  const int nsl = MODE == 1 ? K / 128 : (K + 63) / 64;          // promotion slices (= activation scale blocks)
+  const int NT = MODE == 1 ? (p.F + 127) / 128 : p.d / 256;     // weight tiles per expert
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFpStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->sfull[b], 1);
+      mbar_init(&bars->sempty[b], 16);          // the promotion warps of both CTAs
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(&bars->tmem_slot, 512);
+  tc_fence_before();
+  cluster_sync();                               // both CTAs' barriers and tensor memory exist
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+  const uint32_t lead_full0 = dsmem_map(smem_u32(&bars->full[0]), 0);
+  const uint32_t lead_sempty0 = dsmem_map(smem_u32(&bars->sempty[0]), 0);
+  pdl_wait();   // routing, the quantized activation rows and their scales come from the preceding kernels
+
+  // items per expert: NT weight tiles x ceil(n_e / 256) chunks; s_cum = exclusive prefix over experts
+  if (warp == 2) {
+    int run = 0;
+    for (int e0 = 0; e0 < n_exp; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < n_exp ? NT * ((p.offsets[e + 1] - p.offsets[e] + 255) / 256) : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (e < n_exp) s_cum[e] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_cum[n_exp] = run;
+  }
+  __syncthreads();
+  const int n_items = s_cum[n_exp];
+  int ecur = 0;
+  // item -> expert e, weight tile t, chunk c (items increase along every role's walk)
+  auto decode = [&](int item, int& e, int& t, int& c) {
+    while (s_cum[ecur + 1] <= item) ++ecur;
+    e = ecur;
+    const int nch = (p.offsets[e + 1] - p.offsets[e] + 255) / 256;
+    t = (item - s_cum[e]) / nch;
+    c = (item - s_cum[e]) % nch;
+  };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer (both CTAs) ------------------------------
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();   // token rows and weight tiles are each read by several items
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = pair; item < n_items && ok; item += n_pairs) {
+        int e, t, c;
+        decode(item, e, t, c);
+        const int nf = MODE == 1 ? min(128, p.F - t * 128) : 128;   // weight rows this CTA holds
+        const int tok0 = p.offsets[e] + c * 256 + (int)rank * 128;
+        const int wrow = MODE == 1 ? e * 2 * p.F + (int)rank * p.F + t * 128 : e * p.d + t * 256 + (int)rank * 128;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kFpStages;
+          if (!mbar_wait(&bars->empty[s], ((it / kFpStages) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a = tiles + (size_t)s * kFpStage;
+          if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], 2 * (kFpATile + (uint32_t)nf * 128));
+          const uint32_t bar = lead_full0 + (uint32_t)(s * sizeof(uint64_t));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tma_load_2d_pair(&tmX, bar, a + q * 4096, kb * 128, tok0 + q * 32, pol);
+          if (MODE == 1) {
+            for (int h = 0; h < nf / 64; ++h)
+              tma_load_2d_pair(&tmW, bar, a + kFpATile + h * 8192, kb * 128, wrow + h * 64, pol);
+          } else {
+            tma_load_2d_pair(&tmW, bar, a + kFpATile, kb * 128, wrow, pol);
+          }
+        }
+      }
+      // tail: every stage released once more, i.e. the leader's last commits (multicast to this CTA)
+      // have arrived here before the CTA may leave
+      for (int i = 0; i < kFpStages && ok; ++i, ++it)
+        ok = mbar_wait(&bars->empty[it % kFpStages], ((it / kFpStages) & 1) ^ 1, err, DEV_ERR_TIMEOUT_PRODUCER);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader) ------------------------------
+    if (rank == 0 && lane == 0) {
+      uint32_t it = 0, g = 0;
+      bool ok = true;
+      for (int item = pair; item < n_items && ok; item += n_pairs) {
+        int e, t, c;
+        decode(item, e, t, c);
+        const int nf = MODE == 1 ? min(128, p.F - t * 128) : 128;
+        const uint32_t idesc = idesc_e4m3_f32(256, 2 * nf);
+        for (int kb = 0; kb < nkb && ok; ++kb, ++it) {
+          const int s = it % kFpStages;
+          if (!mbar_wait(&bars->full[s], (it / kFpStages) & 1, err, DEV_ERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* a = tiles + (size_t)s * kFpStage;
+          const uint64_t ad = smem_desc_sw128(smem_u32(a));
+          const uint64_t bd = smem_desc_sw128(smem_u32(a + kFpATile));
+          // MODE 1: one 128-deep slice per stage; MODE 2: two 64-deep slices (none past F)
+          const int per = MODE == 1 ? 1 : 2;
+          for (int h = 0; h < per; ++h) {
+            if (kb * per + h >= nsl) break;
+            const uint32_t b = g & 1;
+            if (!mbar_wait(&bars->sempty[b], ((g >> 1) & 1) ^ 1, err, DEV_ERR_TIMEOUT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            constexpr int kSteps = MODE == 1 ? 4 : 2;        // 32 K per instruction
+#pragma unroll
+            for (int k = 0; k < kSteps; ++k)
+              umma_e4m3_pair(tmem + b * 256, desc_advance(ad, (h * kSteps + k) * 32), desc_advance(bd, (h * kSteps + k) * 32),
+                             idesc, k != 0);
+            umma_commit_pair(&bars->sfull[b]);
+            ++g;
+          }
+          umma_commit_pair(&bars->empty[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------ promotion + epilogue (warps 2-9 of both CTAs) ------------------------------
+    // Warps w and w + 4 read TMEM lanes 32 (w % 4) .. (token rows of this CTA) and split the columns:
+    // MODE 1 the gate columns [ch nf/2, (ch + 1) nf/2) and the matching up columns nf + ..., MODE 2
+    // the output columns [128 ch, 128 ch + 128).
+    const int q = warp & 3, ch = (warp - 2) >> 2;
+    const int lrow = q * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    const int nwb = p.w_scale_cols;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int item = pair; item < n_items; item += n_pairs) {
+      int e, t, c;
+      decode(item, e, t, c);
+      const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
+      const int nf = MODE == 1 ? min(128, p.F - t * 128) : 128;
+      const int half = nf / 2;                   // MODE 1: SwiGLU features of this thread
+      const int tl = c * 256 + (int)rank * 128 + lrow;
+      const bool valid = tl < n_e;
+      const size_t token = (size_t)(off + (valid ? tl : 0));
+      // scale rows (128-row tiles of the weight matrix) of this thread's column blocks
+      const int r0 = MODE == 1 ? (e * 2 * p.F + t * 128 + ch * half) / 128 : (e * p.d + t * 256 + ch * 128) / 128;
+      const int r1 = MODE == 1 ? (e * 2 * p.F + p.F + t * 128 + ch * half) / 128 : r0;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      // the scales of slice sl + 1 are loaded while slice sl is promoted
+      const float* pa = p.a_scale + token * p.a_scale_cols;
+      const float* pw0 = p.w_scale + (size_t)r0 * nwb;
+      const float* pw1 = p.w_scale + (size_t)r1 * nwb;
+      float sa_n = valid ? __ldg(pa) : 0.f, sw0_n = __ldg(pw0), sw1_n = MODE == 1 ? __ldg(pw1) : 0.f;
+      for (int sl = 0; sl < nsl; ++sl, ++g) {
+        const float sa = sa_n, sw0 = sw0_n, sw1 = sw1_n;
+        if (sl + 1 < nsl) {
+          const int kb1 = MODE == 1 ? sl + 1 : (sl + 1) >> 1;
+          sa_n = valid ? __ldg(pa + sl + 1) : 0.f;
+          sw0_n = __ldg(pw0 + kb1);
+          if (MODE == 1) sw1_n = __ldg(pw1 + kb1);
+        }
+        const float c0s = sw0 * sa;
+        const float c1s = MODE == 1 ? sw1 * sa : 0.f;
+        const uint32_t b = g & 1;
+        ok = ok && mbar_wait(&bars->sfull[b], (g >> 1) & 1, err, DEV_ERR_TIMEOUT_EPILOGUE);
+        tc_fence_after();
+        const uint32_t ta = tq + b * 256;
+        // two 16-column TMEM loads in flight per wait: the 128 accumulators and 32 loaded values fit the
+        // registers, and a slice takes four load round trips
+        if (MODE == 1) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j * 16 < half) {
+              uint32_t v[2][16];
+              tmem_ld16_nowait(ta + ch * half + j * 16, v[0]);
+              tmem_ld16_nowait(ta + nf + ch * half + j * 16, v[1]);
+              tmem_wait_ld16();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                acc[j * 16 + i] = __fmaf_rn(__uint_as_float(v[0][i]), c0s, acc[j * 16 + i]);
+                acc[64 + j * 16 + i] = __fmaf_rn(__uint_as_float(v[1][i]), c1s, acc[64 + j * 16 + i]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            uint32_t v[2][16];
+            tmem_ld16_nowait(ta + ch * 128 + j * 16, v[0]);
+            tmem_ld16_nowait(ta + ch * 128 + j * 16 + 16, v[1]);
+            tmem_wait_ld16();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc[j * 16 + i] = __fmaf_rn(__uint_as_float(v[0][i]), c0s, acc[j * 16 + i]);
+              acc[j * 16 + 16 + i] = __fmaf_rn(__uint_as_float(v[1][i]), c0s, acc[j * 16 + 16 + i]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(lead_sempty0 + b * (uint32_t)sizeof(uint64_t));
+      }
+      if (MODE == 2) {
+        if (ok && valid) {
+          float4* dst = reinterpret_cast<float4*>(p.y_out + token * p.d + t * 256 + ch * 128);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        }
+      } else {
+        // SwiGLU of this thread's features (gate acc[i], up acc[64 + i]), e4m3 per (token, 64 features)
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          if (i < half) {
+            const float gg = acc[i], uu = acc[64 + i];
+            acc[i] = gg / (1.f + __expf(-gg)) * uu;
+            amax = fmaxf(amax, fabsf(acc[i]));
+          }
+        }
+        if (half < 64) {
+          // the 64-feature block is shared with warp w ^ 4 (same token rows, the other half): exchange
+          amx[ch * 128 + lrow] = amax;
+          f8_epi_sync();
+          amax = fmaxf(amax, amx[(ch ^ 1) * 128 + lrow]);
+          f8_epi_sync();
+        }
+        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+        if (ok && valid) {
+          const int f0 = t * 128 + ch * half;      // first feature of this thread
+          uint8_t* dst = p.hq_out + token * p.F + f0;
+#pragma unroll
+          for (int i = 0; i < 64; i += 16) {
+            if (i < half) {
+              uint4 w;
+              w.x = e4m3x2(acc[i] * inv, acc[i + 1] * inv) | (e4m3x2(acc[i + 2] * inv, acc[i + 3] * inv) << 16);
+              w.y = e4m3x2(acc[i + 4] * inv, acc[i + 5] * inv) | (e4m3x2(acc[i + 6] * inv, acc[i + 7] * inv) << 16);
+              w.z = e4m3x2(acc[i + 8] * inv, acc[i + 9] * inv) | (e4m3x2(acc[i + 10] * inv, acc[i + 11] * inv) << 16);
+              w.w = e4m3x2(acc[i + 12] * inv, acc[i + 13] * inv) | (e4m3x2(acc[i + 14] * inv, acc[i + 15] * inv) << 16);
+              *reinterpret_cast<uint4*>(dst + i) = w;
+            }
+          }
+          if (half == 64 || ch == 0) p.hs_out[token * (p.F / 64) + f0 / 64] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();                               // no CTA leaves while the pair's MMAs or arrivals may touch it
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
+template <int MODE>
+cudaError_t launch_f8_pair(const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp, int n_ctas,
+                           int* err, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(expert_f8_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kFpSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(expert_f8_pair_kernel<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_ctas & ~1);
+  cfg.blockDim = dim3(kFpThreads);
+  cfg.dynamicSmemBytes = kFpSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, expert_f8_pair_kernel<MODE>, w, x, p, n_exp, err);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    // say which resource the launch exceeded
+    cudaFuncAttributes fa{};
+    cudaGetLastError();
+    if (cudaFuncGetAttributes(&fa, expert_f8_pair_kernel<MODE>) == cudaSuccess) {
+      fprintf(stderr, "expert_f8_pair_kernel<%d>: %s (registers %d, max threads %d, static smem %zu, dynamic %zu)\n",
+              MODE, cudaGetErrorString(e), fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, kFpSmem);
+    }
+  }
+  return e;
+}
+
 template <int MODE>
 cudaError_t launch_f8(const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp, int n_ctas,
                       int* err, cudaStream_t st) {
@@ -373,6 +734,15 @@ cudaError_t gather_rows_q8(const GatherSrc& src, const int32_t* slot, int n_rows
                     src.g, slot, n_rows, top_k, d, xq, xs);
   return launch_k(gather_rows_q8_kernel<true>, dim3((warps + 7) / 8), dim3(256), 0, st, 1, src.xn, src.x, src.r, src.g,
                   slot, n_rows, top_k, d, xq, xs);
+}
+
+cudaError_t gemm_expert_f8_pair(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p,
+                                int n_exp, int n_ctas, int* err, cudaStream_t st) {
+  if (!p.w_scale || !p.a_scale || !p.offsets || n_exp <= 0 || n_exp > kFpMaxExp || n_ctas < 2) return cudaErrorInvalidValue;
+  if (mode == 1 && (p.d % 128 || p.F % 64 || p.a_scale_cols != p.d / 128 || !p.hq_out || !p.hs_out))
+    return cudaErrorInvalidValue;
+  if (mode == 2 && (p.d % 256 || p.F % 64 || p.a_scale_cols != p.F / 64 || !p.y_out)) return cudaErrorInvalidValue;
+  return mode == 1 ? launch_f8_pair<1>(w, x, p, n_exp, n_ctas, err, st) : launch_f8_pair<2>(w, x, p, n_exp, n_ctas, err, st);
 }
 
 cudaError_t gemm_expert_f8(int mode, const CUtensorMap& w, const CUtensorMap& x, const ExpertParams& p, int n_exp,
