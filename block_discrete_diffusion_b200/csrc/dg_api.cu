@@ -391,6 +391,8 @@ struct dg_seqs {
   float* rr;
   bool route_fused;             // fold the FFN RMSNorm + router into the O epilogue (DG_ROUTE_FUSED, default on)
   bool expert_merged;           // bf16, narrow chunks: gate|up and down in one launch (DG_EXPERT_MERGED, default on)
+  bool head_fused_batch;        // several canvases: the fused head + sampler once per canvas (DG_HEAD_FUSED_BATCH,
+                                // default on), else the dense head GEMM + the sampler over all logits
   int32_t* head_off;            // {0, R}: all rows as one "expert" for the persistent head GEMM
   int32_t* cursor;              // per-expert row cursors of the multi-CTA bucketing
   int32_t* topk_done;           // launch counter of the top-k kernel that also buckets
@@ -628,6 +630,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   if (const char* v = getenv("DG_ROUTE_FUSED")) s->route_fused = atoi(v) != 0;
   s->expert_merged = true;
   if (const char* v = getenv("DG_EXPERT_MERGED")) s->expert_merged = atoi(v) != 0;
+  s->head_fused_batch = true;
+  if (const char* v = getenv("DG_HEAD_FUSED_BATCH")) s->head_fused_batch = atoi(v) != 0;
   s->dstep = reinterpret_cast<int*>(b + L.dstep);
   s->bsteps = reinterpret_cast<int*>(b + L.bsteps);
   s->attn_plan_P = -1;
@@ -1062,29 +1066,44 @@ dg_status issue_step(dg_seqs* s, const dg_sampler_params* p, int32_t* d_ids, uin
   a.d_step = d_step;
   a.t_start = p->t_start;
   a.t_end = p->t_end;
-  if (s->L.R == kCanvas && s->head_nv > 0) {
-    // one canvas: the head's logits folded into the sampler's per-row reductions tile by tile in
-    // TMEM (the logits reach HBM only as the optional debug copy), then the step rule
-    HeadSamplerArgs hs{};
-    hs.d = c.d_model;
-    hs.vocab = c.vocab;
-    hs.seq_P = s->seqP;
-    hs.commit_in = d_commit;
-    hs.inv_temp = a.inv_temp;
-    hs.seed = p->seed;
-    hs.step = s->step;
-    hs.partial = s->hsamp;
-    hs.logits_out = d_logits_out;
-    hs.d_step = d_step;
-    hs.t_start = p->t_start;
-    hs.t_end = p->t_end;
-    hs.max_steps = p->max_steps;
+  if (s->head_nv > 0 && (s->L.R == kCanvas || s->head_fused_batch)) {
+    // the head's logits folded into the sampler's per-row reductions tile by tile in TMEM (the logits
+    // reach HBM only as the optional debug copy), then the step rule; one canvas per pass (each pass
+    // streams the head once: at 32 canvases 32 passes of 0.37 ms against a dense head GEMM of 11.7 ms that
+    // writes 8.6 GB of logits and a sampler pass of 4.8 ms that reads them)
     const int n_ctas = head_sampler_ctas(c.vocab, s->head_nv, s->m->n_sms);
-    a.partial = s->hsamp;
-    a.n_chunks = n_ctas;
-    LAUNCH(s, DG_K_HEAD, 3,
-           head_sampler_run(s->xn_map, s->head_nv == 256 ? s->m->head_map : s->m->head_map128, s->head_nv, hs, n_ctas,
-                            a, s->err, s->st));
+    for (int i = 0; i < s->n_seq; ++i) {
+      HeadSamplerArgs hs{};
+      hs.d = c.d_model;
+      hs.vocab = c.vocab;
+      hs.row0 = i * kCanvas;
+      hs.seq_P = s->seqP + i;
+      hs.commit_in = d_commit + (size_t)i * kCanvas;
+      hs.inv_temp = a.inv_temp;
+      hs.seed = p->seed + (uint64_t)i;       // sequence i's stream
+      hs.step = s->step;
+      hs.partial = s->hsamp;
+      hs.logits_out = d_logits_out ? d_logits_out + (size_t)i * kCanvas * c.vocab : nullptr;
+      hs.d_step = d_step;
+      hs.t_start = p->t_start;
+      hs.t_end = p->t_end;
+      hs.max_steps = p->max_steps;
+      SamplerArgs ai = a;
+      ai.n_seq = 1;
+      ai.seq_P = s->seqP + i;
+      ai.ids_in = d_ids + (size_t)i * kCanvas;
+      ai.commit_in = d_commit + (size_t)i * kCanvas;
+      ai.ids_out = d_ids + (size_t)i * kCanvas;
+      ai.commit_out = d_commit + (size_t)i * kCanvas;
+      ai.entropy = d_entropy + (size_t)i * kCanvas;
+      ai.stop = d_stop + i;
+      ai.seed = p->seed + (uint64_t)i;
+      ai.partial = s->hsamp;
+      ai.n_chunks = n_ctas;
+      LAUNCH(s, DG_K_HEAD, 3,
+             head_sampler_run(s->xn_map, s->head_nv == 256 ? s->m->head_map : s->m->head_map128, s->head_nv, hs,
+                              n_ctas, ai, s->err, s->st));
+    }
     return DG_OK;
   }
   if (s->L.R <= kCanvas) {

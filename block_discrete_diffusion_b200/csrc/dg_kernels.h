@@ -251,6 +251,7 @@ int sampler_chunks(int vocab);
 // vocabulary head fused with the sampler's reductions, one canvas (head_sampler.cu)
 struct HeadSamplerArgs {
   int d, vocab;
+  int row0;                // first row of this canvas in the normed-row map (canvas c of a batch: 256 c)
   const int* seq_P;        // committed length of the sequence (device; nullptr -> 0)
   const uint8_t* commit_in;
   float inv_temp;

@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(kHsThreads, 1)
       for (int kb = 0; kb < npre; ++kb) {
         uint8_t* a = tiles + (size_t)kb * C::kStage;
         mbar_arrive_expect_tx(&bars->full[kb], 2 * kHsATile);
-        tma_load_2d(&tmA, &bars->full[kb], a, kb * 64, 0);
-        tma_load_2d(&tmA, &bars->full[kb], a + kHsATile, kb * 64, 128);
+        tma_load_2d(&tmA, &bars->full[kb], a, kb * 64, p.row0);
+        tma_load_2d(&tmA, &bars->full[kb], a + kHsATile, kb * 64, p.row0 + 128);
       }
       uint32_t it = 0;
       bool ok = true;
@@ -205,8 +205,8 @@ __global__ void __launch_bounds__(kHsThreads, 1)
           }
           uint8_t* a = tiles + (size_t)s * C::kStage;
           mbar_arrive_expect_tx(&bars->full[s], C::kStage);
-          tma_load_2d(&tmA, &bars->full[s], a, kb * 64, 0);
-          tma_load_2d(&tmA, &bars->full[s], a + kHsATile, kb * 64, 128);
+          tma_load_2d(&tmA, &bars->full[s], a, kb * 64, p.row0);
+          tma_load_2d(&tmA, &bars->full[s], a + kHsATile, kb * 64, p.row0 + 128);
           tma_load_2d_hint(&tmB, &bars->full[s], a + 2 * kHsATile, kb * 64, item * NV, pol_w);
         }
       }
@@ -384,7 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHsThreads, 1)
           uint8_t* a = tiles + (size_t)s * kHpStage;
           if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], 2 * kHpStage);   // both CTAs' bytes
           const uint32_t bar = lead_full0 + (uint32_t)(s * sizeof(uint64_t));
-          tma_load_2d_pair(&tmA, bar, a, kb * 64, (int)rank * 128, pol_a);                       // canvas rows
+          tma_load_2d_pair(&tmA, bar, a, kb * 64, p.row0 + (int)rank * 128, pol_a);                       // canvas rows
           tma_load_2d_pair(&tmB, bar, a + kHsATile, kb * 64, item * NV + (int)rank * 128, pol_w);  // head rows
         }
       }
