@@ -75,6 +75,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int DH>
+__device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int seq, int h, int j, __nv_bfloat16* out,
+                                          int lane);
+
+template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, AttnParams p, int n_seq, __nv_bfloat16* out, int* err) {
@@ -369,25 +373,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 9) tmem_dealloc(tmem, C::kTmemCols);
+  if (p.n_splits > 1 && p.merge_in_cluster) {
+    // the pair's splits are the CTAs of this cluster (cluster dims (1, n_splits, 1)): once every split's
+    // partials are written (the barrier's release / acquire at cluster scope makes them visible), CTA
+    // `split` merges its share of the pair's 256 rows, one warp per row
+    cluster_sync();
+    const int per = (256 + p.n_splits - 1) / p.n_splits;
+    const int q1 = min(256, (split + 1) * per);
+    for (int q = split * per + warp; q < q1; q += kAttnThreads / 32) {
+      const int rr = pair * 256 + q;
+      const int g = rr / p.rows_per_seq, j = rr % p.rows_per_seq;
+      if (g < G && j < p.Tq) merge_row<DH>(p, n_seq, seq, kvh * G + g, j, out, lane);
+    }
+  }
 }
 
 // One warp per (sequence, query head, row): combine the split partials (lane s < n_splits holds
 // split s's (m, l)) and write the row of the token-major attention output
-// [seq*rows_per_seq + j][h*dh + c] in bf16; each lane owns dh/32 consecutive columns.
+// [seq*rows_per_seq + j][h*dh + c] in bf16; each lane owns dh/32 consecutive columns.  Loads bypass
+// L1 (in the in-cluster merge the partials come from other CTAs of the same launch).
 template <int DH>
-__global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
-  pdl_trigger();
-  pdl_wait();
-  const int warp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (warp >= n_seq * p.n_q * p.Tq) return;
-  const int j = warp % p.Tq;
-  const int sh = warp / p.Tq;          // seq * n_q + h
-  const int seq = sh / p.n_q, h = sh % p.n_q;
+__device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int seq, int h, int j, __nv_bfloat16* out,
+                                          int lane) {
+  const int sh = seq * p.n_q + h;
   const size_t stride = (size_t)n_seq * p.n_q * p.rows_per_seq;
   const size_t r0 = (size_t)sh * p.rows_per_seq + j;
   float ms = -INFINITY, ls = 0.f;
   if (lane < p.n_splits) {
-    const float2 v = *reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2);
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2));
     ms = v.x;
     ls = v.y;
   }
@@ -410,10 +423,10 @@ __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
       for (int c = 0; c < kPer; ++c) v[u][c] = 0.f;
       if (s < p.n_splits) {
         if constexpr (kPer == 4) {
-          const float4 q = *reinterpret_cast<const float4*>(src);
+          const float4 q = __ldcg(reinterpret_cast<const float4*>(src));
           v[u][0] = q.x; v[u][1] = q.y; v[u][2] = q.z; v[u][3] = q.w;
         } else {
-          const float2 q = *reinterpret_cast<const float2*>(src);
+          const float2 q = __ldcg(reinterpret_cast<const float2*>(src));
           v[u][0] = q.x; v[u][1] = q.y;
         }
       }
@@ -437,6 +450,17 @@ __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
 }
 
 template <int DH>
+__global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (warp >= n_seq * p.n_q * p.Tq) return;
+  const int j = warp % p.Tq;
+  const int sh = warp / p.Tq;          // seq * n_q + h
+  merge_row<DH>(p, n_seq, sh / p.n_q, sh % p.n_q, j, out, lane);
+}
+
+template <int DH>
 static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
   using C = AttnCfg<DH>;
@@ -449,14 +473,38 @@ static cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, con
   }
   const int G = p.n_q / p.n_kv;
   dim3 grid((G * p.rows_per_seq + 255) / 256, p.n_splits, n_seq * p.n_kv);
-  return launch_k(attn_fwd_kernel<DH>, grid, dim3(kAttnThreads), C::kSmemBytes, st, 1, tq, tk, tv, p, n_seq, out,
-                  err);
+  if (!(p.n_splits > 1 && p.merge_in_cluster))
+    return launch_k(attn_fwd_kernel<DH>, grid, dim3(kAttnThreads), C::kSmemBytes, st, 1, tq, tk, tv, p, n_seq, out,
+                    err);
+  // the splits of a query-tile pair as one cluster (1, n_splits, 1)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  attr[n].id = cudaLaunchAttributeClusterDimension;
+  attr[n].val.clusterDim.x = 1;
+  attr[n].val.clusterDim.y = p.n_splits;
+  attr[n].val.clusterDim.z = 1;
+  ++n;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<DH>, tq, tk, tv, p, n_seq, out, err);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // n_splits == 1: the attention output is written directly to `out`; otherwise the partials are
-// left for attention_merge.
+// merged inside the launch (merge_in_cluster, n_splits <= 8) or left for attention_merge.
 cudaError_t attention_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const AttnParams& p, int n_seq, __nv_bfloat16* out, int* err, cudaStream_t st) {
+  if (p.merge_in_cluster && p.n_splits > 8) return cudaErrorInvalidValue;   // portable cluster size
   if (p.dh == 128) return launch_attn<128>(tq, tk, tv, p, n_seq, out, err, st);
   if (p.dh == 64) return launch_attn<64>(tq, tk, tv, p, n_seq, out, err, st);
   return cudaErrorInvalidValue;

@@ -410,6 +410,7 @@ struct dg_seqs {
   int step;
   bool block_open;
   int max_splits;   // upper bound on attention key splits (DG_ATTN_MAX_SPLITS, default: no extra bound)
+  bool attn_cluster_merge;   // key splits merged inside the attention launch (DG_ATTN_CLUSTER_MERGE=1; off by default)
   int pre_bytes;    // bytes per weight row the gate|up GEMM brings into L2 before its wait (DG_EXPERT_PREFETCH)
   bool prefetch_early;   // merged expert launch: the top-k launch issues that prefetch too (DG_PREFETCH_EARLY=1)
   int head_nv;      // one canvas: tiling of the fused head + sampler (kHeadSamplerPair: CTA pairs; 128 or 256
@@ -653,6 +654,8 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->next_pair = 0;
   s->max_splits = kMaxSplits;
   if (const char* v = getenv("DG_ATTN_MAX_SPLITS")) s->max_splits = std::max(1, atoi(v));
+  s->attn_cluster_merge = false;
+  if (const char* v = getenv("DG_ATTN_CLUSTER_MERGE")) s->attn_cluster_merge = atoi(v) != 0;
   s->pre_bytes = 1 << 20;   // capped at the row length: the whole first tile
   s->head_nv = kHeadSamplerPair;   // CTA pairs: the fastest form measured on B200 (0.44 vs 0.47 ms at V 262144)
   if (const char* v = getenv("DG_HEAD_SAMPLER")) {
@@ -798,14 +801,23 @@ dg_status run_layer(dg_seqs* s, int l, float* x, int rows, int n_local, int seq_
   ap.seq_base = seq_base;
   ap.cache_seq_stride = s->n_seq * c.n_kv;
   ap.layer = l;
-  const int sp = std::min(std::min(s->L.split_cap, s->max_splits), ntiles);
+  int sp = std::min(std::min(s->L.split_cap, s->max_splits), ntiles);
+  // With DG_ATTN_CLUSTER_MERGE=1, the splits of a query-tile pair merged inside the attention launch over a
+  // cluster of at most 8 CTAs, for direct calls whose launch is one wave (with several waves the merging
+  // CTAs hold their SMs from the next wave, and inside the device-resident loop's graph the step got slower).
+  // Off by default: at batch 1 it saved 0.08 ms per step behind a 2048-token prompt but cost 22 us per layer
+  // behind 4096 positions.
+  const int units = ((c.n_q / c.n_kv) * kCanvas + 255) / 256 * n_local * c.n_kv;
+  const bool cmerge = s->attn_cluster_merge && s->attn_plan_P < 0 && sp > 1 && units * std::min(sp, 8) <= s->m->n_sms;
+  if (cmerge) sp = std::min(sp, 8);
   ap.tiles_per_split = (ntiles + sp - 1) / sp;
   ap.n_splits = (ntiles + ap.tiles_per_split - 1) / ap.tiles_per_split;
   ap.seq_P = s->seqP;
   ap.opart = s->opart;
   ap.ml = s->ml;
+  ap.merge_in_cluster = cmerge ? 1 : 0;
   LAUNCH(s, DG_K_ATTN, 1, attention_fwd(s->q_map, s->k_map, s->v_map, ap, n_local, s->attn, s->err, st));
-  if (ap.n_splits > 1) LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
+  if (ap.n_splits > 1 && !ap.merge_in_cluster) LAUNCH(s, DG_K_ATTN_MERGE, 1, attention_merge(ap, n_local, s->attn, st));
 
   // Few rows: the FFN RMSNorm and the router fold into the O epilogue (the router is linear and the
   // RMSNorm scales a row by one factor: logits = (x' g) W^T / rms(x')), and the gather forms the

@@ -126,6 +126,8 @@ struct AttnParams {
   const int* seq_P;
   float* opart;          // [split][seq][n_q][rows_per_seq][dh] un-normalised partial outputs
   float* ml;             // [split][seq][n_q][rows_per_seq][2] (running max in log2 units, sum)
+  int merge_in_cluster;  // n_splits > 1: the splits of a query-tile pair form a thread-block cluster and
+                         // merge their partials after a cluster barrier (no attention_merge launch)
 };
 
 cudaError_t gemm_dense(int bn, int epi, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,

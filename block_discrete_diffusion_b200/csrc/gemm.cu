@@ -191,6 +191,7 @@ struct RouterFrags {
   uint32_t b[4][8][2];
   float2 g[8][2];
 };
+template <bool WITH_B>
 __device__ __forceinline__ void router_frags_load(const EpiParams& ep, int n0, RouterFrags& f) {
   constexpr int NW = kGemmThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,6 +201,7 @@ __device__ __forceinline__ void router_frags_load(const EpiParams& ep, int n0, R
     f.g[ks][0] = __ldg(reinterpret_cast<const float2*>(ep.rg + n0 + 16 * ks + 2 * tig));
     f.g[ks][1] = __ldg(reinterpret_cast<const float2*>(ep.rg + n0 + 16 * ks + 8 + 2 * tig));
   }
+  if constexpr (!WITH_B) return;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int nt = warp + NW * j;
@@ -214,13 +216,32 @@ __device__ __forceinline__ void router_frags_load(const EpiParams& ep, int n0, R
   }
 }
 
+// The tile's 128 columns of the router weights W[e][n0 + c] into shared memory with asynchronous copies
+// (rows of kRwPitch bytes: 256 + 16, so that the eight rows an ldmatrix reads fall in different banks).
+constexpr int kRwPitch = 272;
+__device__ __forceinline__ void router_w_to_smem(const EpiParams& ep, int n0, uint8_t* wr_s) {
+  for (int i = threadIdx.x; i < ep.n_exp * 16; i += kGemmThreads) {
+    const int e = i >> 4, c16 = i & 15;
+    const __nv_bfloat16* src = ep.rw + (size_t)e * ep.ldo + n0 + c16 * 8;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(wr_s + e * kRwPitch + c16 * 16)),
+                 "l"(src)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // The router's share of the tile (ep.rw): rpart[n0/128][row][e] = sum over the tile's 128 columns c of
 // bf16(x'[row][c] g[c]) * W[e][c], for the RPC updated rows held in shared memory.  A small product
 // (RPC x n_exp x 128), so it runs on warp-level mma.sync (16 rows x 8 experts x 16 columns per
 // instruction, fp32 accumulation) inside the epilogue; warp w takes the 8-expert groups w, w + 4, ...
-template <int RPC>
+template <int RPC, bool B_SMEM>
 __device__ __forceinline__ void router_partial_from_smem(const EpiParams& ep, const RouterFrags& f, const float* t,
-                                                         int rs, int row0, int n0, int M) {
+                                                         int rs, int row0, int n0, int M, const uint8_t* wr_s) {
   static_assert(RPC % 16 == 0, "16-row blocks");
   constexpr int NW = kGemmThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -249,8 +270,22 @@ __device__ __forceinline__ void router_partial_from_smem(const EpiParams& ep, co
       const int nt = warp + NW * j;
       if (nt < ep.n_exp / 8) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (B_SMEM) {
+          // B fragments of two column steps per ldmatrix.x4: lanes 8 m .. 8 m + 7 address the group's rows at
+          // columns 16 (ks + m / 2) + 8 (m % 2)
+          const int mi = lane >> 3;
+          const uint32_t rowa = smem_u32(wr_s + (nt * 8 + (lane & 7)) * kRwPitch) + (uint32_t)(((mi >> 1) * 16 + (mi & 1) * 8) * 2);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_bf16_m16n8k16(c, a[ks], f.b[j][ks][0], f.b[j][ks][1]);
+          for (int ks = 0; ks < 8; ks += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(rowa + ks * 32, b0, b1, b2, b3);
+            mma_bf16_m16n8k16(c, a[ks], b0, b1);
+            mma_bf16_m16n8k16(c, a[ks + 1], b2, b3);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) mma_bf16_m16n8k16(c, a[ks], f.b[j][ks][0], f.b[j][ks][1]);
+        }
         const int e = nt * 8 + 2 * tig;
         if (ra < M) *reinterpret_cast<float2*>(out + (size_t)ra * ep.n_exp + e) = make_float2(c[0], c[1]);
         if (ra + 8 < M) *reinterpret_cast<float2*>(out + (size_t)(ra + 8) * ep.n_exp + e) = make_float2(c[2], c[3]);
@@ -349,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
   tc_fence_after();
   RouterFrags rf;
   if constexpr (EPI == EPI_RESID && BN == 128) {
-    if (ep.rw) router_frags_load(ep, n0, rf);
+    if (ep.rw) router_frags_load<Z == 1>(ep, n0, rf);   // Z > 1: the weights go to shared memory below
   }
   const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
 
@@ -372,7 +407,7 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       if constexpr (EPI == EPI_RESID && BN == 128) {
         if (ep.rw) {
           __syncthreads();
-          router_partial_from_smem<128>(ep, rf, red, RS, m0, n0, M);
+          router_partial_from_smem<128, false>(ep, rf, red, RS, m0, n0, M, nullptr);
         }
       }
     }
@@ -403,6 +438,13 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
     // every slot of the tile is written (the barrier's release / acquire at cluster scope makes the
     // peers' global stores visible), and this CTA's shared tile is free again
     cluster_sync();
+    // the folded router's weight columns into the shared memory past the reduced rows (in flight during the
+    // reduction and the residual epilogue)
+    uint8_t* wr_s = reinterpret_cast<uint8_t*>(red + RPC * RS);
+    if constexpr (EPI == EPI_RESID && BN == 128) {
+      static_assert((size_t)RPC * RS * 4 + 128 * kRwPitch <= (size_t)C::kStages * C::kStageBytes, "router staging");
+      if (ep.rw) router_w_to_smem(ep, n0, wr_s);
+    }
     {
       constexpr int IT = RPC * F4 / kGemmThreads;           // float4 per thread
       constexpr int B = IT < 16 / Z ? IT : 16 / Z;          // iterations whose Z loads are in flight together
@@ -432,8 +474,9 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       epilogue_from_smem<BN, EPI, RPC>(ep, red, RS, m0 + zz * RPC, n0, M, N);
       if constexpr (EPI == EPI_RESID && BN == 128) {
         if (ep.rw) {
+          asm volatile("cp.async.wait_all;" ::: "memory");
           __syncthreads();
-          router_partial_from_smem<RPC>(ep, rf, red, RS, m0 + zz * RPC, n0, M);
+          router_partial_from_smem<RPC, true>(ep, rf, red, RS, m0 + zz * RPC, n0, M, wr_s);
         }
       }
     }

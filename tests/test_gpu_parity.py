@@ -175,15 +175,19 @@ def _layer_case(dg, cfg, P, seed, router_std=None):
     ("tiny", 0, 256, False, "folded"), ("tiny", 128, 256, False, "folded"), ("tiny", 300, 256, False, "folded"),
     ("tiny", 0, 44, True, "folded"), ("tiny", 256, 128, True, "folded"), ("tiny", 200, 56, True, "folded"),
     ("tiny", 384, 256, True, "folded"), ("tiny", 128, 256, False, "separate"), ("tiny", 200, 56, True, "separate"),
+    ("tiny", 300, 256, False, "cluster_merge"),
     ("one_layer", 4096, 256, False, "folded"), ("one_layer", 2048, 200, True, "folded"),
-    ("one_layer", 4096, 256, False, "separate"),
+    ("one_layer", 4096, 256, False, "separate"), ("one_layer", 4096, 256, False, "cluster_merge"),
 ])
 def test_layer_matches_oracle(dg, monkeypatch, cfg_name, P, n_rows, causal, route):
     """One layer (attention block, then MoE block) on canvas rows (bidirectional) or on a prefill
     chunk (causal, ragged row counts), against a committed prefix of P positions.  route "folded":
     the FFN RMSNorm and the router folded into the O-projection epilogue (the default for up to 1024
-    rows); "separate": DG_ROUTE_FUSED=0, an RMSNorm launch and a router GEMM."""
-    monkeypatch.setenv("DG_ROUTE_FUSED", "1" if route == "folded" else "0")
+    rows) and the attention's key splits merged by a launch of their own (the defaults); "separate":
+    DG_ROUTE_FUSED=0, an RMSNorm launch and a router GEMM; "cluster_merge": DG_ATTN_CLUSTER_MERGE=1,
+    the key splits merged inside the attention launch over a thread-block cluster."""
+    monkeypatch.setenv("DG_ROUTE_FUSED", "0" if route == "separate" else "1")
+    monkeypatch.setenv("DG_ATTN_CLUSTER_MERGE", "1" if route == "cluster_merge" else "0")
     if cfg_name == "tiny":
         cfg, router_std = synthetic.TINY, None
     else:
