@@ -96,6 +96,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int G = p.n_q / p.n_kv;
   const int cseq = p.seq_base + seq;
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);

@@ -112,6 +112,10 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                      ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* stage_out = reinterpret_cast<float*>(tiles + (size_t)kF8Stages * kF8Stage);
   // [2][kF8MaxSl][32 tokens] combined scales s_w * s_a per (weight-row half, slice, token) of a chunk
@@ -397,6 +401,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFpThreads, 1)
                           ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* amx = reinterpret_cast<float*>(tiles + (size_t)kFpStages * kFpStage);   // [2][128]: half-block amax
   int* s_cum = reinterpret_cast<int*>(amx + 256);                                // first item of each expert

@@ -317,6 +317,10 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
   const int kb0 = zz * nk_all / Z;
   const int nk = (zz + 1) * nk_all / Z - kb0;
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -552,6 +556,10 @@ __global__ void __launch_bounds__(FP8 ? kExpThreadsFp8 : kExpThreads, 1)
                        ExpertParams p, int n_exp, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
   uint8_t* tiles = align1024(smem_raw);
   using C = ExpCfg<BN, FP8>;
   constexpr int kExpStages = C::kStages;
@@ -849,6 +857,12 @@ __global__ void __launch_bounds__(kExpThreads, 1)
                          ExpertParams p, int n_exp, int* done, int* err) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmWu);
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmWd);
+    tma_prefetch_desc(&tmH);
+  }
   uint8_t* tiles = align1024(smem_raw);
   using C = ExpCfg<BN, false>;
   constexpr int kStages = C::kStages;

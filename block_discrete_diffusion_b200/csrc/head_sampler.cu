@@ -151,6 +151,10 @@ __global__ void __launch_bounds__(kHsThreads, 1)
   using C = HsCfg<NV>;
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   HsBarriers* bars = reinterpret_cast<HsBarriers*>(tiles + (size_t)C::kStages * C::kStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -339,6 +343,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHsThreads, 1)
   constexpr int NV = 256;                       // vocabulary rows per item (128 per CTA)
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
+  if (threadIdx.x == 0) {   // descriptors into the TMA unit's cache while the previous kernel still runs
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   HpBarriers* bars = reinterpret_cast<HpBarriers*>(tiles + (size_t)kHpStages * kHpStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
