@@ -226,9 +226,9 @@ def run_steps(dg, seqs, prm, st, k, state, nvtx=False):
 # 1,028,473,600 + 3,732,224.  Set to None when the kernel changes until it is captured again.
 EXPERT_UP_TRAFFIC_BF16 = 1_028_473_600 + 3_732_224
 # DRAM bytes (read + write) of one merged gate|up -> down launch at batch 1 (bf16), from an ncu capture of
-# that kernel on the one-layer workload (profiles/expert_updown_one_layer_b1.md): 1,536,471,296 +
-# 4,139,776.  None when the kernel changes until it is captured again.
-EXPERT_UPDOWN_TRAFFIC_BF16 = 1_536_471_296 + 4_139_776
+# that kernel on the one-layer workload (profiles/expert_updown_one_layer_b1.md): 1,536,429,824 +
+# 6,081,280.  None when the kernel changes until it is captured again.
+EXPERT_UPDOWN_TRAFFIC_BF16 = 1_536_429_824 + 6_081_280
 
 # DRAM bytes (read + write) of one sampler_partial_kernel launch on the 256 x 262144 sampler workload,
 # from an ncu capture of this kernel: 268,503,552 + 3,422,720.  None when the kernel changes until it is

@@ -37,8 +37,8 @@ def _tiny(wdtype, head_scale=50.0, seed=0):
 PAIR_CASES = [(1, 50.0, "pair"), (1, 1.0, "pair")] if os.environ.get("DG_TEST_FP8_PAIR") == "1" else []
 
 
-@pytest.mark.parametrize("wdtype,head_scale,experts", [(0, 50.0, "expand"), (1, 50.0, "expand"), (1, 1.0, "expand")]
-                         + PAIR_CASES)
+@pytest.mark.parametrize("wdtype,head_scale,experts", [(0, 50.0, "expand"), (1, 50.0, "expand"), (1, 1.0, "expand"),
+                                                        (0, 50.0, "dense_head")] + PAIR_CASES)
 def test_batched_sequences_match_their_oracles(dg, monkeypatch, wdtype, head_scale, experts):
     """Three sequences (prompts of 128, 300 and 0 tokens) prefilled, initialised and stepped in one
     batch; each sequence's hidden states, logits and sampler decisions match its own oracle run
@@ -46,12 +46,16 @@ def test_batched_sequences_match_their_oracles(dg, monkeypatch, wdtype, head_sca
     entropies judged with the derived large-logit tolerances; head x1: the base tolerances.  The tiny
     model routes hundreds of tokens to each expert: with FP8 weights the expert GEMMs run on the
     CTA-pair e4m3 x e4m3 kernels ("pair"), or with DG_FP8_PAIR=0 on the kernels that expand the
-    weights to bf16 ("expand").  The e4m3 kernels also quantize the expert inputs (per token and 128
+    weights to bf16 ("expand"); "dense_head" runs the batch's head as one dense GEMM and the sampler over
+    its logits instead of the fused head + sampler per canvas.  The e4m3 kernels also quantize the expert inputs (per token and 128
     channels / 64 features), which the oracle does not: the hidden states and logits are still judged
     against the oracle at 6e-2, and the sampler's decisions on the GPU's own logits with the base
     tolerances (at large logits the quantized activations move decisions that the oracle's exact
     activations fix)."""
     monkeypatch.setenv("DG_FP8_PAIR", "1" if experts == "pair" else "0")
+    # "dense_head": the batch's head as one dense GEMM over all canvases, then the sampler over the logits
+    # (DG_HEAD_FUSED_BATCH=0); otherwise the fused head + sampler once per canvas
+    monkeypatch.setenv("DG_HEAD_FUSED_BATCH", "0" if experts == "dense_head" else "1")
     e4m3_act = wdtype == 1 and experts == "pair"
     cfg, w = _tiny(wdtype, head_scale)
     tol = HIDDEN_TOL if wdtype == 0 else HIDDEN_TOL_FP8

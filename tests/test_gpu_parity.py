@@ -312,13 +312,18 @@ def _diagnose(hg, r, l, keep, cfg):
     return "; ".join(out)
 
 
-@pytest.mark.parametrize("top_k,head,router,prompt_len,n_steps", [
-    (8, "x1", "unit", 128, 4), (8, "x1", "unit", 300, 3), (8, "x50", "unit", 128, 48), (8, "x50", "unit", 300, 6),
-    (8, "copy", "unit", 128, 48),
-    (2, "x1", "stated", 128, 48),      # the tiny configuration as stated: top-2, head x1, 48-step adaptive run
-    (2, "x1", "unit", 128, 12), (2, "x50", "unit", 300, 48), (2, "copy", "stated", 128, 48),
+@pytest.mark.parametrize("top_k,head,router,prompt_len,n_steps,head_impl", [
+    (8, "x1", "unit", 128, 4, "pair"), (8, "x1", "unit", 300, 3, "pair"), (8, "x50", "unit", 128, 48, "pair"),
+    (8, "x50", "unit", 300, 6, "pair"), (8, "copy", "unit", 128, 48, "pair"),
+    (2, "x1", "stated", 128, 48, "pair"),   # the tiny configuration as stated: top-2, head x1, 48-step adaptive run
+    (2, "x1", "unit", 128, 12, "pair"), (2, "x50", "unit", 300, 48, "pair"), (2, "copy", "stated", 128, 48, "pair"),
+    (8, "x50", "unit", 128, 6, "unfused"), (8, "copy", "unit", 300, 6, "nv128"),
 ])
-def test_canvas_steps_match_oracle(dg, top_k, head, router, prompt_len, n_steps):
+def test_canvas_steps_match_oracle(dg, monkeypatch, top_k, head, router, prompt_len, n_steps, head_impl):
+    """head_impl: the vocabulary head + sampler of the step as the fused CTA-pair kernel (the default),
+    the fused single-CTA kernel with 128 vocabulary rows per tile (DG_HEAD_SAMPLER=128), or the head GEMM
+    followed by the sampler kernels (DG_HEAD_SAMPLER=0)."""
+    monkeypatch.setenv("DG_HEAD_SAMPLER", {"pair": "2", "nv128": "128", "unfused": "0"}[head_impl])
     cfg, w, model, M = _tiny_model_pair(dg, head, top_k=top_k, router=router)
     max_ctx = 1024
     seqs = dg.dg_seqs_create(model, 1, max_ctx)
