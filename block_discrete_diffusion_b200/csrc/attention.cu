@@ -74,7 +74,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-template <int DH>
+template <int DH, bool CG>
 __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int seq, int h, int j, __nv_bfloat16* out,
                                           int lane);
 
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int q = split * per + warp; q < q1; q += kAttnThreads / 32) {
       const int rr = pair * 256 + q;
       const int g = rr / p.rows_per_seq, j = rr % p.rows_per_seq;
-      if (g < G && j < p.Tq) merge_row<DH>(p, n_seq, seq, kvh * G + g, j, out, lane);
+      if (g < G && j < p.Tq) merge_row<DH, true>(p, n_seq, seq, kvh * G + g, j, out, lane);
     }
   }
 }
@@ -396,8 +396,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // One warp per (sequence, query head, row): combine the split partials (lane s < n_splits holds
 // split s's (m, l)) and write the row of the token-major attention output
 // [seq*rows_per_seq + j][h*dh + c] in bf16; each lane owns dh/32 consecutive columns.  Loads bypass
-// L1 (in the in-cluster merge the partials come from other CTAs of the same launch).
-template <int DH>
+// L1 when CG (in the in-cluster merge the partials come from other CTAs of the same launch).
+template <typename T>
+__device__ __forceinline__ T ld_partial(const T* p, bool cg) {
+  return cg ? __ldcg(p) : *p;
+}
+template <int DH, bool CG>
 __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int seq, int h, int j, __nv_bfloat16* out,
                                           int lane) {
   const int sh = seq * p.n_q + h;
@@ -405,7 +409,7 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
   const size_t r0 = (size_t)sh * p.rows_per_seq + j;
   float ms = -INFINITY, ls = 0.f;
   if (lane < p.n_splits) {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2));
+    const float2 v = ld_partial(reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2), CG);
     ms = v.x;
     ls = v.y;
   }
@@ -428,10 +432,10 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
       for (int c = 0; c < kPer; ++c) v[u][c] = 0.f;
       if (s < p.n_splits) {
         if constexpr (kPer == 4) {
-          const float4 q = __ldcg(reinterpret_cast<const float4*>(src));
+          const float4 q = ld_partial(reinterpret_cast<const float4*>(src), CG);
           v[u][0] = q.x; v[u][1] = q.y; v[u][2] = q.z; v[u][3] = q.w;
         } else {
-          const float2 q = __ldcg(reinterpret_cast<const float2*>(src));
+          const float2 q = ld_partial(reinterpret_cast<const float2*>(src), CG);
           v[u][0] = q.x; v[u][1] = q.y;
         }
       }
@@ -462,7 +466,7 @@ __global__ void attn_merge_kernel(AttnParams p, int n_seq, __nv_bfloat16* out) {
   if (warp >= n_seq * p.n_q * p.Tq) return;
   const int j = warp % p.Tq;
   const int sh = warp / p.Tq;          // seq * n_q + h
-  merge_row<DH>(p, n_seq, sh / p.n_q, sh % p.n_q, j, out, lane);
+  merge_row<DH, false>(p, n_seq, sh / p.n_q, sh % p.n_q, j, out, lane);
 }
 
 template <int DH>
