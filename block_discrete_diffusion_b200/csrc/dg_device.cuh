@@ -18,6 +18,7 @@ enum : int {
   DEV_ERR_TIMEOUT_EPILOGUE = 3,   // epilogue waited too long for the accumulator
   DEV_ERR_TIMEOUT_ATTN = 4,       // attention pipeline wait ran out
   DEV_ERR_BAD_INDEX = 5,          // an id or index outside its range was seen and skipped
+  DEV_ERR_TIMEOUT_ROUTE = 6,      // a top-k CTA waited too long for the expert offsets of its launch
 };
 
 // Every spin-wait gives up after this many nanoseconds of %globaltimer and reports an error.

@@ -202,6 +202,23 @@ struct ExpertPrefetchArgs {
 cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
                         int32_t* sel, float* gate, int32_t* counts, const FusedAssignArgs* fused,
                         const RouterNormArgs* norm, const ExpertPrefetchArgs* prefetch, cudaStream_t st);
+// One canvas: top-k, bucketing and the gather in one launch (router_topk_gather_kernel; two rows per CTA,
+// all CTAs resident, so (n_rows + 1) / 2 <= n_sms).  sync: 3 zero-initialised ints (left zero on exit).
+struct TopkGatherLaunch {
+  GatherSrc src;
+  __nv_bfloat16* xp;
+  int d;
+  int32_t* sync;
+  int32_t* offsets;
+  int32_t* cursor;
+  int32_t* slot;
+  int32_t* zero;
+  int n_zero;
+  int* err;
+};
+cudaError_t router_topk_gather(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
+                               int32_t* sel, float* gate, int32_t* counts, const RouterNormArgs* norm,
+                               const TopkGatherLaunch& g, int n_sms, cudaStream_t st);
 // expert offsets and the bucketed row of every (token, rank) assignment; *n_launched = kernels used
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,
                         int32_t* offsets, int32_t* cursor, int32_t* slot, int* n_launched, cudaStream_t st);

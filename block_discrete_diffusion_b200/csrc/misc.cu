@@ -128,6 +128,19 @@ struct FusedAssign {   // the last CTA of the top-k launch also buckets the assi
   int32_t* slot;
 };
 
+struct TopkGatherArgs {   // router_topk_gather_kernel: the gather's source and destination, the bucketing state
+  GatherSrc src;
+  __nv_bfloat16* xp;
+  int d;
+  int32_t* sync;          // [3] zero-initialised: arrivals, offsets ready, leavers
+  int32_t* offsets;       // [n_exp + 1]
+  int32_t* cursor;        // [n_exp]
+  int32_t* slot;          // [n_rows * top_k]
+  int32_t* zero;          // nullable: n_zero ints cleared (the merged expert launch's counters)
+  int n_zero;
+  int* err;
+};
+
 struct ExpertPrefetch {   // w == nullptr: none
   const uint8_t* w;
   int n_ctas, F, d, row_bytes;
@@ -376,23 +389,15 @@ __device__ __forceinline__ uint4 norm8(const float4 (&x)[2], const float4 (&g)[2
                     pack_bf16x2(b.x * r * gb.x, b.y * r * gb.y), pack_bf16x2(b.z * r * gb.z, b.w * r * gb.w));
 }
 
-// xp[slot[t*k + r]] = row t for every rank r: one warp per token reads the row once.  The row is
-// xn[t] (bf16), or with FROM_X the FFN RMSNorm formed here, bf16(x[t] * rr[t] * g).
+// Row t into its k bucketed rows (lane r < top_k holds rank r's row `my_slot`), one warp: the row is
+// read once (xn[t], or with FROM_X the FFN RMSNorm formed here, bf16(x[t] * rr[t] * g)).
 template <bool FROM_X>
-__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const float* __restrict__ x,
-                                   const float* __restrict__ rr, const float* __restrict__ g,
-                                   const int32_t* __restrict__ slot, int n_rows, int top_k, int d,
-                                   __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ zero, int n_zero) {
-  pdl_trigger();
-  pdl_wait();
-  if (zero && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (t >= n_rows) return;
+__device__ __forceinline__ void gather_row(const __nv_bfloat16* __restrict__ xn, const float* __restrict__ x,
+                                           const float* __restrict__ rr, const float* __restrict__ g, int t,
+                                           int my_slot, int top_k, int d, __nv_bfloat16* __restrict__ xp, int lane) {
   const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
   const float* xr = x + (size_t)t * d;
   const float r = FROM_X ? rr[t] : 0.f;
-  const int my_slot = lane < top_k ? slot[(size_t)t * top_k + lane] : 0;   // rank `lane`'s row, loaded once
   const int n16 = d / 8;   // 16-byte chunks (8 elements) per bf16 row
   for (int c0 = 0; c0 < n16; c0 += 32 * 4) {
     uint4 v[4];
@@ -426,6 +431,114 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const f
         if (c < n16) dst[c] = v[u];
       }
     }
+  }
+}
+
+// xp[slot[t*k + r]] = row t for every rank r: one warp per token.
+template <bool FROM_X>
+__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn, const float* __restrict__ x,
+                                   const float* __restrict__ rr, const float* __restrict__ g,
+                                   const int32_t* __restrict__ slot, int n_rows, int top_k, int d,
+                                   __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ zero, int n_zero) {
+  pdl_trigger();
+  pdl_wait();
+  if (zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= n_rows) return;
+  const int my_slot = lane < top_k ? slot[(size_t)t * top_k + lane] : 0;   // rank `lane`'s row, loaded once
+  gather_row<FROM_X>(xn, x, rr, g, t, my_slot, top_k, d, xp, lane);
+}
+
+// One canvas, the gather folded into the top-k launch: one warp per row, two rows per CTA, every CTA
+// resident at once (the grid fits the SMs).  Each warp takes its row's top-k (as router_topk_kernel);
+// the last CTA to finish publishes the expert offsets (exclusive prefix of the counts) as cursors and
+// raises a flag; every warp, once the flag is up (bounded wait), takes a bucketed row per rank with an
+// atomic on its expert's cursor (row order inside an expert is free: each expert-GEMM column reads its
+// own row, the combine sums a token's rows in rank order) and copies its normed row there.  The last
+// CTA to leave lowers the flags for the next launch.  sync: [0] arrivals, [1] offsets ready, [2] leavers.
+template <int V, bool FROM_X>
+__global__ void router_topk_gather_kernel(const float* __restrict__ logits, int n_parts, size_t part_stride,
+                                          int n_rows, int n_exp, int top_k, int32_t* __restrict__ sel,
+                                          float* __restrict__ gate, int32_t* __restrict__ counts, RouterNorm rn,
+                                          TopkGatherArgs ga) {
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row < n_rows)
+    router_topk_row<V>(logits, n_parts, part_stride, row, n_rows, n_exp, top_k, sel, gate, counts, rn, lane);
+  __shared__ int s_last;
+  __shared__ int s_wsum[2];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ga.sync + 0, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    // offsets: exclusive prefix of the counts (n_exp <= 256; 64 threads, 4 experts each)
+    int c[4], tot = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = threadIdx.x * 4 + i;
+      c[i] = e < n_exp ? __ldcg(counts + e) : 0;
+      tot += c[i];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[threadIdx.x >> 5] = incl;
+    __syncthreads();
+    int run = incl - tot + ((threadIdx.x >> 5) ? s_wsum[0] : 0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = threadIdx.x * 4 + i;
+      if (e < n_exp) {
+        ga.offsets[e] = run;
+        ga.cursor[e] = run;
+        counts[e] = 0;      // consumed: cleared for the next layer's router
+      }
+      run += c[i];
+    }
+    if (threadIdx.x == 0) ga.offsets[n_exp] = s_wsum[0] + s_wsum[1];
+    for (int i = threadIdx.x; i < ga.n_zero; i += blockDim.x) ga.zero[i] = 0;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) atomicExch(ga.sync + 1, 1);
+  }
+  __shared__ int s_ready;
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    int ready = atomicAdd(ga.sync + 1, 0);
+    for (uint32_t i = 1; ready == 0; ++i) {
+      if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        report_error(ga.err, DEV_ERR_TIMEOUT_ROUTE);
+        break;
+      }
+      ready = atomicAdd(ga.sync + 1, 0);
+    }
+    s_ready = ready;
+  }
+  __syncthreads();
+  __threadfence();
+  // without the offsets (the wait ran out) the cursors are not valid: no row is taken or written
+  if (s_ready && row < n_rows) {
+    int my_slot = 0;
+    if (lane < top_k) {
+      const int e = sel[(size_t)row * top_k + lane];   // written by this lane above
+      my_slot = atomicAdd(ga.cursor + e, 1);
+      ga.slot[(size_t)row * top_k + lane] = my_slot;
+    }
+    gather_row<FROM_X>(ga.src.xn, ga.src.x, ga.src.r, ga.src.g, row, my_slot, top_k, ga.d, ga.xp, lane);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(ga.sync + 2, 1) == (int)gridDim.x - 1) {
+    ga.sync[0] = 0;
+    ga.sync[1] = 0;
+    ga.sync[2] = 0;
   }
 }
 
@@ -568,6 +681,35 @@ cudaError_t router_topk(const float* logits, int n_parts, size_t part_stride, in
   DG_TOPK_CASE(4)
   DG_TOPK_CASE(8)
 #undef DG_TOPK_CASE
+  return cudaErrorInvalidValue;
+}
+cudaError_t router_topk_gather(const float* logits, int n_parts, size_t part_stride, int n_rows, int n_exp, int top_k,
+                               int32_t* sel, float* gate, int32_t* counts, const RouterNormArgs* norm,
+                               const TopkGatherLaunch& g, int n_sms, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  const int V = (n_exp + 31) / 32;
+  const int blocks = (n_rows + 1) / 2;
+  if (n_exp > 256 || top_k > 32 || g.d % 8 || blocks > n_sms || !g.sync || !g.offsets || !g.cursor || !g.slot || !g.xp ||
+      (!g.src.xn && (!g.src.x || !g.src.r || !g.src.g)))
+    return cudaErrorInvalidValue;   // every CTA must be resident at once: the grid fits the SMs
+  RouterNorm rn{};
+  if (norm) {
+    if (!norm->ssq || !norm->r_out || !norm->logits_out || norm->n_ssq <= 0 || norm->d <= 0) return cudaErrorInvalidValue;
+    rn = RouterNorm{norm->ssq, norm->n_ssq, norm->d, norm->eps, norm->r_out, norm->logits_out};
+  }
+  const TopkGatherArgs ga{g.src, g.xp, g.d, g.sync, g.offsets, g.cursor, g.slot, g.zero, g.n_zero, g.err};
+  const bool fx = g.src.xn == nullptr;
+#define DG_TG_CASE(V_)                                                                                              \
+  if (V == V_)                                                                                                      \
+    return fx ? launch_k(router_topk_gather_kernel<V_, true>, dim3(blocks), dim3(64), 0, st, 1, logits, n_parts,     \
+                         part_stride, n_rows, n_exp, top_k, sel, gate, counts, rn, ga)                              \
+              : launch_k(router_topk_gather_kernel<V_, false>, dim3(blocks), dim3(64), 0, st, 1, logits, n_parts,    \
+                         part_stride, n_rows, n_exp, top_k, sel, gate, counts, rn, ga);
+  DG_TG_CASE(1)
+  DG_TG_CASE(2)
+  DG_TG_CASE(4)
+  DG_TG_CASE(8)
+#undef DG_TG_CASE
   return cudaErrorInvalidValue;
 }
 cudaError_t assign_rows(const int32_t* sel, const float* gate, int32_t* counts, int n_rows, int top_k, int n_exp,

@@ -178,6 +178,7 @@ def _layer_case(dg, cfg, P, seed, router_std=None):
     ("tiny", 300, 256, False, "cluster_merge"),
     ("one_layer", 4096, 256, False, "folded"), ("one_layer", 2048, 200, True, "folded"),
     ("one_layer", 4096, 256, False, "separate"), ("one_layer", 4096, 256, False, "cluster_merge"),
+    ("one_layer", 2048, 256, False, "topk_gather"), ("tiny", 128, 256, False, "topk_gather"),
 ])
 def test_layer_matches_oracle(dg, monkeypatch, cfg_name, P, n_rows, causal, route):
     """One layer (attention block, then MoE block) on canvas rows (bidirectional) or on a prefill
@@ -185,9 +186,12 @@ def test_layer_matches_oracle(dg, monkeypatch, cfg_name, P, n_rows, causal, rout
     the FFN RMSNorm and the router folded into the O-projection epilogue (the default for up to 1024
     rows) and the attention's key splits merged by a launch of their own (the defaults); "separate":
     DG_ROUTE_FUSED=0, an RMSNorm launch and a router GEMM; "cluster_merge": DG_ATTN_CLUSTER_MERGE=1,
-    the key splits merged inside the attention launch over a thread-block cluster."""
+    the key splits merged inside the attention launch over a thread-block cluster; "topk_gather":
+    DG_TOPK_GATHER=1, the routed rows bucketed and gathered inside the top-k launch (by default a
+    gather launch of their own)."""
     monkeypatch.setenv("DG_ROUTE_FUSED", "0" if route == "separate" else "1")
     monkeypatch.setenv("DG_ATTN_CLUSTER_MERGE", "1" if route == "cluster_merge" else "0")
+    monkeypatch.setenv("DG_TOPK_GATHER", "1" if route == "topk_gather" else "0")
     if cfg_name == "tiny":
         cfg, router_std = synthetic.TINY, None
     else:
