@@ -219,7 +219,7 @@ dg_status dg_sample(const float *d_logits, int n_seq, int vocab, const dg_sample
                     const int32_t *d_seq_P, int32_t *d_ids, uint8_t *d_commit, float *d_entropy, int32_t *d_stop,
                     void *ws, size_t ws_bytes, void *stream);
 
-/* dg_sample without a workspace argument.  The paper has no counterpart of this entry point: it is
+/* dg_sample without a workspace argument.  The method's description has no counterpart of this entry point: it is
  * an interface of this library only.  For callers that cannot allocate device memory -- a server whose pool owns all
  * free HBM, a real-time loop that must not allocate, a C component with no CUDA allocator -- the
  * sampler's per-(row, vocabulary chunk) partial results live in a static device array of the
