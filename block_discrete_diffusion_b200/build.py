@@ -55,8 +55,9 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if errors:
         raise RuntimeError("nvcc failed for " + ", ".join(s for s, _ in errors))
     objs = [o for _, o, _ in results]
+    # --no-undefined: a symbol one source declares and none defines fails here, not at load time
     subprocess.run([_nvcc(), *ARCH, "-shared", "-o", LIB + ".tmp", *objs, "-lcudart_static", "-ldl", "-lrt",
-                    "-lpthread"], check=True)
+                    "-lpthread", "-Xlinker", "--no-undefined"], check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
