@@ -354,11 +354,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (row_valid) {
         p.ml[prw * 2 + 0] = -INFINITY;
         p.ml[prw * 2 + 1] = 0.f;
-        float4* o4 = reinterpret_cast<float4*>(p.opart + prw * DH);
-        for (int c = 0; c < DH / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint4* o8 = reinterpret_cast<uint4*>(p.opart + prw * DH);
+        for (int c = 0; c < DH / 8; ++c) o8[c] = make_uint4(0u, 0u, 0u, 0u);
       }
     } else {
-      float4* o4 = reinterpret_cast<float4*>(p.opart + prw * DH);
+      // the partial row in bf16 (un-normalised, values up to l times the largest |v|): half the bytes of
+      // fp32 for the store here and the merge's loads, one more rounding of 2^-9 relative
+      uint4* o8 = reinterpret_cast<uint4*>(p.opart + prw * DH);
 #pragma unroll
       for (int cb = 0; cb < DH; cb += 32) {
         float o[32];
@@ -366,7 +368,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
         if (row_valid && ok) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) o4[(cb + i) / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+          for (int i = 0; i < 32; i += 8)
+            o8[(cb + i) / 8] = make_uint4(pack_bf16x2(o[i], o[i + 1]), pack_bf16x2(o[i + 2], o[i + 3]),
+                                          pack_bf16x2(o[i + 4], o[i + 5]), pack_bf16x2(o[i + 6], o[i + 7]));
         }
       }
       if (row_valid && ok) {
@@ -427,16 +431,16 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int s = s0 + u;
-      const float* src = p.opart + ((size_t)s * stride + r0) * DH + lane * kPer;
+      const __nv_bfloat16* src = p.opart + ((size_t)s * stride + r0) * DH + lane * kPer;
 #pragma unroll
       for (int c = 0; c < kPer; ++c) v[u][c] = 0.f;
       if (s < p.n_splits) {
         if constexpr (kPer == 4) {
-          const float4 q = ld_partial(reinterpret_cast<const float4*>(src), CG);
-          v[u][0] = q.x; v[u][1] = q.y; v[u][2] = q.z; v[u][3] = q.w;
+          const uint2 q = ld_partial(reinterpret_cast<const uint2*>(src), CG);
+          v[u][0] = bf16_lo(q.x); v[u][1] = bf16_hi(q.x); v[u][2] = bf16_lo(q.y); v[u][3] = bf16_hi(q.y);
         } else {
-          const float2 q = ld_partial(reinterpret_cast<const float2*>(src), CG);
-          v[u][0] = q.x; v[u][1] = q.y;
+          const uint32_t q = ld_partial(reinterpret_cast<const uint32_t*>(src), CG);
+          v[u][0] = bf16_lo(q); v[u][1] = bf16_hi(q);
         }
       }
     }

@@ -239,7 +239,7 @@ WsLayout ws_layout(const dg_model_config& c, int n_seq, int max_ctx) {
   L.x = take(4 * R * d);
   L.xn = take(2 * R * d);
   L.q = take(2 * (size_t)n_seq * nq * kCanvas * dh);
-  L.opart = take(4 * (size_t)L.split_cap * n_seq * nq * kCanvas * dh);
+  L.opart = take(2 * (size_t)L.split_cap * n_seq * nq * kCanvas * dh);
   L.ml = take(8 * (size_t)L.split_cap * n_seq * nq * kCanvas);
   L.attn = take(2 * R * nq * dh);
   L.rlog = take(4 * R * c.n_exp);
@@ -369,7 +369,8 @@ struct dg_seqs {
   uint8_t* ws;
   // typed workspace views
   int *err, *seqP;
-  float *x, *opart, *ml, *rlog, *gate, *y, *logits, *samp, *hsamp, *splitk;
+  float *x, *ml, *rlog, *gate, *y, *logits, *samp, *hsamp, *splitk;
+  __nv_bfloat16* opart;   // attention key-split partial outputs
   __nv_bfloat16 *xn, *q, *attn, *xp, *hb;
   int32_t *sel, *counts, *offsets, *slot, *cids, *cstop;
   uint8_t* ccommit;
@@ -592,7 +593,7 @@ DG_API dg_status dg_seqs_create(dg_model* m, int n_seq, int max_ctx, void* kv, s
   s->x = reinterpret_cast<float*>(b + L.x);
   s->xn = reinterpret_cast<__nv_bfloat16*>(b + L.xn);
   s->q = reinterpret_cast<__nv_bfloat16*>(b + L.q);
-  s->opart = reinterpret_cast<float*>(b + L.opart);
+  s->opart = reinterpret_cast<__nv_bfloat16*>(b + L.opart);
   s->ml = reinterpret_cast<float*>(b + L.ml);
   s->attn = reinterpret_cast<__nv_bfloat16*>(b + L.attn);
   s->rlog = reinterpret_cast<float*>(b + L.rlog);

@@ -124,7 +124,7 @@ struct AttnParams {
   int layer;
   int n_splits, tiles_per_split;
   const int* seq_P;
-  float* opart;          // [split][seq][n_q][rows_per_seq][dh] un-normalised partial outputs
+  __nv_bfloat16* opart;  // [split][seq][n_q][rows_per_seq][dh] un-normalised partial outputs (bf16)
   float* ml;             // [split][seq][n_q][rows_per_seq][2] (running max in log2 units, sum)
   int merge_in_cluster;  // n_splits > 1: the splits of a query-tile pair form a thread-block cluster and
                          // merge their partials after a cluster barrier (no attention_merge launch)
