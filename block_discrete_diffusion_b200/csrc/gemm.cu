@@ -432,9 +432,19 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
       }
     }
     __syncthreads();
-    // slot zz of this tile: [128][BN] fp32, written with coalesced 16-byte stores
+    // slot zz of this tile: [128][BN], written with coalesced stores.  The projections whose outputs are
+    // bf16 (Q/K/V) or small next to the fp32 residual they are added to (O) keep their partials in bf16
+    // (half the bytes through L2; one more rounding of 2^-9 relative per partial); the fp32 router
+    // logits keep fp32 partials.
+    constexpr bool kBfPart = EPI != EPI_F32;
     float* slots = ep.part + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * Z * 128 * BN;
-    {
+    if constexpr (kBfPart) {
+      uint2* dst = reinterpret_cast<uint2*>(slots) + (size_t)zz * 128 * F4;
+      for (int i = threadIdx.x; i < 128 * F4; i += kGemmThreads) {
+        const float4 v = *reinterpret_cast<const float4*>(red + (i / F4) * RS + 4 * (i % F4));
+        __stcg(dst + i, make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
+      }
+    } else {
       float4* dst = reinterpret_cast<float4*>(slots + (size_t)zz * 128 * BN);
       for (int i = threadIdx.x; i < 128 * F4; i += kGemmThreads)
         __stcg(dst + i, *reinterpret_cast<const float4*>(red + (i / F4) * RS + 4 * (i % F4)));
@@ -460,7 +470,14 @@ __global__ void __launch_bounds__(kGemmThreads, DenseCfg<BN>::kMinBlocks)
           const int i = threadIdx.x + (i0 + b) * kGemmThreads;
           const size_t off = (size_t)(zz * RPC + i / F4) * BN + 4 * (i % F4);
 #pragma unroll
-          for (int z = 0; z < Z; ++z) v[b][z] = __ldcg(reinterpret_cast<const float4*>(slots + (size_t)z * 128 * BN + off));
+          for (int z = 0; z < Z; ++z) {
+            if constexpr (kBfPart) {
+              const uint2 q = __ldcg(reinterpret_cast<const uint2*>(slots) + ((size_t)z * 128 * BN + off) / 4);
+              v[b][z] = make_float4(bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y));
+            } else {
+              v[b][z] = __ldcg(reinterpret_cast<const float4*>(slots + (size_t)z * 128 * BN + off));
+            }
+          }
         }
 #pragma unroll
         for (int b = 0; b < B; ++b) {
