@@ -411,23 +411,11 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
   const int sh = seq * p.n_q + h;
   const size_t stride = (size_t)n_seq * p.n_q * p.rows_per_seq;
   const size_t r0 = (size_t)sh * p.rows_per_seq + j;
-  float ms = -INFINITY, ls = 0.f;
-  if (lane < p.n_splits) {
-    const float2 v = ld_partial(reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2), CG);
-    ms = v.x;
-    ls = v.y;
-  }
-  const float M = warp_max(ms);
-  const float wgt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-  const float den = warp_sum(wgt * ls);
-  const float inv = den > 0.f ? 1.f / den : 0.f;
   constexpr int kPer = DH / 32;
-  float acc[kPer];
-#pragma unroll
-  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
-  // splits in groups of 8: the group's loads are all issued before they are summed (in split order)
-  for (int s0 = 0; s0 < p.n_splits; s0 += 8) {
-    float v[8][kPer];
+  // splits in groups of 8: a group's loads are all issued before they are summed (in split order); the
+  // first group's loads are issued together with the (m, l) loads, before the weights are reduced
+  float v[8][kPer];
+  auto load_group = [&](int s0) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int s = s0 + u;
@@ -444,6 +432,22 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
         }
       }
     }
+  };
+  float ms = -INFINITY, ls = 0.f;
+  if (lane < p.n_splits) {
+    const float2 q = ld_partial(reinterpret_cast<const float2*>(p.ml + (lane * stride + r0) * 2), CG);
+    ms = q.x;
+    ls = q.y;
+  }
+  load_group(0);
+  const float M = warp_max(ms);
+  const float wgt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+  const float den = warp_sum(wgt * ls);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  float acc[kPer];
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+  for (int s0 = 0;;) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const float ws = __shfl_sync(0xffffffffu, wgt, (s0 + u) & 31);
@@ -452,6 +456,9 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int n_seq, int se
         for (int c = 0; c < kPer; ++c) acc[c] += ws * v[u][c];
       }
     }
+    s0 += 8;
+    if (s0 >= p.n_splits) break;
+    load_group(s0);
   }
   __nv_bfloat16* dst = out + ((size_t)seq * p.rows_per_seq + j) * (p.n_q * DH) + h * DH + lane * kPer;
   if constexpr (kPer == 4) {
